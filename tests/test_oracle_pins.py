@@ -1,0 +1,485 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the oracle itself.
+
+Each pin targets a mistake the oracle could plausibly make: a transposed factor, a dropped
+rank term, a wrong softmax normalisation, a reversed summation order, a double rounding,
+a wrong tie-break, a wrong leader.  Sources: the xKV page (section 2.2 cross-layer
+factorization, 2.3 selective reconstruction, section 4 dense reconstruction) and the
+Stochastic KV Routing page (inference sharing strategy S, Algorithm 2 load/update skip,
+the 32K Qwen3-8B memory figure).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from cross_layer_compressed_b200 import synth
+
+
+def _f32(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+
+
+def _sdpa64(q, K, V):
+    """torch SDPA in fp64 on CPU; q [Hq][hd], K/V [Hkv][T][hd] with GQA by repeat."""
+    Hq, hd = q.shape
+    Hkv = K.shape[0]
+    G = Hq // Hkv
+    Kr = torch.as_tensor(K, dtype=torch.float64).repeat_interleave(G, 0)
+    Vr = torch.as_tensor(V, dtype=torch.float64).repeat_interleave(G, 0)
+    qq = torch.as_tensor(q, dtype=torch.float64)[:, None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qq, Kr, Vr)
+    return o[:, 0, :].numpy()
+
+
+# ------------------------------------------------------------------ rounding helper
+@pytest.mark.parametrize("x,bits", [
+    (1.0, 0x3F80),
+    (1.0 + 2 ** -8, 0x3F80),                 # exact half-way: ties to even (down)
+    (1.0 + 3 * 2 ** -8, 0x3F82),             # exact half-way: ties to even (up)
+    (1.0 + 2 ** -8 + 2 ** -40, 0x3F81),      # above half-way; an fp32 detour would tie down
+    (-(1.0 + 2 ** -8 + 2 ** -40), 0xBF81),
+    (3.0e38, 0x7F62),
+    (1e39, 0x7F80),                          # overflow to +inf
+    (2.0 ** -133, 0x0001),                   # smallest bf16 subnormal
+    (0.0, 0x0000),
+])
+def test_round_bf16_nearest_even_single_step(ora, x, bits):
+    assert ora.round_bf16(x) == bits
+
+
+# ---------------------------------------------------- xKV 2.2: factorization pins
+def _window_svd(L, W, d_kv, seed):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((L, W * d_kv))
+    U, s, Vt = np.linalg.svd(X, full_matrices=False)
+    A = U * s[None, :]                     # L x r (r = min(L, W*d_kv))
+    return X, A, Vt                        # X = A @ Vt
+
+
+def test_full_rank_factors_reconstruct_the_window(ora):
+    """Full-rank SVD factors rebuild each layer's block of the concatenated cache."""
+    L, W, d_kv = 48, 3, 8
+    X, A, Vt = _window_svd(L, W, d_kv, 1)
+    A32 = A.astype(np.float32)
+    for layer in range(W):
+        Bl = Vt[:, layer * d_kv:(layer + 1) * d_kv]          # r x d_kv
+        Bt32 = np.ascontiguousarray(Bl.T.astype(np.float32))  # stored column-major
+        rec = ora.reconstruct_rows(_f32(A32), _f32(Bt32), 0, L)
+        ref = X[:, layer * d_kv:(layer + 1) * d_kv]
+        assert np.max(np.abs(rec - ref)) <= 2e-6 * np.max(np.abs(ref))
+        # and exactly the product of the stored factors (library matmul in fp64)
+        exact = A32.astype(np.float64) @ Bt32.astype(np.float64).T
+        assert np.max(np.abs(rec - exact)) <= 1e-12 * np.max(np.abs(exact))
+
+
+def test_truncated_rank_drops_exactly_the_tail(ora):
+    """Rank-r factors give the best rank-r approximation: the residual's spectral norm is
+    the (r+1)-th singular value (Eckart-Young)."""
+    L, W, d_kv, r = 40, 2, 8, 5
+    X, A, Vt = _window_svd(L, W, d_kv, 2)
+    s = np.linalg.svd(X, compute_uv=False)
+    A32 = np.ascontiguousarray(A[:, :r].astype(np.float32))
+    rec = np.hstack([ora.reconstruct_rows(_f32(A32), _f32(np.ascontiguousarray(
+        Vt[:r, l * d_kv:(l + 1) * d_kv].T.astype(np.float32))), 0, L) for l in range(W)])
+    resid = np.linalg.norm(X - rec, 2)
+    assert abs(resid - s[r]) <= 1e-5 * s[0]
+
+
+# ---------------------------------------- dense reconstruction = plain attention
+def _xkv_case(L, W, Hq, Hkv, hd, seed, chunk=8):
+    """W=1 full-rank factors of random K and V caches (fp32 storage)."""
+    d_kv = Hkv * hd
+    rng = np.random.default_rng(seed)
+    XK = rng.standard_normal((L, d_kv)) * 0.5
+    XV = rng.standard_normal((L, d_kv))
+    out = {}
+    for tag, X in (("k", XK), ("v", XV)):
+        U, s, Vt = np.linalg.svd(X, full_matrices=False)
+        out["A" + tag] = np.ascontiguousarray((U * s).astype(np.float32))[None]
+        out["B" + tag + "t"] = np.ascontiguousarray(Vt.T.astype(np.float32))[None]
+    q = (rng.standard_normal((1, Hq, hd)) * 0.7).astype(np.float32)
+    return XK, XV, out, q
+
+
+def _khat(out, tag, Hkv, hd):
+    A = out["A" + tag][0].astype(np.float64)
+    Bt = out["B" + tag + "t"][0].astype(np.float64)
+    X = A @ Bt.T                                                  # L x d_kv
+    return np.stack([X[:, g * hd:(g + 1) * hd] for g in range(Hkv)])  # Hkv x L x hd
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (4, 4), (5, 1)])
+def test_dense_reconstruction_equals_sdpa(ora, Hq, Hkv):
+    L, hd, C = 64, 16, 8
+    XK, XV, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 3)
+    o = ora.reconstruct_attend(_f32(f["Ak"]), _f32(f["Av"]), _f32(f["Bkt"]), _f32(f["Bvt"]),
+                               _f32(q), None, C)
+    K, V = _khat(f, "k", Hkv, hd), _khat(f, "v", Hkv, hd)
+    ref = _sdpa64(q[0], K, V)
+    assert np.max(np.abs(o[0] - ref)) <= 1e-6 * np.max(np.abs(ref))
+    # against the uncompressed caches: the factorization is lossless at full rank
+    Ko = np.stack([XK[:, g * hd:(g + 1) * hd] for g in range(Hkv)])
+    Vo = np.stack([XV[:, g * hd:(g + 1) * hd] for g in range(Hkv)])
+    ref0 = _sdpa64(q[0], Ko, Vo)
+    assert np.max(np.abs(o[0] - ref0)) <= 1e-5 * np.max(np.abs(ref0))
+
+
+def test_selecting_every_chunk_equals_dense(ora):
+    L, hd, C, Hq, Hkv = 64, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 4)
+    args = [_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")] + [_f32(q)]
+    dense = ora.reconstruct_attend(*args, None, C)
+    sel = np.tile(np.arange(L // C, dtype=np.int32), (1, Hkv, 1))
+    assert np.array_equal(ora.reconstruct_attend(*args, sel, C), dense)
+
+
+def test_selective_equals_sdpa_over_selected_rows(ora):
+    L, hd, C, Hq, Hkv = 128, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 5)
+    sel = np.array([[[0, 3, 7, 15], [1, 2, 9, 14]]], dtype=np.int32)
+    o = ora.reconstruct_attend(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")], _f32(q),
+                               sel, C)
+    K, V = _khat(f, "k", Hkv, hd), _khat(f, "v", Hkv, hd)
+    G = Hq // Hkv
+    for g in range(Hkv):
+        rows = np.concatenate([np.arange(c * C, (c + 1) * C) for c in sel[0, g]])
+        ref = _sdpa64(q[0, g * G:(g + 1) * G], K[g:g + 1, rows], V[g:g + 1, rows])
+        assert np.max(np.abs(o[0, g * G:(g + 1) * G] - ref)) <= 1e-6 * np.max(np.abs(ref))
+
+
+def test_softmax_shift_invariance_through_an_extra_rank_term(ora):
+    """Adding u to every key row (a rank-1 term: a ones column in A^K, u in B^K) shifts each
+    head's logits by a constant, which softmax ignores.  Catches a dropped rank term or a
+    missing normalisation."""
+    L, hd, C, Hq, Hkv = 64, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 6)
+    rng = np.random.default_rng(60)
+    u = rng.standard_normal(Hkv * hd).astype(np.float32) * 3
+    Ak2 = np.concatenate([f["Ak"], np.ones((1, L, 1), np.float32)], axis=2)
+    Bkt2 = np.concatenate([f["Bkt"], u[None, :, None]], axis=2)
+    sel = np.array([[[0, 2, 5], [1, 6, 7]]], dtype=np.int32)
+    base = ora.reconstruct_attend(_f32(f["Ak"]), _f32(f["Av"]), _f32(f["Bkt"]), _f32(f["Bvt"]),
+                                  _f32(q), sel, C)
+    shifted = ora.reconstruct_attend(_f32(Ak2), _f32(f["Av"]), _f32(Bkt2), _f32(f["Bvt"]),
+                                     _f32(q), sel, C)
+    assert np.max(np.abs(base - shifted)) <= 1e-5 * np.max(np.abs(base))
+    # ... whereas adding it to only some rows must change the result
+    Ak3 = Ak2.copy()
+    Ak3[0, :8, -1] = 0.0
+    moved = ora.reconstruct_attend(_f32(Ak3), _f32(f["Av"]), _f32(Bkt2), _f32(f["Bvt"]),
+                                   _f32(q), sel, C)
+    assert np.max(np.abs(base - moved)) > 1e-3 * np.max(np.abs(base))
+
+
+def test_chunk_permutation_invariance(ora):
+    L, hd, C, Hq, Hkv = 64, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 7)
+    nC = L // C
+    perm = np.random.default_rng(70).permutation(nC)       # new chunk i holds old perm[i]
+    inv = np.argsort(perm)
+    rows = np.concatenate([np.arange(p * C, (p + 1) * C) for p in perm])
+    sel = np.array([[[0, 1, 4, 6], [2, 3, 5, 7]]], dtype=np.int32)
+    sel_p = np.sort(inv[sel], axis=2).astype(np.int32)
+    a = ora.reconstruct_attend(_f32(f["Ak"]), _f32(f["Av"]), _f32(f["Bkt"]), _f32(f["Bvt"]),
+                               _f32(q), sel, C)
+    b = ora.reconstruct_attend(_f32(np.ascontiguousarray(f["Ak"][:, rows])),
+                               _f32(np.ascontiguousarray(f["Av"][:, rows])), _f32(f["Bkt"]),
+                               _f32(f["Bvt"]), _f32(q), sel_p, C)
+    assert np.max(np.abs(a - b)) <= 1e-6 * np.max(np.abs(a))
+
+
+def test_zero_query_gives_mean_of_selected_values(ora):
+    """q = 0: uniform weights, so out = (mean of the selected A^V rows) B^V_g (closed form)."""
+    L, hd, C, Hq, Hkv = 64, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 8)
+    q0 = np.zeros_like(q)
+    sel = np.array([[[1, 5], [0, 7]]], dtype=np.int32)
+    o = ora.reconstruct_attend(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")], _f32(q0),
+                               sel, C)
+    Av = f["Av"][0].astype(np.float64)
+    Bvt = f["Bvt"][0].astype(np.float64)
+    G = Hq // Hkv
+    for g in range(Hkv):
+        rows = np.concatenate([np.arange(c * C, (c + 1) * C) for c in sel[0, g]])
+        ref = Av[rows].mean(0) @ Bvt[g * hd:(g + 1) * hd].T
+        for h in range(G):
+            assert np.max(np.abs(o[0, g * G + h] - ref)) <= 1e-6 * np.max(np.abs(ref))
+
+
+def test_one_sharp_chunk_dominates(ora):
+    """A query aligned with one row's key at large scale puts all weight on that row."""
+    L, hd, C, Hq, Hkv = 32, 16, 8, 2, 1
+    _, _, f, _ = _xkv_case(L, 1, Hq, Hkv, hd, 9)
+    K = _khat(f, "k", Hkv, hd)[0]
+    V = _khat(f, "v", Hkv, hd)[0]
+    t = 13
+    q = np.stack([K[t] * 400.0, K[t] * 400.0])[None].astype(np.float32)
+    o = ora.reconstruct_attend(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")], _f32(q),
+                               None, C)
+    assert np.max(np.abs(o[0, 0] - V[t])) <= 1e-5 * np.max(np.abs(V[t]))
+
+
+def test_bf16_inputs_are_widened_exactly(ora):
+    """bf16 storage: the oracle must read each value exactly (compare with the same inputs
+    widened by torch)."""
+    L, hd, C, Hq, Hkv = 32, 16, 8, 4, 2
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 10)
+    bf = {k: torch.from_numpy(v).to(torch.bfloat16) for k, v in f.items()}
+    qb = torch.from_numpy(q).to(torch.bfloat16)
+    o = ora.reconstruct_attend(bf["Ak"], bf["Av"], bf["Bkt"], bf["Bvt"], qb, None, C)
+    o32 = ora.reconstruct_attend(*[bf[k].float() for k in ("Ak", "Av", "Bkt", "Bvt")],
+                                 qb.float(), None, C)
+    assert np.array_equal(o, o32)
+
+
+# ------------------------------------------------------------ landmark scoring pins
+def test_score_integer_dot_products_and_group_max(ora):
+    """Small integers are exact in bf16 and their dot products are exact in fp64."""
+    rng = np.random.default_rng(11)
+    B, Hkv, G, nC, hd = 2, 3, 4, 10, 16
+    lm = rng.integers(-8, 9, size=(B, Hkv, nC, hd))
+    q = rng.integers(-8, 9, size=(B, Hkv * G, hd))
+    s = ora.score_landmarks(torch.tensor(lm, dtype=torch.bfloat16),
+                            torch.tensor(q, dtype=torch.bfloat16))
+    ref = np.einsum("bgcd,bghd->bgch", lm, q.reshape(B, Hkv, G, hd)).max(-1)
+    assert np.array_equal(s, ref.astype(np.float64))
+
+
+def test_score_sums_in_ascending_dimension_order(ora):
+    """lm = [2^53, 1, -2^53, 0...], q = 1: ascending order gives (2^53 + 1) - 2^53 = 0 in
+    fp64 (2^53 + 1 rounds to 2^53); the exact value, or a descending sum, gives 1."""
+    hd = 8
+    lm = np.zeros((1, 1, 1, hd))
+    lm[0, 0, 0, :3] = [2.0 ** 53, 1.0, -(2.0 ** 53)]
+    q = np.ones((1, 1, hd))
+    s = ora.score_landmarks(torch.tensor(lm, dtype=torch.bfloat16),
+                            torch.tensor(q, dtype=torch.bfloat16))
+    assert s[0, 0, 0] == 0.0
+
+
+def test_score_fp32_products_exact(ora):
+    """fp32 x fp32 products have at most 48 significant bits: exact in fp64, so a single
+    product is reproduced exactly."""
+    rng = np.random.default_rng(12)
+    a = rng.standard_normal(5).astype(np.float32)
+    b = rng.standard_normal(5).astype(np.float32)
+    for x, y in zip(a, b):
+        lm = np.zeros((1, 1, 1, 4), np.float32)
+        q = np.zeros((1, 1, 4), np.float32)
+        lm[0, 0, 0, 2] = x
+        q[0, 0, 2] = y
+        s = ora.score_landmarks(_f32(lm), _f32(q))
+        assert s[0, 0, 0] == float(x) * float(y)
+
+
+# ------------------------------------------------------------------ selection pins
+def _brute_force_select(scores, k, forced):
+    """Exhaustive: the unique k-subset of candidates such that every member precedes every
+    non-member under (score descending, index ascending)."""
+    n = len(scores)
+    cand = [c for c in range(n) if c not in forced]
+    k = min(k, len(cand))
+    hits = []
+    for sub in itertools.combinations(cand, k):
+        rest = [c for c in cand if c not in sub]
+        ok = all((scores[a] > scores[b]) or (scores[a] == scores[b] and a < b)
+                 for a in sub for b in rest)
+        if ok:
+            hits.append(sorted(set(sub) | set(forced)))
+    assert len(hits) == 1
+    return hits[0]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_matches_brute_force_with_ties(ora, seed):
+    rng = np.random.default_rng(100 + seed)
+    n = 12
+    scores = rng.integers(-3, 4, size=n).astype(np.float64)   # many exact ties
+    for k, sink, recent in [(4, 1, 1), (3, 0, 0), (2, 2, 3), (4, 0, 2), (0, 1, 1)]:
+        forced = sorted(set(range(sink)) | set(range(n - recent, n)))
+        want = _brute_force_select(scores, k, forced)
+        got = ora.select_chunks(scores[None, None, :], k, sink, recent)[0, 0]
+        assert list(got) == want
+
+
+def test_select_k_at_least_candidates_takes_everything(ora):
+    s = np.arange(10, dtype=np.float64)[None, None, :]
+    assert list(ora.select_chunks(s, 50, 1, 2)[0, 0]) == list(range(10))
+    # sink and recent overlapping on a tiny context
+    assert list(ora.select_chunks(s[:, :, :3], 1, 2, 2)[0, 0]) == [0, 1, 2]
+    assert ora.n_selected(3, 1, 2, 2) == 3
+
+
+def test_select_orders_negative_zero_below_positive_zero(ora):
+    s = np.array([[[5.0, -0.0, 0.0, -1.0]]])
+    assert list(ora.select_chunks(s, 2, 0, 0)[0, 0]) == [0, 2]
+
+
+def test_select_is_per_unit(ora):
+    s = np.array([[[1.0, 9.0, 3.0, 2.0], [9.0, 1.0, 2.0, 3.0]],
+                  [[0.0, 0.0, 0.0, 0.0], [1.0, 2.0, 3.0, 4.0]]])
+    got = ora.select_chunks(s, 1, 0, 1)
+    assert got.tolist() == [[[1, 3], [0, 3]], [[0, 3], [2, 3]]]
+
+
+# --------------------------------------------------------------- landmark pins
+def test_landmarks_are_chunk_means_of_reconstructed_keys(ora):
+    """Linearity: mean_t(A[t] B) = (mean_t A[t]) B; the oracle rounds once to fp32."""
+    w = synth.reduced(synth.TINY_SR_F32, batch=1, ctx_len=64)
+    x = synth.np_xkv_layer_inputs(w, 0, 0)
+    lm = ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk)
+    A = x["Ak"][0].double().numpy()
+    Bt = x["Bkt"][0].double().numpy()
+    abar = A.reshape(-1, w.chunk, A.shape[1]).mean(1)                 # nC x r
+    ref = (abar @ Bt.T).reshape(-1, w.n_kv_heads, w.head_dim).transpose(1, 0, 2)
+    ulp = np.spacing(np.abs(ref).astype(np.float32))
+    assert np.all(np.abs(lm[0].astype(np.float64) - ref) <= ulp)
+
+
+def test_landmarks_bf16_within_one_ulp_of_exact_mean(ora):
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=1, ctx_len=64, rank_k=32, rank_v=32,
+                      n_kv_heads=2, n_q_heads=4, head_dim=16, n_needles=0)
+    x = synth.np_xkv_layer_inputs(w, 0, 0)
+    lm = ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk)
+    got = ora.as_float64(ora.to_torch(lm))
+    A = x["Ak"][0].double().numpy()
+    Bt = x["Bkt"][0].double().numpy()
+    ref = (A.reshape(-1, w.chunk, A.shape[1]).mean(1) @ Bt.T).reshape(
+        -1, w.n_kv_heads, w.head_dim).transpose(1, 0, 2)
+    half_ulp = np.abs(ref) * 2.0 ** -8                                 # bf16: 8 bits
+    assert np.all(np.abs(got[0] - ref) <= half_ulp * 1.0000001)
+
+
+# --------------------------------------------------------------------- R-CLA pins
+def test_leader_map_nearest_previous_leader(ora):
+    S = list(range(0, 36, 4))
+    lo = ora.leader_map(S, 36)
+    assert lo.tolist() == [4 * (l // 4) for l in range(36)]
+    lo2 = ora.leader_map([0, 1, 5, 6, 20], 24)
+    want = [0, 1, 1, 1, 1, 5, 6] + [6] * 13 + [20] * 4
+    assert lo2.tolist() == want
+    with pytest.raises(ValueError):
+        ora.leader_map([3, 7], 10)                                    # layer 0 has no leader
+
+
+def _rcla_case(B=2, Hkv=2, G=2, hd=16, L_max=40, length=30, n_lead=3, seed=20):
+    rng = np.random.default_rng(seed)
+    K = np.zeros((n_lead, B, Hkv, L_max, hd), np.float32)
+    V = np.zeros((n_lead, B, Hkv, L_max, hd), np.float32)
+    K[..., :length, :] = rng.standard_normal((n_lead, B, Hkv, length, hd))
+    V[..., :length, :] = rng.standard_normal((n_lead, B, Hkv, length, hd))
+    q = rng.standard_normal((B, Hkv * G, hd)).astype(np.float32)
+    kn = rng.standard_normal((B, Hkv, hd)).astype(np.float32)
+    vn = rng.standard_normal((B, Hkv, hd)).astype(np.float32)
+    return K, V, q, kn, vn
+
+
+def test_rcla_leader_update_then_attend_equals_sdpa(ora):
+    K, V, q, kn, vn = _rcla_case()
+    S = [0, 2, 5]
+    lo = ora.leader_map(S, 8)
+    length = 30
+    K0, V0 = K.copy(), V.copy()
+    o = ora.rcla_decode_attend(5, lo, K, V, length, _f32(kn), _f32(vn), _f32(q))
+    slot = 2
+    assert np.array_equal(K[slot, :, :, length], kn) and np.array_equal(V[slot, :, :, length], vn)
+    mask = np.ones(K.shape, bool)
+    mask[slot, :, :, length] = False
+    assert np.array_equal(K[mask], K0[mask])                          # nothing else written
+    for b in range(2):
+        ref = _sdpa64(q[b], K[slot, b, :, :length + 1], V[slot, b, :, :length + 1])
+        assert np.max(np.abs(o[b] - ref)) <= 1e-6 * np.max(np.abs(ref))
+
+
+def test_rcla_non_leader_reads_leader_cache_and_writes_nothing(ora):
+    K, V, q, _, _ = _rcla_case(seed=21)
+    lo = ora.leader_map([0, 2, 5], 8)
+    K0 = K.copy()
+    o = ora.rcla_decode_attend(4, lo, K, V, 31, None, None, _f32(q))  # leader of 4 is 2
+    assert np.array_equal(K, K0)
+    for b in range(2):
+        ref = _sdpa64(q[b], K[1, b, :, :31], V[1, b, :, :31])
+        assert np.max(np.abs(o[b] - ref)) <= 1e-6 * np.max(np.abs(ref))
+    with pytest.raises(ValueError):                                   # non-leader owns no cache
+        ora.rcla_decode_attend(4, lo, K, V, 31, _f32(np.zeros((2, 2, 16))),
+                               _f32(np.zeros((2, 2, 16))), _f32(q))
+
+
+def test_rcla_single_row_returns_that_value(ora):
+    """len = 0 with an update: one row, weight 1, so out = v_new (closed form)."""
+    K, V, q, kn, vn = _rcla_case(length=0, seed=22)
+    lo = ora.leader_map([0], 2)
+    o = ora.rcla_decode_attend(0, lo, K, V, 0, _f32(kn), _f32(vn), _f32(q))
+    G = 2
+    for b in range(2):
+        for h in range(4):
+            assert np.array_equal(o[b, h], vn[b, h // G])
+
+
+# ------------------------------------------------------------------ footprint pins
+def test_footprint_equals_bytes_of_generated_tensors(ora):
+    """xKV 2.2 storage O(L*r + W*r*d): compare the closed form with the bytes of the
+    tensors the generator actually builds."""
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=1, ctx_len=64, rank_k=32, rank_v=48,
+                      n_layers=5, window=2, n_kv_heads=2, n_q_heads=4, head_dim=16,
+                      n_needles=0)
+    total = 0
+    for win in range(w.n_windows):
+        x = synth.np_xkv_layer_inputs(w, 0, win * w.window)
+        total += x["Ak"].nbytes + x["Av"].nbytes
+    for layer in range(w.n_layers):
+        x = synth.np_xkv_layer_inputs(w, 0, layer)
+        total += x["Bkt"].nbytes + x["Bvt"].nbytes
+    got = ora.footprint_bytes(w.batch, w.n_kv_heads, w.head_dim, w.ctx_len, w.chunk, w.rank_k,
+                              w.rank_v, 1, w.n_layers, w.window, False)
+    assert got == total
+    lm_bytes = w.n_layers * w.n_chunks * w.d_kv * 2
+    assert ora.footprint_bytes(w.batch, w.n_kv_heads, w.head_dim, w.ctx_len, w.chunk, w.rank_k,
+                               w.rank_v, 1, w.n_layers, w.window, True) == total + lm_bytes
+
+
+def test_footprint_is_smaller_than_dense_by_the_page_formula(ora):
+    """For W layers of L tokens: W*L*d (dense, per K or V) vs L*r + W*r*d."""
+    L, W, r, d = 32768, 4, 512, 1024
+    got = ora.footprint_bytes(1, 8, 128, L, 8, r, r, 1, W, W, False)
+    assert got == 2 * (L * r + W * r * d) * 2
+    assert got < 2 * W * L * d * 2
+
+
+def test_rcla_cache_bytes_match_the_page(ora):
+    """Stochastic KV Routing page: Qwen3-8B at 32K, one cache per 4 layers, 4.6 -> 1.1 GB (4x)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "rcla_qwen3_8b_32k_kv_bytes.txt")
+    g = {}
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, v = line.split()
+            g[k] = float(v)
+    n = int(g["n_layers"])
+    leaders = len(range(0, n, int(g["leader_stride"])))
+    dense = ora.rcla_cache_bytes(1, int(g["n_kv_heads"]), int(g["head_dim"]), int(g["ctx_len"]),
+                                 1, n)
+    shared = ora.rcla_cache_bytes(1, int(g["n_kv_heads"]), int(g["head_dim"]), int(g["ctx_len"]),
+                                  1, leaders)
+    assert dense == n * int(g["ctx_len"]) * 2 * int(g["n_kv_heads"]) * int(g["head_dim"]) * 2
+    assert dense / shared == g["ratio"]
+    gib = 2.0 ** 30
+    # the page prints one decimal without a unit; in GiB both agree to within 3 %
+    assert abs(dense / gib - g["dense_gb"]) <= 0.03 * g["dense_gb"]
+    assert abs(shared / gib - g["shared_gb"]) <= 0.03 * g["shared_gb"]
+
+
+# ------------------------------------------------------------ workload sanity
+def test_needles_are_selected_by_the_oracle(ora):
+    """The planted needle chunks reach the top-k of every (sequence, KV head)."""
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=1024, rank_k=128, rank_v=64,
+                      n_kv_heads=2, n_q_heads=8, head_dim=128, top_k=8)
+    x = synth.np_xkv_layer_inputs(w, 0, 1)
+    lm = ora.to_torch(ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    s = ora.score_landmarks(lm, x["q"])
+    sel = ora.select_chunks(s, w.top_k, w.n_sink, w.n_recent)
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            assert set(x["needles"][b].tolist()) <= set(sel[b, g].tolist())
