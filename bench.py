@@ -1,0 +1,507 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark over a cross-layer-compressed KV cache (one JSON line).
+
+A step is one decode step of every layer for every sequence of the workload: for the
+selective xKV workloads, landmark scoring, chunk selection and reconstruct+attend per
+layer; for dense reconstruction, reconstruct+attend; for R-CLA, the leader update and
+attention per layer.  Layers run in order (a layer's query depends on the previous
+layer's output in a real model).  Inputs are synthetic, seeded, generated on the device
+before timing; the cache (bases, matrices, landmarks, leader caches) stays resident.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl cuda|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of the
+workload (sequences are independent: no collective on the data path); value is the
+aggregate over ranks, timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn tokens/s (batch×steps) at 32K ctx; HBM GB/s vs 8 TB/s peak"
+DEFAULT_WORKLOAD = "llama8b_sr_32k"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=16)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ident = vis.split(",")[device_index] if vis else str(device_index)
+        self.ident = ident
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------ workloads
+class XkvStep:
+    """Device-resident xKV workload (selective or dense) and its decode step."""
+
+    def __init__(self, w, seed, dev):
+        import torch
+        from cross_layer_compressed_b200 import synth
+        from cross_layer_compressed_b200 import xkv
+        self.w, self.dev, self.xkv = w, dev, xkv
+        self.d = xkv.dims_of(w)
+        self.cache = synth.torch_xkv_cache(w, seed, device=dev)
+        dt = self.cache["Ak"].dtype
+        self.dense = w.mode == "dense"
+        self.lm = None
+        if not self.dense:
+            self.lm = torch.empty((w.n_layers, w.batch, w.n_kv_heads, w.n_chunks, w.head_dim),
+                                  dtype=dt, device=dev)
+            for l in range(w.n_layers):
+                xkv.xkv_build_landmarks(self.d, self.cache["Ak"][l // w.window],
+                                        self.cache["Bkt"][l], self.lm[l])
+        self.qpool = synth.torch_queries(w, seed, self.cache, device=dev)   # [nq][N][B][Hq][hd]
+        self.n_sel = 0 if self.dense else w.n_sel
+        mode = xkv.XKV_MODE_DENSE if self.dense else xkv.XKV_MODE_SELECTIVE
+        self.ws = torch.empty(xkv.xkv_workspace_bytes(self.d, self.n_sel, mode),
+                              dtype=torch.uint8, device=dev)
+        self.scores = torch.empty((w.batch, w.n_kv_heads, max(w.n_chunks, 1)),
+                                  dtype=torch.float64, device=dev)
+        self.sel = torch.empty((w.n_layers, w.batch, w.n_kv_heads, max(self.n_sel, 1)),
+                               dtype=torch.int32, device=dev)
+        self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
+                               dtype=torch.float32, device=dev)
+        self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
+        self.launches_per_step = w.n_layers * (2 if self.dense else 4)
+        torch.cuda.synchronize()
+
+    def resident_bytes(self):
+        n = sum(t.numel() * t.element_size() for t in self.cache.values())
+        if self.lm is not None:
+            n += self.lm.numel() * self.lm.element_size()
+        return n
+
+    def step(self, slot=None, q=None, attend_events=None):
+        w, xkv, d = self.w, self.xkv, self.d
+        qq = self.qpool[slot] if q is None else q
+        for l in range(w.n_layers):
+            win = l // w.window
+            if not self.dense:
+                xkv.xkv_score_landmarks(d, self.lm[l], qq[l], self.scores)
+                xkv.xkv_select_chunks(d, self.scores, w.top_k, w.n_sink, w.n_recent, self.sel[l])
+            if attend_events is not None:
+                attend_events[l][0].record()
+            xkv.xkv_reconstruct_attend(d, self.cache["Ak"][win], self.cache["Av"][win],
+                                       self.cache["Bkt"][l], self.cache["Bvt"][l], qq[l],
+                                       None if self.dense else self.sel[l], self.n_sel,
+                                       self.out[l], self.ws)
+            if attend_events is not None:
+                attend_events[l][1].record()
+
+    def attend_bytes(self, slots):
+        """Algorithmic bytes of each reconstruct+attend launch (per layer), averaged over
+        the query slots used: the union over KV heads of the selected rows of A^K and A^V
+        per sequence, B_l (K and V), the selection, q and out."""
+        import torch
+        w = self.w
+        e = self.cache["Ak"].element_size()
+        per_launch = []
+        for slot in slots:
+            self.step(slot)                    # recompute this slot's selections (untimed)
+            torch.cuda.synchronize()
+            for l in range(w.n_layers):
+                if self.dense:
+                    rows = w.batch * w.ctx_len
+                else:
+                    mask = torch.zeros((w.batch, w.n_chunks), dtype=torch.bool, device=self.dev)
+                    mask.scatter_(1, self.sel[l].reshape(w.batch, -1).long(), True)
+                    rows = int(mask.sum().item()) * w.chunk
+                nbytes = (rows * (w.rank_k + w.rank_v) * e
+                          + w.batch * w.d_kv * (w.rank_k + w.rank_v) * e
+                          + w.batch * w.n_q_heads * w.head_dim * (e + 4)
+                          + (0 if self.dense else w.batch * w.n_kv_heads * self.n_sel * 4))
+                per_launch.append(nbytes)
+        return float(np.mean(per_launch))
+
+    def step_bytes(self, attend_bytes_per_launch):
+        w = self.w
+        e = self.cache["Ak"].element_size()
+        lm = 0 if self.dense else w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * e
+        sc = 0 if self.dense else w.batch * w.n_kv_heads * w.n_chunks * 8 * 2
+        return w.n_layers * (attend_bytes_per_launch + lm + sc)
+
+    def io_bytes(self):
+        w = self.w
+        return (self.q_in.numel() * self.q_in.element_size(),
+                self.out.numel() * self.out.element_size())
+
+
+class RclaStep:
+    """Device-resident R-CLA workload and its decode step (leaders append, then attend)."""
+
+    def __init__(self, w, seed, dev):
+        import torch
+        from cross_layer_compressed_b200 import synth
+        from cross_layer_compressed_b200 import xkv
+        self.w, self.dev, self.xkv = w, dev, xkv
+        self.d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+        c = synth.torch_rcla_cache(w, seed, device=dev)
+        self.K, self.V, self.kn, self.vn = c["K_lead"], c["V_lead"], c["k_new"], c["v_new"]
+        self.S = synth.leader_set(w)
+        self.lo = [max(s for s in self.S if s <= l) for l in range(w.n_layers)]
+        self.qpool = synth.torch_queries(w, seed, None, device=dev)
+        self.ws = torch.empty(xkv.xkv_workspace_bytes(self.d, 0, xkv.XKV_MODE_RCLA),
+                              dtype=torch.uint8, device=dev)
+        self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
+                               dtype=torch.float32, device=dev)
+        self.q_in = torch.empty_like(self.qpool[0])
+        self.len = w.ctx_len
+        self.launches_per_step = w.n_layers * 2
+        self.step_index = 0
+        torch.cuda.synchronize()
+
+    def resident_bytes(self):
+        return 2 * self.K.numel() * self.K.element_size()
+
+    def step(self, slot=None, q=None, attend_events=None):
+        w, xkv = self.w, self.xkv
+        qq = self.qpool[slot] if q is None else q
+        # cache length cycles within the capacity so every step does the same work
+        length = w.ctx_len + (self.step_index % max(w.extra_rows, 1))
+        self.step_index += 1
+        ns = slot if slot is not None else 0
+        for l in range(w.n_layers):
+            leader = self.lo[l] == l
+            si = self.S.index(self.lo[l])
+            if attend_events is not None:
+                attend_events[l][0].record()
+            xkv.rcla_decode_attend(self.d, l, self.lo, self.K, self.V, w.L_max,
+                                   length if leader else length + 1,
+                                   self.kn[ns, si] if leader else None,
+                                   self.vn[ns, si] if leader else None, qq[l], self.out[l],
+                                   self.ws)
+            if attend_events is not None:
+                attend_events[l][1].record()
+
+    def attend_bytes(self, slots):
+        w = self.w
+        e = self.K.element_size()
+        rows = w.ctx_len + 1
+        per_layer = []
+        for l in range(w.n_layers):
+            leader = self.lo[l] == l
+            b = (w.batch * w.n_kv_heads * rows * w.head_dim * 2 * e
+                 + w.batch * w.n_q_heads * w.head_dim * (e + 4)
+                 + (w.batch * w.n_kv_heads * w.head_dim * 2 * e * 2 if leader else 0))
+            per_layer.append(b)
+        return float(np.mean(per_layer))
+
+    def step_bytes(self, attend_bytes_per_launch):
+        return self.w.n_layers * attend_bytes_per_launch
+
+    def io_bytes(self):
+        return (self.q_in.numel() * self.q_in.element_size(),
+                self.out.numel() * self.out.element_size())
+
+
+# --------------------------------------------------------------------- CPU baseline
+def cpu_baseline(w, seed, budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of one decode step, extrapolated."""
+    import torch
+    import oracle
+    from cross_layer_compressed_b200 import synth
+    oracle.build()
+    if w.mode == "rcla":
+        wl = synth.reduced(w, batch=1, n_layers=1, extra_rows=1)
+        x = synth.np_rcla_inputs(wl, seed, len_rows=w.ctx_len)
+        K = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+        V = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+        t0 = time.perf_counter()
+        oracle.rcla_decode_attend(0, [0], K, V, w.ctx_len, x["k_new"][0], x["v_new"][0],
+                                  x["q"][0])
+        dt = time.perf_counter() - t0
+        scale = w.batch * w.n_layers
+        sample = f"1 sequence x 1 layer (all {w.n_kv_heads} KV heads) of the {w.batch}-sequence x {w.n_layers}-layer step, extrapolated x{scale}"
+    else:
+        # one sequence, one layer, `heads` KV heads: scores, selection, reconstruct+attend
+        rng = np.random.default_rng(seed)
+        wl = synth.reduced(w, batch=1, n_layers=1, ctx_len=w.ctx_len, n_needles=0)
+        Ak = synth.to_storage(synth.np_basis(wl, seed, 0, 0, "k")[None], w.dtype)
+        Av = synth.to_storage(synth.np_basis(wl, seed, 0, 0, "v")[None], w.dtype)
+        Bkt = synth.to_storage(synth.np_recon_t(wl, seed, 0, 0, "k")[None], w.dtype)
+        Bvt = synth.to_storage(synth.np_recon_t(wl, seed, 0, 0, "v")[None], w.dtype)
+        q = synth.to_storage(synth.np_queries(wl, seed, 0, 0), w.dtype)
+        lm = synth.to_storage(rng.standard_normal((1, w.n_kv_heads, w.n_chunks, w.head_dim))
+                              * 1e-2, w.dtype) if w.mode != "dense" else None
+        t0 = time.perf_counter()
+        if lm is not None:
+            s = oracle.score_landmarks(lm, q)
+            sel = oracle.select_chunks(s, w.top_k, w.n_sink, w.n_recent)
+        else:
+            sel = None
+        heads = 0
+        for g in range(w.n_kv_heads):
+            oracle.reconstruct_attend(Ak, Av, Bkt, Bvt, q, sel, w.chunk, units=[(0, g)])
+            heads += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = (time.perf_counter() - t0) * w.n_kv_heads / heads
+        scale = w.batch * w.n_layers
+        sample = (f"1 sequence x 1 layer ({heads} of {w.n_kv_heads} KV heads timed, scaled to "
+                  f"all) of the {w.batch}-sequence x {w.n_layers}-layer step, extrapolated x{scale}")
+    step_s = dt * scale
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": sample, "sample_seconds": round(dt, 3)}
+
+
+def reference_arm(args, w, rank, world):
+    """--impl reference: the oracle on the host cores, one bounded sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    budget = max(0.5, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, args.seed, budget_s=budget)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = cpu_baseline(w, args.seed, budget_s=budget)
+        vals.append(r["value"])
+        secs.append(r["sample_seconds"])
+    v = float(np.mean(vals))
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.batch / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "ctx_len": w.ctx_len,
+                       "n_layers": w.n_layers},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- driver
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from cross_layer_compressed_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    assert args.warmup >= 3 or os.environ.get("XKV_BENCH_ALLOW_SHORT"), "need >= 3 warm-up steps"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from cross_layer_compressed_b200 import build
+    build.build()
+    wl = RclaStep(w, args.seed + rank, dev) if w.mode == "rcla" else XkvStep(w, args.seed + rank, dev)
+    nq = wl.qpool.shape[0]
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- device-resident timing
+    for s in range(args.warmup):
+        wl.step(s % nq)
+    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+          for _ in range(w.n_layers)]
+    attend_ms = []
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        wl.step(s % nq, attend_events=ev)
+        # attention-launch events of this step are read after the timed region
+        attend_ms.append(ev)
+        ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+              for _ in range(w.n_layers)]
+    stop.record(stream)
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop))
+    per_launch = [a.elapsed_time(b) for step in attend_ms for a, b in step]
+    attend_avg_ms = float(np.mean(per_launch))
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        q_host = torch.empty(wl.qpool.shape, dtype=wl.qpool.dtype, pin_memory=True)
+        q_host.copy_(wl.qpool.cpu())
+        out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
+        for s in range(args.warmup):
+            wl.q_in.copy_(q_host[s % nq], non_blocking=True)
+            wl.step(q=wl.q_in)
+            out_host.copy_(wl.out, non_blocking=True)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.steps):
+            wl.q_in.copy_(q_host[s % nq], non_blocking=True)
+            wl.step(q=wl.q_in)
+            out_host.copy_(wl.out, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        h2d, d2h = wl.io_bytes()
+        e2e = {"value": world * w.batch * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---------------- algorithmic bytes (untimed: selections recomputed per slot)
+    slots = sorted({s % nq for s in range(args.steps)})[:4]
+    bytes_launch = wl.attend_bytes(slots)
+    step_bytes = wl.step_bytes(bytes_launch)
+    hbm_peak, _, peak_kind = measured_peaks()
+    achieved = bytes_launch / (attend_avg_ms / 1e3) / 1e9
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
+    if os.path.exists(tr_path):
+        try:
+            with open(tr_path) as f:
+                traffic = json.load(f).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.seed)
+    if rank == 0:
+        ms_step = elapsed_ms / args.steps
+        value = world * w.batch * args.steps / (elapsed_ms / 1e3)
+        cfg = {"workload": w.name, "batch": w.batch, "ctx_len": w.ctx_len,
+               "n_layers": w.n_layers, "heads_q_kv": [w.n_q_heads, w.n_kv_heads],
+               "head_dim": w.head_dim, "parallelism": f"replicas x{world}",
+               "l2": f"inputs larger than L2: {wl.resident_bytes() / 1e9:.1f} GB resident, "
+                     f"{step_bytes / 1e9:.2f} GB algorithmic per step"}
+        if w.mode != "rcla":
+            cfg.update({"window": w.window, "ranks_k_v": [w.rank_k, w.rank_v], "chunk": w.chunk,
+                        "mode": w.mode})
+        if w.mode == "sr":
+            cfg.update({"top_k": w.top_k, "n_sink": w.n_sink, "n_recent": w.n_recent,
+                        "n_sel": w.n_sel})
+        if w.mode == "rcla":
+            cfg.update({"leaders": len(wl.S), "ctx_rows": f"{w.ctx_len}..{w.L_max}"})
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": cfg,
+            "step_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "kernel": "reconstruct_attend" if w.mode != "rcla"
+                         else "rcla_decode_attend", "achieved": achieved, "peak": hbm_peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+                         "frac_of_8tbs": achieved / 8000.0, "traffic": traffic,
+                         "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms},
+            "gpu_launches": wl.launches_per_step * args.steps,
+            "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,317 @@
+// C ABI of the xKV decode-attention library (declared in include/xkv.h).
+//
+// Every entry point validates its arguments on the host before touching CUDA, so an
+// argument error launches nothing and needs no GPU.  Launch failures map to
+// XKV_ERR_CUDA.  The message of the last non-OK status is kept per calling thread.
+//
+// Host-side fault injection for tests: XKV_FAULT="<entry point>:<status code>" makes
+// that entry point return the status before launching anything.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "xkv_internal.cuh"
+
+using namespace xkv;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+xkv_status fail(xkv_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+xkv_status ok() {
+    g_last_error.clear();
+    return XKV_OK;
+}
+
+// XKV_FAULT="name:code" -> that status for the named entry point (tests only).
+bool injected(const char *name, xkv_status *st) {
+    const char *f = getenv("XKV_FAULT");
+    if (!f) return false;
+    const char *colon = strchr(f, ':');
+    if (!colon || (size_t)(colon - f) != strlen(name) || strncmp(f, name, colon - f) != 0)
+        return false;
+    *st = (xkv_status)atoi(colon + 1);
+    g_last_error = std::string("injected fault in ") + name;
+    return true;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t esize(const xkv_dims &d) { return d.dtype == XKV_F32 ? 4 : 2; }
+
+// Checks shared by every call that takes dims.  `need_xkv` adds the chunk / rank rules.
+xkv_status check_dims(const xkv_dims *d, bool need_xkv, const char *who) {
+    if (!d) return fail(XKV_ERR_INVALID_ARG, "%s: dims is NULL", who);
+    if (d->batch <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->ctx_len <= 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: batch, heads and ctx_len must be positive", who);
+    if (d->n_q_heads % d->n_kv_heads)
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_q_heads %% n_kv_heads != 0", who);
+    if (d->n_q_heads / d->n_kv_heads > 16)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: more than 16 query heads per KV head", who);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: head_dim must be 64 or 128", who);
+    if (d->dtype != XKV_F32 && d->dtype != XKV_BF16)
+        return fail(XKV_ERR_INVALID_ARG, "%s: unknown dtype %d", who, d->dtype);
+    if (d->batch > 65535 || d->n_kv_heads > 65535)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: batch or n_kv_heads above 65535", who);
+    if (need_xkv) {
+        if (d->chunk <= 0 || d->chunk % 8 || d->ctx_len % d->chunk)
+            return fail(XKV_ERR_INVALID_ARG, "%s: chunk must be a positive multiple of 8 "
+                        "dividing ctx_len", who);
+        if (d->rank_k <= 0 || d->rank_v <= 0 || d->rank_k % 16 || d->rank_v % 16)
+            return fail(XKV_ERR_INVALID_ARG, "%s: ranks must be positive multiples of 16", who);
+        if (d->rank_k > 1024 || d->rank_v > 1024)
+            return fail(XKV_ERR_UNSUPPORTED, "%s: rank above 1024", who);
+    }
+    return XKV_OK;
+}
+
+// The library is built for sm_100a only; check the current device once per device.
+xkv_status check_device(const char *who) {
+    static int checked[64] = {0};  // 0 unknown, 1 ok, 2 wrong arch
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(XKV_ERR_CUDA, "%s: cudaGetDevice: %s", who, cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return XKV_OK;
+    if (!checked[dev]) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    if (checked[dev] != 1)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: needs a compute capability 10.0 device", who);
+    return XKV_OK;
+}
+
+xkv_status launched(cudaError_t e, const char *who) {
+    if (e != cudaSuccess)
+        return fail(XKV_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+    return ok();
+}
+
+int64_t n_forced(int64_t nC, int n_sink, int n_recent) {
+    int64_t f = 0;
+    const int64_t sink = n_sink < nC ? n_sink : nC;
+    const int64_t rec_lo = nC - n_recent > sink ? nC - n_recent : sink;
+    f = sink + (nC - rec_lo);
+    return f;
+}
+
+// Split plans of the two attention paths (rows = rows attended per unit).
+SplitPlan plan_xkv(const xkv_dims &d, int64_t rows) {
+    const int G = d.n_q_heads / d.n_kv_heads;
+    const int64_t max_rows = 16384 / G < 1024 ? 16384 / G : 1024;
+    return plan_splits(rows, (int64_t)d.batch * d.n_kv_heads, 64, max_rows);
+}
+
+SplitPlan plan_rcla(const xkv_dims &d, int64_t rows) {
+    const int G = d.n_q_heads / d.n_kv_heads;
+    return plan_splits(rows, (int64_t)d.batch * d.n_kv_heads, 256, 16384 / G);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *xkv_last_error(void) { return g_last_error.c_str(); }
+
+int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t n_recent) {
+    if (n_chunks < 0 || top_k < 0 || n_sink < 0 || n_recent < 0) return -1;
+    const int64_t f = n_forced(n_chunks, n_sink, n_recent);
+    const int64_t cand = n_chunks - f;
+    return (top_k < cand ? top_k : cand) + f;
+}
+
+size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
+    if (mode == XKV_MODE_RCLA) {
+        if (check_dims(dims, false, "xkv_workspace_bytes") != XKV_OK) return 0;
+        return partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
+    }
+    if (check_dims(dims, true, "xkv_workspace_bytes") != XKV_OK) return 0;
+    int64_t rows;
+    if (mode == XKV_MODE_SELECTIVE) {
+        if (n_sel <= 0 || (int64_t)n_sel > dims->ctx_len / dims->chunk) return 0;
+        rows = (int64_t)n_sel * dims->chunk;
+    } else if (mode == XKV_MODE_DENSE) {
+        rows = dims->ctx_len;
+    } else {
+        return 0;
+    }
+    return partial_bytes(*dims, (int)plan_xkv(*dims, rows).n_bound);
+}
+
+int64_t xkv_footprint_bytes(const xkv_dims *d, int32_t n_layers, int32_t window,
+                            int32_t with_landmarks) {
+    if (check_dims(d, true, "xkv_footprint_bytes") != XKV_OK || n_layers <= 0 || window <= 0)
+        return -1;
+    const int64_t e = (int64_t)esize(*d);
+    const int64_t n_win = (n_layers + window - 1) / window;
+    const int64_t d_kv = (int64_t)d->n_kv_heads * d->head_dim;
+    const int64_t r = (int64_t)d->rank_k + d->rank_v;
+    int64_t per_seq = n_win * d->ctx_len * r * e + (int64_t)n_layers * r * d_kv * e;
+    if (with_landmarks) per_seq += (int64_t)n_layers * (d->ctx_len / d->chunk) * d_kv * e;
+    return (int64_t)d->batch * per_seq;
+}
+
+int64_t rcla_cache_bytes(const xkv_dims *d, int32_t n_leaders, int64_t L_max) {
+    if (check_dims(d, false, "rcla_cache_bytes") != XKV_OK || n_leaders <= 0 || L_max <= 0)
+        return -1;
+    return (int64_t)n_leaders * d->batch * d->n_kv_heads * L_max * d->head_dim * 2 *
+           (int64_t)esize(*d);
+}
+
+xkv_status xkv_build_landmarks(const xkv_dims *dims, const void *Ak_win, const void *Bkt_layer,
+                               void *lm_layer, void *stream) {
+    const char *who = "xkv_build_landmarks";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!Ak_win || !Bkt_layer || !lm_layer)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(Ak_win) || !aligned16(Bkt_layer) || !aligned16(lm_layer))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (dims->ctx_len / dims->chunk > (int64_t)65535 * 16)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: too many chunks", who);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_build_landmarks(*dims, Ak_win, Bkt_layer, lm_layer,
+                                           (cudaStream_t)stream), who);
+}
+
+xkv_status xkv_score_landmarks(const xkv_dims *dims, const void *lm_layer, const void *q,
+                               double *scores, void *stream) {
+    const char *who = "xkv_score_landmarks";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!lm_layer || !q || !scores)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(lm_layer) || !aligned16(q) || !aligned16(scores))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (dims->ctx_len / dims->chunk > (int64_t)65535 * 128)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: too many chunks", who);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_score(*dims, lm_layer, q, scores, (cudaStream_t)stream), who);
+}
+
+xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t top_k,
+                             int32_t n_sink, int32_t n_recent, int32_t *sel,
+                             int32_t *n_sel_out, void *stream) {
+    const char *who = "xkv_select_chunks";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!scores || !sel) return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(scores) || !aligned16(sel))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (top_k < 0 || n_sink < 0 || n_recent < 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: top_k, n_sink, n_recent must be >= 0", who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (nC > 16384)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: more than 16384 chunks per unit", who);
+    const int64_t n_sel = xkv_n_selected(nC, top_k, n_sink, n_recent);
+    if (n_sel_out) *n_sel_out = (int32_t)n_sel;
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_select(*dims, scores, top_k, n_sink, n_recent, sel, (int)n_sel,
+                                  (cudaStream_t)stream), who);
+}
+
+xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
+                                  const void *Bkt_layer, const void *Bvt_layer, const void *q,
+                                  const int32_t *sel, int32_t n_sel, float *out, void *ws,
+                                  size_t ws_bytes, void *stream) {
+    const char *who = "xkv_reconstruct_attend";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!Ak_win || !Av_win || !Bkt_layer || !Bvt_layer || !q || !out || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(Ak_win) || !aligned16(Av_win) || !aligned16(Bkt_layer) ||
+        !aligned16(Bvt_layer) || !aligned16(q) || !aligned16(out) || !aligned16(ws) ||
+        (sel && !aligned16(sel)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (sel && (n_sel <= 0 || n_sel > nC))
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_sel must be in [1, n_chunks]", who);
+    const int64_t rows = sel ? (int64_t)n_sel * dims->chunk : dims->ctx_len;
+    const SplitPlan plan = plan_xkv(*dims, rows);
+    if (plan.n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    const size_t need = partial_bytes(*dims, plan.n_split);
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    float *partials = (float *)ws;
+    cudaError_t e = launch_attend_simt(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
+                                       n_sel, plan, partials, s);
+    if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, s);
+    return launched(e, who);
+}
+
+xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t *leader_of,
+                              int32_t n_layers, void *K_lead, void *V_lead, int64_t L_max,
+                              int64_t len, const void *k_new, const void *v_new, const void *q,
+                              float *out, void *ws, size_t ws_bytes, void *stream) {
+    const char *who = "rcla_decode_attend";
+    xkv_status st;
+    if ((st = check_dims(dims, false, who)) != XKV_OK) return st;
+    if (!leader_of || !K_lead || !V_lead || !q || !out || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL pointer", who);
+    if (!aligned16(K_lead) || !aligned16(V_lead) || !aligned16(q) || !aligned16(out) ||
+        !aligned16(ws) || (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (n_layers <= 0 || layer < 0 || layer >= n_layers)
+        return fail(XKV_ERR_INVALID_ARG, "%s: layer outside [0, n_layers)", who);
+    if (leader_of[0] != 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: layer 0 must be a leader", who);
+    int slot = 0, lead = leader_of[layer];
+    for (int l = 0; l < n_layers; ++l) {
+        const int32_t s = leader_of[l];
+        if (s < 0 || s > l || leader_of[s] != s)
+            return fail(XKV_ERR_INVALID_ARG, "%s: leader_of[%d] = %d is not an earlier leader",
+                        who, l, s);
+        if (l < lead && s == l) ++slot;
+    }
+    const bool is_leader = lead == layer;
+    if ((k_new == nullptr) != (v_new == nullptr))
+        return fail(XKV_ERR_INVALID_ARG, "%s: give both k_new and v_new or neither", who);
+    if (!is_leader && k_new)
+        return fail(XKV_ERR_INVALID_ARG, "%s: layer %d is not a leader and owns no cache", who,
+                    layer);
+    const bool update = is_leader && k_new;
+    const int64_t n_rows = len + (update ? 1 : 0);
+    if (len < 0 || L_max <= 0 || n_rows > L_max || n_rows <= 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: need 0 < rows attended <= L_max", who);
+    const SplitPlan plan = plan_rcla(*dims, n_rows);
+    if (plan.n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    const size_t need = partial_bytes(*dims, plan.n_split);
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    float *partials = (float *)ws;
+    cudaError_t e = launch_rcla(*dims, slot, L_max, n_rows, update ? len : -1, K_lead, V_lead,
+                                k_new, v_new, q, plan, partials, s);
+    if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, s);
+    return launched(e, who);
+}
+
+}  // extern "C"

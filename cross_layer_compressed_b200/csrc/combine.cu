@@ -1,0 +1,56 @@
+// Merge of split-K partial attention results (flash-decoding): each split s of a
+// (sequence, query head) left (m_s, l_s, acc_s) with acc_s = sum_t exp(z_t - m_s) v_t
+// over its rows.  out = sum_s exp(m_s - M) acc_s / sum_s exp(m_s - M) l_s, M = max m_s.
+#include "xkv_internal.cuh"
+
+namespace xkv {
+namespace {
+
+__global__ void __launch_bounds__(128) k_combine(const float *__restrict__ partials,
+                                                 float *__restrict__ out, int n_split,
+                                                 int BH, int hd) {
+    const int bh = blockIdx.x;
+    const int j = threadIdx.x;
+    const size_t stride = (size_t)BH * (hd + 2);
+    const float *p = partials + (size_t)bh * (hd + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, p[s * stride]);
+    float l = 0.f, acc = 0.f;
+    for (int s = 0; s < n_split; ++s) {
+        const float w = expf(p[s * stride] - M);
+        l = fmaf(w, p[s * stride + 1], l);
+        if (j < hd) acc = fmaf(w, p[s * stride + 2 + j], acc);
+    }
+    if (j < hd) out[(size_t)bh * hd + j] = acc / l;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
+                           cudaStream_t s) {
+    const int BH = d.batch * d.n_q_heads;
+    k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim);
+    return cudaGetLastError();
+}
+
+SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max_rows) {
+    // Aim for about four CTAs per SM over the 148 SMs of a B200, with at least
+    // min_rows rows per split and at most max_rows (the logits held in shared memory).
+    const int64_t target_ctas = 148 * 4;
+    int64_t n = (target_ctas + units - 1) / units;
+    n = n < (rows + min_rows - 1) / min_rows ? n : (rows + min_rows - 1) / min_rows;
+    const int64_t n_hi = (rows + max_rows - 1) / max_rows;
+    if (n < n_hi) n = n_hi;
+    if (n < 1) n = 1;
+    SplitPlan p;
+    p.n_bound = n;
+    p.rows_per_split = (rows + n - 1) / n;
+    p.n_split = (int)((rows + p.rows_per_split - 1) / p.rows_per_split);  // no empty split
+    return p;
+}
+
+size_t partial_bytes(const xkv_dims &d, int n_split) {
+    return (size_t)n_split * d.batch * d.n_q_heads * (d.head_dim + 2) * sizeof(float);
+}
+
+}  // namespace xkv

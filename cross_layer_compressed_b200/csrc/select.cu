@@ -1,0 +1,184 @@
+// Chunk selection (xKV page, section 2.3: keep the chunks most relevant to the query,
+// plus the always-kept sink and recent chunks).
+//
+// One CTA per (sequence, KV head).  Scores become 64-bit keys that order like the
+// doubles (-0 below +0); an 8-pass MSB-first radix select finds the key T of the k-th
+// best candidate and how many candidates equal to T are still needed; those are taken
+// in ascending index (the tie-break), found with a block-wide prefix count.  A second
+// prefix count writes the selected chunks in ascending order.  No floating-point
+// arithmetic is involved, so the result is exactly the oracle's.
+#include "xkv_internal.cuh"
+
+namespace xkv {
+namespace {
+
+constexpr int SEL_THREADS = 1024;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
+
+// Exclusive prefix sum of one value per thread over the CTA; also returns the total.
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned *warp_tot,
+                                                         unsigned *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        unsigned t = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += t;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        unsigned w = warp_tot[lane];
+        unsigned winc = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            unsigned t = __shfl_up_sync(0xffffffffu, winc, off);
+            if (lane >= off) winc += t;
+        }
+        warp_tot[lane] = winc - w;  // exclusive warp offsets
+        if (lane == 31) *total = winc;
+    }
+    __syncthreads();
+    const unsigned r = warp_tot[warp] + inc - v;
+    __syncthreads();  // warp_tot may be reused by the caller
+    return r;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict__ scores,
+                                                        int32_t *__restrict__ sel, int64_t nC_,
+                                                        int top_k, int n_sink, int n_recent,
+                                                        int n_sel) {
+    extern __shared__ unsigned long long keys[];  // [nC]
+    __shared__ unsigned hist[256];
+    __shared__ unsigned warp_tot[SEL_WARPS];
+    __shared__ unsigned s_total;
+    __shared__ unsigned long long s_prefix;
+    __shared__ unsigned s_krem;
+
+    const int nC = (int)nC_;
+    const int unit = blockIdx.x;
+    const double *s = scores + (size_t)unit * nC;
+    auto forced = [&](int c) { return c < n_sink || c >= nC - n_recent; };
+
+    unsigned nf_local = 0;
+    for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
+        keys[c] = order_key(s[c]);
+        nf_local += forced(c) ? 1u : 0u;
+    }
+    (void)block_exclusive_scan(nf_local, warp_tot, &s_total);  // also a barrier
+    const int n_forced = (int)s_total;
+    const int n_cand = nC - n_forced;
+    const int k_eff = min(top_k, n_cand);
+
+    // 0: take no candidate, 1: take every candidate, 2: threshold select
+    const int mode = k_eff == 0 ? 0 : (k_eff == n_cand ? 1 : 2);
+    unsigned long long T = 0;
+    unsigned krem = 0;
+    if (mode == 2) {
+        if (threadIdx.x == 0) {
+            s_prefix = 0ull;
+            s_krem = (unsigned)k_eff;
+        }
+        unsigned long long mask = 0ull;
+        for (int shift = 56; shift >= 0; shift -= 8) {
+            for (int i = threadIdx.x; i < 256; i += SEL_THREADS) hist[i] = 0u;
+            __syncthreads();
+            const unsigned long long prefix = s_prefix;
+            for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
+                const unsigned long long k = keys[c];
+                if (!forced(c) && (k & mask) == prefix)
+                    atomicAdd(&hist[(unsigned)(k >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (threadIdx.x < 32) {
+                const int lane = threadIdx.x;
+                const unsigned need = s_krem;
+                unsigned cnt[8], tot = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    cnt[i] = hist[255 - (lane * 8 + i)];  // lanes walk the digits downwards
+                    tot += cnt[i];
+                }
+                unsigned inc = tot;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    unsigned t = __shfl_up_sync(0xffffffffu, inc, off);
+                    if (lane >= off) inc += t;
+                }
+                const unsigned exc = inc - tot;
+                if (exc < need && need <= inc) {
+                    unsigned cum = exc;
+                    for (int i = 0; i < 8; ++i) {
+                        if (cum + cnt[i] >= need) {
+                            const unsigned long long D = (unsigned long long)(255 - (lane * 8 + i));
+                            s_prefix = prefix | (D << shift);
+                            s_krem = need - cum;
+                            break;
+                        }
+                        cum += cnt[i];
+                    }
+                }
+            }
+            mask |= 255ull << shift;
+            __syncthreads();
+        }
+        T = s_prefix;
+        krem = s_krem;
+    }
+
+    // Each thread owns a contiguous run of chunks so prefix counts follow chunk order.
+    const int ipt = (nC + SEL_THREADS - 1) / SEL_THREADS;
+    const int lo = min(nC, (int)threadIdx.x * ipt), hi = min(nC, lo + ipt);
+    unsigned eq_local = 0;
+    if (mode == 2)
+        for (int c = lo; c < hi; ++c) eq_local += (!forced(c) && keys[c] == T) ? 1u : 0u;
+    unsigned eq_rank = block_exclusive_scan(eq_local, warp_tot, &s_total);
+
+    // selection flags for the thread's run, as a bit mask (ipt <= 16)
+    unsigned flags = 0, n_local = 0;
+    for (int c = lo; c < hi; ++c) {
+        bool take;
+        if (forced(c)) {
+            take = true;
+        } else if (mode == 0) {
+            take = false;
+        } else if (mode == 1) {
+            take = true;
+        } else {
+            const unsigned long long k = keys[c];
+            if (k > T) {
+                take = true;
+            } else if (k == T) {
+                take = eq_rank < krem;
+                ++eq_rank;
+            } else {
+                take = false;
+            }
+        }
+        if (take) {
+            flags |= 1u << (c - lo);
+            ++n_local;
+        }
+    }
+    unsigned pos = block_exclusive_scan(n_local, warp_tot, &s_total);
+    int32_t *out = sel + (size_t)unit * n_sel;
+    for (int c = lo; c < hi; ++c)
+        if ((flags >> (c - lo)) & 1u) {
+            if (pos < (unsigned)n_sel) out[pos] = c;
+            ++pos;
+        }
+}
+
+}  // namespace
+
+cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, int n_sink,
+                          int n_recent, int32_t *sel, int n_sel, cudaStream_t s) {
+    const int64_t nC = d.ctx_len / d.chunk;
+    const size_t smem = (size_t)nC * sizeof(unsigned long long);
+    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_select<<<d.batch * d.n_kv_heads, SEL_THREADS, smem, s>>>(scores, sel, nC, top_k, n_sink,
+                                                               n_recent, n_sel);
+    return cudaGetLastError();
+}
+
+}  // namespace xkv

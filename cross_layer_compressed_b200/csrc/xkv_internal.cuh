@@ -1,0 +1,100 @@
+// Internal declarations shared by the kernels and the C-ABI layer of the xKV decode
+// library.  Nothing here is part of the public ABI (include/xkv.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "xkv.h"
+
+namespace xkv {
+
+// ------------------------------------------------------------------ launch plans
+// Work split of one attention call: `n_split` CTAs per (sequence, KV head) unit, each
+// over a contiguous range of the unit's rows.  Partials go to the workspace as
+// [n_split][B][Hq][hd + 2] fp32 = (running max m, sum l, unnormalised acc[hd]).
+struct SplitPlan {
+    int n_split;             // CTAs per unit (no split is empty)
+    int64_t rows_per_split;
+    int64_t n_bound;         // >= n_split and nondecreasing in `rows`: sizes workspaces
+};
+
+// A workspace sized with n_bound for the largest row count fits every smaller call.
+SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max_rows);
+
+size_t partial_bytes(const xkv_dims &d, int n_split);
+
+// ------------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error; arguments were validated by the caller.
+cudaError_t launch_build_landmarks(const xkv_dims &d, const void *Ak, const void *Bkt, void *lm,
+                                   cudaStream_t s);
+cudaError_t launch_score(const xkv_dims &d, const void *lm, const void *q, double *scores,
+                         cudaStream_t s);
+cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, int n_sink,
+                          int n_recent, int32_t *sel, int n_sel, cudaStream_t s);
+cudaError_t launch_attend_simt(const xkv_dims &d, const void *Ak, const void *Av,
+                               const void *Bkt, const void *Bvt, const void *q,
+                               const int32_t *sel, int n_sel, const SplitPlan &plan,
+                               float *partials, cudaStream_t s);
+cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,
+                        int64_t update_row, void *K, void *V, const void *k_new,
+                        const void *v_new, const void *q, const SplitPlan &plan,
+                        float *partials, cudaStream_t s);
+cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
+                           cudaStream_t s);
+
+// ------------------------------------------------------------------ device helpers
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float f32(float x) { return x; }
+    static __device__ __forceinline__ double f64(float x) { return (double)x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ double f64(__nv_bfloat16 x) {
+        return (double)__bfloat162float(x);  // both widenings are exact
+    }
+};
+
+// Widen the low / high bf16 of a packed pair to fp32 (exact: a bf16 is the top half of
+// an fp32 bit pattern).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Round an fp64 value to the nearest bf16, ties to even, in one step (no fp32 detour).
+// Method: round-half-even at bit 45 of the binary64 pattern by adding
+// (2^44 - 1) + (bit 45) and truncating, then re-bias the exponent from 1023 to 127.
+// Values below the bf16 normal range are first rounded to the fixed subnormal quantum
+// 2^-133 (exactly representable in fp64), so the result is exact there too.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+    uint64_t u = (uint64_t)__double_as_longlong(x);
+    uint64_t sign = u >> 63;
+    uint64_t mag = u & 0x7fffffffffffffffull;
+    if (mag == 0) return (uint16_t)(sign << 15);
+    int e = (int)(mag >> 52) - 1023;  // unbiased exponent (normal fp64 inputs)
+    if (e >= 128) return (uint16_t)((sign << 15) | 0x7f80u);  // overflow -> inf
+    if (e < -126) {
+        // subnormal bf16 range: k = rint(|x| * 2^133), value k * 2^-133, k <= 128
+        double k = rint(fabs(x) * 0x1p133);
+        uint32_t bits = (uint32_t)k;  // k == 128 is the smallest normal, same encoding
+        return (uint16_t)((sign << 15) | bits);
+    }
+    uint64_t lsb = (mag >> 45) & 1ull;
+    mag += 0x00000FFFFFFFFFFFull + lsb;  // 2^44 - 1 + lsb
+    int e2 = (int)(mag >> 52) - 1023;
+    if (e2 >= 128) return (uint16_t)((sign << 15) | 0x7f80u);
+    uint32_t man7 = (uint32_t)((mag >> 45) & 0x7f);
+    return (uint16_t)((sign << 15) | ((uint32_t)(e2 + 127) << 7) | man7);
+}
+
+// Key under which a larger double compares larger and -0 < +0.
+__device__ __forceinline__ unsigned long long order_key(double s) {
+    unsigned long long u = (unsigned long long)__double_as_longlong(s);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+}  // namespace xkv

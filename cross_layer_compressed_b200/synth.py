@@ -41,7 +41,8 @@ __all__ = [
     "LLAMA8B_DENSE_128K", "QWEN14B_SR_16K", "reduced", "leader_set",
     "np_basis", "np_recon_t", "np_queries", "np_needle_chunks", "np_plant_needles",
     "np_xkv_layer_inputs", "np_rcla_inputs", "to_storage",
-    "torch_xkv_cache", "torch_queries", "torch_rcla_cache",
+    "torch_xkv_cache", "torch_xkv_layer", "torch_queries", "torch_layer_queries",
+    "torch_rcla_cache",
 ]
 
 
@@ -284,31 +285,53 @@ def _tdtype(dtype: str):
     return torch.float32 if dtype == "f32" else torch.bfloat16
 
 
+def _t_basis(w: Workload, seed: int, seq: int, win: int, which: str, device):
+    import torch
+    r = w.rank_k if which == "k" else w.rank_v
+    g = _tgen(seed, "Ak" if which == "k" else "Av", seq, win, device=device)
+    x = torch.randn((w.ctx_len, r), generator=g, device=device, dtype=torch.float32)
+    qf, _ = torch.linalg.qr(x)
+    s = torch.exp(-torch.arange(r, device=device, dtype=torch.float32) / w.tau)
+    return (qf * s[None, :]).to(_tdtype(w.dtype))
+
+
+def _t_recon_t(w: Workload, seed: int, seq: int, layer: int, which: str, device):
+    import torch
+    r = w.rank_k if which == "k" else w.rank_v
+    g = _tgen(seed, "Bk" if which == "k" else "Bv", seq, layer, device=device)
+    return (torch.randn((w.d_kv, r), generator=g, device=device) / math.sqrt(r)).to(
+        _tdtype(w.dtype))
+
+
 def torch_xkv_cache(w: Workload, seed: int, device="cuda") -> dict:
     """Full xKV cache on a device: Ak, Av [n_win][B][L][r], Bkt, Bvt [N][B][d_kv][r]."""
     import torch
     dt = _tdtype(w.dtype)
-    L = w.ctx_len
-    Ak = torch.empty((w.n_windows, w.batch, L, w.rank_k), dtype=dt, device=device)
-    Av = torch.empty((w.n_windows, w.batch, L, w.rank_v), dtype=dt, device=device)
-    for which, T, r in (("k", Ak, w.rank_k), ("v", Av, w.rank_v)):
-        s = torch.exp(-torch.arange(r, device=device, dtype=torch.float32) / w.tau)
-        for win in range(w.n_windows):
-            for b in range(w.batch):
-                g = _tgen(seed, "Ak" if which == "k" else "Av", b, win, device=device)
-                x = torch.randn((L, r), generator=g, device=device, dtype=torch.float32)
-                qf, _ = torch.linalg.qr(x)
-                T[win, b].copy_((qf * s[None, :]).to(dt))
-                del x, qf
+    Ak = torch.empty((w.n_windows, w.batch, w.ctx_len, w.rank_k), dtype=dt, device=device)
+    Av = torch.empty((w.n_windows, w.batch, w.ctx_len, w.rank_v), dtype=dt, device=device)
+    for win in range(w.n_windows):
+        for b in range(w.batch):
+            Ak[win, b].copy_(_t_basis(w, seed, b, win, "k", device))
+            Av[win, b].copy_(_t_basis(w, seed, b, win, "v", device))
     Bkt = torch.empty((w.n_layers, w.batch, w.d_kv, w.rank_k), dtype=dt, device=device)
     Bvt = torch.empty((w.n_layers, w.batch, w.d_kv, w.rank_v), dtype=dt, device=device)
-    for which, T, r in (("k", Bkt, w.rank_k), ("v", Bvt, w.rank_v)):
-        for l in range(w.n_layers):
-            for b in range(w.batch):
-                g = _tgen(seed, "Bk" if which == "k" else "Bv", b, l, device=device)
-                T[l, b].copy_((torch.randn((w.d_kv, r), generator=g, device=device)
-                               / math.sqrt(r)).to(dt))
+    for l in range(w.n_layers):
+        for b in range(w.batch):
+            Bkt[l, b].copy_(_t_recon_t(w, seed, b, l, "k", device))
+            Bvt[l, b].copy_(_t_recon_t(w, seed, b, l, "v", device))
     return dict(Ak=Ak, Av=Av, Bkt=Bkt, Bvt=Bvt)
+
+
+def torch_xkv_layer(w: Workload, seed: int, layer: int, device="cuda") -> dict:
+    """One layer's slice of torch_xkv_cache (same values): Ak, Av [B][L][r], Bkt, Bvt
+    [B][d_kv][r]."""
+    import torch
+    win = layer // w.window
+    return dict(
+        Ak=torch.stack([_t_basis(w, seed, b, win, "k", device) for b in range(w.batch)]),
+        Av=torch.stack([_t_basis(w, seed, b, win, "v", device) for b in range(w.batch)]),
+        Bkt=torch.stack([_t_recon_t(w, seed, b, layer, "k", device) for b in range(w.batch)]),
+        Bvt=torch.stack([_t_recon_t(w, seed, b, layer, "v", device) for b in range(w.batch)]))
 
 
 def torch_needle_chunks(w: Workload, seed: int) -> list:
@@ -340,6 +363,26 @@ def torch_queries(w: Workload, seed: int, cache: dict | None = None, device="cud
                 u = (d / d.norm(dim=-1, keepdim=True)).sum(0)                     # H x hd
                 q[:, l, b] += lam * u.repeat_interleave(G, dim=0)[None]
     return q.to(dt)
+
+
+def torch_layer_queries(w: Workload, seed: int, layer: int, layer_cache: dict, slot: int = 0,
+                        device="cuda"):
+    """Query slot `slot` of one layer, [B][Hq][hd], as torch_queries builds it (needles
+    from the layer's factors)."""
+    import torch
+    g = _tgen(seed, "q", slot, layer, device=device)
+    q = torch.randn((w.batch, w.n_q_heads, w.head_dim), generator=g, device=device) \
+        * w.head_dim ** -0.25
+    if w.n_needles:
+        lam = 4.0 * w.head_dim ** 0.25
+        C, hd, G = w.chunk, w.head_dim, w.group
+        for b, nd in enumerate(torch_needle_chunks(w, seed)):
+            A = layer_cache["Ak"][b].float()
+            abar = torch.stack([A[n * C:(n + 1) * C].mean(0) for n in nd])
+            d = (abar @ layer_cache["Bkt"][b].float().T).view(len(nd), w.n_kv_heads, hd)
+            u = (d / d.norm(dim=-1, keepdim=True)).sum(0)
+            q[b] += lam * u.repeat_interleave(G, dim=0)
+    return q.to(_tdtype(w.dtype))
 
 
 def torch_rcla_cache(w: Workload, seed: int, device="cuda") -> dict:

@@ -1,0 +1,188 @@
+/*
+ * xkv.h -- C ABI of the B200 (sm_100a) decode-attention library for a
+ * cross-layer-compressed KV cache.
+ *
+ * The operations follow two pages:
+ *  [xKV]   "xKV: Cross-Layer KV-Cache Compression via Aligned Singular Vector
+ *          Extraction" (technical summary).  Section 2.2, cross-layer factorization
+ *          (CLF): each window of W layers keeps one shared token basis A (L x r) and
+ *          one small reconstruction matrix B_l (r x d_kv) per layer.  Section 2.3,
+ *          selective reconstruction (SR): landmark-based chunk selection, then only
+ *          the selected rows of K = A B_l (and V) are rebuilt.  Section 4, dense
+ *          reconstruction (all rows).
+ *  [R-CLA] "Stochastic KV Routing: adaptive depth-wise cache sharing".  Inference
+ *          with a fixed sharing set S: a layer outside S reuses the KV cache of the
+ *          nearest previous layer in S and skips its own K/V load and update
+ *          (the page's Algorithm 2).
+ *
+ * Conventions for every call
+ *  - All tensor arguments are DEVICE pointers to dense row-major arrays (last index
+ *    fastest) in the layouts stated below, unless marked "host".  The caller owns
+ *    every buffer; the library never allocates, frees or keeps a pointer after the
+ *    call returns.
+ *  - Storage type (dims->dtype): XKV_F32 or XKV_BF16, shared by the factors,
+ *    landmarks, queries and caches of a call.  Outputs are fp32; scores are fp64.
+ *  - Every pointer the kernels read or write must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and return after the launches are queued.
+ *  - Every call returns an xkv_status; no C++ exception crosses the ABI.  On a
+ *    non-OK status nothing was launched (argument errors) or a launch failed
+ *    (XKV_ERR_CUDA); xkv_last_error() gives a message for the calling thread.
+ *  - Query head h belongs to KV group g = h / G, G = n_q_heads / n_kv_heads.
+ *  - Inputs holding NaN or Inf are outside the contract.
+ *  - The library runs on compute capability 10.0 devices only (XKV_ERR_UNSUPPORTED
+ *    otherwise).
+ */
+#ifndef XKV_H
+#define XKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    XKV_OK = 0,
+    XKV_ERR_INVALID_ARG = 1, /* a pointer, size, alignment or layout rule is broken */
+    XKV_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels handle */
+    XKV_ERR_CUDA = 3,        /* a CUDA runtime call or a launch failed */
+    XKV_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up */
+    XKV_ERR_INTERNAL = 5     /* a device-side consistency check failed */
+} xkv_status;
+
+typedef enum { XKV_F32 = 0, XKV_BF16 = 1 } xkv_dtype;
+
+typedef enum { XKV_MODE_SELECTIVE = 0, XKV_MODE_DENSE = 1, XKV_MODE_RCLA = 2 } xkv_mode;
+
+/*
+ * Shapes of one decode call.
+ *   batch       B  sequences
+ *   n_q_heads   Hq query heads; n_kv_heads Hkv KV heads (Hq % Hkv == 0, G = Hq/Hkv <= 16)
+ *   head_dim    hd in {64, 128}
+ *   ctx_len     L  tokens in the compressed cache (xKV) or rows of cache capacity
+ *                  L_max (R-CLA workspace sizing only)
+ *   chunk       C  tokens per landmark chunk (xKV; L % C == 0; C % 8 == 0)
+ *   rank_k/v    r_K, r_V ranks of the key / value bases (multiples of 16, <= 1024)
+ *   dtype       xkv_dtype
+ * d_kv = Hkv * hd, nC = L / C.
+ */
+typedef struct {
+    int32_t batch;
+    int32_t n_q_heads;
+    int32_t n_kv_heads;
+    int32_t head_dim;
+    int64_t ctx_len;
+    int32_t chunk;
+    int32_t rank_k;
+    int32_t rank_v;
+    int32_t dtype;
+} xkv_dims;
+
+/*
+ * Landmark keys of one layer [xKV 2.3, "landmark-based chunk selection"], built once
+ * per cache (not part of a decode step).  The landmark of chunk c of KV head g is the
+ * mean of the chunk's reconstructed key rows:
+ *   lm[b][g][c][j] = round( (1/C) * sum_{t = cC}^{cC+C-1} (A^K[b][t] . B^K_l[:, g*hd + j]) )
+ * accumulated in fp64 and rounded to nearest-even into the storage type.
+ *   Ak_win    [B][L][r_K]      the layer's window basis A^K
+ *   Bkt_layer [B][d_kv][r_K]   B^K_l stored column-major (element (i, j) at j*r_K + i)
+ *   lm_layer  [B][Hkv][nC][hd] output
+ */
+xkv_status xkv_build_landmarks(const xkv_dims *dims, const void *Ak_win, const void *Bkt_layer,
+                               void *lm_layer, void *stream);
+
+/*
+ * Landmark scores of one layer [xKV 2.3; the query-relevance step of SR]:
+ *   scores[b][g][c] = max_{h in group g} sum_{d=0}^{hd-1} lm[b][g][c][d] * q[b][h][d]
+ * Each product is formed exactly in fp64 and the sum runs in fp64 in ascending d,
+ * so the value is reproducible bit for bit; the max orders -0 below +0.  Unscaled
+ * (a positive scale does not change the ranking).
+ *   lm_layer [B][Hkv][nC][hd], q [B][Hq][hd], scores [B][Hkv][nC] fp64 (output)
+ */
+xkv_status xkv_score_landmarks(const xkv_dims *dims, const void *lm_layer, const void *q,
+                               double *scores, void *stream);
+
+/*
+ * Chunk selection [xKV 2.3: "the sparse subset most relevant to the current query"]:
+ * per (b, g), the forced chunks F = {0..n_sink-1} U {nC-n_recent..nC-1} plus the
+ * top_k of the remaining chunks under (score descending, chunk index ascending),
+ * written in ascending chunk order.  n_sel = min(top_k, nC - |F|) + |F| chunks per
+ * unit; *n_sel_out (host pointer, may be NULL) receives it, computed on the host.
+ *   scores [B][Hkv][nC] fp64, sel [B][Hkv][n_sel] int32 (output)
+ * nC <= 16384.
+ */
+xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t top_k,
+                             int32_t n_sink, int32_t n_recent, int32_t *sel,
+                             int32_t *n_sel_out, void *stream);
+
+/*
+ * Selective (or dense) reconstruction followed by GQA attention
+ * [xKV 2.3 "only the rows of the selected tokens are reconstructed from the shared
+ * basis and the per-layer matrices"; xKV 4, dense reconstruction].
+ * For each (b, g) let T = the C rows of every chunk in sel[b][g] (sel != NULL), or
+ * all L rows (sel == NULL, dense).  With K_hat[t] = A^K[b][t] B^K_l[:, g-slice] and
+ * V_hat[t] = A^V[b][t] B^V_l[:, g-slice] (never written to memory):
+ *   z[h][t] = q[b][h] . K_hat[t] / sqrt(hd),  p = softmax_t(z),
+ *   out[b][h] = sum_t p[h][t] V_hat[t]                       for every h in group g.
+ *   Ak_win [B][L][r_K], Av_win [B][L][r_V]          the layer's window bases
+ *   Bkt_layer [B][d_kv][r_K], Bvt_layer [B][d_kv][r_V] (column-major B_l)
+ *   q [B][Hq][hd]; sel [B][Hkv][n_sel] int32 ascending chunk indices, or NULL
+ *   out [B][Hq][hd] fp32 (output)
+ *   ws, ws_bytes: scratch of at least xkv_workspace_bytes(dims, n_sel, mode) bytes
+ *   (mode = XKV_MODE_SELECTIVE, or XKV_MODE_DENSE when sel == NULL).
+ */
+xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
+                                  const void *Bkt_layer, const void *Bvt_layer, const void *q,
+                                  const int32_t *sel, int32_t n_sel, float *out, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * Decode attention of layer `layer` under R-CLA sharing [R-CLA, inference strategy S
+ * and Algorithm 2].  leader_of (HOST, [n_layers]) maps each layer to the layer whose
+ * cache it reads: leader_of[0] == 0, leader_of[l] <= l, leader_of[leader_of[l]] ==
+ * leader_of[l]; the leaders are S = {l : leader_of[l] == l}, and the cache slot of
+ * leader s is |{s' in S : s' < s}|.
+ *   K_lead, V_lead [n_lead][B][Hkv][L_max][hd] leader-only caches
+ *   len    rows valid in the leader's cache when the call starts
+ *   k_new, v_new [B][Hkv][hd]: only for a leader layer (both or neither).  When given,
+ *          the call first writes them at row `len` of the layer's own cache (the
+ *          update) and attends len+1 rows; otherwise it attends `len` rows.  A
+ *          non-leader owns no cache and gets XKV_ERR_INVALID_ARG if given a row.
+ *   q [B][Hq][hd], out [B][Hq][hd] fp32 (output)
+ *   ws, ws_bytes: scratch of at least xkv_workspace_bytes(dims with ctx_len = L_max,
+ *          0, XKV_MODE_RCLA) bytes.
+ * dims->chunk, rank_k and rank_v are ignored.
+ */
+xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t *leader_of,
+                              int32_t n_layers, void *K_lead, void *V_lead, int64_t L_max,
+                              int64_t len, const void *k_new, const void *v_new, const void *q,
+                              float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Scratch bytes the attention calls need (the split-K partial results). 0 on bad dims. */
+size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode);
+
+/* Chunks selected per (b, g): min(top_k, nC - |F|) + |F|; -1 on bad arguments. */
+int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t n_recent);
+
+/*
+ * Bytes of the compressed cache [xKV 2.2 storage, O(L*r + W*r*d) per window]: for
+ * each sequence, ceil(n_layers / W) bases (L x (r_K + r_V)) and n_layers matrix pairs
+ * ((r_K + r_V) x d_kv), plus the landmark keys (n_layers x nC x d_kv) when
+ * with_landmarks != 0.  -1 on bad arguments.
+ */
+int64_t xkv_footprint_bytes(const xkv_dims *dims, int32_t n_layers, int32_t window,
+                            int32_t with_landmarks);
+
+/* Bytes of the leader-only K and V caches [R-CLA]: n_leaders x B x Hkv x L_max x hd x 2. */
+int64_t rcla_cache_bytes(const xkv_dims *dims, int32_t n_leaders, int64_t L_max);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char *xkv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XKV_H */

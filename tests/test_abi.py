@@ -1,0 +1,158 @@
+"""Host side of the C ABI (no GPU needed): the library loads, exports every entry point
+include/xkv.h declares, rejects bad arguments before touching CUDA, propagates injected
+faults, and its size helpers agree with the oracle's closed forms."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def xkv():
+    from cross_layer_compressed_b200 import build
+    build.build()
+    from cross_layer_compressed_b200 import xkv as m
+    return m
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "xkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(xkv):
+    names = _declared_functions()
+    assert {"xkv_score_landmarks", "xkv_select_chunks", "xkv_reconstruct_attend",
+            "rcla_decode_attend", "xkv_build_landmarks"} <= set(names)
+    lib = ctypes.CDLL(xkv.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_built_for_sm100a_only():
+    """The in-tree build targets sm_100a (checked from the build flags, not the binary)."""
+    from cross_layer_compressed_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in build.FLAGS
+
+
+FAKE = 0x10000  # aligned, never dereferenced on the host
+
+
+def _d(xkv, **kw):
+    base = dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, ctx_len=1024, chunk=8,
+                rank_k=64, rank_v=64, dtype=xkv.XKV_BF16)
+    base.update(kw)
+    return xkv.dims(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_q_heads=6, n_kv_heads=4), 1),          # Hq % Hkv
+    (dict(head_dim=96), 2),                         # unsupported head_dim
+    (dict(chunk=12), 1),                            # chunk not a multiple of 8
+    (dict(ctx_len=1004), 1),                        # L % C
+    (dict(rank_k=40), 1),                           # rank not a multiple of 16
+    (dict(rank_v=2048), 2),                         # rank above 1024
+    (dict(batch=0), 1),
+    (dict(dtype=7), 1),
+    (dict(n_q_heads=34, n_kv_heads=2), 2),          # G > 16
+])
+def test_bad_dims_rejected_without_launch(xkv, kw, status):
+    d = _d(xkv, **kw)
+    st = xkv.xkv_score_landmarks(d, FAKE, FAKE, FAKE, stream=0, check=False)
+    assert st == status
+    assert xkv.last_error()
+
+
+def test_null_and_misaligned_pointers_rejected(xkv):
+    d = _d(xkv)
+    assert xkv.xkv_score_landmarks(d, 0, FAKE, FAKE, stream=0, check=False) == 1
+    assert xkv.xkv_score_landmarks(d, FAKE + 8, FAKE, FAKE, stream=0, check=False) == 1
+    assert "aligned" in xkv.last_error()
+    assert xkv.xkv_build_landmarks(d, FAKE, FAKE + 2, FAKE, stream=0, check=False) == 1
+    assert xkv.xkv_select_chunks(d, FAKE, -1, 1, 1, FAKE, stream=0, check=False) == 1
+    ws = xkv.xkv_workspace_bytes(d, 10, xkv.XKV_MODE_SELECTIVE)
+    assert xkv.xkv_reconstruct_attend(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, ws,
+                                      stream=0, check=False) == 1      # n_sel = 0
+    assert xkv.xkv_reconstruct_attend(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 129, FAKE, FAKE,
+                                      ws, stream=0, check=False) == 1  # n_sel > nC
+
+
+def test_workspace_too_small_rejected(xkv):
+    d = _d(xkv)
+    ws = xkv.xkv_workspace_bytes(d, 20, xkv.XKV_MODE_SELECTIVE)
+    assert ws > 0
+    st = xkv.xkv_reconstruct_attend(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 20, FAKE, FAKE,
+                                    ws - 4, stream=0, check=False)
+    assert st == 1 and "workspace" in xkv.last_error()
+
+
+def test_workspace_bound_covers_every_smaller_call(xkv):
+    """A workspace sized for the largest row count fits every smaller call (the split
+    count used by a call never exceeds the bound)."""
+    for G, Hkv, B in [(4, 8, 8), (5, 8, 1), (1, 2, 3), (16, 1, 1)]:
+        d = _d(xkv, n_q_heads=G * Hkv, n_kv_heads=Hkv, batch=B, ctx_len=4096)
+        big = xkv.xkv_workspace_bytes(d, 512, xkv.XKV_MODE_SELECTIVE)
+        for n in range(1, 513, 7):
+            assert xkv.xkv_workspace_bytes(d, n, xkv.XKV_MODE_SELECTIVE) <= big
+        dr = _d(xkv, n_q_heads=G * Hkv, n_kv_heads=Hkv, batch=B, ctx_len=40000)
+        big_r = xkv.xkv_workspace_bytes(dr, 0, xkv.XKV_MODE_RCLA)
+        for L in list(range(1, 40000, 997)) + [40000]:
+            dd = _d(xkv, n_q_heads=G * Hkv, n_kv_heads=Hkv, batch=B, ctx_len=L)
+            assert xkv.xkv_workspace_bytes(dd, 0, xkv.XKV_MODE_RCLA) <= big_r
+
+
+def test_rcla_leader_rules(xkv):
+    d = _d(xkv)
+    ws = xkv.xkv_workspace_bytes(_d(xkv, ctx_len=64), 0, xkv.XKV_MODE_RCLA)
+    lo = [0, 0, 2, 2]
+
+    def call(layer, leader_of, length=10, kn=None, vn=None, L_max=64):
+        return xkv.rcla_decode_attend(d, layer, leader_of, FAKE, FAKE, L_max, length, kn, vn,
+                                      FAKE, FAKE, FAKE, ws, stream=0, check=False)
+    assert call(1, lo, kn=FAKE, vn=FAKE) == 1            # non-leader with a new row
+    assert "not a leader" in xkv.last_error()
+    assert call(2, lo, kn=FAKE) == 1                     # k_new without v_new
+    assert call(0, [1, 1, 2, 2]) == 1                    # layer 0 not a leader
+    assert call(3, [0, 0, 3, 2]) == 1                    # leader_of[2] = 3 > 2
+    assert call(3, [0, 0, 1, 1]) == 1                    # 1 is not a leader
+    assert call(4, lo) == 1                              # layer out of range
+    assert call(2, lo, length=64, kn=FAKE, vn=FAKE) == 1  # no room for the new row
+    assert call(0, lo, length=0) == 1                    # nothing to attend
+
+
+def test_fault_injection_propagates_before_any_launch(xkv, monkeypatch):
+    """XKV_FAULT makes a valid call return the injected status on the host (no GPU)."""
+    d = _d(xkv)
+    monkeypatch.setenv("XKV_FAULT", "xkv_score_landmarks:3")
+    assert xkv.xkv_score_landmarks(d, FAKE, FAKE, FAKE, stream=0, check=False) == 3
+    assert "injected" in xkv.last_error()
+    with pytest.raises(xkv.XkvError) as ei:
+        xkv.xkv_score_landmarks(d, FAKE, FAKE, FAKE, stream=0)
+    assert ei.value.status == xkv.XKV_ERR_CUDA
+    monkeypatch.setenv("XKV_FAULT", "rcla_decode_attend:4")
+    ws = xkv.xkv_workspace_bytes(_d(xkv, ctx_len=64), 0, xkv.XKV_MODE_RCLA)
+    assert xkv.rcla_decode_attend(d, 1, [0, 0], FAKE, FAKE, 64, 10, None, None, FAKE, FAKE,
+                                  FAKE, ws, stream=0, check=False) == 4
+    # other entry points are unaffected (they fail later, on the device check)
+    monkeypatch.setenv("XKV_FAULT", "xkv_select_chunks:5")
+    assert xkv.xkv_score_landmarks(d, FAKE, 0, FAKE, stream=0, check=False) == 1
+
+
+def test_size_helpers_match_oracle(xkv, ora):
+    for (B, Hkv, hd, L, C, rk, rv, dt, N, W, lm) in [
+            (8, 8, 128, 32768, 8, 512, 768, 1, 32, 4, 1), (1, 2, 64, 1024, 8, 64, 64, 0, 2, 2, 0),
+            (64, 8, 128, 16384, 8, 512, 768, 1, 48, 4, 1), (3, 2, 64, 96, 16, 32, 48, 1, 5, 2, 1)]:
+        d = xkv.dims(B, Hkv * 4, Hkv, hd, L, C, rk, rv, dt)
+        assert xkv.xkv_footprint_bytes(d, N, W, lm) == ora.footprint_bytes(
+            B, Hkv, hd, L, C, rk, rv, dt, N, W, lm)
+    for nC, k, s, r in [(4096, 256, 1, 4), (10, 50, 1, 2), (3, 1, 2, 2), (128, 16, 1, 1),
+                        (7, 0, 0, 0), (5, 2, 9, 0), (5, 2, 0, 9)]:
+        assert xkv.xkv_n_selected(nC, k, s, r) == ora.n_selected(nC, k, s, r)
+    d = xkv.dims(16, 32, 8, 128, 32832, dtype=1)
+    assert xkv.rcla_cache_bytes(d, 9, 32832) == ora.rcla_cache_bytes(16, 8, 128, 32832, 1, 9)

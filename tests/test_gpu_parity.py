@@ -1,0 +1,325 @@
+"""GPU parity: every entry point of the CUDA library against the CPU oracle, element by
+element, on seeded synthetic inputs at sizes the oracle finishes in seconds (several
+tiles, ragged tails), plus edge cases.  Scores and selections must match bit for bit;
+attention outputs within the tolerances of parity_util.TOL."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from cross_layer_compressed_b200 import synth
+from parity_util import bf16_ulp_diff, compare_outputs
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+
+
+@pytest.fixture(scope="module")
+def xkv():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from cross_layer_compressed_b200 import build
+    build.build()
+    from cross_layer_compressed_b200 import xkv as m
+    return m
+
+
+# Small workloads (each spans several CTAs and ends on a ragged tile)
+TINY = synth.TINY_SR_F32                                                  # as specified
+LLAMA_R = synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=2048, top_k=24)
+QWEN14_R = synth.reduced(synth.QWEN14B_SR_16K, batch=2, ctx_len=1024, top_k=20)
+DENSE_R = synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=1024)
+SMALL_HD64 = dataclasses.replace(synth.reduced(synth.LLAMA8B_SR_32K, batch=3, ctx_len=1536,
+                                               top_k=11, n_needles=0),
+                                 head_dim=64, n_kv_heads=2, n_q_heads=6, rank_k=96, rank_v=80,
+                                 name="hd64_g3")
+XKV_CASES = [TINY, LLAMA_R, QWEN14_R, SMALL_HD64]
+
+
+def _dev(t):
+    return t.to(DEV).contiguous()
+
+
+def _host_lm(ora, lm_np):
+    return ora.to_torch(lm_np)
+
+
+def _layer_inputs(w, layer=1):
+    return synth.np_xkv_layer_inputs(w, seed=0, layer=min(layer, w.n_layers - 1))
+
+
+# ------------------------------------------------------------------------ landmarks
+@pytest.mark.parametrize("w", XKV_CASES, ids=lambda w: w.name)
+def test_landmarks_match_oracle(xkv, ora, w):
+    x = _layer_inputs(w)
+    ref = ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk)
+    d = xkv.dims_of(w)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    lm = torch.empty((w.batch, w.n_kv_heads, w.n_chunks, w.head_dim), dtype=dt, device=DEV)
+    xkv.xkv_build_landmarks(d, _dev(x["Ak"]), _dev(x["Bkt"]), lm)
+    torch.cuda.synchronize()
+    got = lm.cpu()
+    if w.dtype == "f32":
+        g = got.numpy()
+        # fp64 accumulation in a different order, one rounding to fp32: at most 1 ulp
+        assert np.all(np.abs(g.astype(np.float64) - ref.astype(np.float64))
+                      <= np.spacing(np.abs(ref)))
+    else:
+        gu = got.view(torch.int16).numpy().view(np.uint16)
+        diff = bf16_ulp_diff(gu, ref)
+        assert diff.max() <= 1
+        assert (diff > 0).mean() < 1e-4
+
+
+# ------------------------------------------------------------------------- scoring
+@pytest.mark.parametrize("w", XKV_CASES, ids=lambda w: w.name)
+def test_scores_bit_exact(xkv, ora, w):
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    ref = ora.score_landmarks(lm, x["q"])
+    scores = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
+    xkv.xkv_score_landmarks(xkv.dims_of(w), _dev(lm), _dev(x["q"]), scores)
+    torch.cuda.synchronize()
+    got = scores.cpu().numpy()
+    assert np.array_equal(got.view(np.uint64), ref.view(np.uint64))
+
+
+def test_scores_bit_exact_heavy_cancellation(xkv, ora):
+    """Values whose fp64 sums round differently in any other order (2^53 + 1 - 2^53)."""
+    B, Hkv, G, hd, nC = 1, 2, 4, 128, 200
+    rng = np.random.default_rng(3)
+    lm = rng.integers(-4, 5, size=(B, Hkv, nC, hd)).astype(np.float64)
+    lm[..., 0] = 2.0 ** 53
+    lm[..., 1] = 1.0
+    lm[..., 2] = -(2.0 ** 53)
+    q = np.ones((B, Hkv * G, hd))
+    q[:, :, 3:] = rng.integers(-3, 4, size=(B, Hkv * G, hd - 3))
+    lm_t = torch.tensor(lm, dtype=torch.bfloat16)
+    q_t = torch.tensor(q, dtype=torch.bfloat16)
+    ref = ora.score_landmarks(lm_t, q_t)
+    d = xkv.dims(B, Hkv * G, Hkv, hd, nC * 8, 8, 16, 16, xkv.XKV_BF16)
+    scores = torch.empty((B, Hkv, nC), dtype=torch.float64, device=DEV)
+    xkv.xkv_score_landmarks(d, _dev(lm_t), _dev(q_t), scores)
+    torch.cuda.synchronize()
+    assert np.array_equal(scores.cpu().numpy().view(np.uint64), ref.view(np.uint64))
+
+
+# ------------------------------------------------------------------------ selection
+def _run_select(xkv, scores_np, top_k, n_sink, n_recent, chunk=8):
+    B, Hkv, nC = scores_np.shape
+    d = xkv.dims(B, Hkv, Hkv, 64, nC * chunk, chunk, 16, 16, xkv.XKV_BF16)
+    n_sel = xkv.xkv_n_selected(nC, top_k, n_sink, n_recent)
+    sel = torch.full((B, Hkv, n_sel), -7, dtype=torch.int32, device=DEV)
+    got_n = xkv.xkv_select_chunks(d, torch.from_numpy(scores_np).to(DEV), top_k, n_sink,
+                                  n_recent, sel)
+    torch.cuda.synchronize()
+    assert got_n == n_sel
+    return sel.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", XKV_CASES, ids=lambda w: w.name)
+def test_select_bit_exact(xkv, ora, w):
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    s = ora.score_landmarks(lm, x["q"])
+    ref = ora.select_chunks(s, w.top_k, w.n_sink, w.n_recent)
+    got = _run_select(xkv, s, w.top_k, w.n_sink, w.n_recent, w.chunk)
+    assert np.array_equal(got, ref)
+    for b, nd in enumerate(x["needles"]):
+        for g in range(w.n_kv_heads):
+            assert set(nd.tolist()) <= set(got[b, g].tolist())
+
+
+@pytest.mark.parametrize("nC,top_k,n_sink,n_recent", [
+    (4096, 256, 1, 4), (4097 - 1, 0, 1, 4), (1000, 990, 1, 4), (1000, 995, 1, 4),
+    (1000, 2000, 1, 4), (37, 5, 3, 3), (5, 2, 3, 3), (16384, 128, 1, 4), (1, 1, 0, 0),
+    (2048, 1, 0, 0), (3000, 2999, 0, 0), (777, 100, 0, 9)])
+def test_select_edge_cases_with_ties(xkv, ora, nC, top_k, n_sink, n_recent):
+    rng = np.random.default_rng(nC + top_k)
+    B, Hkv = 2, 3
+    s = rng.integers(-20, 21, size=(B, Hkv, nC)).astype(np.float64)   # heavy exact ties
+    s[0, 0] = 1.0                                                      # all tied
+    s[1, 2, ::2] = -0.0
+    s[1, 2, 1::2] = 0.0                                               # signed zeros
+    ref = ora.select_chunks(s, top_k, n_sink, n_recent)
+    got = _run_select(xkv, s, top_k, n_sink, n_recent)
+    assert np.array_equal(got, ref)
+
+
+def test_select_distinct_scores_extremes(xkv, ora):
+    rng = np.random.default_rng(9)
+    s = rng.standard_normal((1, 2, 3000)) * 1e300
+    s[0, 1, :10] = [1e-320, -1e-320, 5e-324, -5e-324, 1e308, -1e308, 0, -0.0,
+                    1, -1]
+    ref = ora.select_chunks(s, 77, 2, 2)
+    assert np.array_equal(_run_select(xkv, s, 77, 2, 2), ref)
+
+
+# ------------------------------------------------------------ reconstruct + attend
+def _attend(xkv, w, x, sel, dense=False):
+    d = xkv.dims_of(w)
+    n_sel = 0 if dense else sel.shape[2]
+    mode = xkv.XKV_MODE_DENSE if dense else xkv.XKV_MODE_SELECTIVE
+    ws = torch.empty(max(1, xkv.xkv_workspace_bytes(d, n_sel, mode)), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), device=DEV)
+    sel_d = None if dense else torch.from_numpy(sel).to(DEV)
+    xkv.xkv_reconstruct_attend(d, _dev(x["Ak"]), _dev(x["Av"]), _dev(x["Bkt"]), _dev(x["Bvt"]),
+                               _dev(x["q"]), sel_d, n_sel, out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", XKV_CASES, ids=lambda w: w.name)
+def test_reconstruct_attend_selective(xkv, ora, w):
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    got = _attend(xkv, w, x, sel)
+    compare_outputs(got, ref, w.dtype)
+
+
+@pytest.mark.parametrize("w", [DENSE_R, TINY], ids=lambda w: w.name)
+def test_reconstruct_attend_dense(xkv, ora, w):
+    x = _layer_inputs(w)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], None, w.chunk)
+    got = _attend(xkv, w, x, None, dense=True)
+    compare_outputs(got, ref, w.dtype)
+
+
+@pytest.mark.parametrize("n_sel", [1, 3, 17, 128])
+def test_reconstruct_attend_selection_sizes(xkv, ora, n_sel):
+    """One chunk (8 rows, a single partial tile) up to every chunk."""
+    w = dataclasses.replace(LLAMA_R, ctx_len=1024, batch=1)
+    x = _layer_inputs(w)
+    rng = np.random.default_rng(n_sel)
+    sel = np.stack([np.sort(rng.choice(w.n_chunks, n_sel, replace=False))
+                    for _ in range(w.n_kv_heads)])[None].astype(np.int32)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(_attend(xkv, w, x, sel), ref, w.dtype)
+
+
+def test_pipeline_end_to_end_tiny(xkv, ora):
+    """The whole decode step of the tiny fp32 workload on the GPU (landmarks built on the
+    GPU too) against the oracle's pipeline."""
+    w = TINY
+    d = xkv.dims_of(w)
+    for layer in range(w.n_layers):
+        x = _layer_inputs(w, layer)
+        lm_ref = ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk)
+        s_ref = ora.score_landmarks(ora.to_torch(lm_ref), x["q"])
+        sel_ref = ora.select_chunks(s_ref, w.top_k, w.n_sink, w.n_recent)
+        o_ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel_ref,
+                                       w.chunk)
+        lm = torch.empty((w.batch, w.n_kv_heads, w.n_chunks, w.head_dim), device=DEV)
+        xkv.xkv_build_landmarks(d, _dev(x["Ak"]), _dev(x["Bkt"]), lm)
+        sc = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
+        xkv.xkv_score_landmarks(d, lm, _dev(x["q"]), sc)
+        sel = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
+        xkv.xkv_select_chunks(d, sc, w.top_k, w.n_sink, w.n_recent, sel)
+        ws = torch.empty(xkv.xkv_workspace_bytes(d, w.n_sel, 0), dtype=torch.uint8, device=DEV)
+        out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+        xkv.xkv_reconstruct_attend(d, _dev(x["Ak"]), _dev(x["Av"]), _dev(x["Bkt"]),
+                                   _dev(x["Bvt"]), _dev(x["q"]), sel, w.n_sel, out, ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(lm.cpu().numpy(), lm_ref)
+        assert np.array_equal(sc.cpu().numpy().view(np.uint64), s_ref.view(np.uint64))
+        assert np.array_equal(sel.cpu().numpy(), sel_ref)
+        compare_outputs(out.cpu().numpy(), o_ref, w.dtype)
+
+
+# ----------------------------------------------------------------------------- R-CLA
+RCLA_R = synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=2, ctx_len=1500, n_layers=8,
+                       extra_rows=8)
+
+
+@pytest.mark.parametrize("w", [RCLA_R, dataclasses.replace(RCLA_R, dtype="f32", head_dim=64,
+                                                            n_q_heads=10, n_kv_heads=2,
+                                                            name="rcla_f32_g5")],
+                         ids=lambda w: w.name)
+def test_rcla_decode_step_matches_oracle(xkv, ora, w):
+    """One decode step over all layers: leaders append their new row, then every layer
+    attends its leader's cache; outputs and the caches after the step must agree."""
+    length = w.ctx_len
+    x = synth.np_rcla_inputs(w, seed=0, len_rows=length)
+    S = synth.leader_set(w)
+    lo = ora.leader_map(S, w.n_layers)
+    K_ref = ora.as_float64(x["K_lead"]).astype(np.float32) if w.dtype == "f32" else \
+        x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    V_ref = ora.as_float64(x["V_lead"]).astype(np.float32) if w.dtype == "f32" else \
+        x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    K = _dev(x["K_lead"])
+    V = _dev(x["V_lead"])
+    d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                     device=DEV)
+    for layer in range(w.n_layers):
+        leader = lo[layer] == layer
+        slot = S.index(lo[layer])
+        kn = x["k_new"][slot] if leader else None
+        vn = x["v_new"][slot] if leader else None
+        n = length if leader else length + 1
+        ref = ora.rcla_decode_attend(layer, lo, K_ref, V_ref, n, kn, vn, x["q"][layer])
+        out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+        xkv.rcla_decode_attend(d, layer, lo, K, V, w.L_max, n,
+                               _dev(kn) if leader else None, _dev(vn) if leader else None,
+                               _dev(x["q"][layer]), out, ws)
+        torch.cuda.synchronize()
+        compare_outputs(out.cpu().numpy(), ref, w.dtype)
+    if w.dtype == "f32":
+        assert np.array_equal(K.cpu().numpy(), K_ref) and np.array_equal(V.cpu().numpy(), V_ref)
+    else:
+        assert np.array_equal(K.cpu().view(torch.int16).numpy().view(np.uint16), K_ref)
+        assert np.array_equal(V.cpu().view(torch.int16).numpy().view(np.uint16), V_ref)
+
+
+@pytest.mark.parametrize("length", [0, 1, 127, 128, 129, 4095])
+def test_rcla_lengths(xkv, ora, length):
+    """From a single (new) row up to several tiles and splits, ragged tails."""
+    w = synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=1, ctx_len=max(length, 1), n_layers=2,
+                      extra_rows=1, outlier_frac=0.0)
+    x = synth.np_rcla_inputs(w, seed=length, len_rows=length)
+    lo = ora.leader_map([0], 2)
+    K_ref = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    V_ref = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    ref = ora.rcla_decode_attend(0, lo, K_ref, V_ref, length, x["k_new"][0], x["v_new"][0],
+                                 x["q"][0])
+    d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+    K, V = _dev(x["K_lead"]), _dev(x["V_lead"])
+    xkv.rcla_decode_attend(d, 0, lo, K, V, w.L_max, length, _dev(x["k_new"][0]),
+                           _dev(x["v_new"][0]), _dev(x["q"][0]), out, ws)
+    torch.cuda.synchronize()
+    compare_outputs(out.cpu().numpy(), ref, w.dtype)
+    assert np.array_equal(K.cpu().view(torch.int16).numpy().view(np.uint16), K_ref)
+
+
+def test_rcla_outlier_values_are_attended(xkv, ora):
+    """Rows whose V is 20x larger (1% of tokens) dominate nothing by themselves but must be
+    carried exactly: compare against the oracle with the outliers present."""
+    w = synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=2, ctx_len=3000, n_layers=1,
+                      extra_rows=0)
+    x = synth.np_rcla_inputs(w, seed=5, len_rows=3000)
+    lo = [0]
+    K_ref = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    V_ref = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    ref = ora.rcla_decode_attend(0, lo, K_ref, V_ref, 3000, None, None, x["q"][0])
+    d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+    xkv.rcla_decode_attend(d, 0, lo, _dev(x["K_lead"]), _dev(x["V_lead"]), w.L_max, 3000,
+                           None, None, _dev(x["q"][0]), out, ws)
+    torch.cuda.synchronize()
+    compare_outputs(out.cpu().numpy(), ref, w.dtype)
+
+
+def test_unsupported_device_paths_fail_loudly(xkv):
+    """Argument errors surface as exceptions from the binding (no silent fallback)."""
+    d = xkv.dims(1, 4, 2, 64, 64, 8, 16, 16, xkv.XKV_BF16)
+    with pytest.raises(xkv.XkvError):
+        xkv.xkv_score_landmarks(d, None, None, None)
