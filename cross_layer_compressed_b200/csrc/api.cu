@@ -141,7 +141,7 @@ int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t 
 size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
     if (mode == XKV_MODE_RCLA) {
         if (check_dims(dims, false, "xkv_workspace_bytes") != XKV_OK) return 0;
-        return partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
+        return WS_HEADER + partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
     }
     if (check_dims(dims, true, "xkv_workspace_bytes") != XKV_OK) return 0;
     int64_t rows;
@@ -153,7 +153,12 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
     } else {
         return 0;
     }
-    return partial_bytes(*dims, (int)plan_xkv(*dims, rows).n_bound);
+    int64_t n = plan_xkv(*dims, rows).n_bound;
+    if (attend_tc_supported(*dims)) {
+        const int n_tc = tc_splits(*dims, (int)(rows / dims->chunk));
+        if (n_tc > n) n = n_tc;
+    }
+    return WS_HEADER + partial_bytes(*dims, (int)n);
 }
 
 int64_t xkv_footprint_bytes(const xkv_dims *d, int32_t n_layers, int32_t window,
@@ -248,19 +253,31 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     if (sel && (n_sel <= 0 || n_sel > nC))
         return fail(XKV_ERR_INVALID_ARG, "%s: n_sel must be in [1, n_chunks]", who);
     const int64_t rows = sel ? (int64_t)n_sel * dims->chunk : dims->ctx_len;
+    const bool use_tc = attend_tc_supported(*dims) && !getenv("XKV_FORCE_SIMT");
     const SplitPlan plan = plan_xkv(*dims, rows);
-    if (plan.n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    const size_t need = partial_bytes(*dims, plan.n_split);
+    const int n_split = use_tc ? tc_splits(*dims, (int)(rows / dims->chunk)) : plan.n_split;
+    if (n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    const size_t need = WS_HEADER + partial_bytes(*dims, n_split);
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
     if (injected(who, &st)) return st;
     if ((st = check_device(who)) != XKV_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    float *partials = (float *)ws;
-    cudaError_t e = launch_attend_simt(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
-                                       n_sel, plan, partials, s);
-    if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, s);
+    unsigned *status = (unsigned *)ws;
+    float *partials = (float *)((char *)ws + WS_HEADER);
+    cudaError_t e;
+    int used_split = n_split;
+    if (use_tc) {
+        e = launch_attend_tc(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
+                             sel ? n_sel : (int)(dims->ctx_len / dims->chunk), partials, status,
+                             &used_split, s);
+        if (e == cudaSuccess) e = launch_combine(*dims, used_split, partials, out, status, s);
+    } else {
+        e = launch_attend_simt(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel, plan,
+                               partials, s);
+        if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, nullptr, s);
+    }
     return launched(e, who);
 }
 
@@ -300,17 +317,17 @@ xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t
         return fail(XKV_ERR_INVALID_ARG, "%s: need 0 < rows attended <= L_max", who);
     const SplitPlan plan = plan_rcla(*dims, n_rows);
     if (plan.n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    const size_t need = partial_bytes(*dims, plan.n_split);
+    const size_t need = WS_HEADER + partial_bytes(*dims, plan.n_split);
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
     if (injected(who, &st)) return st;
     if ((st = check_device(who)) != XKV_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    float *partials = (float *)ws;
+    float *partials = (float *)((char *)ws + WS_HEADER);
     cudaError_t e = launch_rcla(*dims, slot, L_max, n_rows, update ? len : -1, K_lead, V_lead,
                                 k_new, v_new, q, plan, partials, s);
-    if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, s);
+    if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, nullptr, s);
     return launched(e, who);
 }
 

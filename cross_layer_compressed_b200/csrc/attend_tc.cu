@@ -1,0 +1,601 @@
+// Selective / dense reconstruction + GQA attention on the 5th-generation tensor cores.
+//
+// xKV page, section 2.3 (selective reconstruction) and section 4 (dense): for each
+// (sequence b, KV head g) only the rows T of the selected chunks are rebuilt,
+//   K_hat = A^K[T] B^K_l[:, g],  V_hat = A^V[T] B^V_l[:, g],
+// and the G query heads of the group attend over them.  The two rebuilds are dense
+// GEMMs (rank 512 / 768 deep) and run as tcgen05.mma (bf16 in, fp32 accumulate in
+// tensor memory); K_hat and V_hat never leave the SM.
+//
+// Work item = (b, g, a run of <= 256 selected rows).  Persistent kernel: one CTA per SM
+// walks the items; roles are warp-specialised:
+//   warp 0      TMA producer.  Per 64-wide rank slice it loads, into one pipeline stage,
+//               the item's A rows (one 8-row x 128-byte box per row group, so any set
+//               of chunks is gathered with no index arithmetic in the MMA path) and the
+//               matching 128 x 64 slice of B_l's group-g columns (B_l is stored
+//               column-major, so that slice is K-major).  Stages are released by the
+//               MMAs' completion (tcgen05.commit).
+//   warp 1      allocates the 512 TMEM columns; one thread issues the MMAs.
+//               Key phase:   D_K[tok][j]  (cols   0..255) += A^K[tok][k] . B^K[j][k]
+//                            (M = 128 tokens per MMA, N = hd = 128)
+//               Value phase: D_V[j][tok]  (cols 256..511) += B^V[j][k] . A^V[tok][k]
+//                            (M = hd = 128, N = tokens rounded up to 16)
+//               so keys come out one token per TMEM lane and values one head-dim per
+//               lane -- each epilogue thread then needs no cross-thread reduction.
+//   warps 2-5   epilogue.  Key epilogue: thread = token, logits z_h = q_h . K_hat (fp32),
+//               then the exact max / sum of the item's rows.  Value epilogue: thread =
+//               output column j, o_h[j] = sum_t p_h[t] V_hat[t][j].  Partials
+//               (m, l, o) go to the workspace; the combine kernel merges items.
+// The key MMAs of item i+1 overlap the value epilogue of item i (separate TMEM columns);
+// the producer runs ahead across items, so the HBM stream does not stop between items.
+//
+// Every wait on an mbarrier is bounded; on expiry the CTA records XKV_ERR_TIMEOUT in the
+// workspace status word, drains its own copies and MMAs (again bounded), frees TMEM and
+// returns; the combine kernel then writes NaN outputs.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "xkv_internal.cuh"
+
+namespace xkv {
+namespace {
+
+constexpr int TC_STAGES = 4;
+constexpr int TC_ROWS = 256;                 // rows per work item
+constexpr int TC_KS = 64;                    // rank slice per stage: 128 bytes of bf16
+constexpr int TC_HD = 128;
+constexpr int A_TILE = TC_ROWS * TC_KS * 2;  // 32 KB: 32 row groups of 8 x 128 B
+constexpr int B_TILE = TC_HD * TC_KS * 2;    // 16 KB
+constexpr int STAGE_BYTES = A_TILE + B_TILE;
+constexpr int TC_THREADS = 192;
+constexpr uint32_t SPIN_LIMIT = 1u << 24;
+
+struct TcShared {
+    uint64_t full[TC_STAGES];
+    uint64_t empty[TC_STAGES];
+    uint64_t kdone, vdone, kfree, vfree, idle;
+    uint32_t tmem_base;
+    int abort;
+    int issued[TC_STAGES];
+    float red[4][16];
+};
+
+struct TcParams {
+    const __nv_bfloat16 *q;   // [B][Hq][hd]
+    const int32_t *sel;       // [B][Hkv][n_sel] or null (dense)
+    float *partials;          // [n_split][B][Hq][hd + 2]
+    unsigned *status;         // workspace status word
+    int64_t L;
+    int n_sel;                // chunks per unit
+    int C;
+    int rk, rv;
+    int Hq, Hkv, B;
+    int chunks_per_item;
+    int n_split;
+    int n_items;
+    float qscale;             // log2(e) / sqrt(hd)
+};
+
+// ----------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t su32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of parity `parity`; false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared *sh) {
+    for (uint32_t i = 0; i < SPIN_LIMIT; ++i) {
+        if (mbar_test(b, parity)) return true;
+        if (*(volatile int *)&sh->abort) return false;
+    }
+    return false;
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(su32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (leading offset unused for this layout; version 1).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                     uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            su32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, "
+        "%26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+          "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier of the 128 epilogue threads that also ORs `flag` over them, so that a decision
+// taken after a bounded wait is the same in every epilogue thread.
+__device__ __forceinline__ bool epi_bar_any(bool flag) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pin, pout;\n\t"
+        "setp.ne.u32 pin, %1, 0;\n\t"
+        "bar.red.or.pred pout, 1, 128, pin;\n\t"
+        "selp.u32 %0, 1, 0, pout;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag)
+        : "memory");
+    return r != 0;
+}
+
+struct Item {
+    int b, g, split, c0, nch, nr;
+};
+__device__ __forceinline__ Item decode(const TcParams &p, int item) {
+    Item it;
+    const int u = item / p.n_split;
+    it.split = item % p.n_split;
+    it.b = u / p.Hkv;
+    it.g = u % p.Hkv;
+    it.c0 = it.split * p.chunks_per_item;
+    it.nch = min(p.chunks_per_item, p.n_sel - it.c0);
+    it.nr = it.nch * p.C;
+    return it;
+}
+
+__device__ void abort_cta(TcShared *sh, const TcParams &p) {
+    *(volatile int *)&sh->abort = 1;
+    if (p.status) atomicOr(p.status, 1u << XKV_ERR_TIMEOUT);
+}
+
+template <int G>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_xkv_tc(const __grid_constant__ CUtensorMap tmAk, const __grid_constant__ CUtensorMap tmAv,
+             const __grid_constant__ CUtensorMap tmBk, const __grid_constant__ CUtensorMap tmBv,
+             const TcParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    TcShared *sh = reinterpret_cast<TcShared *>(smem + TC_STAGES * STAGE_BYTES);
+    float *qs = reinterpret_cast<float *>(sh + 1);       // [hd][G]
+    float *zs = qs + TC_HD * G;                          // [TC_ROWS][G]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nC = p.L / p.C;
+    const int gpc = p.C / 8;                             // 8-row groups per chunk
+
+    if (threadIdx.x == 0 && blockIdx.x == 0 && p.status) *p.status = 0u;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&sh->full[s], 1);
+            mbar_init(&sh->empty[s], 1);
+            sh->issued[s] = 0;
+        }
+        mbar_init(&sh->kdone, 1);
+        mbar_init(&sh->vdone, 1);
+        mbar_init(&sh->kfree, 1);
+        mbar_init(&sh->vfree, 1);
+        mbar_init(&sh->idle, 1);
+        sh->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_tmap(&tmAk);
+        prefetch_tmap(&tmAv);
+        prefetch_tmap(&tmBk);
+        prefetch_tmap(&tmBv);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         su32(&sh->tmem_base))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        int it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+            const Item w = decode(p, item);
+            const int ng = w.nr / 8;
+            int row = 0;
+            if (lane < ng) {
+                const int ci = lane / gpc, sub = lane % gpc;
+                int64_t c = w.c0 + ci;
+                if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
+                c = min64(max64(c, 0), nC - 1);  // out-of-range indices are clamped
+                row = (int)((int64_t)w.b * p.L + c * p.C + sub * 8);
+            }
+            const int brow = (w.b * p.Hkv + w.g) * TC_HD;
+            for (int phase = 0; phase < 2 && ok; ++phase) {
+                const int nks = (phase == 0 ? p.rk : p.rv) / TC_KS;
+                const CUtensorMap *mA = phase == 0 ? &tmAk : &tmAv;
+                const CUtensorMap *mB = phase == 0 ? &tmBk : &tmBv;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % TC_STAGES, n = it / TC_STAGES;
+                    int got = 0;
+                    if (lane == 0) {
+                        got = mbar_wait(&sh->empty[s], (n & 1) ^ 1, sh) ? 1 : 0;
+                        if (!got) abort_cta(sh, p);
+                    }
+                    if (!__shfl_sync(0xffffffffu, got, 0)) {  // same decision in every lane
+                        ok = false;
+                        break;
+                    }
+                    unsigned char *st = smem + s * STAGE_BYTES;
+                    if (lane == 0) {
+                        mbar_expect_tx(&sh->full[s], (uint32_t)(ng * 1024 + B_TILE));
+                        sh->issued[s] = n + 1;
+                    }
+                    __syncwarp();
+                    if (lane < ng) tma_load_2d(mA, &sh->full[s], st + lane * 1024, ks * TC_KS, row);
+                    if (lane == 0) tma_load_2d(mB, &sh->full[s], st + A_TILE, ks * TC_KS, brow);
+                }
+            }
+        }
+        if (!ok && lane == 0) {  // drain this CTA's copies in flight before exiting
+            for (int s = 0; s < TC_STAGES; ++s)
+                if (sh->issued[s] > 0) {
+                    for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
+                        if (mbar_test(&sh->full[s], (sh->issued[s] - 1) & 1)) break;
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t smem_base = su32(smem);
+            int it = 0, ic = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++ic) {
+                const Item w = decode(p, item);
+                const int nr16 = (w.nr + 15) & ~15;
+                const uint32_t idK = idesc_bf16(128, TC_HD);
+                const uint32_t idV = idesc_bf16(128, nr16);
+                // key phase into columns [0, 256)
+                if (!mbar_wait(&sh->kfree, (ic & 1) ^ 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                tc_fence_after();
+                const int nk = p.rk / TC_KS;
+                for (int ks = 0; ks < nk && ok; ++ks, ++it) {
+                    const int s = it % TC_STAGES, n = it / TC_STAGES;
+                    if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
+#pragma unroll
+                    for (int kk = 0; kk < TC_KS / 16; ++kk) {
+                        const uint32_t acc = (ks | kk) ? 1u : 0u;
+                        umma(tmem, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), idK, acc);
+                        if (w.nr > 128)
+                            umma(tmem + 128, sdesc(a0 + 16384 + kk * 32), sdesc(b0 + kk * 32), idK,
+                                 acc);
+                    }
+                    umma_commit(&sh->empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&sh->kdone);
+                // value phase into columns [256, 512)
+                if (!mbar_wait(&sh->vfree, (ic & 1) ^ 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                tc_fence_after();
+                const int nv = p.rv / TC_KS;
+                for (int ks = 0; ks < nv && ok; ++ks, ++it) {
+                    const int s = it % TC_STAGES, n = it / TC_STAGES;
+                    if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
+#pragma unroll
+                    for (int kk = 0; kk < TC_KS / 16; ++kk)
+                        umma(tmem + 256, sdesc(b0 + kk * 32), sdesc(a0 + kk * 32), idV,
+                             (ks | kk) ? 1u : 0u);
+                    umma_commit(&sh->empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&sh->vdone);
+            }
+            // all MMAs issued by this thread have completed once `idle` fires
+            umma_commit(&sh->idle);
+            for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
+                if (mbar_test(&sh->idle, 0)) break;
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;          // 0..127
+        const int quad = warp & 3;                // TMEM lane quadrant of this warp
+        const int ew = warp - 2;                  // epilogue warp 0..3
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        int ic = 0;
+        for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++ic) {
+            const Item w = decode(p, item);
+            epi_bar();
+            const __nv_bfloat16 *qg = p.q + ((size_t)w.b * p.Hq + (size_t)w.g * G) * TC_HD;
+            for (int e = et; e < G * TC_HD; e += 128) {
+                const int h = e / TC_HD, j = e % TC_HD;
+                qs[j * G + h] = __bfloat162float(qg[e]) * p.qscale;
+            }
+            epi_bar();
+            {
+                const bool fail = !mbar_wait(&sh->kdone, ic & 1, sh);
+                if (fail) abort_cta(sh, p);
+                if (epi_bar_any(fail)) break;
+            }
+            tc_fence_after();
+            // key epilogue: thread = token (quad*32 + lane within each 128-row half)
+            for (int half = 0; half < (w.nr > 128 ? 2 : 1); ++half) {
+                float acc[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < TC_HD; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + half * 128 + c0, v);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float *qd = qs + (c0 + c) * G;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) acc[h] = fmaf(v[c], qd[h], acc[h]);
+                    }
+                }
+                const int t = half * 128 + quad * 32 + lane;
+                if (t < w.nr) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) zs[t * G + h] = acc[h];
+                }
+            }
+            tc_fence_before();
+            epi_bar();
+            if (et == 0) mbar_arrive(&sh->kfree);
+            // exact softmax statistics of the item's rows (log2 domain)
+            float m[G], l[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) m[h] = -INFINITY;
+            for (int t = et; t < w.nr; t += 128)
+#pragma unroll
+                for (int h = 0; h < G; ++h) m[h] = fmaxf(m[h], zs[t * G + h]);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1)
+                    m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
+                if (lane == 0) sh->red[ew][h] = m[h];
+            }
+            epi_bar();
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+                m[h] = fmaxf(fmaxf(sh->red[0][h], sh->red[1][h]), fmaxf(sh->red[2][h], sh->red[3][h]));
+            epi_bar();
+#pragma unroll
+            for (int h = 0; h < G; ++h) l[h] = 0.f;
+            for (int t = et; t < w.nr; t += 128)
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float pv = exp2f(zs[t * G + h] - m[h]);
+                    zs[t * G + h] = pv;
+                    l[h] += pv;
+                }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+                if (lane == 0) sh->red[ew][h] = l[h];
+            }
+            epi_bar();
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+                l[h] = (sh->red[0][h] + sh->red[1][h]) + (sh->red[2][h] + sh->red[3][h]);
+            // value epilogue: thread = output column j = quad*32 + lane
+            {
+                const bool fail = !mbar_wait(&sh->vdone, ic & 1, sh);
+                if (fail) abort_cta(sh, p);
+                if (epi_bar_any(fail)) break;
+            }
+            tc_fence_after();
+            float o[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) o[h] = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < w.nr; c0 += 32) {
+                float v[32];
+                tmem_ld32(tmem + lane_base + 256 + c0, v);
+                const int nc = min(32, w.nr - c0);
+                if (nc == 32) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float *pz = zs + (c0 + c) * G;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) o[h] = fmaf(pz[h], v[c], o[h]);
+                    }
+                } else {
+                    for (int c = 0; c < nc; ++c) {
+                        const float *pz = zs + (c0 + c) * G;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) o[h] = fmaf(pz[h], v[c], o[h]);
+                    }
+                }
+            }
+            tc_fence_before();
+            epi_bar();
+            if (et == 0) mbar_arrive(&sh->vfree);
+            const int j = quad * 32 + lane;
+            float *dst = p.partials + (((size_t)w.split * p.B + w.b) * p.Hq + (size_t)w.g * G) *
+                                          (TC_HD + 2);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                dst[h * (TC_HD + 2) + 2 + j] = o[h];
+                if (et == 0) {
+                    dst[h * (TC_HD + 2)] = m[h] * 0.6931471805599453f;  // back to natural log
+                    dst[h * (TC_HD + 2) + 1] = l[h];
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
+                     : "memory");
+}
+
+// ----------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
+    }
+    return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows][cols] array with a 128-byte-swizzled box of
+// box_rows x 64 elements.
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)TC_KS, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int G>
+cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s) {
+    const size_t smem = 1024 + (size_t)TC_STAGES * STAGE_BYTES + sizeof(TcShared) +
+                        sizeof(float) * ((size_t)TC_HD * G + (size_t)TC_ROWS * G);
+    auto k = k_xkv_tc<G>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
+    k<<<grid, TC_THREADS, smem, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attend_tc_supported(const xkv_dims &d) {
+    return d.dtype == XKV_BF16 && d.head_dim == TC_HD && d.rank_k % TC_KS == 0 &&
+           d.rank_v % TC_KS == 0 && TC_ROWS % d.chunk == 0 && encode_fn() != nullptr;
+}
+
+int tc_splits(const xkv_dims &d, int n_sel) {
+    const int64_t rows = (int64_t)n_sel * d.chunk;
+    return (int)((rows + TC_ROWS - 1) / TC_ROWS);
+}
+
+cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
+                             const void *Bvt, const void *q, const int32_t *sel, int n_sel,
+                             float *partials, unsigned *status, int *n_split_out,
+                             cudaStream_t s) {
+    const int64_t d_kv = (int64_t)d.n_kv_heads * d.head_dim;
+    CUtensorMap maps[4];
+    if (!make_map(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8) ||
+        !make_map(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8) ||
+        !make_map(&maps[2], Bkt, (uint64_t)d.batch * d_kv, d.rank_k, TC_HD) ||
+        !make_map(&maps[3], Bvt, (uint64_t)d.batch * d_kv, d.rank_v, TC_HD))
+        return cudaErrorInvalidValue;
+    TcParams p;
+    p.q = (const __nv_bfloat16 *)q;
+    p.sel = sel;
+    p.partials = partials;
+    p.status = status;
+    p.L = d.ctx_len;
+    p.n_sel = n_sel;
+    p.C = d.chunk;
+    p.rk = d.rank_k;
+    p.rv = d.rank_v;
+    p.Hq = d.n_q_heads;
+    p.Hkv = d.n_kv_heads;
+    p.B = d.batch;
+    const int n_split = tc_splits(d, n_sel);
+    p.chunks_per_item = (n_sel + n_split - 1) / n_split;
+    p.n_split = (n_sel + p.chunks_per_item - 1) / p.chunks_per_item;
+    p.n_items = d.batch * d.n_kv_heads * p.n_split;
+    p.qscale = 1.4426950408889634f / sqrtf((float)d.head_dim);
+    *n_split_out = p.n_split;
+    switch (d.n_q_heads / d.n_kv_heads) {
+#define XKV_G(GG) \
+    case GG: return launch_g<GG>(maps, p, s);
+        XKV_G(1) XKV_G(2) XKV_G(3) XKV_G(4) XKV_G(5) XKV_G(6) XKV_G(7) XKV_G(8)
+        XKV_G(9) XKV_G(10) XKV_G(11) XKV_G(12) XKV_G(13) XKV_G(14) XKV_G(15) XKV_G(16)
+#undef XKV_G
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace xkv

@@ -8,9 +8,14 @@ namespace {
 
 __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ partials,
                                                  float *__restrict__ out, int n_split,
-                                                 int BH, int hd) {
+                                                 int BH, int hd,
+                                                 const unsigned *__restrict__ status) {
     const int bh = blockIdx.x;
     const int j = threadIdx.x;
+    if (status && *(volatile const unsigned *)status) {  // the attention kernel gave up
+        if (j < hd) out[(size_t)bh * hd + j] = __int_as_float(0x7fc00000);
+        return;
+    }
     const size_t stride = (size_t)BH * (hd + 2);
     const float *p = partials + (size_t)bh * (hd + 2);
     float M = -INFINITY;
@@ -27,9 +32,9 @@ __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ parti
 }  // namespace
 
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
-                           cudaStream_t s) {
+                           const unsigned *status, cudaStream_t s) {
     const int BH = d.batch * d.n_q_heads;
-    k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim);
+    k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
     return cudaGetLastError();
 }
 

@@ -42,7 +42,18 @@ cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_ro
                         const void *v_new, const void *q, const SplitPlan &plan,
                         float *partials, cudaStream_t s);
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
-                           cudaStream_t s);
+                           const unsigned *status, cudaStream_t s);
+// tensor-core path (bf16, head_dim 128, ranks multiple of 64, chunk dividing 256)
+bool attend_tc_supported(const xkv_dims &d);
+int tc_splits(const xkv_dims &d, int n_sel);
+cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
+                             const void *Bvt, const void *q, const int32_t *sel, int n_sel,
+                             float *partials, unsigned *status, int *n_split_out,
+                             cudaStream_t s);
+
+// Workspace layout: a 256-byte header (word 0: device status bits, 1 << xkv_status) and
+// then the partials.
+constexpr size_t WS_HEADER = 256;
 
 // ------------------------------------------------------------------ device helpers
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
