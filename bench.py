@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -359,6 +361,24 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ rank aggregation
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank number over all ranks (the timed region's length)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(batch_per_rank: int, steps: int, world: int,
+                           max_elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank decodes its own batch (weak scaling)."""
+    return world * batch_per_rank * steps / (max_elapsed_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- driver
 def main():
     args = parse()
@@ -367,6 +387,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from cross_layer_compressed_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.batch)
     if args.impl == "reference":
         reference_arm(args, w, rank, world)
         return
@@ -391,13 +414,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---------------- device-resident timing
     for s in range(args.warmup):
         wl.step(s % nq)
@@ -419,7 +435,7 @@ def main():
     stop.record(stream)
     barrier()
     clk = clocks.stop()
-    elapsed_ms = max_over_ranks(start.elapsed_time(stop))
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
     per_launch = [a.elapsed_time(b) for step in attend_ms for a, b in step]
     attend_avg_ms = float(np.mean(per_launch))
 
@@ -443,9 +459,10 @@ def main():
             out_host.copy_(wl.out, non_blocking=True)
         e1.record(stream)
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d, d2h = wl.io_bytes()
-        e2e = {"value": world * w.batch * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": aggregate_tokens_per_s(w.batch, args.steps, world, e2e_ms),
+               "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---------------- algorithmic bytes (untimed: selections recomputed per slot)
@@ -468,7 +485,7 @@ def main():
         cpu = cpu_baseline(w, args.seed)
     if rank == 0:
         ms_step = elapsed_ms / args.steps
-        value = world * w.batch * args.steps / (elapsed_ms / 1e3)
+        value = aggregate_tokens_per_s(w.batch, args.steps, world, elapsed_ms)
         cfg = {"workload": w.name, "batch": w.batch, "ctx_len": w.ctx_len,
                "n_layers": w.n_layers, "heads_q_kv": [w.n_q_heads, w.n_kv_heads],
                "head_dim": w.head_dim, "parallelism": f"replicas x{world}",

@@ -154,7 +154,7 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
         return 0;
     }
     int64_t n = plan_xkv(*dims, rows).n_bound;
-    if (attend_tc_supported(*dims)) {
+    if (attend_tc_shape_ok(*dims)) {
         const int n_tc = tc_splits(*dims, (int)(rows / dims->chunk));
         if (n_tc > n) n = n_tc;
     }
@@ -253,21 +253,23 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     if (sel && (n_sel <= 0 || n_sel > nC))
         return fail(XKV_ERR_INVALID_ARG, "%s: n_sel must be in [1, n_chunks]", who);
     const int64_t rows = sel ? (int64_t)n_sel * dims->chunk : dims->ctx_len;
-    const bool use_tc = attend_tc_supported(*dims) && !getenv("XKV_FORCE_SIMT");
     const SplitPlan plan = plan_xkv(*dims, rows);
-    const int n_split = use_tc ? tc_splits(*dims, (int)(rows / dims->chunk)) : plan.n_split;
-    if (n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    const size_t need = WS_HEADER + partial_bytes(*dims, n_split);
+    const int n_tc = attend_tc_shape_ok(*dims) ? tc_splits(*dims, (int)(rows / dims->chunk)) : 0;
+    if (plan.n_split > 65535 || n_tc > 65535)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    // the same amount xkv_workspace_bytes reports, whichever kernel runs
+    const size_t need = WS_HEADER + partial_bytes(*dims, (int)(n_tc > plan.n_bound ? n_tc : plan.n_bound));
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
     if (injected(who, &st)) return st;
     if ((st = check_device(who)) != XKV_OK) return st;
+    const bool use_tc = n_tc > 0 && attend_tc_supported(*dims) && !getenv("XKV_FORCE_SIMT");
     cudaStream_t s = (cudaStream_t)stream;
     unsigned *status = (unsigned *)ws;
     float *partials = (float *)((char *)ws + WS_HEADER);
     cudaError_t e;
-    int used_split = n_split;
+    int used_split = n_tc;
     if (use_tc) {
         e = launch_attend_tc(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
                              sel ? n_sel : (int)(dims->ctx_len / dims->chunk), partials, status,

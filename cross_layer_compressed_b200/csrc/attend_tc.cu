@@ -548,9 +548,13 @@ cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s)
 
 }  // namespace
 
-bool attend_tc_supported(const xkv_dims &d) {
+bool attend_tc_shape_ok(const xkv_dims &d) {
     return d.dtype == XKV_BF16 && d.head_dim == TC_HD && d.rank_k % TC_KS == 0 &&
-           d.rank_v % TC_KS == 0 && TC_ROWS % d.chunk == 0 && encode_fn() != nullptr;
+           d.rank_v % TC_KS == 0 && TC_ROWS % d.chunk == 0;
+}
+
+bool attend_tc_supported(const xkv_dims &d) {
+    return attend_tc_shape_ok(d) && encode_fn() != nullptr;
 }
 
 int tc_splits(const xkv_dims &d, int n_sel) {

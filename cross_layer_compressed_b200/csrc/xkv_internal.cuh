@@ -44,7 +44,8 @@ cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_ro
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
                            const unsigned *status, cudaStream_t s);
 // tensor-core path (bf16, head_dim 128, ranks multiple of 64, chunk dividing 256)
-bool attend_tc_supported(const xkv_dims &d);
+bool attend_tc_shape_ok(const xkv_dims &d);   // shapes only (sizes workspaces)
+bool attend_tc_supported(const xkv_dims &d);  // shapes and a driver with TMA maps
 int tc_splits(const xkv_dims &d, int n_sel);
 cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
                              const void *Bvt, const void *q, const int32_t *sel, int n_sel,

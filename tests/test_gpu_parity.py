@@ -181,6 +181,17 @@ def test_reconstruct_attend_selective(xkv, ora, w):
     compare_outputs(got, ref, w.dtype)
 
 
+@pytest.mark.parametrize("w", [LLAMA_R, QWEN14_R], ids=lambda w: w.name)
+def test_reconstruct_attend_cuda_core_path_bf16(xkv, ora, w, monkeypatch):
+    """The CUDA-core kernel on bf16 shapes the tensor-core kernel normally takes."""
+    monkeypatch.setenv("XKV_FORCE_SIMT", "1")
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(_attend(xkv, w, x, sel), ref, w.dtype)
+
+
 @pytest.mark.parametrize("w", [DENSE_R, TINY], ids=lambda w: w.name)
 def test_reconstruct_attend_dense(xkv, ora, w):
     x = _layer_inputs(w)
