@@ -127,6 +127,8 @@ SplitPlan plan_rcla(const xkv_dims &d, int64_t rows) {
 
 }  // namespace
 
+void xkv::set_last_error(const char *msg) { g_last_error = msg; }
+
 extern "C" {
 
 const char *xkv_last_error(void) { return g_last_error.c_str(); }

@@ -52,6 +52,9 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
                              float *partials, unsigned *status, int *n_split_out,
                              cudaStream_t s);
 
+// Sets the calling thread's xkv_last_error() message (defined with the C ABI layer).
+void set_last_error(const char *msg);
+
 // Workspace layout: a 256-byte header (word 0: device status bits, 1 << xkv_status) and
 // then the partials.
 constexpr size_t WS_HEADER = 256;

@@ -52,6 +52,8 @@ _sigs = {
                                ctypes.c_int),
     "rcla_decode_attend": ([_D, _i32, _vp, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                             _sz, _vp], ctypes.c_int),
+    "xkv_reconstruct_attend_noalloc": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp],
+                                       ctypes.c_int),
     "xkv_workspace_bytes": ([_D, _i32, _i32], _sz),
     "xkv_n_selected": ([_i64, _i32, _i32, _i32], _i64),
     "xkv_footprint_bytes": ([_D, _i32, _i32, _i32], _i64),
@@ -143,6 +145,18 @@ def xkv_reconstruct_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
                                      _ptr(Bkt_layer), _ptr(Bvt_layer), _ptr(q), _ptr(sel),
                                      int(n_sel), _ptr(out), _ptr(ws), int(ws_bytes),
                                      _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_reconstruct_attend_noalloc(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
+                                   n_sel, out, stream=None, check=True):
+    """xkv_reconstruct_attend with the library's fixed scratch array instead of a
+    workspace, for callers that cannot allocate device memory (see include/xkv.h)."""
+    st = _lib.xkv_reconstruct_attend_noalloc(ctypes.byref(d), _ptr(Ak_win), _ptr(Av_win),
+                                             _ptr(Bkt_layer), _ptr(Bvt_layer), _ptr(q),
+                                             _ptr(sel), int(n_sel), _ptr(out), _stream(stream))
     if check:
         _check(st)
     return st

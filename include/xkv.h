@@ -160,6 +160,27 @@ xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t
                               int64_t len, const void *k_new, const void *v_new, const void *q,
                               float *out, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * xkv_reconstruct_attend without a workspace, for callers that cannot allocate device
+ * memory (engine plugin hooks handed no workspace, processes whose HBM is reserved by a
+ * serving engine's KV pool, paths where an allocation's device synchronisation is not
+ * allowed).  No counterpart on the pages: this is a library convenience.
+ *   Same arguments, layouts and results as xkv_reconstruct_attend, minus ws / ws_bytes.
+ *   Scratch: a fixed 16 MiB array of device memory inside the library, held by every
+ *   GPU that loads the library until the process exits.  A call whose scratch need
+ *   (xkv_workspace_bytes) exceeds 16 MiB returns XKV_ERR_UNSUPPORTED.
+ *   The first call on a device (with that device current) looks up the array's device
+ *   address once; make that first call before any stream capture.
+ *   Every call on a device shares the one array: calls whose kernels overlap on the GPU
+ *   (different streams, or graphs replayed concurrently) race and give wrong results.
+ *   Calls queued on one stream are safe.  The function calls no allocator.
+ */
+xkv_status xkv_reconstruct_attend_noalloc(const xkv_dims *dims, const void *Ak_win,
+                                          const void *Av_win, const void *Bkt_layer,
+                                          const void *Bvt_layer, const void *q,
+                                          const int32_t *sel, int32_t n_sel, float *out,
+                                          void *stream);
+
 /* Scratch bytes the attention calls need (the split-K partial results). 0 on bad dims. */
 size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode);
 
