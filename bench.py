@@ -47,6 +47,8 @@ def parse():
                    help="override the workload's batch (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch every call directly instead of replaying a captured step")
     return p.parse_args()
 
 
@@ -414,12 +416,41 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # ---------------- device-resident timing
-    for s in range(args.warmup):
+    # ---------------- capture: one CUDA graph per query slot (the xKV steps are
+    # stateless; the R-CLA step advances its cache length, so it launches directly)
+    use_graph = not args.no_graph and w.mode != "rcla"
+    for s in range(args.warmup):                    # also initialises the library's caches
         wl.step(s % nq)
-    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-          for _ in range(w.n_layers)]
-    attend_ms = []
+    torch.cuda.synchronize(dev)
+    graphs = {}
+    e2e_graph = None
+    if use_graph:
+        for slot in sorted({s % nq for s in range(max(args.steps, args.warmup))}):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                wl.step(slot)
+            graphs[slot] = g
+        if not args.no_e2e:
+            e2e_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(e2e_graph):
+                wl.step(q=wl.q_in)
+        torch.cuda.synchronize(dev)
+
+    def run_step(s):
+        if use_graph:
+            graphs[s % nq].replay()
+        else:
+            wl.step(s % nq)
+
+    def run_e2e_step():
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            wl.step(q=wl.q_in)
+
+    # ---------------- device-resident timing (the reported value)
+    for s in range(args.warmup):
+        run_step(s)
     clocks = ClockSampler(local)
     barrier()
     clocks.start()
@@ -427,16 +458,23 @@ def main():
     stop = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for s in range(args.steps):
-        wl.step(s % nq, attend_events=ev)
-        # attention-launch events of this step are read after the timed region
-        attend_ms.append(ev)
-        ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-              for _ in range(w.n_layers)]
+        run_step(s)
     stop.record(stream)
     barrier()
     clk = clocks.stop()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
-    per_launch = [a.elapsed_time(b) for step in attend_ms for a, b in step]
+
+    # ---------------- per-launch time of the attention kernel: the same steps launched
+    # directly, CUDA events around every attention call on the launching stream
+    ev_steps = []
+    barrier()
+    for s in range(args.steps):
+        ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+              for _ in range(w.n_layers)]
+        wl.step(s % nq, attend_events=ev)
+        ev_steps.append(ev)
+    barrier()
+    per_launch = [a.elapsed_time(b) for step in ev_steps for a, b in step]
     attend_avg_ms = float(np.mean(per_launch))
 
     # ---------------- end to end through the public API with host buffers
@@ -447,7 +485,7 @@ def main():
         out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
         for s in range(args.warmup):
             wl.q_in.copy_(q_host[s % nq], non_blocking=True)
-            wl.step(q=wl.q_in)
+            run_e2e_step()
             out_host.copy_(wl.out, non_blocking=True)
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -455,15 +493,14 @@ def main():
         e0.record(stream)
         for s in range(args.steps):
             wl.q_in.copy_(q_host[s % nq], non_blocking=True)
-            wl.step(q=wl.q_in)
+            run_e2e_step()
             out_host.copy_(wl.out, non_blocking=True)
         e1.record(stream)
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d, d2h = wl.io_bytes()
         e2e = {"value": aggregate_tokens_per_s(w.batch, args.steps, world, e2e_ms),
-               "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---------------- algorithmic bytes (untimed: selections recomputed per slot)
     slots = sorted({s % nq for s in range(args.steps)})[:4]
@@ -512,6 +549,7 @@ def main():
                          "frac_of_8tbs": achieved / 8000.0, "traffic": traffic,
                          "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms},
             "gpu_launches": wl.launches_per_step * args.steps,
+            "cuda_graph": use_graph,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

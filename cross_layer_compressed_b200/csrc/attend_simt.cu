@@ -150,7 +150,7 @@ cudaError_t launch_g(const xkv_dims &d, const void *Ak, const void *Av, const vo
                                          (size_t)plan.rows_per_split * G);
     const int64_t rows = sel ? (int64_t)n_sel * d.chunk : d.ctx_len;
     auto k = k_attend_simt<T, G>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    set_smem_limit((const void *)k, smem);
     dim3 grid(plan.n_split, d.n_kv_heads, d.batch);
     k<<<grid, AT_THREADS, smem, s>>>((const T *)Ak, (const T *)Av, (const T *)Bkt,
                                      (const T *)Bvt, (const T *)q, sel, n_sel, d.ctx_len,

@@ -539,7 +539,7 @@ cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s)
     const size_t smem = 1024 + (size_t)TC_STAGES * STAGE_BYTES + sizeof(TcShared) +
                         sizeof(float) * ((size_t)TC_HD * G + (size_t)TC_ROWS * G);
     auto k = k_xkv_tc<G>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
     k<<<grid, TC_THREADS, smem, s>>>(maps[0], maps[1], maps[2], maps[3], p);

@@ -1,6 +1,10 @@
 // Merge of split-K partial attention results (flash-decoding): each split s of a
 // (sequence, query head) left (m_s, l_s, acc_s) with acc_s = sum_t exp(z_t - m_s) v_t
 // over its rows.  out = sum_s exp(m_s - M) acc_s / sum_s exp(m_s - M) l_s, M = max m_s.
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "xkv_internal.cuh"
 
 namespace xkv {
@@ -52,6 +56,20 @@ SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max
     p.rows_per_split = (rows + n - 1) / n;
     p.n_split = (int)((rows + p.rows_per_split - 1) / p.rows_per_split);  // no empty split
     return p;
+}
+
+cudaError_t set_smem_limit(const void *kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &cur = done[std::make_pair(kernel, dev)];
+    if (bytes <= cur) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) cur = bytes;
+    return e;
 }
 
 size_t partial_bytes(const xkv_dims &d, int n_split) {

@@ -153,7 +153,7 @@ cudaError_t launch_g(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,
                         sizeof(float) * ((size_t)d.head_dim * G + 2 * G +
                                          (size_t)plan.rows_per_split * G);
     auto k = k_rcla<T, G>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    set_smem_limit((const void *)k, smem);
     dim3 grid(plan.n_split, d.n_kv_heads, d.batch);
     k<<<grid, RC_THREADS, smem, s>>>((T *)K, (T *)V, (const T *)k_new, (const T *)v_new,
                                      (const T *)q, slot, d.n_q_heads, d.n_kv_heads, d.head_dim,

@@ -83,7 +83,7 @@ cudaError_t launch_t(const xkv_dims &d, const void *lm, const void *q, double *s
 #define XKV_SCORE_CASE(GG)                                                                  \
     case GG: {                                                                              \
         auto k = k_score<T, GG>;                                                            \
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+        set_smem_limit((const void *)k, smem);    \
         k<<<grid, SC_ROWS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,         \
                                       d.head_dim, G);                                       \
         break;                                                                              \
@@ -96,7 +96,7 @@ cudaError_t launch_t(const xkv_dims &d, const void *lm, const void *q, double *s
         XKV_SCORE_CASE(8)
         default: {
             auto k = k_score<T, 0>;
-            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            set_smem_limit((const void *)k, smem);
             k<<<grid, SC_ROWS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,
                                           d.head_dim, G);
         }

@@ -175,7 +175,7 @@ cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, in
                           int n_recent, int32_t *sel, int n_sel, cudaStream_t s) {
     const int64_t nC = d.ctx_len / d.chunk;
     const size_t smem = (size_t)nC * sizeof(unsigned long long);
-    cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    set_smem_limit((const void *)k_select, smem);
     k_select<<<d.batch * d.n_kv_heads, SEL_THREADS, smem, s>>>(scores, sel, nC, top_k, n_sink,
                                                                n_recent, n_sel);
     return cudaGetLastError();

@@ -25,6 +25,11 @@ SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max
 
 size_t partial_bytes(const xkv_dims &d, int n_split);
 
+// Raises a kernel's dynamic shared-memory limit on the current device only when a call
+// needs more than was set before, so steady-state calls (and stream captures) make no
+// attribute calls.
+cudaError_t set_smem_limit(const void *kernel, size_t bytes);
+
 // ------------------------------------------------------------------ launchers
 // Each returns cudaSuccess or the launch error; arguments were validated by the caller.
 cudaError_t launch_build_landmarks(const xkv_dims &d, const void *Ak, const void *Bkt, void *lm,
