@@ -8,26 +8,29 @@
 // tensor memory); K_hat and V_hat never leave the SM.
 //
 // Work item = (b, g, a run of <= 256 selected rows).  Persistent kernel: one CTA per SM
-// walks the items; roles are warp-specialised:
-//   warp 0      TMA producer.  Per 64-wide rank slice it loads, into one pipeline stage,
-//               the item's A rows (one 8-row x 128-byte box per row group, so any set
-//               of chunks is gathered with no index arithmetic in the MMA path) and the
-//               matching 128 x 64 slice of B_l's group-g columns (B_l is stored
-//               column-major, so that slice is K-major).  Stages are released by the
-//               MMAs' completion (tcgen05.commit).
-//   warp 1      allocates the 512 TMEM columns; one thread issues the MMAs.
-//               Key phase:   D_K[tok][j]  (cols   0..255) += A^K[tok][k] . B^K[j][k]
-//                            (M = 128 tokens per MMA, N = hd = 128)
-//               Value phase: D_V[j][tok]  (cols 256..511) += B^V[j][k] . A^V[tok][k]
-//                            (M = hd = 128, N = tokens rounded up to 16)
-//               so keys come out one token per TMEM lane and values one head-dim per
-//               lane -- each epilogue thread then needs no cross-thread reduction.
-//   warps 2-5   epilogue.  Key epilogue: thread = token, logits z_h = q_h . K_hat (fp32),
-//               then the exact max / sum of the item's rows.  Value epilogue: thread =
-//               output column j, o_h[j] = sum_t p_h[t] V_hat[t][j].  Partials
-//               (m, l, o) go to the workspace; the combine kernel merges items.
+// walks the items.  The pipeline streams 64-wide rank slices: a stage holds the item's
+// rows of A for that slice (256 x 128 B, 128-byte-swizzled 8-row atoms) and the 128 x 64
+// slice of B_l's group-g columns.  Roles (warp-specialised):
+//   warp 0        allocates the 512 TMEM columns; one thread issues the MMAs.
+//                 Key phase:   D_K[tok][j]  (cols   0..255) += A^K[tok][k] . B^K[j][k]
+//                              (M = 128 tokens per MMA, N = hd = 128)
+//                 Value phase: D_V[j][tok]  (cols 256..511) += B^V[j][k] . A^V[tok][k]
+//                              (M = hd = 128, N = tokens rounded up to 16)
+//                 so keys come out one token per TMEM lane and values one head-dim per
+//                 lane: neither epilogue needs a cross-thread reduction.
+//   warps 1-4     TMA producers.  Each 8-row group of the item's A rows is one 8 x 64
+//                 box (a selected chunk is 8 contiguous rows, so a group is one 128-byte
+//                 swizzle atom); the groups are spread over the four warps because the
+//                 per-box cost of the tensor-copy unit, not bandwidth, bounds how fast one
+//                 warp can feed a stage.  Warp 1 also loads the 16 KB B slice.
+//   warps 5-12    epilogue in two groups of four (group 1 takes rows / tokens 128..255).
+//                 Key epilogue: thread = token, logits z_h = q_h . K_hat (fp32); then the
+//                 exact max / sum of the item's rows.  Value epilogue: thread = output
+//                 column j, o_h[j] = sum_t p_h[t] V_hat[t][j]; the groups' halves are
+//                 summed in shared memory.  Partials (m, l, o) go to the workspace and
+//                 the combine kernel merges an item's splits.
 // The key MMAs of item i+1 overlap the value epilogue of item i (separate TMEM columns);
-// the producer runs ahead across items, so the HBM stream does not stop between items.
+// the producers run ahead across items, so the HBM stream does not stop between items.
 //
 // Every wait on an mbarrier is bounded; on expiry the CTA records XKV_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs (again bounded), frees TMEM and
@@ -47,17 +50,18 @@ constexpr int TC_HD = 128;
 constexpr int A_TILE = TC_ROWS * TC_KS * 2;  // 32 KB: 32 row groups of 8 x 128 B
 constexpr int B_TILE = TC_HD * TC_KS * 2;    // 16 KB
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
-constexpr int TC_THREADS = 192;
+constexpr int W_MMA = 0, W_LOAD = 1, N_LOAD = 4, W_EPI = 5, N_EPI = 8;
+constexpr int TC_THREADS = 32 * (W_EPI + N_EPI);       // 416
+constexpr int EPI_THREADS = 32 * N_EPI;                // 256
 constexpr uint32_t SPIN_LIMIT = 1u << 24;
 
 struct TcShared {
-    uint64_t full[TC_STAGES];
-    uint64_t empty[TC_STAGES];
+    uint64_t full[TC_STAGES];     // one arrival + the stage's bytes
+    uint64_t empty[TC_STAGES];    // MMA commit
     uint64_t kdone, vdone, kfree, vfree, idle;
     uint32_t tmem_base;
     int abort;
-    int issued[TC_STAGES];
-    float red[4][16];
+    float red[N_EPI][16];
 };
 
 struct TcParams {
@@ -153,7 +157,7 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 // 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
@@ -170,18 +174,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Barrier of the 128 epilogue threads that also ORs `flag` over them, so that a decision
+// Named barrier 1: the epilogue threads.
+__device__ __forceinline__ void epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+}
+// Epilogue barrier that also ORs `flag` over the epilogue threads, so that a decision
 // taken after a bounded wait is the same in every epilogue thread.
 __device__ __forceinline__ bool epi_bar_any(bool flag) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pin, pout;\n\t"
         "setp.ne.u32 pin, %1, 0;\n\t"
-        "bar.red.or.pred pout, 1, 128, pin;\n\t"
+        "bar.red.or.pred pout, 1, %2, pin;\n\t"
         "selp.u32 %0, 1, 0, pout;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)flag)
+        : "r"((uint32_t)flag), "n"(EPI_THREADS)
         : "memory");
     return r != 0;
 }
@@ -206,6 +213,17 @@ __device__ void abort_cta(TcShared *sh, const TcParams &p) {
     if (p.status) atomicOr(p.status, 1u << XKV_ERR_TIMEOUT);
 }
 
+// One warp-uniform bounded wait: lane 0 polls, every lane gets the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t *b, uint32_t parity, TcShared *sh,
+                                          const TcParams &p, int lane) {
+    int got = 0;
+    if (lane == 0) {
+        got = mbar_wait(b, parity, sh) ? 1 : 0;
+        if (!got) abort_cta(sh, p);
+    }
+    return __shfl_sync(0xffffffffu, got, 0) != 0;
+}
+
 template <int G>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_xkv_tc(const __grid_constant__ CUtensorMap tmAk, const __grid_constant__ CUtensorMap tmAv,
@@ -216,6 +234,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     TcShared *sh = reinterpret_cast<TcShared *>(smem + TC_STAGES * STAGE_BYTES);
     float *qs = reinterpret_cast<float *>(sh + 1);       // [hd][G]
     float *zs = qs + TC_HD * G;                          // [TC_ROWS][G]
+    float *os = zs + TC_ROWS * G;                        // [G][hd]: group 1's value partials
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nC = p.L / p.C;
     const int gpc = p.C / 8;                             // 8-row groups per chunk
@@ -225,7 +244,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int s = 0; s < TC_STAGES; ++s) {
             mbar_init(&sh->full[s], 1);
             mbar_init(&sh->empty[s], 1);
-            sh->issued[s] = 0;
         }
         mbar_init(&sh->kdone, 1);
         mbar_init(&sh->vdone, 1);
@@ -239,7 +257,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prefetch_tmap(&tmBk);
         prefetch_tmap(&tmBv);
     }
-    if (warp == 1) {
+    if (warp == W_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                          su32(&sh->tmem_base))
                      : "memory");
@@ -250,19 +268,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp >= W_LOAD && warp < W_LOAD + N_LOAD) {
+        // ------------------------------------------------------------ TMA producers
+        const int pi = warp - W_LOAD;              // row groups pi, pi + 4, ... of an item
         int it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
             const Item w = decode(p, item);
             const int ng = w.nr / 8;
+            const int gi = pi + N_LOAD * lane;
             int row = 0;
-            if (lane < ng) {
-                const int ci = lane / gpc, sub = lane % gpc;
+            if (gi < ng) {
+                const int ci = gi / gpc, sub = gi % gpc;
                 int64_t c = w.c0 + ci;
                 if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
-                c = min64(max64(c, 0), nC - 1);  // out-of-range indices are clamped
+                c = min64(max64(c, 0), nC - 1);        // out-of-range indices are clamped
                 row = (int)((int64_t)w.b * p.L + c * p.C + sub * 8);
             }
             const int brow = (w.b * p.Hkv + w.g) * TC_HD;
@@ -272,34 +292,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const CUtensorMap *mB = phase == 0 ? &tmBk : &tmBv;
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % TC_STAGES, n = it / TC_STAGES;
-                    int got = 0;
-                    if (lane == 0) {
-                        got = mbar_wait(&sh->empty[s], (n & 1) ^ 1, sh) ? 1 : 0;
-                        if (!got) abort_cta(sh, p);
-                    }
-                    if (!__shfl_sync(0xffffffffu, got, 0)) {  // same decision in every lane
+                    if (!warp_wait(&sh->empty[s], (n & 1) ^ 1, sh, p, lane)) {
                         ok = false;
                         break;
                     }
                     unsigned char *st = smem + s * STAGE_BYTES;
-                    if (lane == 0) {
+                    if (pi == 0 && lane == 0) {
+                        // the stage's one arrival, with every byte its four warps will load
                         mbar_expect_tx(&sh->full[s], (uint32_t)(ng * 1024 + B_TILE));
-                        sh->issued[s] = n + 1;
+                        tma_load_2d(mB, &sh->full[s], st + A_TILE, ks * TC_KS, brow);
                     }
+                    if (gi < ng) tma_load_2d(mA, &sh->full[s], st + gi * 1024, ks * TC_KS, row);
                     __syncwarp();
-                    if (lane < ng) tma_load_2d(mA, &sh->full[s], st + lane * 1024, ks * TC_KS, row);
-                    if (lane == 0) tma_load_2d(mB, &sh->full[s], st + A_TILE, ks * TC_KS, brow);
                 }
             }
         }
-        if (!ok && lane == 0) {  // drain this CTA's copies in flight before exiting
+        if (!ok && pi == 0 && lane == 0) {  // give this CTA's copies time to land
             for (int s = 0; s < TC_STAGES; ++s)
-                if (sh->issued[s] > 0) {
-                    for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
-                        if (mbar_test(&sh->full[s], (sh->issued[s] - 1) & 1)) break;
-                }
+                for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
+                    if (mbar_test(&sh->full[s], 0) || mbar_test(&sh->full[s], 1)) break;
         }
-    } else if (warp == 1) {
+    } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t smem_base = su32(smem);
@@ -357,35 +370,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;          // 0..127
+        const int et = threadIdx.x - 32 * W_EPI;  // 0..255
+        const int ew = warp - W_EPI;              // 0..7
+        const int grp = ew >> 2;                  // rows / tokens [128 grp, 128 grp + 128)
         const int quad = warp & 3;                // TMEM lane quadrant of this warp
-        const int ew = warp - 2;                  // epilogue warp 0..3
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         int ic = 0;
         for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++ic) {
             const Item w = decode(p, item);
             epi_bar();
             const __nv_bfloat16 *qg = p.q + ((size_t)w.b * p.Hq + (size_t)w.g * G) * TC_HD;
-            for (int e = et; e < G * TC_HD; e += 128) {
+            for (int e = et; e < G * TC_HD; e += EPI_THREADS) {
                 const int h = e / TC_HD, j = e % TC_HD;
                 qs[j * G + h] = __bfloat162float(qg[e]) * p.qscale;
             }
-            epi_bar();
             {
                 const bool fail = !mbar_wait(&sh->kdone, ic & 1, sh);
                 if (fail) abort_cta(sh, p);
-                if (epi_bar_any(fail)) break;
+                if (epi_bar_any(fail)) break;     // also publishes qs
             }
             tc_fence_after();
-            // key epilogue: thread = token (quad*32 + lane within each 128-row half)
-            for (int half = 0; half < (w.nr > 128 ? 2 : 1); ++half) {
+            // key epilogue: thread = token grp*128 + quad*32 + lane
+            if (grp * 128 < w.nr) {
                 float acc[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll 1
                 for (int c0 = 0; c0 < TC_HD; c0 += 32) {
                     float v[32];
-                    tmem_ld32(tmem + lane_base + half * 128 + c0, v);
+                    tmem_ld32(tmem + lane_base + grp * 128 + c0, v);
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const float *qd = qs + (c0 + c) * G;
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         for (int h = 0; h < G; ++h) acc[h] = fmaf(v[c], qd[h], acc[h]);
                     }
                 }
-                const int t = half * 128 + quad * 32 + lane;
+                const int t = grp * 128 + quad * 32 + lane;
                 if (t < w.nr) {
 #pragma unroll
                     for (int h = 0; h < G; ++h) zs[t * G + h] = acc[h];
@@ -406,7 +419,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             float m[G], l[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) m[h] = -INFINITY;
-            for (int t = et; t < w.nr; t += 128)
+            for (int t = et; t < w.nr; t += EPI_THREADS)
 #pragma unroll
                 for (int h = 0; h < G; ++h) m[h] = fmaxf(m[h], zs[t * G + h]);
 #pragma unroll
@@ -418,12 +431,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             epi_bar();
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-                m[h] = fmaxf(fmaxf(sh->red[0][h], sh->red[1][h]), fmaxf(sh->red[2][h], sh->red[3][h]));
+            for (int h = 0; h < G; ++h) {
+                float mm = sh->red[0][h];
+#pragma unroll
+                for (int k = 1; k < N_EPI; ++k) mm = fmaxf(mm, sh->red[k][h]);
+                m[h] = mm;
+            }
             epi_bar();
 #pragma unroll
             for (int h = 0; h < G; ++h) l[h] = 0.f;
-            for (int t = et; t < w.nr; t += 128)
+            for (int t = et; t < w.nr; t += EPI_THREADS)
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     const float pv = exp2f(zs[t * G + h] - m[h]);
@@ -436,34 +453,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int off = 16; off; off >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
                 if (lane == 0) sh->red[ew][h] = l[h];
             }
-            epi_bar();
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-                l[h] = (sh->red[0][h] + sh->red[1][h]) + (sh->red[2][h] + sh->red[3][h]);
-            // value epilogue: thread = output column j = quad*32 + lane
             {
                 const bool fail = !mbar_wait(&sh->vdone, ic & 1, sh);
                 if (fail) abort_cta(sh, p);
-                if (epi_bar_any(fail)) break;
+                if (epi_bar_any(fail)) break;     // also publishes p (zs) and red
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float ll = 0.f;
+#pragma unroll
+                for (int k = 0; k < N_EPI; ++k) ll += sh->red[k][h];
+                l[h] = ll;
             }
             tc_fence_after();
+            // value epilogue: thread = output column j; tokens [128 grp, 128 grp + 128)
             float o[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) o[h] = 0.f;
+            const int tend = min(w.nr, grp * 128 + 128);
 #pragma unroll 1
-            for (int c0 = 0; c0 < w.nr; c0 += 32) {
+            for (int c0 = grp * 128; c0 < tend; c0 += 32) {
                 float v[32];
                 tmem_ld32(tmem + lane_base + 256 + c0, v);
-                const int nc = min(32, w.nr - c0);
-                if (nc == 32) {
+                const int nc = tend - c0;      // >= 1; columns past it are not attended
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float *pz = zs + (c0 + c) * G;
-#pragma unroll
-                        for (int h = 0; h < G; ++h) o[h] = fmaf(pz[h], v[c], o[h]);
-                    }
-                } else {
-                    for (int c = 0; c < nc; ++c) {
+                for (int c = 0; c < 32; ++c) {
+                    if (c < nc) {
                         const float *pz = zs + (c0 + c) * G;
 #pragma unroll
                         for (int h = 0; h < G; ++h) o[h] = fmaf(pz[h], v[c], o[h]);
@@ -471,17 +486,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
             }
             tc_fence_before();
+            const int j = quad * 32 + lane;
+            if (grp == 1) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) os[h * TC_HD + j] = o[h];
+            }
             epi_bar();
             if (et == 0) mbar_arrive(&sh->vfree);
-            const int j = quad * 32 + lane;
-            float *dst = p.partials + (((size_t)w.split * p.B + w.b) * p.Hq + (size_t)w.g * G) *
-                                          (TC_HD + 2);
+            if (grp == 0) {
+                float *dst = p.partials + (((size_t)w.split * p.B + w.b) * p.Hq + (size_t)w.g * G) *
+                                              (TC_HD + 2);
+                const bool two = w.nr > 128;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                dst[h * (TC_HD + 2) + 2 + j] = o[h];
-                if (et == 0) {
-                    dst[h * (TC_HD + 2)] = m[h] * 0.6931471805599453f;  // back to natural log
-                    dst[h * (TC_HD + 2) + 1] = l[h];
+                for (int h = 0; h < G; ++h) {
+                    dst[h * (TC_HD + 2) + 2 + j] = two ? o[h] + os[h * TC_HD + j] : o[h];
+                    if (et == 0) {
+                        dst[h * (TC_HD + 2)] = m[h] * 0.6931471805599453f;  // natural log
+                        dst[h * (TC_HD + 2) + 1] = l[h];
+                    }
                 }
             }
         }
@@ -489,7 +511,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1)
+    if (warp == W_MMA)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
                      : "memory");
 }
@@ -537,7 +559,8 @@ int sm_count() {
 template <int G>
 cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s) {
     const size_t smem = 1024 + (size_t)TC_STAGES * STAGE_BYTES + sizeof(TcShared) +
-                        sizeof(float) * ((size_t)TC_HD * G + (size_t)TC_ROWS * G);
+                        sizeof(float) * ((size_t)TC_HD * G + (size_t)TC_ROWS * G +
+                                         (size_t)G * TC_HD);
     auto k = k_xkv_tc<G>;
     cudaError_t e = set_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
