@@ -293,7 +293,7 @@ def cpu_baseline(w, seed, budget_s=20.0):
     from cross_layer_compressed_b200 import synth
     oracle.build()
     if w.mode == "rcla":
-        wl = synth.reduced(w, batch=1, n_layers=1, extra_rows=1)
+        wl = synth.reduced(w, batch=1, n_layers=1, ctx_len=w.ctx_len, extra_rows=1)
         x = synth.np_rcla_inputs(wl, seed, len_rows=w.ctx_len)
         K = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
         V = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()

@@ -5,69 +5,87 @@
 // product exact in fp64 and the sum in ascending d, so the value is reproducible bit for
 // bit on any IEEE-754 machine.  HBM-bound: one pass over the landmarks.
 //
-// One thread per chunk, 128 chunks per CTA.  The CTA's landmark rows are one contiguous
-// block of memory; it is copied into shared memory with coalesced 16-byte loads and an
-// XOR swizzle on the 16-byte column so that the row-per-thread reads are conflict-free.
 #include "xkv_internal.cuh"
 
 namespace xkv {
 namespace {
 
-constexpr int SC_ROWS = 128;
+constexpr int SC_THREADS = 256;
+constexpr int SC_CPT = 2;      // chunks per thread: 2G independent fp64 chains
 constexpr int SC_MAXG = 16;
 
+// One thread scores SC_CPT chunks (rows c, c + 256 of the CTA's block).  Each row is read
+// with 16-byte loads straight from global memory: a warp's 32 rows are one contiguous
+// 8 KB run, and the rest of each 128-byte line is an L1 hit on the next loads.  The
+// query of the group sits in shared memory in fp64, [d][G], so every step of the
+// d-loop is one broadcast read per head pair.
 template <typename T, int G>
-__global__ void __launch_bounds__(SC_ROWS) k_score(const T *__restrict__ lm,
-                                                   const T *__restrict__ q,
-                                                   double *__restrict__ scores, int64_t nC,
-                                                   int Hq, int Hkv, int hd, int g_rt) {
+__global__ void __launch_bounds__(SC_THREADS) k_score(const T *__restrict__ lm,
+                                                      const T *__restrict__ q,
+                                                      double *__restrict__ scores, int64_t nC,
+                                                      int Hq, int Hkv, int hd, int g_rt) {
     constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
-    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NG = G > 0 ? G : SC_MAXG;
+    extern __shared__ __align__(16) double qs[];   // [hd][ng]
     const int ng = G > 0 ? G : g_rt;
     const int b = blockIdx.z, g = blockIdx.y;
-    const int64_t c0 = (int64_t)blockIdx.x * SC_ROWS;
-    const int rows = (int)min64(SC_ROWS, nC - c0);
-    const int vpr = hd / EPV;  // 16-byte vectors per row (8..32)
-
-    double *qs = reinterpret_cast<double *>(smem);               // [hd][ng]
-    uint4 *tile = reinterpret_cast<uint4 *>(smem + (size_t)hd * ng * sizeof(double));
-
     const T *qb = q + ((size_t)b * Hq + (size_t)g * ng) * hd;
-    for (int e = threadIdx.x; e < hd * ng; e += blockDim.x) {
+    for (int e = threadIdx.x; e < hd * ng; e += SC_THREADS) {
         const int h = e / hd, dd = e % hd;
         qs[dd * ng + h] = Elem<T>::f64(qb[(size_t)h * hd + dd]);
     }
-    const uint4 *src = reinterpret_cast<const uint4 *>(lm + (((size_t)b * Hkv + g) * nC + c0) * hd);
-    for (int e = threadIdx.x; e < rows * vpr; e += blockDim.x) {
-        const int r = e / vpr, v = e % vpr;
-        tile[r * vpr + (v ^ (r & 7))] = __ldg(src + e);
-    }
     __syncthreads();
-    const int r = threadIdx.x;
-    if (r >= rows) return;
-
-    double acc[G > 0 ? G : SC_MAXG];
+    const int64_t cbase = (int64_t)blockIdx.x * SC_THREADS * SC_CPT + threadIdx.x;
+    const int vpr = hd / EPV;
+    const uint4 *rows[SC_CPT];
+    bool valid[SC_CPT];
 #pragma unroll
-    for (int h = 0; h < (G > 0 ? G : SC_MAXG); ++h) acc[h] = 0.0;
+    for (int i = 0; i < SC_CPT; ++i) {
+        const int64_t c = cbase + (int64_t)i * SC_THREADS;
+        valid[i] = c < nC;
+        rows[i] = reinterpret_cast<const uint4 *>(lm + (((size_t)b * Hkv + g) * nC +
+                                                        (valid[i] ? c : 0)) * hd);
+    }
+    double acc[SC_CPT][NG];
+#pragma unroll
+    for (int i = 0; i < SC_CPT; ++i)
+#pragma unroll
+        for (int h = 0; h < NG; ++h) acc[i][h] = 0.0;
+#pragma unroll 2
     for (int v = 0; v < vpr; ++v) {
-        const uint4 w = tile[r * vpr + (v ^ (r & 7))];
-        const T *e = reinterpret_cast<const T *>(&w);
+        uint4 w[SC_CPT];
+#pragma unroll
+        for (int i = 0; i < SC_CPT; ++i) w[i] = __ldg(rows[i] + v);
 #pragma unroll
         for (int k = 0; k < EPV; ++k) {
-            const double x = Elem<T>::f64(e[k]);
             const double *qd = qs + (v * EPV + k) * ng;
+            double x[SC_CPT];
+#pragma unroll
+            for (int i = 0; i < SC_CPT; ++i) x[i] = Elem<T>::f64(reinterpret_cast<const T *>(&w[i])[k]);
             if constexpr (G > 0) {
 #pragma unroll
-                for (int h = 0; h < G; ++h) acc[h] = fma(x, qd[h], acc[h]);  // exact product
+                for (int h = 0; h < G; ++h) {
+                    const double qv = qd[h];
+#pragma unroll
+                    for (int i = 0; i < SC_CPT; ++i) acc[i][h] = fma(x[i], qv, acc[i][h]);  // exact product
+                }
             } else {
-                for (int h = 0; h < ng; ++h) acc[h] = fma(x, qd[h], acc[h]);
+                for (int h = 0; h < ng; ++h) {
+                    const double qv = qd[h];
+#pragma unroll
+                    for (int i = 0; i < SC_CPT; ++i) acc[i][h] = fma(x[i], qv, acc[i][h]);
+                }
             }
         }
     }
-    double best = acc[0];
-    for (int h = 1; h < ng; ++h)
-        if (order_key(acc[h]) > order_key(best)) best = acc[h];
-    scores[((size_t)b * Hkv + g) * nC + c0 + r] = best;
+#pragma unroll
+    for (int i = 0; i < SC_CPT; ++i) {
+        if (!valid[i]) continue;
+        double best = acc[i][0];
+        for (int h = 1; h < ng; ++h)
+            if (order_key(acc[i][h]) > order_key(best)) best = acc[i][h];
+        scores[((size_t)b * Hkv + g) * nC + cbase + (int64_t)i * SC_THREADS] = best;
+    }
 }
 
 template <typename T>
@@ -75,17 +93,17 @@ cudaError_t launch_t(const xkv_dims &d, const void *lm, const void *q, double *s
                      cudaStream_t s) {
     const int G = d.n_q_heads / d.n_kv_heads;
     const int64_t nC = d.ctx_len / d.chunk;
-    dim3 grid((unsigned)((nC + SC_ROWS - 1) / SC_ROWS), d.n_kv_heads, d.batch);
-    const size_t smem = (size_t)d.head_dim * G * sizeof(double) +
-                        (size_t)SC_ROWS * d.head_dim * sizeof(T);
+    const int64_t per_cta = (int64_t)SC_THREADS * SC_CPT;
+    dim3 grid((unsigned)((nC + per_cta - 1) / per_cta), d.n_kv_heads, d.batch);
+    const size_t smem = (size_t)d.head_dim * G * sizeof(double);
     const T *l = (const T *)lm;
     const T *qq = (const T *)q;
 #define XKV_SCORE_CASE(GG)                                                                  \
     case GG: {                                                                              \
         auto k = k_score<T, GG>;                                                            \
-        set_smem_limit((const void *)k, smem);    \
-        k<<<grid, SC_ROWS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,         \
-                                      d.head_dim, G);                                       \
+        set_smem_limit((const void *)k, smem);                                              \
+        k<<<grid, SC_THREADS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,      \
+                                         d.head_dim, G);                                    \
         break;                                                                              \
     }
     switch (G) {
@@ -97,8 +115,8 @@ cudaError_t launch_t(const xkv_dims &d, const void *lm, const void *q, double *s
         default: {
             auto k = k_score<T, 0>;
             set_smem_limit((const void *)k, smem);
-            k<<<grid, SC_ROWS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,
-                                          d.head_dim, G);
+            k<<<grid, SC_THREADS, smem, s>>>(l, qq, scores, nC, d.n_q_heads, d.n_kv_heads,
+                                             d.head_dim, G);
         }
     }
 #undef XKV_SCORE_CASE

@@ -2,9 +2,11 @@
 // plus the always-kept sink and recent chunks).
 //
 // One CTA per (sequence, KV head).  Scores become 64-bit keys that order like the
-// doubles (-0 below +0); an 8-pass MSB-first radix select finds the key T of the k-th
-// best candidate and how many candidates equal to T are still needed; those are taken
-// in ascending index (the tie-break), found with a block-wide prefix count.  A second
+// doubles (-0 below +0); an MSB-first radix select over 8-bit digits narrows a key prefix
+// T (under a mask M) holding the k-th best candidate and counts how many candidates with
+// that prefix are still needed.  It stops early once every candidate with the prefix is
+// needed; otherwise after 8 passes T is the k-th key itself and the remaining ties are
+// taken in ascending index (the tie-break), found with a block-wide prefix count.  A second
 // prefix count writes the selected chunks in ascending order.  No floating-point
 // arithmetic is involved, so the result is exactly the oracle's.
 #include "xkv_internal.cuh"
@@ -52,8 +54,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     __shared__ unsigned hist[256];
     __shared__ unsigned warp_tot[SEL_WARPS];
     __shared__ unsigned s_total;
-    __shared__ unsigned long long s_prefix;
+    __shared__ unsigned long long s_prefix, s_mask;
     __shared__ unsigned s_krem;
+    __shared__ int s_done;
 
     const int nC = (int)nC_;
     const int unit = blockIdx.x;
@@ -72,12 +75,14 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
 
     // 0: take no candidate, 1: take every candidate, 2: threshold select
     const int mode = k_eff == 0 ? 0 : (k_eff == n_cand ? 1 : 2);
-    unsigned long long T = 0;
+    unsigned long long T = 0, M = 0;
     unsigned krem = 0;
     if (mode == 2) {
         if (threadIdx.x == 0) {
             s_prefix = 0ull;
+            s_mask = 0ull;
             s_krem = (unsigned)k_eff;
+            s_done = 0;
         }
         unsigned long long mask = 0ull;
         for (int shift = 56; shift >= 0; shift -= 8) {
@@ -112,7 +117,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
                         if (cum + cnt[i] >= need) {
                             const unsigned long long D = (unsigned long long)(255 - (lane * 8 + i));
                             s_prefix = prefix | (D << shift);
+                            s_mask = mask | (255ull << shift);
                             s_krem = need - cum;
+                            s_done = cnt[i] == need - cum;  // the whole bin is needed
                             break;
                         }
                         cum += cnt[i];
@@ -121,8 +128,10 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
             }
             mask |= 255ull << shift;
             __syncthreads();
+            if (s_done) break;                          // uniform: read after the barrier
         }
         T = s_prefix;
+        M = s_mask;
         krem = s_krem;
     }
 
@@ -131,7 +140,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     const int lo = min(nC, (int)threadIdx.x * ipt), hi = min(nC, lo + ipt);
     unsigned eq_local = 0;
     if (mode == 2)
-        for (int c = lo; c < hi; ++c) eq_local += (!forced(c) && keys[c] == T) ? 1u : 0u;
+        for (int c = lo; c < hi; ++c) eq_local += (!forced(c) && (keys[c] & M) == T) ? 1u : 0u;
     unsigned eq_rank = block_exclusive_scan(eq_local, warp_tot, &s_total);
 
     // selection flags for the thread's run, as a bit mask (ipt <= 16)
@@ -145,7 +154,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
         } else if (mode == 1) {
             take = true;
         } else {
-            const unsigned long long k = keys[c];
+            const unsigned long long k = keys[c] & M;
             if (k > T) {
                 take = true;
             } else if (k == T) {

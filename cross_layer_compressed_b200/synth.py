@@ -14,9 +14,11 @@ Workloads (shapes and value recipes follow the cross-layer KV pages):
   B_l (r x d_kv) with entries ~ N(0, 1/r) (variance 1/r).
 * Queries ~ N(0, 1/sqrt(hd)) (variance 1/sqrt(hd)).
 * "Needle" chunks (Llama-3.1-8B 32K workload): per sequence, a few chunk indices
-  outside the sink and recent chunks; every query head h of KV group g gets
-  lambda * sum_n u_n added, u_n the unit direction of needle n's mean key
-  (mean of the chunk's A rows times B_l's group-g columns), lambda = 4 * hd^(1/4).
+  outside the sink and recent chunks; query head j of a KV group g (j = 0..G-1 within
+  the group) gets lambda * u_n added for needle n = j mod n_needles, u_n the unit
+  direction of needle n's mean key (mean of the chunk's A rows times B_l's group-g
+  columns), lambda = 4 * hd^(1/4).  One needle per head keeps the needles from
+  interfering; the group max still reaches each of them.
 * R-CLA leader caches (Stochastic KV Routing page, inference sharing strategy S):
   K, V ~ N(0, 1); 1% of token positions per sequence (shared by leaders and heads)
   have their V row multiplied by 20 (a large value range, as on the VASE page).
@@ -198,17 +200,18 @@ def np_needle_chunks(w: Workload, seed: int, seq: int) -> np.ndarray:
 
 def np_plant_needles(w: Workload, q: np.ndarray, Ak_seq: np.ndarray, Bkt_seq: np.ndarray,
                      needles: np.ndarray, seq: int) -> None:
-    """Add lambda * sum_n u_n to every head of each KV group (in place, one sequence)."""
+    """Add lambda * u_(j mod n) to head j of each KV group (in place, one sequence)."""
     lam = 4.0 * w.head_dim ** 0.25
     C, hd, G = w.chunk, w.head_dim, w.group
     for g in range(w.n_kv_heads):
         Bg = Bkt_seq[g * hd:(g + 1) * hd, :]               # hd x r
-        acc = np.zeros(hd)
+        u = []
         for n in needles:
             abar = Ak_seq[n * C:(n + 1) * C, :].mean(axis=0)
             d = Bg @ abar
-            acc += d / np.linalg.norm(d)
-        q[seq, g * G:(g + 1) * G, :] += lam * acc[None, :]
+            u.append(d / np.linalg.norm(d))
+        for j in range(G):
+            q[seq, g * G + j, :] += lam * u[j % len(u)]
 
 
 def to_storage(x: np.ndarray, dtype: str):
@@ -360,8 +363,9 @@ def torch_queries(w: Workload, seed: int, cache: dict | None = None, device="cud
                 abar = torch.stack([A[n * C:(n + 1) * C].mean(0) for n in nd])   # n x r
                 Bt = cache["Bkt"][l, b].float()                                   # d_kv x r
                 d = (abar @ Bt.T).view(len(nd), w.n_kv_heads, hd)                 # n x H x hd
-                u = (d / d.norm(dim=-1, keepdim=True)).sum(0)                     # H x hd
-                q[:, l, b] += lam * u.repeat_interleave(G, dim=0)[None]
+                u = d / d.norm(dim=-1, keepdim=True)                              # n x H x hd
+                pick = torch.tensor([j % len(nd) for j in range(G)], device=device)
+                q[:, l, b] += lam * u[pick].permute(1, 0, 2).reshape(-1, hd)[None]
     return q.to(dt)
 
 
@@ -380,8 +384,9 @@ def torch_layer_queries(w: Workload, seed: int, layer: int, layer_cache: dict, s
             A = layer_cache["Ak"][b].float()
             abar = torch.stack([A[n * C:(n + 1) * C].mean(0) for n in nd])
             d = (abar @ layer_cache["Bkt"][b].float().T).view(len(nd), w.n_kv_heads, hd)
-            u = (d / d.norm(dim=-1, keepdim=True)).sum(0)
-            q[b] += lam * u.repeat_interleave(G, dim=0)
+            u = d / d.norm(dim=-1, keepdim=True)                                  # n x H x hd
+            pick = torch.tensor([j % len(nd) for j in range(G)], device=device)
+            q[b] += lam * u[pick].permute(1, 0, 2).reshape(-1, hd)
     return q.to(_tdtype(w.dtype))
 
 
