@@ -153,7 +153,8 @@ class XkvStep:
         self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
                                dtype=torch.float32, device=dev)
         self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
-        self.launches_per_step = w.n_layers * (2 if self.dense else 4)
+        # our kernels per layer: score + select (selective only), attention, split combine
+        self.launches_per_step = w.n_layers * ((0 if self.dense else 2) + 2)
         torch.cuda.synchronize()
 
     def resident_bytes(self):
@@ -363,6 +364,28 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def profiled_traffic(workload: str, kernel: str, source: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and workload,
+    or None when there is none or the kernel's source changed since the capture."""
+    import glob
+    import hashlib
+    src = os.path.join(ROOT, "cross_layer_compressed_b200", "csrc", source)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    for path in glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_{workload}*.md")):
+        fields = {}
+        for line in open(path):
+            if ":" in line and not line.startswith(" "):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        key = f"traffic_bytes_per_launch_{workload}"
+        if fields.get("source_sha256_prefix") == sha and key in fields:
+            return float(fields[key])
+    return None
+
+
 # ------------------------------------------------------------------ rank aggregation
 def max_over_ranks(x: float, world: int, device) -> float:
     """Max of a per-rank number over all ranks (the timed region's length)."""
@@ -508,14 +531,8 @@ def main():
     step_bytes = wl.step_bytes(bytes_launch)
     hbm_peak, _, peak_kind = measured_peaks()
     achieved = bytes_launch / (attend_avg_ms / 1e3) / 1e9
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
-    if os.path.exists(tr_path):
-        try:
-            with open(tr_path) as f:
-                traffic = json.load(f).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = profiled_traffic(w.name, "k_xkv_tc" if w.mode != "rcla" else "k_rcla",
+                               "attend_tc.cu" if w.mode != "rcla" else "rcla.cu")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -121,8 +121,17 @@ SplitPlan plan_xkv(const xkv_dims &d, int64_t rows) {
 }
 
 SplitPlan plan_rcla(const xkv_dims &d, int64_t rows) {
+    // at most 4096 / G rows per split (the logits of a split stay in shared memory), in
+    // whole 256-row tiles once a split spans more than one tile
     const int G = d.n_q_heads / d.n_kv_heads;
-    return plan_splits(rows, (int64_t)d.batch * d.n_kv_heads, 256, 16384 / G);
+    int64_t cap = (4096 / G) / 256 * 256;
+    if (cap < 256) cap = 256;
+    SplitPlan p = plan_splits(rows, (int64_t)d.batch * d.n_kv_heads, 256, cap);
+    if (rows > 256) {
+        p.rows_per_split = (p.rows_per_split + 255) / 256 * 256;
+        p.n_split = (int)((rows + p.rows_per_split - 1) / p.rows_per_split);
+    }
+    return p;
 }
 
 }  // namespace
@@ -143,7 +152,8 @@ int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t 
 size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
     if (mode == XKV_MODE_RCLA) {
         if (check_dims(dims, false, "xkv_workspace_bytes") != XKV_OK) return 0;
-        return WS_HEADER + partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
+        return ws_header_bytes(*dims) +
+               partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
     }
     if (check_dims(dims, true, "xkv_workspace_bytes") != XKV_OK) return 0;
     int64_t rows;
@@ -160,7 +170,7 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
         const int n_tc = tc_splits(*dims, (int)(rows / dims->chunk));
         if (n_tc > n) n = n_tc;
     }
-    return WS_HEADER + partial_bytes(*dims, (int)n);
+    return ws_header_bytes(*dims) + partial_bytes(*dims, (int)n);
 }
 
 int64_t xkv_footprint_bytes(const xkv_dims *d, int32_t n_layers, int32_t window,
@@ -260,7 +270,8 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     if (plan.n_split > 65535 || n_tc > 65535)
         return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
     // the same amount xkv_workspace_bytes reports, whichever kernel runs
-    const size_t need = WS_HEADER + partial_bytes(*dims, (int)(n_tc > plan.n_bound ? n_tc : plan.n_bound));
+    const size_t need = ws_header_bytes(*dims) +
+                        partial_bytes(*dims, (int)(n_tc > plan.n_bound ? n_tc : plan.n_bound));
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
@@ -268,11 +279,12 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     if ((st = check_device(who)) != XKV_OK) return st;
     const bool use_tc = n_tc > 0 && attend_tc_supported(*dims) && !getenv("XKV_FORCE_SIMT");
     cudaStream_t s = (cudaStream_t)stream;
+    const size_t hdr = ws_header_bytes(*dims);
     unsigned *status = (unsigned *)ws;
-    float *partials = (float *)((char *)ws + WS_HEADER);
+    float *partials = (float *)((char *)ws + hdr);
     cudaError_t e;
-    int used_split = n_tc;
     if (use_tc) {
+        int used_split = n_tc;
         e = launch_attend_tc(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
                              sel ? n_sel : (int)(dims->ctx_len / dims->chunk), partials, status,
                              &used_split, s);
@@ -321,14 +333,14 @@ xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t
         return fail(XKV_ERR_INVALID_ARG, "%s: need 0 < rows attended <= L_max", who);
     const SplitPlan plan = plan_rcla(*dims, n_rows);
     if (plan.n_split > 65535) return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    const size_t need = WS_HEADER + partial_bytes(*dims, plan.n_split);
+    const size_t need = ws_header_bytes(*dims) + partial_bytes(*dims, plan.n_split);
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
     if (injected(who, &st)) return st;
     if ((st = check_device(who)) != XKV_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    float *partials = (float *)((char *)ws + WS_HEADER);
+    float *partials = (float *)((char *)ws + ws_header_bytes(*dims));
     cudaError_t e = launch_rcla(*dims, slot, L_max, n_rows, update ? len : -1, K_lead, V_lead,
                                 k_new, v_new, q, plan, partials, s);
     if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, nullptr, s);

@@ -35,10 +35,7 @@
 // Every wait on an mbarrier is bounded; on expiry the CTA records XKV_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs (again bounded), frees TMEM and
 // returns; the combine kernel then writes NaN outputs.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "xkv_internal.cuh"
+#include "sm100_util.cuh"
 
 namespace xkv {
 namespace {
@@ -81,31 +78,6 @@ struct TcParams {
 };
 
 // ----------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t su32(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(su32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 // Bounded wait for the phase of parity `parity`; false on timeout or abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared *sh) {
     for (uint32_t i = 0; i < SPIN_LIMIT; ++i) {
@@ -113,17 +85,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared
         if (*(volatile int *)&sh->abort) return false;
     }
     return false;
-}
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
-                                            int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(su32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (leading offset unused for this layout; version 1).
@@ -517,45 +478,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
-    }
-    return fn;
-}
-
-// 2D bf16 tensor map over a row-major [rows][cols] array with a 128-byte-swizzled box of
-// box_rows x 64 elements.
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)TC_KS, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <int G>
 cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s) {
     const size_t smem = 1024 + (size_t)TC_STAGES * STAGE_BYTES + sizeof(TcShared) +
@@ -577,7 +499,7 @@ bool attend_tc_shape_ok(const xkv_dims &d) {
 }
 
 bool attend_tc_supported(const xkv_dims &d) {
-    return attend_tc_shape_ok(d) && encode_fn() != nullptr;
+    return attend_tc_shape_ok(d) && tma_available();
 }
 
 int tc_splits(const xkv_dims &d, int n_sel) {
@@ -591,10 +513,10 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
                              cudaStream_t s) {
     const int64_t d_kv = (int64_t)d.n_kv_heads * d.head_dim;
     CUtensorMap maps[4];
-    if (!make_map(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8) ||
-        !make_map(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8) ||
-        !make_map(&maps[2], Bkt, (uint64_t)d.batch * d_kv, d.rank_k, TC_HD) ||
-        !make_map(&maps[3], Bvt, (uint64_t)d.batch * d_kv, d.rank_v, TC_HD))
+    if (!make_map_bf16_sw128(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8) ||
+        !make_map_bf16_sw128(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8) ||
+        !make_map_bf16_sw128(&maps[2], Bkt, (uint64_t)d.batch * d_kv, d.rank_k, TC_HD) ||
+        !make_map_bf16_sw128(&maps[3], Bvt, (uint64_t)d.batch * d_kv, d.rank_v, TC_HD))
         return cudaErrorInvalidValue;
     TcParams p;
     p.q = (const __nv_bfloat16 *)q;

@@ -62,7 +62,7 @@ void set_last_error(const char *msg);
 
 // Workspace layout: a 256-byte header (word 0: device status bits, 1 << xkv_status) and
 // then the partials.
-constexpr size_t WS_HEADER = 256;
+inline size_t ws_header_bytes(const xkv_dims &) { return 256; }
 
 // ------------------------------------------------------------------ device helpers
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
