@@ -497,6 +497,9 @@ cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_ro
                         int64_t update_row, void *K, void *V, const void *k_new,
                         const void *v_new, const void *q, const SplitPlan &plan,
                         float *partials, cudaStream_t s) {
+    if (rcla_tc_ok(d, slot, L_max, plan))
+        return launch_rcla_tc(d, slot, L_max, n_rows, update_row, K, V, k_new, v_new, q, plan,
+                              partials, s);
     if (rcla_tma_ok(d, slot, L_max, plan)) {
         switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_R(GG)                                                                             \

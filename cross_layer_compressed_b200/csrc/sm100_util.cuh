@@ -130,6 +130,5 @@ bool tma_available();
 // (128 bytes) written to shared memory with the 128-byte swizzle.
 bool make_map_bf16_sw128(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                          uint32_t box_rows);
-int sm_count();
 
 }  // namespace xkv

@@ -46,6 +46,14 @@ cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_ro
                         int64_t update_row, void *K, void *V, const void *k_new,
                         const void *v_new, const void *q, const SplitPlan &plan,
                         float *partials, cudaStream_t s);
+// R-CLA on the tensor cores (bf16, head_dim 128, G in {1, 2, 4, 5, 8}, splits of at most
+// 1024 rows); launch_rcla picks it when rcla_tc_ok holds
+bool rcla_tc_ok(const xkv_dims &d, int slot, int64_t L_max, const SplitPlan &plan);
+cudaError_t launch_rcla_tc(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,
+                           int64_t update_row, void *K, void *V, const void *k_new,
+                           const void *v_new, const void *q, const SplitPlan &plan,
+                           float *partials, cudaStream_t s);
+int sm_count();   // multiprocessors of the current device (cached)
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
                            const unsigned *status, cudaStream_t s);
 // tensor-core path (bf16, head_dim 128, ranks multiple of 64, chunk dividing 256)

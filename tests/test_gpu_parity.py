@@ -105,6 +105,23 @@ def test_scores_bit_exact_heavy_cancellation(xkv, ora):
     assert np.array_equal(scores.cpu().numpy().view(np.uint64), ref.view(np.uint64))
 
 
+@pytest.mark.parametrize("hd,G,nC", [(64, 1, 37), (64, 8, 100), (128, 2, 33), (128, 8, 65),
+                                     (64, 4, 1), (128, 5, 300)])
+def test_scores_bit_exact_shapes(xkv, ora, hd, G, nC):
+    """Every head size and group size of the bf16 scoring kernels, with row counts that
+    end in a partial warp batch."""
+    B, Hkv = 2, 3
+    rng = np.random.default_rng(hd * 1000 + G * 10 + nC)
+    lm_t = torch.tensor(rng.standard_normal((B, Hkv, nC, hd)), dtype=torch.bfloat16)
+    q_t = torch.tensor(rng.standard_normal((B, Hkv * G, hd)), dtype=torch.bfloat16)
+    ref = ora.score_landmarks(lm_t, q_t)
+    d = xkv.dims(B, Hkv * G, Hkv, hd, nC * 8, 8, 16, 16, xkv.XKV_BF16)
+    scores = torch.full((B, Hkv, nC), float("nan"), dtype=torch.float64, device=DEV)
+    xkv.xkv_score_landmarks(d, _dev(lm_t), _dev(q_t), scores)
+    torch.cuda.synchronize()
+    assert np.array_equal(scores.cpu().numpy().view(np.uint64), ref.view(np.uint64))
+
+
 # ------------------------------------------------------------------------ selection
 def _run_select(xkv, scores_np, top_k, n_sink, n_recent, chunk=8):
     B, Hkv, nC = scores_np.shape
@@ -307,6 +324,36 @@ def test_rcla_lengths(xkv, ora, length):
     torch.cuda.synchronize()
     compare_outputs(out.cpu().numpy(), ref, w.dtype)
     assert np.array_equal(K.cpu().view(torch.int16).numpy().view(np.uint16), K_ref)
+
+
+@pytest.mark.parametrize("G,length", [(1, 700), (2, 1300), (5, 2100), (8, 900), (4, 5000)])
+def test_rcla_group_sizes(xkv, ora, G, length):
+    """Every group size of the bf16 kernels; a leader appends, then a follower attends."""
+    w = dataclasses.replace(
+        synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=2, ctx_len=length, n_layers=2,
+                      extra_rows=2, outlier_frac=0.01),
+        n_kv_heads=2, n_q_heads=2 * G, name=f"rcla_g{G}")
+    x = synth.np_rcla_inputs(w, seed=G, len_rows=length)
+    lo = ora.leader_map([0], 2)
+    K_ref = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    V_ref = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                     device=DEV)
+    K, V = _dev(x["K_lead"]), _dev(x["V_lead"])
+    for layer in (0, 1):
+        leader = layer == 0
+        n = length if leader else length + 1
+        kn = x["k_new"][0] if leader else None
+        vn = x["v_new"][0] if leader else None
+        ref = ora.rcla_decode_attend(layer, lo, K_ref, V_ref, n, kn, vn, x["q"][layer])
+        out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+        xkv.rcla_decode_attend(d, layer, lo, K, V, w.L_max, n, _dev(kn) if leader else None,
+                               _dev(vn) if leader else None, _dev(x["q"][layer]), out, ws)
+        torch.cuda.synchronize()
+        compare_outputs(out.cpu().numpy(), ref, w.dtype)
+    assert np.array_equal(K.cpu().view(torch.int16).numpy().view(np.uint16), K_ref)
+    assert np.array_equal(V.cpu().view(torch.int16).numpy().view(np.uint16), V_ref)
 
 
 def test_rcla_outlier_values_are_attended(xkv, ora):
