@@ -21,9 +21,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -63,62 +61,62 @@ def measured_peaks():
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+    """This GPU's SM clock and clock-event (throttle) reasons, polled through NVML (the
+    source nvidia-smi reads) every ~2 ms on a thread while the timed region runs, so a
+    region of a few milliseconds still gets samples."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device_index: int):
         import torch
-        self.proc = None
-        self.path = None
+        self.nvml = None
+        self.handle = None
+        self.thread = None
         try:
+            import pynvml
+            pynvml.nvmlInit()
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nvml = pynvml
         except Exception:
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-            ident = vis.split(",")[device_index] if vis else str(device_index)
-        self.ident = ident
+            self.nvml = None
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while not self.done.is_set():
+            try:
+                self.sm.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                self.mask |= nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                pass
+            self.done.wait(0.002)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.ident, "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        import threading
+        self.sm, self.mask = [], 0
+        if self.nvml is None:
+            return
+        self.done = threading.Event()
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
+        self.done.set()
+        self.thread.join(timeout=5)
+        self.thread = None
+        if not self.sm:
+            return None
         try:
-            self.proc.wait(timeout=5)
+            mx = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+            mx = max(self.sm)
+        reasons = sorted(n for n, bit in self.REASONS.items() if self.mask & bit)
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": mx,
+                "samples": len(self.sm), "reasons": reasons, "source": "nvml"}
 
 
 # ------------------------------------------------------------------------ workloads
@@ -531,8 +529,8 @@ def main():
     step_bytes = wl.step_bytes(bytes_launch)
     hbm_peak, _, peak_kind = measured_peaks()
     achieved = bytes_launch / (attend_avg_ms / 1e3) / 1e9
-    traffic = profiled_traffic(w.name, "k_xkv_tc" if w.mode != "rcla" else "k_rcla",
-                               "attend_tc.cu" if w.mode != "rcla" else "rcla.cu")
+    traffic = profiled_traffic(w.name, "k_xkv_tc" if w.mode != "rcla" else "k_rcla_tc",
+                               "attend_tc.cu" if w.mode != "rcla" else "rcla_tc.cu")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

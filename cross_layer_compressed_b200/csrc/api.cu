@@ -282,7 +282,10 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     const size_t hdr = ws_header_bytes(*dims);
     unsigned *status = (unsigned *)ws;
     float *partials = (float *)((char *)ws + hdr);
-    cudaError_t e;
+    // device-side errors of this call (timeouts, selections out of range) are OR-ed
+    // into the status word; the combine kernel turns a non-zero word into NaN outputs
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return launched(e, who);
     if (use_tc) {
         int used_split = n_tc;
         e = launch_attend_tc(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
@@ -291,8 +294,8 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
         if (e == cudaSuccess) e = launch_combine(*dims, used_split, partials, out, status, s);
     } else {
         e = launch_attend_simt(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel, plan,
-                               partials, s);
-        if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, nullptr, s);
+                               partials, status, s);
+        if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, status, s);
     }
     return launched(e, who);
 }

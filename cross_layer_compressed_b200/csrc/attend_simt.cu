@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(AT_THREADS) k_attend_simt(
     const T *__restrict__ Ak, const T *__restrict__ Av, const T *__restrict__ Bkt,
     const T *__restrict__ Bvt, const T *__restrict__ q, const int32_t *__restrict__ sel,
     int n_sel, int64_t L, int C, int rk, int rv, int Hq, int Hkv, int hd, int64_t rows_total,
-    int64_t rows_per_split, float *__restrict__ partials) {
+    int64_t rows_per_split, float *__restrict__ partials, unsigned *__restrict__ status) {
     extern __shared__ __align__(16) float sm[];
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int B = gridDim.z;
@@ -40,9 +40,12 @@ __global__ void __launch_bounds__(AT_THREADS) k_attend_simt(
     const int d_kv = Hkv * hd;
     const int32_t *su = sel ? sel + ((size_t)b * Hkv + g) * n_sel : nullptr;
     const int64_t nC = L / C;
-    auto token = [&](int64_t i) -> int64_t {  // out-of-range chunk indices are clamped
+    auto token = [&](int64_t i) -> int64_t {
         if (!su) return i;
-        const int64_t c = min64(max64(su[i / C], 0), nC - 1);
+        const int64_t c0 = su[i / C];
+        if ((c0 < 0 || c0 >= nC) && status)   // the call fails (NaN outputs); reads stay
+            atomicOr(status, 1u << XKV_ERR_INVALID_ARG);   // in bounds
+        const int64_t c = min64(max64(c0, 0), nC - 1);
         return c * C + i % C;
     };
     const float scale = 1.0f / sqrtf((float)hd);
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(AT_THREADS) k_attend_simt(
 template <typename T, int G>
 cudaError_t launch_g(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
                      const void *Bvt, const void *q, const int32_t *sel, int n_sel,
-                     const SplitPlan &plan, float *partials, cudaStream_t s) {
+                     const SplitPlan &plan, float *partials, unsigned *status, cudaStream_t s) {
     const int rmax = d.rank_k > d.rank_v ? d.rank_k : d.rank_v;
     const size_t smem = sizeof(float) * ((size_t)AT_RT * rmax + (size_t)AT_RT * d.head_dim +
                                          (size_t)G * d.head_dim + 2 * G +
@@ -155,17 +158,18 @@ cudaError_t launch_g(const xkv_dims &d, const void *Ak, const void *Av, const vo
     k<<<grid, AT_THREADS, smem, s>>>((const T *)Ak, (const T *)Av, (const T *)Bkt,
                                      (const T *)Bvt, (const T *)q, sel, n_sel, d.ctx_len,
                                      d.chunk, d.rank_k, d.rank_v, d.n_q_heads, d.n_kv_heads,
-                                     d.head_dim, rows, plan.rows_per_split, partials);
+                                     d.head_dim, rows, plan.rows_per_split, partials, status);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_t(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
                      const void *Bvt, const void *q, const int32_t *sel, int n_sel,
-                     const SplitPlan &plan, float *partials, cudaStream_t s) {
+                     const SplitPlan &plan, float *partials, unsigned *status, cudaStream_t s) {
     switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_G(GG) \
-    case GG: return launch_g<T, GG>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials, s);
+    case GG:                                                                               \
+        return launch_g<T, GG>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials, status, s);
         XKV_G(1) XKV_G(2) XKV_G(3) XKV_G(4) XKV_G(5) XKV_G(6) XKV_G(7) XKV_G(8)
         XKV_G(9) XKV_G(10) XKV_G(11) XKV_G(12) XKV_G(13) XKV_G(14) XKV_G(15) XKV_G(16)
 #undef XKV_G
@@ -178,10 +182,11 @@ cudaError_t launch_t(const xkv_dims &d, const void *Ak, const void *Av, const vo
 cudaError_t launch_attend_simt(const xkv_dims &d, const void *Ak, const void *Av,
                                const void *Bkt, const void *Bvt, const void *q,
                                const int32_t *sel, int n_sel, const SplitPlan &plan,
-                               float *partials, cudaStream_t s) {
+                               float *partials, unsigned *status, cudaStream_t s) {
     return d.dtype == XKV_F32
-               ? launch_t<float>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials, s)
-               : launch_t<__nv_bfloat16>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials, s);
+               ? launch_t<float>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials, status, s)
+               : launch_t<__nv_bfloat16>(d, Ak, Av, Bkt, Bvt, q, sel, n_sel, plan, partials,
+                                         status, s);
 }
 
 }  // namespace xkv

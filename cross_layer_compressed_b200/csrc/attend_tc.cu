@@ -157,10 +157,14 @@ __device__ __forceinline__ bool epi_bar_any(bool flag) {
 struct Item {
     int b, g, split, c0, nch, nr;
 };
+// Items run split-major: the B * Hkv units of one row range are consecutive, so the KV
+// heads that read the same rows of A (every row, in dense mode) run side by side and
+// share them through L2 instead of each streaming the window from DRAM.
 __device__ __forceinline__ Item decode(const TcParams &p, int item) {
     Item it;
-    const int u = item / p.n_split;
-    it.split = item % p.n_split;
+    const int units = p.B * p.Hkv;
+    const int u = item % units;
+    it.split = item / units;
     it.b = u / p.Hkv;
     it.g = u % p.Hkv;
     it.c0 = it.split * p.chunks_per_item;
@@ -200,7 +204,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int64_t nC = p.L / p.C;
     const int gpc = p.C / 8;                             // 8-row groups per chunk
 
-    if (threadIdx.x == 0 && blockIdx.x == 0 && p.status) *p.status = 0u;
     if (threadIdx.x == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
             mbar_init(&sh->full[s], 1);
@@ -232,20 +235,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (warp >= W_LOAD && warp < W_LOAD + N_LOAD) {
         // ------------------------------------------------------------ TMA producers
         const int pi = warp - W_LOAD;              // row groups pi, pi + 4, ... of an item
+        const int gi = pi + N_LOAD * lane;
+        // global row of this lane's 8-row group in an item (-1: none)
+        auto group_row = [&](const Item &w) -> int64_t {
+            if (gi >= w.nr / 8) return -1;
+            const int ci = gi / gpc, sub = gi % gpc;
+            int64_t c = w.c0 + ci;
+            if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
+            if ((c < 0 || c >= nC) && p.status)             // the call fails: NaN outputs
+                atomicOr(p.status, 1u << XKV_ERR_INVALID_ARG);
+            c = min64(max64(c, 0), nC - 1);                 // and the copy stays in bounds
+            return (int64_t)w.b * p.L + c * p.C + sub * 8;
+        };
         int it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
             const Item w = decode(p, item);
             const int ng = w.nr / 8;
-            const int gi = pi + N_LOAD * lane;
-            int row = 0;
-            if (gi < ng) {
-                const int ci = gi / gpc, sub = gi % gpc;
-                int64_t c = w.c0 + ci;
-                if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
-                c = min64(max64(c, 0), nC - 1);        // out-of-range indices are clamped
-                row = (int)((int64_t)w.b * p.L + c * p.C + sub * 8);
-            }
+            const int64_t grow = group_row(w);
+            const int row = grow < 0 ? 0 : (int)grow;
             const int brow = (w.b * p.Hkv + w.g) * TC_HD;
             for (int phase = 0; phase < 2 && ok; ++phase) {
                 const int nks = (phase == 0 ? p.rk : p.rv) / TC_KS;

@@ -64,9 +64,19 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     auto forced = [&](int c) { return c < n_sink || c >= nC - n_recent; };
 
     unsigned nf_local = 0;
+    bool nan_seen = false;
     for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
-        keys[c] = order_key(s[c]);
+        const double v = s[c];
+        nan_seen |= isnan(v);
+        keys[c] = order_key(v);
         nf_local += forced(c) ? 1u : 0u;
+    }
+    // a NaN score marks a failed scoring launch: the unit selects nothing (-1 entries),
+    // which makes the attention call that consumes it fail with NaN outputs
+    if (__syncthreads_or(nan_seen)) {
+        for (int i = threadIdx.x; i < n_sel; i += SEL_THREADS)
+            sel[(size_t)unit * n_sel + i] = -1;
+        return;
     }
     (void)block_exclusive_scan(nf_local, warp_tot, &s_total);  // also a barrier
     const int n_forced = (int)s_total;

@@ -41,7 +41,7 @@ cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, in
 cudaError_t launch_attend_simt(const xkv_dims &d, const void *Ak, const void *Av,
                                const void *Bkt, const void *Bvt, const void *q,
                                const int32_t *sel, int n_sel, const SplitPlan &plan,
-                               float *partials, cudaStream_t s);
+                               float *partials, unsigned *status, cudaStream_t s);
 cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,
                         int64_t update_row, void *K, void *V, const void *k_new,
                         const void *v_new, const void *q, const SplitPlan &plan,

@@ -100,6 +100,8 @@ xkv_status xkv_build_landmarks(const xkv_dims *dims, const void *Ak_win, const v
  * so the value is reproducible bit for bit; the max orders -0 below +0.  Unscaled
  * (a positive scale does not change the ranking).
  *   lm_layer [B][Hkv][nC][hd], q [B][Hq][hd], scores [B][Hkv][nC] fp64 (output)
+ * A score of NaN marks a failed launch (a bounded device-side wait gave up); scores
+ * are never NaN otherwise.
  */
 xkv_status xkv_score_landmarks(const xkv_dims *dims, const void *lm_layer, const void *q,
                                double *scores, void *stream);
@@ -111,7 +113,8 @@ xkv_status xkv_score_landmarks(const xkv_dims *dims, const void *lm_layer, const
  * written in ascending chunk order.  n_sel = min(top_k, nC - |F|) + |F| chunks per
  * unit; *n_sel_out (host pointer, may be NULL) receives it, computed on the host.
  *   scores [B][Hkv][nC] fp64, sel [B][Hkv][n_sel] int32 (output)
- * nC <= 16384.
+ * nC <= 16384.  A unit whose scores hold a NaN (a failed scoring launch) gets every
+ * entry -1.
  */
 xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t top_k,
                              int32_t n_sink, int32_t n_recent, int32_t *sel,
@@ -132,6 +135,9 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
  *   out [B][Hq][hd] fp32 (output)
  *   ws, ws_bytes: scratch of at least xkv_workspace_bytes(dims, n_sel, mode) bytes
  *   (mode = XKV_MODE_SELECTIVE, or XKV_MODE_DENSE when sel == NULL).
+ * Device-side failures of the call (an entry of sel outside [0, nC), a bounded wait
+ * that gave up) make every output of the call NaN; the first 4 bytes of ws then hold
+ * the OR of (1 << xkv_status) over the failures seen, until the next call.
  */
 xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
                                   const void *Bkt_layer, const void *Bvt_layer, const void *q,

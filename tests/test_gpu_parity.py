@@ -173,6 +173,20 @@ def test_select_distinct_scores_extremes(xkv, ora):
     assert np.array_equal(_run_select(xkv, s, 77, 2, 2), ref)
 
 
+def test_select_nan_scores_mark_the_unit_failed(xkv, ora):
+    """A NaN score (how a failed scoring launch shows) makes its unit select -1
+    everywhere; the other units are selected as usual."""
+    rng = np.random.default_rng(4)
+    s = rng.standard_normal((2, 3, 500))
+    s[1, 2, 123] = np.nan
+    got = _run_select(xkv, s, 20, 1, 4)
+    assert np.all(got[1, 2] == -1)
+    good = np.ones((2, 3), dtype=bool)
+    good[1, 2] = False
+    ref = ora.select_chunks(np.where(np.isnan(s), 0.0, s), 20, 1, 4)
+    assert np.array_equal(got[good], ref[good])
+
+
 # ------------------------------------------------------------ reconstruct + attend
 def _attend(xkv, w, x, sel, dense=False):
     d = xkv.dims_of(w)
@@ -207,6 +221,37 @@ def test_reconstruct_attend_cuda_core_path_bf16(xkv, ora, w, monkeypatch):
     sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
     ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
     compare_outputs(_attend(xkv, w, x, sel), ref, w.dtype)
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["tensor_core", "cuda_core"])
+def test_reconstruct_attend_invalid_selection_fails_loudly(xkv, ora, monkeypatch, force_simt):
+    """A chunk index outside [0, nC) fails the call on the device: every output is NaN
+    and the workspace status word holds the INVALID_ARG bit; the next call is clean."""
+    if force_simt:
+        monkeypatch.setenv("XKV_FORCE_SIMT", "1")
+    w = LLAMA_R
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    d = xkv.dims_of(w)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, sel.shape[2], xkv.XKV_MODE_SELECTIVE),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.zeros((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+    args = [_dev(x["Ak"]), _dev(x["Av"]), _dev(x["Bkt"]), _dev(x["Bvt"]), _dev(x["q"])]
+    for bad in (-1, w.n_chunks):
+        sel_bad = sel.copy()
+        sel_bad[1, 0, 3] = bad
+        xkv.xkv_reconstruct_attend(d, *args, torch.from_numpy(sel_bad).to(DEV), sel.shape[2],
+                                   out, ws)
+        torch.cuda.synchronize()
+        assert torch.isnan(out).all()
+        status = int(ws[:4].cpu().view(torch.int32).item())
+        assert status & (1 << xkv.XKV_ERR_INVALID_ARG)
+    xkv.xkv_reconstruct_attend(d, *args, torch.from_numpy(sel).to(DEV), sel.shape[2], out, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].cpu().view(torch.int32).item()) == 0
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(out.cpu().numpy(), ref, w.dtype)
 
 
 @pytest.mark.parametrize("w", [DENSE_R, TINY], ids=lambda w: w.name)
