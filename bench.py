@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--batch", type=int, default=0,
                    help="override the workload's batch (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--path", choices=["explicit", "reassociated"], default="explicit",
+                   help="xKV attention: explicit reconstruction (the method as the pages "
+                        "state it) or its rank-space reassociation")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call directly instead of replaying a captured step")
@@ -57,6 +60,15 @@ def measured_peaks():
         return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
     except Exception:
         return 6650.0, 1590.0, "fallback"
+
+
+def measured_tflops_sustained():
+    """Dense bf16 rate of a GEMM timed inside a long loop (the power-capped figure)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured sustained"
+    except Exception:
+        return 1400.0, "fallback sustained"
 
 
 # --------------------------------------------------------------------------- clocks
@@ -123,11 +135,12 @@ class ClockSampler:
 class XkvStep:
     """Device-resident xKV workload (selective or dense) and its decode step."""
 
-    def __init__(self, w, seed, dev):
+    def __init__(self, w, seed, dev, path="explicit"):
         import torch
         from cross_layer_compressed_b200 import synth
         from cross_layer_compressed_b200 import xkv
         self.w, self.dev, self.xkv = w, dev, xkv
+        self.path = path
         self.d = xkv.dims_of(w)
         self.cache = synth.torch_xkv_cache(w, seed, device=dev)
         dt = self.cache["Ak"].dtype
@@ -142,8 +155,12 @@ class XkvStep:
         self.qpool = synth.torch_queries(w, seed, self.cache, device=dev)   # [nq][N][B][Hq][hd]
         self.n_sel = 0 if self.dense else w.n_sel
         mode = xkv.XKV_MODE_DENSE if self.dense else xkv.XKV_MODE_SELECTIVE
+        if path == "reassociated":
+            mode = xkv.XKV_MODE_REASSOC
         self.ws = torch.empty(xkv.xkv_workspace_bytes(self.d, self.n_sel, mode),
                               dtype=torch.uint8, device=dev)
+        self.attend = (xkv.xkv_reassociated_attend if path == "reassociated"
+                       else xkv.xkv_reconstruct_attend)
         self.scores = torch.empty((w.batch, w.n_kv_heads, max(w.n_chunks, 1)),
                                   dtype=torch.float64, device=dev)
         self.sel = torch.empty((w.n_layers, w.batch, w.n_kv_heads, max(self.n_sel, 1)),
@@ -151,8 +168,10 @@ class XkvStep:
         self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
                                dtype=torch.float32, device=dev)
         self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
-        # our kernels per layer: score + select (selective only), attention, split combine
-        self.launches_per_step = w.n_layers * ((0 if self.dense else 2) + 2)
+        # our kernels per layer: score + select (selective only), then attention + split
+        # combine (explicit) or q~ + attention + merge + projection (reassociated)
+        self.launches_per_step = w.n_layers * ((0 if self.dense else 2) +
+                                               (4 if path == "reassociated" else 2))
         torch.cuda.synchronize()
 
     def resident_bytes(self):
@@ -171,10 +190,9 @@ class XkvStep:
                 xkv.xkv_select_chunks(d, self.scores, w.top_k, w.n_sink, w.n_recent, self.sel[l])
             if attend_events is not None:
                 attend_events[l][0].record()
-            xkv.xkv_reconstruct_attend(d, self.cache["Ak"][win], self.cache["Av"][win],
-                                       self.cache["Bkt"][l], self.cache["Bvt"][l], qq[l],
-                                       None if self.dense else self.sel[l], self.n_sel,
-                                       self.out[l], self.ws)
+            self.attend(d, self.cache["Ak"][win], self.cache["Av"][win], self.cache["Bkt"][l],
+                        self.cache["Bvt"][l], qq[l], None if self.dense else self.sel[l],
+                        self.n_sel, self.out[l], self.ws)
             if attend_events is not None:
                 attend_events[l][1].record()
 
@@ -202,6 +220,14 @@ class XkvStep:
                           + (0 if self.dense else w.batch * w.n_kv_heads * self.n_sel * 4))
                 per_launch.append(nbytes)
         return float(np.mean(per_launch))
+
+    def attend_flops(self):
+        """Tensor-core flops of one explicit attention launch: the two reconstruction
+        GEMMs over the attended rows plus q.K_hat and p.V_hat (dense mode: every row)."""
+        w = self.w
+        rows = w.ctx_len if self.dense else w.n_sel * w.chunk
+        return (2.0 * w.batch * w.n_kv_heads * rows * w.head_dim * (w.rank_k + w.rank_v)
+                + 4.0 * w.batch * w.n_q_heads * rows * w.head_dim)
 
     def step_bytes(self, attend_bytes_per_launch):
         w = self.w
@@ -428,7 +454,8 @@ def main():
                                 device_id=dev)
     from cross_layer_compressed_b200 import build
     build.build()
-    wl = RclaStep(w, args.seed + rank, dev) if w.mode == "rcla" else XkvStep(w, args.seed + rank, dev)
+    wl = RclaStep(w, args.seed + rank, dev) if w.mode == "rcla" else \
+        XkvStep(w, args.seed + rank, dev, args.path)
     nq = wl.qpool.shape[0]
     stream = torch.cuda.current_stream(dev)
 
@@ -532,6 +559,26 @@ def main():
     traffic = profiled_traffic(w.name, "k_xkv_tc" if w.mode != "rcla" else "k_rcla_tc",
                                "attend_tc.cu" if w.mode != "rcla" else "rcla_tc.cu")
 
+    kernel = ("rcla_decode_attend" if w.mode == "rcla" else
+              "reassociated_attend" if args.path == "reassociated" else "reconstruct_attend")
+    roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm_peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+                "frac_of_8tbs": achieved / 8000.0, "traffic": traffic,
+                "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms}
+    if w.mode == "dense" and args.path == "explicit":
+        # explicit dense reconstruction is bound by the tensor cores, not by HBM: report
+        # the GEMM rate against the sustained bf16 peak (the kernel runs inside a long
+        # step), keeping the HBM figures alongside
+        tf_peak, tf_kind = measured_tflops_sustained()
+        tflops = wl.attend_flops() / (attend_avg_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": kernel, "achieved": tflops, "peak": tf_peak,
+                    "peak_kind": tf_kind, "unit": "TFLOP/s", "frac": tflops / tf_peak,
+                    "traffic": traffic, "flops_per_launch": wl.attend_flops(),
+                    "hbm_gbs": achieved, "hbm_frac": achieved / hbm_peak,
+                    "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms}
+    if args.path == "reassociated":
+        roofline["traffic"] = None            # the committed captures are of the explicit kernel
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -545,7 +592,7 @@ def main():
                      f"{step_bytes / 1e9:.2f} GB algorithmic per step"}
         if w.mode != "rcla":
             cfg.update({"window": w.window, "ranks_k_v": [w.rank_k, w.rank_v], "chunk": w.chunk,
-                        "mode": w.mode})
+                        "mode": w.mode, "path": args.path})
         if w.mode == "sr":
             cfg.update({"top_k": w.top_k, "n_sink": w.n_sink, "n_recent": w.n_recent,
                         "n_sel": w.n_sel})
@@ -558,11 +605,7 @@ def main():
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": cfg,
             "step_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-            "roofline": {"bound": "hbm", "kernel": "reconstruct_attend" if w.mode != "rcla"
-                         else "rcla_decode_attend", "achieved": achieved, "peak": hbm_peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
-                         "frac_of_8tbs": achieved / 8000.0, "traffic": traffic,
-                         "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms},
+            "roofline": roofline,
             "gpu_launches": wl.launches_per_step * args.steps,
             "cuda_graph": use_graph,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,

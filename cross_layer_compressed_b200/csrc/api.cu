@@ -156,6 +156,12 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
                partial_bytes(*dims, (int)plan_rcla(*dims, dims->ctx_len).n_bound);
     }
     if (check_dims(dims, true, "xkv_workspace_bytes") != XKV_OK) return 0;
+    if (mode == XKV_MODE_REASSOC) {
+        const int64_t nC = dims->ctx_len / dims->chunk;
+        if (n_sel < 0 || n_sel > nC || !attend_ra_shape_ok(*dims)) return 0;
+        const int n = ra_splits(*dims, n_sel ? n_sel : (int)nC);
+        return ws_header_bytes(*dims) + ra_scratch_bytes(*dims, n);
+    }
     int64_t rows;
     if (mode == XKV_MODE_SELECTIVE) {
         if (n_sel <= 0 || (int64_t)n_sel > dims->ctx_len / dims->chunk) return 0;
@@ -297,6 +303,45 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
                                partials, status, s);
         if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, status, s);
     }
+    return launched(e, who);
+}
+
+xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
+                                   const void *Bkt_layer, const void *Bvt_layer, const void *q,
+                                   const int32_t *sel, int32_t n_sel, float *out, void *ws,
+                                   size_t ws_bytes, void *stream) {
+    const char *who = "xkv_reassociated_attend";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!Ak_win || !Av_win || !Bkt_layer || !Bvt_layer || !q || !out || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(Ak_win) || !aligned16(Av_win) || !aligned16(Bkt_layer) ||
+        !aligned16(Bvt_layer) || !aligned16(q) || !aligned16(out) || !aligned16(ws) ||
+        (sel && !aligned16(sel)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (sel && (n_sel <= 0 || n_sel > nC))
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_sel must be in [1, n_chunks]", who);
+    if (!attend_ra_shape_ok(*dims))
+        return fail(XKV_ERR_UNSUPPORTED, "%s: needs bf16, head_dim 128, G in {1,2,4,5,8}, "
+                    "ranks multiple of 128 (r_K <= 1024, or 512 when G > 4; r_V <= 1024) and "
+                    "a chunk dividing 256", who);
+    const int ns = sel ? n_sel : (int)nC;
+    if (ra_splits(*dims, ns) > 65535 || (int64_t)dims->batch * dims->ctx_len >= (1ll << 31))
+        return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    const size_t need = ws_header_bytes(*dims) + ra_scratch_bytes(*dims, ra_splits(*dims, ns));
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    if (!tma_available()) return fail(XKV_ERR_UNSUPPORTED, "%s: no tensor-map encoder", who);
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned *status = (unsigned *)ws;
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess)
+        e = launch_attend_ra(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, ns,
+                             (char *)ws + ws_header_bytes(*dims), status, out, s);
     return launched(e, who);
 }
 

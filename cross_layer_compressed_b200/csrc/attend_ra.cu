@@ -1,0 +1,674 @@
+// Reassociated xKV attention: the same result as reconstruct-then-attend, computed in
+// the rank space of the window's basis.
+//
+// xKV page, section 2.2 (K_hat = A^K B^K_l, V_hat = A^V B^V_l) and section 2.3 (attend
+// over the rows T of the selected chunks).  By associativity,
+//   z_h[t] = q_h . (A^K[t] B^K_g) / sqrt(hd) = A^K[t] . q~_h / sqrt(hd),  q~_h = B^K_g q_h
+//   o_h    = sum_t p_h[t] (A^V[t] B^V_g)    = (sum_t p_h[t] A^V[t]) B^V_g = u_h B^V_g,
+// so a decode step reads the selected rows of A once, does r-deep dot products instead of
+// r x hd GEMMs, and touches B_l only twice per (sequence, KV head): once for q~ and once
+// in the final projection.  Four kernels:
+//   k_qtilde     q~_h = B^K_g q_h (fp32), stored as two bf16 terms (hi + lo, ~16 bits)
+//   k_xkv_ra     per work item (b, g, <= 256 selected rows), on tcgen05:
+//                  logits  D_z[t][n] = A^K[t][:] . Q~[n][:]    (M = 128 rows, N = 8)
+//                  output  D_u[r][n] = sum_t A^V[t][r] P[n][t] (M = 128 columns of A^V,
+//                          read MN-major straight from the staged rows; N = 8)
+//                with P holding each probability as two bf16 terms, as in the R-CLA kernel;
+//                partials (m, l, u) in rank space
+//   k_merge_ra   merges an item's splits in rank space (U_h, L_h)
+//   k_project_ra o_h = U_h B^V_g / L_h
+// Warp roles of k_xkv_ra: warp 0 TMEM + MMA issue, warps 1-4 TMA producers (every 8-row
+// group of an item is one 128-byte-swizzled box per 64 columns, a stage holds 128
+// columns of the item's rows), warps 5-8 epilogue.  Every mbarrier wait is bounded; on
+// expiry the CTA sets XKV_ERR_TIMEOUT in the workspace status word, drains its copies
+// and MMAs (bounded), frees TMEM and returns, and the combine writes NaN outputs.
+#include "sm100_util.cuh"
+
+namespace xkv {
+namespace {
+
+constexpr int RA_ROWS = 256;                    // rows per work item
+constexpr int RA_HALF = RA_ROWS * 128;          // one 64-column half of a stage: 32 KB
+constexpr int RA_STAGE = 2 * RA_HALF;           // 128 columns of the item's rows: 64 KB
+constexpr int RA_STAGES = 3;
+constexpr int RA_QBUF = 16 * 1024;              // Q~: NO rows x r_K, K-major
+constexpr int RA_PBUF = 8 * 1024;               // P: NO rows x 256 tokens, K-major
+constexpr uint32_t TM_Z = 0;                    // logits: 2 token halves x NO columns
+constexpr uint32_t TM_U = 64;                   // output: r_V / 128 blocks x NO columns
+// Q~ and P rows: the hi terms of the G heads, then the lo terms, padded to the MMA's N
+template <int G> struct RaCfg {
+    static constexpr int NO = (2 * G + 7) / 8 * 8;
+    static constexpr int ATOM = NO / 8 * 1024;          // bytes per 64-wide K atom
+    static constexpr int MAXR = RA_QBUF / ATOM * 64;    // r_K the Q~ buffer holds
+};
+constexpr int W_MMA = 0, W_LOAD = 1, N_LOAD = 4, W_EPI = 5, N_EPI = 4;
+constexpr int RA_THREADS = 32 * (W_EPI + N_EPI);  // 288
+constexpr int EPI_THREADS = 32 * N_EPI;           // 128
+constexpr uint32_t RA_SPIN = 1u << 24;
+
+struct RaShared {
+    uint64_t full[RA_STAGES], empty[RA_STAGES];
+    uint64_t q_full, z_full, p_full, o_full, idle;
+    uint32_t tmem_base;
+    int abort;
+    float red[N_EPI][8];
+};
+
+struct RaParams {
+    const __nv_bfloat16 *qt_hi, *qt_lo;   // [B][Hq][r_K]
+    const int32_t *sel;                   // [B][Hkv][n_sel] or null (dense)
+    float *partials;                      // [n_split][B][Hq][r_V + 2]
+    unsigned *status;
+    int64_t L;
+    int n_sel, C, rk, rv, Hq, Hkv, B;
+    int chunks_per_item, n_split, n_items;
+    float qscale;                         // log2(e) / sqrt(hd)
+};
+
+struct RaItem {
+    int b, g, split, c0, nch, nr;
+};
+// split-major, as in the explicit kernel: the heads that read the same rows run together
+__device__ __forceinline__ RaItem ra_decode(const RaParams &p, int item) {
+    RaItem it;
+    const int units = p.B * p.Hkv;
+    const int u = item % units;
+    it.split = item / units;
+    it.b = u / p.Hkv;
+    it.g = u % p.Hkv;
+    it.c0 = it.split * p.chunks_per_item;
+    it.nch = min(p.chunks_per_item, p.n_sel - it.c0);
+    it.nr = it.nch * p.C;
+    return it;
+}
+
+// byte offset of element (n, k) of a K-major 128-byte-swizzled operand: 64-wide K atoms
+// `atom` bytes apart, 8-row groups 1 KB apart inside an atom
+__device__ __forceinline__ uint32_t kmaj_off(int n, int k, int atom) {
+    const int kin = k & 63;
+    return (uint32_t)((k >> 6) * atom + (n >> 3) * 1024 + (n & 7) * 128 +
+                      ((((kin >> 3) ^ (n & 7)) & 7) << 4) + (kin & 7) * 2);
+}
+__device__ __forceinline__ void ra_epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+}
+__device__ __forceinline__ bool ra_epi_bar_any(bool flag) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pin, pout;\n\t"
+        "setp.ne.u32 pin, %1, 0;\n\t"
+        "bar.red.or.pred pout, 1, %2, pin;\n\t"
+        "selp.u32 %0, 1, 0, pout;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag), "n"(EPI_THREADS)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool ra_wait(uint64_t *b, uint32_t parity, RaShared *sh,
+                                        const RaParams &p) {
+    if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
+    if (!*(volatile int *)&sh->abort) {
+        *(volatile int *)&sh->abort = 1;
+        if (p.status) atomicOr(p.status, 1u << XKV_ERR_TIMEOUT);
+    }
+    return false;
+}
+__device__ __forceinline__ bool ra_warp_wait(uint64_t *b, uint32_t parity, RaShared *sh,
+                                             const RaParams &p, int lane) {
+    int got = 0;
+    if (lane == 0) got = ra_wait(b, parity, sh, p) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, got, 0) != 0;
+}
+
+template <int G>
+__global__ void __launch_bounds__(RA_THREADS, 1)
+    k_xkv_ra(const __grid_constant__ CUtensorMap tmAk, const __grid_constant__ CUtensorMap tmAv,
+             const RaParams p) {
+    using Cfg = RaCfg<G>;
+    constexpr int NO = Cfg::NO, ATOM = Cfg::ATOM;
+    static_assert(Cfg::MAXR >= 512, "the Q~ buffer holds a rank-512 query at least");
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    unsigned char *qbuf = smem + RA_STAGES * RA_STAGE;
+    unsigned char *pbuf = qbuf + RA_QBUF;
+    RaShared *sh = reinterpret_cast<RaShared *>(pbuf + RA_PBUF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nC = p.L / p.C;
+    const int gpc = p.C / 8;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RA_STAGES; ++s) {
+            mbar_init(&sh->full[s], 1);
+            mbar_init(&sh->empty[s], 1);
+        }
+        mbar_init(&sh->q_full, 1);
+        mbar_init(&sh->z_full, 1);
+        mbar_init(&sh->p_full, 1);
+        mbar_init(&sh->o_full, 1);
+        mbar_init(&sh->idle, 1);
+        sh->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_tmap(&tmAk);
+        prefetch_tmap(&tmAv);
+    }
+    if (warp == W_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                         su32(&sh->tmem_base))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tcgen05_before();
+    __syncthreads();
+    tcgen05_after();
+    const uint32_t tmem = sh->tmem_base;
+
+    if (warp >= W_LOAD && warp < W_LOAD + N_LOAD) {
+        // ------------------------------------------------------------ TMA producers
+        const int pi = warp - W_LOAD;
+        const int gi = pi + N_LOAD * lane;         // this lane's 8-row group of an item
+        int it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+            const RaItem w = ra_decode(p, item);
+            const int ng = w.nr / 8;
+            // an odd group count is padded to a whole 16-row MMA step with a copy of group
+            // 0: finite rows whose weight is zero
+            const int ngl = (ng + 1) & ~1;
+            int row = 0;
+            if (gi < ngl) {
+                const int gg = gi < ng ? gi : 0;
+                const int ci = gg / gpc, sub = gg % gpc;
+                int64_t c = w.c0 + ci;
+                if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
+                if (gi < ng && (c < 0 || c >= nC) && p.status)   // the call fails: NaN outputs
+                    atomicOr(p.status, 1u << XKV_ERR_INVALID_ARG);
+                c = min64(max64(c, 0), nC - 1);                   // the copy stays in bounds
+                row = (int)((int64_t)w.b * p.L + c * p.C + sub * 8);
+            }
+            for (int phase = 0; phase < 2 && ok; ++phase) {
+                const int nst = (phase == 0 ? p.rk : p.rv) / 128;
+                const CUtensorMap *m = phase == 0 ? &tmAk : &tmAv;
+                for (int st = 0; st < nst; ++st, ++it) {
+                    const int s = it % RA_STAGES, n = it / RA_STAGES;
+                    if (!ra_warp_wait(&sh->empty[s], (n & 1) ^ 1, sh, p, lane)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char *dst = smem + s * RA_STAGE;
+                    if (pi == 0 && lane == 0)
+                        mbar_expect_tx(&sh->full[s], (uint32_t)(ngl * 2 * 1024));
+                    __syncwarp();
+                    if (gi < ngl) {
+                        tma_load_2d(m, &sh->full[s], dst + gi * 1024, st * 128, row);
+                        tma_load_2d(m, &sh->full[s], dst + RA_HALF + gi * 1024, st * 128 + 64,
+                                    row);
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        if (!ok && pi == 0 && lane == 0) {
+            for (int s = 0; s < RA_STAGES; ++s)
+                for (uint32_t i = 0; i < RA_SPIN; ++i)
+                    if (mbar_test(&sh->full[s], 0) || mbar_test(&sh->full[s], 1)) break;
+        }
+    } else if (warp == W_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sbase = su32(smem), qb = su32(qbuf), pb = su32(pbuf);
+            constexpr uint32_t idZ = idesc_f16(128, NO, false, false);
+            constexpr uint32_t idU = idesc_f16(128, NO, true, false);  // A = A^V^T, MN-major
+            int it = 0, ic = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++ic) {
+                const RaItem w = ra_decode(p, item);
+                const int nk16 = ((w.nr / 8 + 1) & ~1) / 2;   // 16-row K steps of the output
+                if (!ra_wait(&sh->q_full, ic & 1, sh, p)) { ok = false; break; }
+                tcgen05_after();
+                const int nsk = p.rk / 128;
+                for (int st = 0; st < nsk && ok; ++st, ++it) {
+                    const int s = it % RA_STAGES, n = it / RA_STAGES;
+                    if (!ra_wait(&sh->full[s], n & 1, sh, p)) { ok = false; break; }
+                    tcgen05_after();
+                    const uint32_t a0 = sbase + s * RA_STAGE;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {      // 16 columns of the stage per step
+                        const uint32_t aoff = (kk >> 2) * RA_HALF + (kk & 3) * 32;
+                        const int k0 = st * 128 + kk * 16;
+                        const uint64_t bq = smem_desc_sw128(qb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32,
+                                                            16, 1024);
+                        const uint32_t acc = (st | kk) ? 1u : 0u;
+                        umma_f16(tmem + TM_Z, smem_desc_sw128(a0 + aoff, 16, 1024), bq, idZ, acc);
+                        if (w.nr > 128)
+                            umma_f16(tmem + TM_Z + NO, smem_desc_sw128(a0 + aoff + 16384, 16, 1024),
+                                     bq, idZ, acc);
+                    }
+                    umma_arrive(&sh->empty[s]);
+                }
+                if (!ok) break;
+                umma_arrive(&sh->z_full);
+                if (!ra_wait(&sh->p_full, ic & 1, sh, p)) { ok = false; break; }
+                tcgen05_after();
+                const int nsv = p.rv / 128;
+                for (int st = 0; st < nsv && ok; ++st, ++it) {
+                    const int s = it % RA_STAGES, n = it / RA_STAGES;
+                    if (!ra_wait(&sh->full[s], n & 1, sh, p)) { ok = false; break; }
+                    tcgen05_after();
+                    const uint32_t a0 = sbase + s * RA_STAGE;
+                    for (int kt = 0; kt < nk16; ++kt) {
+                        const int k0 = kt * 16;
+                        umma_f16(tmem + TM_U + st * NO, smem_desc_sw128(a0 + kt * 2048, RA_HALF, 1024),
+                                 smem_desc_sw128(pb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32, 16, 1024),
+                                 idU, kt ? 1u : 0u);
+                    }
+                    umma_arrive(&sh->empty[s]);
+                }
+                if (!ok) break;
+                umma_arrive(&sh->o_full);
+            }
+            umma_arrive(&sh->idle);
+            for (uint32_t i = 0; i < RA_SPIN; ++i)
+                if (mbar_test(&sh->idle, 0)) break;
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 32 * W_EPI;   // 0..127
+        const int ew = warp - W_EPI;
+        const int quad = warp & 3;
+        const int lrow = quad * 32 + lane;          // TMEM lane: token of a half / column
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        for (int i = et; i < (RA_QBUF + RA_PBUF) / 16; i += EPI_THREADS)   // pad rows = 0
+            reinterpret_cast<uint4 *>(qbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+        ra_epi_bar();
+        auto write_q = [&](int item) {             // Q~ rows: hi of the G heads, then lo
+            const RaItem w = ra_decode(p, item);
+            const size_t base = ((size_t)w.b * p.Hq + (size_t)w.g * G) * p.rk;
+            const int per = p.rk / 8;               // 16-byte pieces per row
+            for (int e = et; e < 2 * G * per; e += EPI_THREADS) {
+                const int n = e / per, c16 = e % per;
+                const __nv_bfloat16 *src = (n < G ? p.qt_hi : p.qt_lo) + base +
+                                           (size_t)(n % G) * p.rk + c16 * 8;
+                const int k = c16 * 8;
+                *reinterpret_cast<uint4 *>(qbuf + kmaj_off(n, k, ATOM)) =
+                    *reinterpret_cast<const uint4 *>(src);
+            }
+        };
+        if (blockIdx.x < p.n_items) write_q(blockIdx.x);
+        fence_async_smem();
+        ra_epi_bar();
+        if (et == 0) mbar_arrive(&sh->q_full);
+        int ic = 0, item = blockIdx.x;
+        for (; item < p.n_items; item += gridDim.x, ++ic) {
+            const RaItem w = ra_decode(p, item);
+            {
+                const bool fail = !ra_wait(&sh->z_full, ic & 1, sh, p);
+                if (ra_epi_bar_any(fail)) break;
+            }
+            tcgen05_after();
+            float z[2][G];
+#pragma unroll
+            for (int th = 0; th < 2; ++th) {
+                if (th * 128 < w.nr) {
+                    float v[NO];
+                    if constexpr (NO == 8)
+                        tmem_load8(tmem + lane_base + TM_Z + th * NO, v);
+                    else
+                        tmem_load16(tmem + lane_base + TM_Z + th * NO, v);
+                    const bool valid = th * 128 + lrow < w.nr;
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        z[th][h] = valid ? (v[h] + v[G + h]) * p.qscale : -INFINITY;
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) z[th][h] = -INFINITY;
+                }
+            }
+            float m[G], l[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                m[h] = fmaxf(z[0][h], z[1][h]);
+#pragma unroll
+                for (int off = 16; off; off >>= 1)
+                    m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
+                if (lane == 0) sh->red[ew][h] = m[h];
+            }
+            ra_epi_bar();
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                m[h] = fmaxf(fmaxf(sh->red[0][h], sh->red[1][h]),
+                             fmaxf(sh->red[2][h], sh->red[3][h]));
+                l[h] = 0.f;
+            }
+            ra_epi_bar();
+#pragma unroll
+            for (int th = 0; th < 2; ++th) {
+                const int k = th * 128 + lrow;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float pv = exp2f(z[th][h] - m[h]);   // 0 past the item's rows
+                    l[h] += pv;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(pv - __bfloat162float(hi));
+                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + kmaj_off(h, k, ATOM)) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + kmaj_off(G + h, k, ATOM)) = lo;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+                if (lane == 0) sh->red[ew][h] = l[h];
+            }
+            fence_async_smem();
+            tcgen05_before();
+            ra_epi_bar();
+            if (et == 0) mbar_arrive(&sh->p_full);
+            // the logit MMAs of this item are done: Q~ takes the next item's rows while
+            // the value MMAs of this one run
+            if (item + (int)gridDim.x < p.n_items) {
+                write_q(item + gridDim.x);
+                fence_async_smem();
+                ra_epi_bar();
+                if (et == 0) mbar_arrive(&sh->q_full);
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+                l[h] = (sh->red[0][h] + sh->red[1][h]) + (sh->red[2][h] + sh->red[3][h]);
+            {
+                const bool fail = !ra_wait(&sh->o_full, ic & 1, sh, p);
+                if (ra_epi_bar_any(fail)) break;
+            }
+            tcgen05_after();
+            float *dst = p.partials + (((size_t)w.split * p.B + w.b) * p.Hq + (size_t)w.g * G) *
+                                          (p.rv + 2);
+            for (int sb = 0; sb < p.rv / 128; ++sb) {
+                float v[NO];
+                if constexpr (NO == 8)
+                    tmem_load8(tmem + lane_base + TM_U + sb * NO, v);
+                else
+                    tmem_load16(tmem + lane_base + TM_U + sb * NO, v);
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    dst[(size_t)h * (p.rv + 2) + 2 + sb * 128 + lrow] = v[h] + v[G + h];
+            }
+            tcgen05_before();
+            if (et == 0) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    dst[(size_t)h * (p.rv + 2)] = m[h] * 0.6931471805599453f;   // natural log
+                    dst[(size_t)h * (p.rv + 2) + 1] = l[h];
+                }
+            }
+            ra_epi_bar();                            // red is rewritten by the next item
+        }
+    }
+    tcgen05_before();
+    __syncthreads();
+    tcgen05_after();
+    if (warp == W_MMA)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+                     : "memory");
+}
+
+// q~[b][h][i] = sum_j q[b][h][j] B^K[b][i][g*hd + j]  (Bkt row g*hd + j holds column j of
+// the group's slice), fp32, then split into the bf16 nearest and the bf16 of the rest.
+// One CTA per (b, g, 128 columns i): warp w takes rows j = w, w + 8, ... of the slice, each
+// lane 4 columns (one 8-byte load per row, all rows' loads in flight), and the 8 warps'
+// sums meet in shared memory.
+constexpr int QT_COLS = 128;
+template <int G>
+__global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict__ q,
+                                                const __nv_bfloat16 *__restrict__ Bkt,
+                                                __nv_bfloat16 *__restrict__ qt_hi,
+                                                __nv_bfloat16 *__restrict__ qt_lo, int Hq,
+                                                int Hkv, int hd, int rk) {
+    __shared__ float qs[G * 128];                  // [G][hd]
+    __shared__ float red[8][G][QT_COLS];
+    const int g = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * QT_COLS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < G * hd; e += blockDim.x)
+        qs[e] = __bfloat162float(q[((size_t)b * Hq + (size_t)g * G) * hd + e]);
+    __syncthreads();
+    const __nv_bfloat16 *Bg = Bkt + ((size_t)b * Hkv * hd + (size_t)g * hd) * rk + i0 + lane * 4;
+    float acc[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[h][c] = 0.f;
+#pragma unroll 4
+    for (int j = warp; j < hd; j += 8) {
+        const uint2 w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
+        const float bv[4] = {bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y)};
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float qv = qs[h * hd + j];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(qv, bv[c], acc[h][c]);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[warp][h][lane * 4 + c] = acc[h][c];
+    __syncthreads();
+    for (int e = threadIdx.x; e < G * QT_COLS; e += blockDim.x) {
+        const int h = e / QT_COLS, c = e % QT_COLS;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += red[w][h][c];
+        const size_t o = ((size_t)b * Hq + (size_t)g * G + h) * rk + i0 + c;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        qt_hi[o] = hi;
+        qt_lo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
+}
+
+// Merge an item's splits in rank space:
+//   M = max_s m_s,  U_h[r] = sum_s e^{m_s - M} u_s[r],  L_h = sum_s e^{m_s - M} l_s.
+// One CTA per (b, h, 256 columns of r): warp w takes the splits s = w, w + 8, ..., each
+// lane 8 columns (coalesced 128-byte rows), so every thread keeps 8 independent loads in
+// flight; the 8 warps' sums meet in shared memory.
+constexpr int MG_THREADS = 256;
+constexpr int MG_COLS = 256;
+__global__ void __launch_bounds__(MG_THREADS) k_merge_ra(const float *__restrict__ partials,
+                                                         float *__restrict__ U,
+                                                         float *__restrict__ Lsum, int n_split,
+                                                         int BH, int rv,
+                                                         const unsigned *__restrict__ status) {
+    __shared__ float red[MG_THREADS / 32][MG_COLS];
+    __shared__ float s_m[MG_THREADS / 32];
+    __shared__ float s_l[MG_THREADS / 32];
+    const int bh = blockIdx.x, r0 = blockIdx.y * MG_COLS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int NW = MG_THREADS / 32;
+    if (status && *(volatile const unsigned *)status) return;   // outputs become NaN anyway
+    const size_t stride = (size_t)BH * (rv + 2);
+    const float *p = partials + (size_t)bh * (rv + 2);
+    float M = -INFINITY;
+    for (int sp = threadIdx.x; sp < n_split; sp += MG_THREADS) M = fmaxf(M, p[sp * stride]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) s_m[warp] = M;
+    __syncthreads();
+    M = s_m[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) M = fmaxf(M, s_m[w]);
+    float acc[8], l = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    for (int sp = warp; sp < n_split; sp += NW) {
+        const float *ps = p + sp * stride;
+        const float wgt = expf(ps[0] - M);
+        l = fmaf(wgt, ps[1], l);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int r = r0 + lane + 32 * k;
+            if (r < rv) acc[k] = fmaf(wgt, ps[2 + r], acc[k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) red[warp][lane + 32 * k] = acc[k];
+    if (lane == 0) s_l[warp] = l;
+    __syncthreads();
+    const int r = r0 + threadIdx.x;
+    if (threadIdx.x < MG_COLS && r < rv) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) sum += red[w][threadIdx.x];
+        U[(size_t)bh * rv + r] = sum;
+    }
+    if (blockIdx.y == 0 && threadIdx.x == 0) {
+        float ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) ls += s_l[w];
+        Lsum[bh] = ls;
+    }
+}
+
+// out[b][h][j] = (U_h . B^V[:, g*hd + j]) / L_h.  One CTA per (b, g, 32 columns j): each
+// warp takes 4 rows j of Bvt, so the group's B^V slice is read once for its G heads with
+// 16-byte loads, several per thread in flight.  Within a warp, lane = 8 * jr + c: row j = j0 + 4 * warp + jr, 16-byte pieces c, c + 8, ... of
+// the row; the 8 lanes of a row then sum their partial dot products with shuffles.
+constexpr int PJ_ROWS = 32;
+template <int G>
+__global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
+                                                    const float *__restrict__ Lsum,
+                                                    const __nv_bfloat16 *__restrict__ Bvt,
+                                                    float *__restrict__ out, int Hq, int Hkv,
+                                                    int hd, int rv,
+                                                    const unsigned *__restrict__ status) {
+    extern __shared__ float Us[];                 // [G][rv]
+    const int g = blockIdx.x, b = blockIdx.y, j0 = blockIdx.z * PJ_ROWS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t bh0 = (size_t)b * Hq + (size_t)g * G;
+    if (status && *(volatile const unsigned *)status) {   // a device-side failure: NaN out
+        for (int e = threadIdx.x; e < G * PJ_ROWS; e += blockDim.x)
+            out[(bh0 + e / PJ_ROWS) * hd + j0 + e % PJ_ROWS] = __int_as_float(0x7fc00000);
+        return;
+    }
+    for (int e = threadIdx.x; e < G * rv; e += blockDim.x) Us[e] = U[bh0 * rv + e];
+    __syncthreads();
+    const int jr = lane >> 3, c = lane & 7;
+    const int j = j0 + warp * 4 + jr;
+    const __nv_bfloat16 *row = Bvt + ((size_t)b * Hkv * hd + (size_t)g * hd + j) * rv;
+    float acc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 4
+    for (int pc = c; pc < rv / 8; pc += 8) {       // 16-byte piece pc: columns 8 pc .. 8 pc + 7
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(row + pc * 8);
+        const float bv[8] = {bf16lo(w4.x), bf16hi(w4.x), bf16lo(w4.y), bf16hi(w4.y),
+                             bf16lo(w4.z), bf16hi(w4.z), bf16lo(w4.w), bf16hi(w4.w)};
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[h] = fmaf(Us[h * rv + pc * 8 + k], bv[k], acc[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int off = 4; off; off >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], off);
+        if (c == 0) out[(bh0 + h) * hd + j] = acc[h] / Lsum[bh0 + h];
+    }
+}
+
+template <int G>
+cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams &p,
+                     const void *q, const void *Bkt, const void *Bvt, __nv_bfloat16 *qt_hi,
+                     __nv_bfloat16 *qt_lo, float *U, float *Lsum, float *out, cudaStream_t s) {
+    k_qtilde<G><<<dim3(d.n_kv_heads, d.batch, d.rank_k / QT_COLS), 256, 0, s>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
+        d.n_kv_heads, d.head_dim, d.rank_k);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = 1024 + (size_t)RA_STAGES * RA_STAGE + RA_QBUF + RA_PBUF + sizeof(RaShared);
+    auto k = k_xkv_ra<G>;
+    if ((e = set_smem_limit((const void *)k, smem)) != cudaSuccess) return e;
+    const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
+    k<<<grid, RA_THREADS, smem, s>>>(maps[0], maps[1], p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int BH = d.batch * d.n_q_heads;
+    k_merge_ra<<<dim3(BH, (d.rank_v + MG_COLS - 1) / MG_COLS), MG_THREADS, 0, s>>>(
+        p.partials, U, Lsum, p.n_split, BH, d.rank_v, p.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t psmem = sizeof(float) * (size_t)G * d.rank_v;
+    auto kp = k_project_ra<G>;
+    if ((e = set_smem_limit((const void *)kp, psmem)) != cudaSuccess) return e;
+    kp<<<dim3(d.n_kv_heads, d.batch, d.head_dim / PJ_ROWS), 256, psmem, s>>>(
+        U, Lsum, (const __nv_bfloat16 *)Bvt, out,
+                                                       d.n_q_heads, d.n_kv_heads, d.head_dim,
+                                                       d.rank_v, p.status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attend_ra_shape_ok(const xkv_dims &d) {
+    const int G = d.n_q_heads / d.n_kv_heads;
+    const int max_rk = G > 4 ? RaCfg<8>::MAXR : RaCfg<4>::MAXR;
+    return d.dtype == XKV_BF16 && d.head_dim == 128 &&
+           (G == 1 || G == 2 || G == 4 || G == 5 || G == 8) && d.rank_k % 128 == 0 &&
+           d.rank_v % 128 == 0 && d.rank_k <= max_rk && d.rank_v <= 1024 &&
+           RA_ROWS % d.chunk == 0;
+}
+
+int ra_splits(const xkv_dims &d, int n_sel) {
+    const int64_t rows = (int64_t)n_sel * d.chunk;
+    return (int)((rows + RA_ROWS - 1) / RA_ROWS);
+}
+
+// scratch: q~ hi and lo [B][Hq][r_K] bf16, U [B][Hq][r_V] and L [B][Hq] fp32, then the
+// partials [n_split][B][Hq][r_V + 2] fp32; each region starts on a 256-byte boundary
+static size_t al256(size_t n) { return (n + 255) / 256 * 256; }
+size_t ra_scratch_bytes(const xkv_dims &d, int n_split) {
+    const size_t bh = (size_t)d.batch * d.n_q_heads;
+    return 2 * al256(bh * d.rank_k * sizeof(__nv_bfloat16)) + al256(bh * d.rank_v * sizeof(float)) +
+           al256(bh * sizeof(float)) + (size_t)n_split * bh * (d.rank_v + 2) * sizeof(float);
+}
+
+cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
+                             const void *Bvt, const void *q, const int32_t *sel, int n_sel,
+                             void *scratch, unsigned *status, float *out, cudaStream_t s) {
+    CUtensorMap maps[2];
+    if (!make_map_bf16_sw128(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8) ||
+        !make_map_bf16_sw128(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8))
+        return cudaErrorInvalidValue;
+    const size_t bh = (size_t)d.batch * d.n_q_heads;
+    const size_t qt_al = al256(bh * d.rank_k * sizeof(__nv_bfloat16));
+    const size_t u_al = al256(bh * d.rank_v * sizeof(float));
+    char *sc = (char *)scratch;
+    __nv_bfloat16 *qt_hi = (__nv_bfloat16 *)sc;
+    __nv_bfloat16 *qt_lo = (__nv_bfloat16 *)(sc + qt_al);
+    float *U = (float *)(sc + 2 * qt_al);
+    float *Lsum = (float *)(sc + 2 * qt_al + u_al);
+    RaParams p;
+    p.qt_hi = qt_hi;
+    p.qt_lo = qt_lo;
+    p.sel = sel;
+    p.partials = (float *)(sc + 2 * qt_al + u_al + al256(bh * sizeof(float)));
+    p.status = status;
+    p.L = d.ctx_len;
+    p.n_sel = n_sel;
+    p.C = d.chunk;
+    p.rk = d.rank_k;
+    p.rv = d.rank_v;
+    p.Hq = d.n_q_heads;
+    p.Hkv = d.n_kv_heads;
+    p.B = d.batch;
+    const int n_split = ra_splits(d, n_sel);
+    p.chunks_per_item = (n_sel + n_split - 1) / n_split;
+    p.n_split = (n_sel + p.chunks_per_item - 1) / p.chunks_per_item;
+    p.n_items = d.batch * d.n_kv_heads * p.n_split;
+    p.qscale = 1.4426950408889634f / sqrtf((float)d.head_dim);
+    switch (d.n_q_heads / d.n_kv_heads) {
+        case 1: return launch_g<1>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        case 2: return launch_g<2>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        case 4: return launch_g<4>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        case 5: return launch_g<5>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        case 8: return launch_g<8>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace xkv

@@ -30,14 +30,14 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned *w
     if (lane == 31) warp_tot[warp] = inc;
     __syncthreads();
     if (warp == 0) {
-        unsigned w = warp_tot[lane];
+        unsigned w = lane < SEL_WARPS ? warp_tot[lane] : 0u;
         unsigned winc = w;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             unsigned t = __shfl_up_sync(0xffffffffu, winc, off);
             if (lane >= off) winc += t;
         }
-        warp_tot[lane] = winc - w;  // exclusive warp offsets
+        if (lane < SEL_WARPS) warp_tot[lane] = winc - w;  // exclusive warp offsets
         if (lane == 31) *total = winc;
     }
     __syncthreads();
@@ -83,8 +83,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     const int n_cand = nC - n_forced;
     const int k_eff = min(top_k, n_cand);
 
-    // 0: take no candidate, 1: take every candidate, 2: threshold select
-    const int mode = k_eff == 0 ? 0 : (k_eff == n_cand ? 1 : 2);
+    // 0: take no candidate, 1: take every candidate, 2: threshold select with ties ranked
+    // by index, 3: threshold select whose whole last bin is taken
+    int mode = k_eff == 0 ? 0 : (k_eff == n_cand ? 1 : 2);
     unsigned long long T = 0, M = 0;
     unsigned krem = 0;
     if (mode == 2) {
@@ -143,15 +144,18 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
         T = s_prefix;
         M = s_mask;
         krem = s_krem;
+        if (s_done) mode = 3;   // every candidate with the prefix is taken: no tie ranks
     }
 
     // Each thread owns a contiguous run of chunks so prefix counts follow chunk order.
     const int ipt = (nC + SEL_THREADS - 1) / SEL_THREADS;
     const int lo = min(nC, (int)threadIdx.x * ipt), hi = min(nC, lo + ipt);
-    unsigned eq_local = 0;
-    if (mode == 2)
+    unsigned eq_rank = 0;
+    if (mode == 2) {                            // uniform: only when ties must be ranked
+        unsigned eq_local = 0;
         for (int c = lo; c < hi; ++c) eq_local += (!forced(c) && (keys[c] & M) == T) ? 1u : 0u;
-    unsigned eq_rank = block_exclusive_scan(eq_local, warp_tot, &s_total);
+        eq_rank = block_exclusive_scan(eq_local, warp_tot, &s_total);
+    }
 
     // selection flags for the thread's run, as a bit mask (ipt <= 16)
     unsigned flags = 0, n_local = 0;
@@ -163,6 +167,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
             take = false;
         } else if (mode == 1) {
             take = true;
+        } else if (mode == 3) {
+            take = (keys[c] & M) >= T;
         } else {
             const unsigned long long k = keys[c] & M;
             if (k > T) {

@@ -54,6 +54,14 @@ cudaError_t launch_rcla_tc(const xkv_dims &d, int slot, int64_t L_max, int64_t n
                            const void *v_new, const void *q, const SplitPlan &plan,
                            float *partials, cudaStream_t s);
 int sm_count();   // multiprocessors of the current device (cached)
+bool tma_available();   // the driver exposes the tensor-map encoder
+// reassociated attention (rank-space logits and values, tcgen05)
+bool attend_ra_shape_ok(const xkv_dims &d);
+int ra_splits(const xkv_dims &d, int n_sel);
+size_t ra_scratch_bytes(const xkv_dims &d, int n_split);
+cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
+                             const void *Bvt, const void *q, const int32_t *sel, int n_sel,
+                             void *scratch, unsigned *status, float *out, cudaStream_t s);
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
                            const unsigned *status, cudaStream_t s);
 // tensor-core path (bf16, head_dim 128, ranks multiple of 64, chunk dividing 256)

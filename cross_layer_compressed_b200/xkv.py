@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libxkv.so")
 XKV_OK, XKV_ERR_INVALID_ARG, XKV_ERR_UNSUPPORTED, XKV_ERR_CUDA, XKV_ERR_TIMEOUT, \
     XKV_ERR_INTERNAL = range(6)
 XKV_F32, XKV_BF16 = 0, 1
-XKV_MODE_SELECTIVE, XKV_MODE_DENSE, XKV_MODE_RCLA = 0, 1, 2
+XKV_MODE_SELECTIVE, XKV_MODE_DENSE, XKV_MODE_RCLA, XKV_MODE_REASSOC = 0, 1, 2, 3
 
 STATUS_NAMES = {0: "XKV_OK", 1: "XKV_ERR_INVALID_ARG", 2: "XKV_ERR_UNSUPPORTED",
                 3: "XKV_ERR_CUDA", 4: "XKV_ERR_TIMEOUT", 5: "XKV_ERR_INTERNAL"}
@@ -52,6 +52,8 @@ _sigs = {
                                ctypes.c_int),
     "rcla_decode_attend": ([_D, _i32, _vp, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                             _sz, _vp], ctypes.c_int),
+    "xkv_reassociated_attend": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp],
+                                ctypes.c_int),
     "xkv_reconstruct_attend_noalloc": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp],
                                        ctypes.c_int),
     "xkv_workspace_bytes": ([_D, _i32, _i32], _sz),
@@ -145,6 +147,19 @@ def xkv_reconstruct_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
                                      _ptr(Bkt_layer), _ptr(Bvt_layer), _ptr(q), _ptr(sel),
                                      int(n_sel), _ptr(out), _ptr(ws), int(ws_bytes),
                                      _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_reassociated_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel,
+                            out, ws, ws_bytes=None, stream=None, check=True):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = _lib.xkv_reassociated_attend(ctypes.byref(d), _ptr(Ak_win), _ptr(Av_win),
+                                      _ptr(Bkt_layer), _ptr(Bvt_layer), _ptr(q), _ptr(sel),
+                                      int(n_sel), _ptr(out), _ptr(ws), int(ws_bytes),
+                                      _stream(stream))
     if check:
         _check(st)
     return st

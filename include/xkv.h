@@ -54,7 +54,12 @@ typedef enum {
 
 typedef enum { XKV_F32 = 0, XKV_BF16 = 1 } xkv_dtype;
 
-typedef enum { XKV_MODE_SELECTIVE = 0, XKV_MODE_DENSE = 1, XKV_MODE_RCLA = 2 } xkv_mode;
+typedef enum {
+    XKV_MODE_SELECTIVE = 0,
+    XKV_MODE_DENSE = 1,
+    XKV_MODE_RCLA = 2,
+    XKV_MODE_REASSOC = 3  /* xkv_reassociated_attend; n_sel = 0 for every row (dense) */
+} xkv_mode;
 
 /*
  * Shapes of one decode call.
@@ -186,6 +191,25 @@ xkv_status xkv_reconstruct_attend_noalloc(const xkv_dims *dims, const void *Ak_w
                                           const void *Bvt_layer, const void *q,
                                           const int32_t *sel, int32_t n_sel, float *out,
                                           void *stream);
+
+/*
+ * The same decode attention as xkv_reconstruct_attend, computed by associativity in the
+ * rank space of the window's basis [xKV 2.2: K_hat = A^K B^K_l, V_hat = A^V B^V_l]:
+ *   q~_h = B^K_g q_h,   z_h[t] = A^K[b][t] . q~_h / sqrt(hd),   p_h = softmax_t(z_h),
+ *   u_h = sum_t p_h[t] A^V[b][t],   out[b][h] = u_h B^V_g
+ * The pages describe the explicit form; this reassociation is exact in real arithmetic
+ * and is not printed there.  It reads the same rows of A once and does r-deep dot
+ * products instead of r x hd GEMMs, so dense reconstruction becomes bound by HBM rather
+ * than by the tensor cores.  Arguments, layouts and failure signalling as for
+ * xkv_reconstruct_attend; ws holds at least
+ * xkv_workspace_bytes(dims, sel ? n_sel : 0, XKV_MODE_REASSOC) bytes.  Runs for bf16,
+ * head_dim 128, G in {1, 2, 4, 5, 8}, ranks multiples of 128 up to 1024 (r_K up to 512
+ * when G > 4) and chunks dividing 256; other shapes return XKV_ERR_UNSUPPORTED.
+ */
+xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
+                                   const void *Bkt_layer, const void *Bvt_layer, const void *q,
+                                   const int32_t *sel, int32_t n_sel, float *out, void *ws,
+                                   size_t ws_bytes, void *stream);
 
 /* Scratch bytes the attention calls need (the split-K partial results). 0 on bad dims. */
 size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode);

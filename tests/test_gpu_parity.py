@@ -303,6 +303,68 @@ def test_pipeline_end_to_end_tiny(xkv, ora):
         compare_outputs(out.cpu().numpy(), o_ref, w.dtype)
 
 
+# ------------------------------------------------------- reassociated (rank space)
+def _reassoc(xkv, w, x, sel):
+    d = xkv.dims_of(w)
+    n_sel = 0 if sel is None else sel.shape[2]
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, n_sel, xkv.XKV_MODE_REASSOC), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), device=DEV)
+    xkv.xkv_reassociated_attend(d, _dev(x["Ak"]), _dev(x["Av"]), _dev(x["Bkt"]), _dev(x["Bvt"]),
+                                _dev(x["q"]), None if sel is None else torch.from_numpy(sel).to(DEV),
+                                n_sel, out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), ws
+
+
+@pytest.mark.parametrize("w", [LLAMA_R, QWEN14_R], ids=lambda w: w.name)
+def test_reassociated_attend_selective(xkv, ora, w):
+    """Rank-space attention equals the oracle's explicit reconstruct-then-attend."""
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(_reassoc(xkv, w, x, sel)[0], ref, w.dtype)
+
+
+def test_reassociated_attend_dense(xkv, ora):
+    w = DENSE_R
+    x = _layer_inputs(w)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], None, w.chunk)
+    compare_outputs(_reassoc(xkv, w, x, None)[0], ref, w.dtype)
+
+
+@pytest.mark.parametrize("n_sel", [1, 3, 17, 33, 128])
+def test_reassociated_selection_sizes(xkv, ora, n_sel):
+    """Items of one chunk, odd 8-row group counts (padded MMA steps), several splits."""
+    w = LLAMA_R
+    x = _layer_inputs(w)
+    rng = np.random.default_rng(n_sel)
+    sel = np.sort(np.stack([np.stack([rng.choice(w.n_chunks, n_sel, replace=False)
+                                      for _ in range(w.n_kv_heads)]) for _ in range(w.batch)]),
+                  axis=2).astype(np.int32)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(_reassoc(xkv, w, x, sel)[0], ref, w.dtype)
+
+
+def test_reassociated_invalid_selection_and_shapes(xkv, ora):
+    w = LLAMA_R
+    x = _layer_inputs(w)
+    sel = np.tile(np.arange(10, dtype=np.int32), (w.batch, w.n_kv_heads, 1))
+    sel[0, 1, 4] = w.n_chunks                       # out of range: NaN outputs, status bit
+    out, ws = _reassoc(xkv, w, x, sel)
+    assert np.isnan(out).all()
+    assert int(ws[:4].cpu().view(torch.int32).item()) & (1 << xkv.XKV_ERR_INVALID_ARG)
+    # fp32 is outside the rank-space kernel: refused before any launch
+    d = xkv.dims_of(TINY)
+    assert xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_REASSOC) == 0
+    dummy = torch.zeros(64, dtype=torch.float32, device=DEV)
+    with pytest.raises(xkv.XkvError) as e:
+        xkv.xkv_reassociated_attend(d, dummy, dummy, dummy, dummy, dummy, None, 0, dummy,
+                                    torch.zeros(1 << 20, dtype=torch.uint8, device=DEV))
+    assert e.value.status == xkv.XKV_ERR_UNSUPPORTED
+
+
 # ----------------------------------------------------------------------------- R-CLA
 RCLA_R = synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=2, ctx_len=1500, n_layers=8,
                        extra_rows=8)
