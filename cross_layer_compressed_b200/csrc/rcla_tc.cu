@@ -181,9 +181,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         if (lane == 0) {
             int it = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-                const RtItem w = rt_decode(p, item);
+            // ring order K(0), K(1), V(0), K(2), V(1), ...: the next item's logits are
+            // computed while the epilogue turns this item's logits into probabilities
+            for (int step = 0; ok; ++step) {
+                const int kitem = blockIdx.x + step * gridDim.x;
+                const int vitem = kitem - gridDim.x;
+                if (vitem >= p.n_items) break;
                 for (int ph = 0; ph < 2 && ok; ++ph) {
+                    const int item = ph == 0 ? kitem : vitem;
+                    if (item < (int)blockIdx.x || item >= p.n_items) continue;
+                    const RtItem w = rt_decode(p, item);
                     const CUtensorMap *m = ph == 0 ? &tmK : &tmV;
                     for (int t = 0; t < w.tiles; ++t, ++it) {
                         const int s = it % S, n = it / S;
@@ -208,66 +215,76 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         const uint32_t sbase = su32(smem), pb = su32(pbuf), qb = su32(qbuf);
         constexpr uint32_t idZ = idesc_f16(128, RT_NZ, false, false);
         constexpr uint32_t idO = idesc_f16(128, NO, true, false);    // A = V^T, MN-major
-        int it = 0, ic = 0;
+        int it = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++ic) {
-            const RtItem w = rt_decode(p, item);
-            const int64_t new_local = p.update_row >= 0 ? p.update_row - w.r0 : -1;
-            const size_t new_off = ((size_t)w.b * p.Hkv + w.g) * RT_HD;
-            // logits
-            if (!rt_warp_wait(&sh->q_full, ic & 1, sh, lane)) { ok = false; break; }
-            tcgen05_after();
-            for (int t = 0; t < w.tiles && ok; ++t, ++it) {
-                const int s = it % S, n = it / S;
-                if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
+        for (int step = 0; ok; ++step) {
+            const int kitem = blockIdx.x + step * gridDim.x;
+            const int vitem = kitem - gridDim.x;
+            if (vitem >= p.n_items) break;
+            if (kitem < p.n_items) {
+                // logits of item kitem (its ordinal among this CTA's items is `step`)
+                const RtItem w = rt_decode(p, kitem);
+                const int64_t new_local = p.update_row >= 0 ? p.update_row - w.r0 : -1;
+                const size_t new_off = ((size_t)w.b * p.Hkv + w.g) * RT_HD;
+                if (!rt_warp_wait(&sh->q_full, step & 1, sh, lane)) { ok = false; break; }
                 tcgen05_after();
-                const int64_t nl = new_local - (int64_t)t * RT_ROWS;
-                if (nl >= 0 && nl < RT_ROWS)
-                    patch_tile(smem + s * RT_TILE, (int)nl, p.k_new + new_off, 0, 0, lane);
-                if (lane == 0) {
-                    const uint32_t a0 = sbase + s * RT_TILE;
+                for (int t = 0; t < w.tiles && ok; ++t, ++it) {
+                    const int s = it % S, n = it / S;
+                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
+                    tcgen05_after();
+                    const int64_t nl = new_local - (int64_t)t * RT_ROWS;
+                    if (nl >= 0 && nl < RT_ROWS)
+                        patch_tile(smem + s * RT_TILE, (int)nl, p.k_new + new_off, 0, 0, lane);
+                    if (lane == 0) {
+                        const uint32_t a0 = sbase + s * RT_TILE;
 #pragma unroll
-                    for (int kk = 0; kk < RT_HD / 16; ++kk)
-                        umma_f16(tmem + TM_Z + t * RT_NZ,
-                                 smem_desc_sw128(a0 + (kk >> 2) * RT_HALF + (kk & 3) * 32, 16, 1024),
-                                 smem_desc_sw128(qb + (kk >> 2) * 1024 + (kk & 3) * 32, 16, 1024),
-                                 idZ, kk ? 1u : 0u);
-                    umma_arrive(&sh->empty[s]);
-                }
-                __syncwarp();
-            }
-            if (!ok) break;
-            if (lane == 0) umma_arrive(&sh->z_full);
-            // output
-            if (!rt_warp_wait(&sh->p_full, ic & 1, sh, lane)) { ok = false; break; }
-            tcgen05_after();
-            for (int t = 0; t < w.tiles && ok; ++t, ++it) {
-                const int s = it % S, n = it / S;
-                if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
-                tcgen05_after();
-                const int rows = min(RT_ROWS, w.nr - t * RT_ROWS);
-                const int nks = (rows + 15) / 16;
-                const int64_t nl = new_local - (int64_t)t * RT_ROWS;
-                const bool has_new = nl >= 0 && nl < RT_ROWS;
-                if (has_new || rows < nks * 16)
-                    patch_tile(smem + s * RT_TILE, has_new ? (int)nl : -1, p.v_new + new_off,
-                               rows, nks * 16, lane);
-                if (lane == 0) {
-                    const uint32_t a0 = sbase + s * RT_TILE;
-                    for (int kk = 0; kk < nks; ++kk) {
-                        const int k0 = t * RT_ROWS + kk * 16;
-                        umma_f16(tmem + TM_O,
-                                 smem_desc_sw128(a0 + kk * 2048, RT_HALF, 1024),
-                                 smem_desc_sw128(pb + (k0 >> 6) * PATOM + ((k0 & 63) >> 4) * 32,
-                                                 16, 1024),
-                                 idO, (t | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < RT_HD / 16; ++kk)
+                            umma_f16(tmem + TM_Z + t * RT_NZ,
+                                     smem_desc_sw128(a0 + (kk >> 2) * RT_HALF + (kk & 3) * 32, 16, 1024),
+                                     smem_desc_sw128(qb + (kk >> 2) * 1024 + (kk & 3) * 32, 16, 1024),
+                                     idZ, kk ? 1u : 0u);
+                        umma_arrive(&sh->empty[s]);
                     }
-                    umma_arrive(&sh->empty[s]);
+                    __syncwarp();
                 }
-                __syncwarp();
+                if (!ok) break;
+                if (lane == 0) umma_arrive(&sh->z_full);
             }
-            if (!ok) break;
-            if (lane == 0) umma_arrive(&sh->o_full);
+            if (vitem >= (int)blockIdx.x) {
+                // output of item vitem (ordinal step - 1)
+                const RtItem w = rt_decode(p, vitem);
+                const int64_t new_local = p.update_row >= 0 ? p.update_row - w.r0 : -1;
+                const size_t new_off = ((size_t)w.b * p.Hkv + w.g) * RT_HD;
+                if (!rt_warp_wait(&sh->p_full, (step - 1) & 1, sh, lane)) { ok = false; break; }
+                tcgen05_after();
+                for (int t = 0; t < w.tiles && ok; ++t, ++it) {
+                    const int s = it % S, n = it / S;
+                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
+                    tcgen05_after();
+                    const int rows = min(RT_ROWS, w.nr - t * RT_ROWS);
+                    const int nks = (rows + 15) / 16;
+                    const int64_t nl = new_local - (int64_t)t * RT_ROWS;
+                    const bool has_new = nl >= 0 && nl < RT_ROWS;
+                    if (has_new || rows < nks * 16)
+                        patch_tile(smem + s * RT_TILE, has_new ? (int)nl : -1, p.v_new + new_off,
+                                   rows, nks * 16, lane);
+                    if (lane == 0) {
+                        const uint32_t a0 = sbase + s * RT_TILE;
+                        for (int kk = 0; kk < nks; ++kk) {
+                            const int k0 = t * RT_ROWS + kk * 16;
+                            umma_f16(tmem + TM_O,
+                                     smem_desc_sw128(a0 + kk * 2048, RT_HALF, 1024),
+                                     smem_desc_sw128(pb + (k0 >> 6) * PATOM + ((k0 & 63) >> 4) * 32,
+                                                     16, 1024),
+                                     idO, (t | kk) ? 1u : 0u);
+                        }
+                        umma_arrive(&sh->empty[s]);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (lane == 0) umma_arrive(&sh->o_full);
+            }
         }
         if (lane == 0) {                            // every MMA issued here has completed
             umma_arrive(&sh->idle);
@@ -330,8 +347,12 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                     for (int h = 0; h < G; ++h) z[t][h] = -INFINITY;
                 }
             }
-            // the logit MMAs of this item are done: Q can take the next item's heads
-            if (item + (int)gridDim.x < p.n_items) write_q(item + gridDim.x);
+            // the logits are read: Q takes the next item's heads and the next item's logit
+            // MMAs may overwrite D_z while this item's softmax runs
+            const bool has_next = item + (int)gridDim.x < p.n_items;
+            if (has_next) write_q(item + gridDim.x);
+            fence_async_smem();
+            tcgen05_before();
             float m[G], l[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -344,6 +365,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 if (lane == 0) sh->red[ew][h] = m[h];
             }
             rt_epi_bar();
+            if (et == 0 && has_next) mbar_arrive(&sh->q_full);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 m[h] = fmaxf(fmaxf(sh->red[0][h], sh->red[1][h]),
@@ -377,7 +399,6 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
             rt_epi_bar();
             if (et == 0) {
                 mbar_arrive(&sh->p_full);
-                if (item + (int)gridDim.x < p.n_items) mbar_arrive(&sh->q_full);
             }
 #pragma unroll
             for (int h = 0; h < G; ++h)
