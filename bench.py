@@ -565,6 +565,13 @@ def main():
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
                 "frac_of_8tbs": achieved / 8000.0, "traffic": traffic,
                 "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms}
+    if w.mode != "rcla" and args.path == "explicit":
+        # the explicit reconstruction is also a tensor-core workload: its GEMM rate
+        # against the sustained bf16 peak, alongside the HBM figures
+        tf_peak, tf_kind = measured_tflops_sustained()
+        tflops = wl.attend_flops() / (attend_avg_ms / 1e3) / 1e12
+        roofline.update({"flops_per_launch": wl.attend_flops(), "tflops": tflops,
+                         "tensor_peak": tf_peak, "tensor_frac": tflops / tf_peak})
     if w.mode == "dense" and args.path == "explicit":
         # explicit dense reconstruction is bound by the tensor cores, not by HBM: report
         # the GEMM rate against the sustained bf16 peak (the kernel runs inside a long

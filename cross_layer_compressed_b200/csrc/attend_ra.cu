@@ -497,6 +497,7 @@ __global__ void __launch_bounds__(MG_THREADS) k_merge_ra(const float *__restrict
     float acc[8], l = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll 4
     for (int sp = warp; sp < n_split; sp += NW) {
         const float *ps = p + sp * stride;
         const float wgt = expf(ps[0] - M);

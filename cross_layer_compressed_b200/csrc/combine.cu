@@ -22,9 +22,12 @@ __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ parti
     }
     const size_t stride = (size_t)BH * (hd + 2);
     const float *p = partials + (size_t)bh * (hd + 2);
+    // the splits' loads are independent: unrolled, several are in flight at once
     float M = -INFINITY;
+#pragma unroll 8
     for (int s = 0; s < n_split; ++s) M = fmaxf(M, p[s * stride]);
     float l = 0.f, acc = 0.f;
+#pragma unroll 8
     for (int s = 0; s < n_split; ++s) {
         const float w = expf(p[s * stride] - M);
         l = fmaf(w, p[s * stride + 1], l);
