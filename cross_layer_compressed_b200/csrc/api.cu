@@ -337,11 +337,10 @@ xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, con
     if ((st = check_device(who)) != XKV_OK) return st;
     if (!tma_available()) return fail(XKV_ERR_UNSUPPORTED, "%s: no tensor-map encoder", who);
     cudaStream_t s = (cudaStream_t)stream;
-    unsigned *status = (unsigned *)ws;
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
-    if (e == cudaSuccess)
-        e = launch_attend_ra(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, ns,
-                             (char *)ws + ws_header_bytes(*dims), status, out, s);
+    unsigned *status = (unsigned *)ws;     // cleared by the call's first kernel
+    const cudaError_t e = launch_attend_ra(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
+                                           ns, (char *)ws + ws_header_bytes(*dims), status,
+                                           out, s);
     return launched(e, who);
 }
 

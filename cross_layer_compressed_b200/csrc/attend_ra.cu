@@ -17,9 +17,13 @@
 //                partials (m, l, u) in rank space
 //   k_merge_ra   merges an item's splits in rank space (U_h, L_h)
 //   k_project_ra o_h = U_h B^V_g / L_h
-// Warp roles of k_xkv_ra: warp 0 TMEM + MMA issue, warps 1-4 TMA producers (every 8-row
-// group of an item is one 128-byte-swizzled box per 64 columns, a stage holds 128
-// columns of the item's rows), warps 5-8 epilogue.  Every mbarrier wait is bounded; on
+// Warp roles of k_xkv_ra: warp 0 TMEM + MMA issue, warps 1-4 TMA producers, warps 5-8
+// epilogue.  A stage holds 128 columns of the item's rows; each 8-row group arrives in
+// one copy of a 3D view of A (64 elements x 8 rows x 2 column blocks) as two consecutive
+// 128-byte-swizzled atoms, so a stage takes one copy per group instead of two (the
+// kernel is bound by the copy engine's per-copy cost: it does almost no arithmetic).
+// The operand descriptors follow the [group][column block][8 rows x 128 B] layout:
+// 8-row groups 2 KB apart, the two column blocks 1 KB apart.  Every mbarrier wait is bounded; on
 // expiry the CTA sets XKV_ERR_TIMEOUT in the workspace status word, drains its copies
 // and MMAs (bounded), frees TMEM and returns, and the combine writes NaN outputs.
 #include "sm100_util.cuh"
@@ -28,8 +32,8 @@ namespace xkv {
 namespace {
 
 constexpr int RA_ROWS = 256;                    // rows per work item
-constexpr int RA_HALF = RA_ROWS * 128;          // one 64-column half of a stage: 32 KB
-constexpr int RA_STAGE = 2 * RA_HALF;           // 128 columns of the item's rows: 64 KB
+constexpr int RA_GROUP = 2048;                  // one 8-row group: two 64-column atoms
+constexpr int RA_STAGE = RA_ROWS / 8 * RA_GROUP;  // 128 columns of the item's rows: 64 KB
 constexpr int RA_STAGES = 3;
 constexpr int RA_QBUF = 16 * 1024;              // Q~: NO rows x r_K, K-major
 constexpr int RA_PBUF = 8 * 1024;               // P: NO rows x 256 tokens, K-major
@@ -198,11 +202,8 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                     if (pi == 0 && lane == 0)
                         mbar_expect_tx(&sh->full[s], (uint32_t)(ngl * 2 * 1024));
                     __syncwarp();
-                    if (gi < ngl) {
-                        tma_load_2d(m, &sh->full[s], dst + gi * 1024, st * 128, row);
-                        tma_load_2d(m, &sh->full[s], dst + RA_HALF + gi * 1024, st * 128 + 64,
-                                    row);
-                    }
+                    if (gi < ngl)   // both 64-column blocks of the group's 8 rows in one copy
+                        tma_load_3d(m, &sh->full[s], dst + gi * RA_GROUP, 0, row, st * 2);
                     __syncwarp();
                 }
             }
@@ -233,15 +234,17 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                     const uint32_t a0 = sbase + s * RA_STAGE;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {      // 16 columns of the stage per step
-                        const uint32_t aoff = (kk >> 2) * RA_HALF + (kk & 3) * 32;
+                        const uint32_t aoff = (kk >> 2) * 1024 + (kk & 3) * 32;
                         const int k0 = st * 128 + kk * 16;
                         const uint64_t bq = smem_desc_sw128(qb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32,
                                                             16, 1024);
                         const uint32_t acc = (st | kk) ? 1u : 0u;
-                        umma_f16(tmem + TM_Z, smem_desc_sw128(a0 + aoff, 16, 1024), bq, idZ, acc);
+                        umma_f16(tmem + TM_Z, smem_desc_sw128(a0 + aoff, 16, RA_GROUP), bq, idZ,
+                                 acc);
                         if (w.nr > 128)
-                            umma_f16(tmem + TM_Z + NO, smem_desc_sw128(a0 + aoff + 16384, 16, 1024),
-                                     bq, idZ, acc);
+                            umma_f16(tmem + TM_Z + NO,
+                                     smem_desc_sw128(a0 + aoff + 16 * RA_GROUP, 16, RA_GROUP), bq,
+                                     idZ, acc);
                     }
                     umma_arrive(&sh->empty[s]);
                 }
@@ -257,7 +260,8 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                     const uint32_t a0 = sbase + s * RA_STAGE;
                     for (int kt = 0; kt < nk16; ++kt) {
                         const int k0 = kt * 16;
-                        umma_f16(tmem + TM_U + st * NO, smem_desc_sw128(a0 + kt * 2048, RA_HALF, 1024),
+                        umma_f16(tmem + TM_U + st * NO,
+                                 smem_desc_sw128(a0 + kt * 2 * RA_GROUP, 1024, RA_GROUP),
                                  smem_desc_sw128(pb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32, 16, 1024),
                                  idU, kt ? 1u : 0u);
                     }
@@ -422,8 +426,12 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
                                                 const __nv_bfloat16 *__restrict__ Bkt,
                                                 __nv_bfloat16 *__restrict__ qt_hi,
                                                 __nv_bfloat16 *__restrict__ qt_lo, int Hq,
-                                                int Hkv, int hd, int rk) {
+                                                int Hkv, int hd, int rk,
+                                                unsigned *__restrict__ status) {
     __shared__ float qs[G * 128];                  // [G][hd]
+    // the call's device-side error word starts clean: this kernel runs first in the call,
+    // so the clear is ordered before every kernel that may set it
+    if (status && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *status = 0u;
     __shared__ float red[8][G][QT_COLS];
     const int g = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * QT_COLS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -436,8 +444,8 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
     for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[h][c] = 0.f;
-#pragma unroll 4
-    for (int j = warp; j < hd; j += 8) {
+#pragma unroll 16
+    for (int j = warp; j < hd; j += 8) {            // every row's load in flight at once
         const uint2 w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
         const float bv[4] = {bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y)};
 #pragma unroll
@@ -580,7 +588,7 @@ cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams 
                      __nv_bfloat16 *qt_lo, float *U, float *Lsum, float *out, cudaStream_t s) {
     k_qtilde<G><<<dim3(d.n_kv_heads, d.batch, d.rank_k / QT_COLS), 256, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
-        d.n_kv_heads, d.head_dim, d.rank_k);
+        d.n_kv_heads, d.head_dim, d.rank_k, p.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = 1024 + (size_t)RA_STAGES * RA_STAGE + RA_QBUF + RA_PBUF + sizeof(RaShared);
@@ -632,8 +640,8 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
                              const void *Bvt, const void *q, const int32_t *sel, int n_sel,
                              void *scratch, unsigned *status, float *out, cudaStream_t s) {
     CUtensorMap maps[2];
-    if (!make_map_bf16_sw128(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8) ||
-        !make_map_bf16_sw128(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8))
+    if (!make_map_bf16_sw128_cb(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 8, 2) ||
+        !make_map_bf16_sw128_cb(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 8, 2))
         return cudaErrorInvalidValue;
     const size_t bh = (size_t)d.batch * d.n_q_heads;
     const size_t qt_al = al256(bh * d.rank_k * sizeof(__nv_bfloat16));

@@ -42,6 +42,14 @@ static __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint6
         "l"(map), "r"(x), "r"(y), "r"(su32(bar))
         : "memory");
 }
+static __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *bar, void *dst,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(su32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(su32(bar))
+        : "memory");
+}
 static __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -130,5 +138,9 @@ bool tma_available();
 // (128 bytes) written to shared memory with the 128-byte swizzle.
 bool make_map_bf16_sw128(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                          uint32_t box_rows);
+// The same array seen as (64 elements, rows, 64-column blocks): a box of box_rows x 64
+// elements x box_cb blocks lands as box_cb consecutive 128-byte-swizzled atoms.
+bool make_map_bf16_sw128_cb(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows, uint32_t box_cb);
 
 }  // namespace xkv

@@ -34,6 +34,24 @@ bool make_map_impl(CUtensorMap *m, const void *base, uint64_t rows, uint64_t col
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D view of the same row-major [rows][cols] array: (64 elements, rows, cols / 64
+// column blocks) with strides (row: cols * 2 bytes, column block: 128 bytes); a box of
+// (64, box_rows, box_cb) lands in shared memory as box_cb consecutive swizzle atoms of
+// box_rows x 128 bytes: several 64-column blocks of the same rows in one copy.
+bool make_map3_impl(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows, uint32_t box_cb) {
+    auto fn = encode_fn();
+    if (!fn || cols % 64) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64u, box_rows, box_cb};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count_impl() {
     static int n = 0;
     if (!n) {
@@ -51,6 +69,10 @@ bool tma_available() { return encode_fn() != nullptr; }
 bool make_map_bf16_sw128(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                          uint32_t box_rows) {
     return make_map_impl(m, base, rows, cols, box_rows);
+}
+bool make_map_bf16_sw128_cb(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows, uint32_t box_cb) {
+    return make_map3_impl(m, base, rows, cols, box_rows, box_cb);
 }
 int sm_count() { return sm_count_impl(); }
 

@@ -27,7 +27,7 @@ def _u16(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def _xkv_layer_check(xkv, ora, w, layer, units, dense=False):
+def _xkv_layer_check(xkv, ora, w, layer, units, dense=False, reassociated=False):
     d = xkv.dims_of(w)
     c = synth.torch_xkv_layer(w, seed=0, layer=layer, device=DEV)
     q = synth.torch_layer_queries(w, 0, layer, c, device=DEV)
@@ -59,11 +59,12 @@ def _xkv_layer_check(xkv, ora, w, layer, units, dense=False):
         host[(b, g)] = (Ak, Bkt_g, lm_ref)
     scores = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
     sel = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
-    ws = torch.empty(xkv.xkv_workspace_bytes(d, w.n_sel, xkv.XKV_MODE_SELECTIVE),
-                     dtype=torch.uint8, device=DEV)
+    mode = xkv.XKV_MODE_REASSOC if reassociated else xkv.XKV_MODE_SELECTIVE
+    attend = xkv.xkv_reassociated_attend if reassociated else xkv.xkv_reconstruct_attend
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, w.n_sel, mode), dtype=torch.uint8, device=DEV)
     xkv.xkv_score_landmarks(d, lm, q, scores)
     xkv.xkv_select_chunks(d, scores, w.top_k, w.n_sink, w.n_recent, sel)
-    xkv.xkv_reconstruct_attend(d, c["Ak"], c["Av"], c["Bkt"], c["Bvt"], q, sel, w.n_sel, out, ws)
+    attend(d, c["Ak"], c["Av"], c["Bkt"], c["Bvt"], q, sel, w.n_sel, out, ws)
     torch.cuda.synchronize()
     sel_h = sel.cpu().numpy()
     # properties of every unit: ascending, in range, forced chunks present, needles kept
@@ -103,6 +104,19 @@ def test_llama8b_selective_32k_full_layer(xkv, ora):
 def test_qwen14b_selective_16k_full_layer(xkv, ora):
     w = synth.QWEN14B_SR_16K
     _xkv_layer_check(xkv, ora, w, layer=9, units=[(0, 7), (63, 2)])
+    torch.cuda.empty_cache()
+
+
+def test_llama8b_selective_32k_full_layer_reassociated(xkv, ora):
+    """The rank-space entry point on the same full-size layer and sampled units."""
+    w = synth.LLAMA8B_SR_32K
+    _xkv_layer_check(xkv, ora, w, layer=5, units=[(3, 5), (7, 0)], reassociated=True)
+    torch.cuda.empty_cache()
+
+
+def test_qwen14b_selective_16k_full_layer_reassociated(xkv, ora):
+    w = synth.QWEN14B_SR_16K
+    _xkv_layer_check(xkv, ora, w, layer=9, units=[(0, 7), (63, 2)], reassociated=True)
     torch.cuda.empty_cache()
 
 
