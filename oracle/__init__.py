@@ -48,6 +48,9 @@ def lib():
                                          i32, vp, vp, vp, vp, vp, vp, i64, vp]
         L.oracle_reconstruct_attend.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32, i32,
                                                 vp, vp, vp, vp, vp, vp, i64, vp]
+        L.oracle_attend_unit_tail.argtypes = [i32, i32, i32, i32, i32, i32, i64, i32, i32,
+                                              i32, i32, vp, vp, vp, vp, vp, vp, i64, vp, vp,
+                                              i64, i64, vp]
         L.oracle_leader_map.argtypes = [vp, i32, i32, vp]
         L.oracle_rcla_decode_attend.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
                                                 i64, i64, vp, vp, vp, vp]
@@ -197,6 +200,40 @@ def reconstruct_attend(Ak, Av, Bkt, Bvt, q, sel, chunk: int, units=None) -> np.n
             _check(lib().oracle_attend_unit(b, g, B, Hq, Hkv, hd, L, chunk, rk, rv, dt, _p(ak),
                                             _p(av), _p(bk), _p(bv), _p(qq), sp, n_sel, _p(out)),
                    "attend_unit")
+    return out
+
+
+def reconstruct_attend_tail(Ak, Av, Bkt, Bvt, q, sel, chunk: int, K_tail, V_tail,
+                            n_tail: int, units=None) -> np.ndarray:
+    """out [B][Hq][hd] fp32: attention over the reconstructed selected rows (all rows when
+    sel is None) followed by the first n_tail rows of K_tail / V_tail [B][Hkv][T_max][hd]
+    (storage type of the factors).  `units` as for reconstruct_attend."""
+    ak, dt = _buf(Ak)
+    av, _ = _buf(Av)
+    bk, _ = _buf(Bkt)
+    bv, _ = _buf(Bvt)
+    qq, _ = _buf(q)
+    kt, _ = _buf(K_tail)
+    vt, _ = _buf(V_tail)
+    B, L, rk = ak.shape
+    rv = av.shape[2]
+    d_kv = bk.shape[1]
+    _, Hq, hd = qq.shape
+    Hkv = d_kv // hd
+    T_max = kt.shape[2]
+    out = np.full((B, Hq, hd), np.nan, dtype=np.float32)
+    n_sel = 0
+    if sel is not None:
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        n_sel = sel.shape[2]
+    for b, g in (units if units is not None else [(b, g) for b in range(B) for g in range(Hkv)]):
+        sp = None
+        if sel is not None:
+            sp = ctypes.c_void_p(sel.ctypes.data + ((b * Hkv + g) * n_sel) * 4)
+        _check(lib().oracle_attend_unit_tail(b, g, B, Hq, Hkv, hd, L, chunk, rk, rv, dt,
+                                             _p(ak), _p(av), _p(bk), _p(bv), _p(qq), sp,
+                                             n_sel, _p(kt), _p(vt), T_max, int(n_tail),
+                                             _p(out)), "attend_unit_tail")
     return out
 
 

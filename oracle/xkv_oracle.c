@@ -388,6 +388,105 @@ int oracle_reconstruct_attend(int B, int Hq, int Hkv, int hd, int64_t L, int C, 
     return 0;
 }
 
+/*
+ * One (sequence b, KV head g) unit attending the reconstructed rows T (as in
+ * oracle_attend_unit) followed by n_tail uncompressed rows of a tail buffer (tokens
+ * generated after the cache was compressed), Kt/Vt [B][Hkv][T_max][hd] in the storage
+ * type.  The pages are silent on generated tokens; the reading taken: they are kept
+ * as they are and always attended, in one softmax with the selected rows.
+ */
+int oracle_attend_unit_tail(int b, int g, int B, int Hq, int Hkv, int hd, int64_t L, int C,
+                            int rk, int rv, int dtype, const void *Ak, const void *Av,
+                            const void *Bkt, const void *Bvt, const void *q,
+                            const int32_t *sel_bg, int64_t n_sel, const void *Kt,
+                            const void *Vt, int64_t T_max, int64_t n_tail, float *out)
+{
+    if (!Ak || !Av || !Bkt || !Bvt || !q || !out || B <= 0 || Hkv <= 0 || Hq % Hkv ||
+        C <= 0 || L % C || b < 0 || b >= B || g < 0 || g >= Hkv || n_tail < 0 ||
+        n_tail > T_max || (n_tail > 0 && (!Kt || !Vt)))
+        return -1;
+    int G = Hq / Hkv;
+    int64_t nC = L / C, d_kv = (int64_t)Hkv * hd;
+    int64_t nT = sel_bg ? n_sel * C : L;
+    if (nT <= 0)
+        return -1;
+    int64_t nR = nT + n_tail;
+    size_t esz = dtype == ORA_F32 ? 4 : 2;
+    const char *ak = (const char *)Ak + (size_t)b * L * rk * esz;
+    const char *av = (const char *)Av + (size_t)b * L * rv * esz;
+    const char *bk = (const char *)Bkt + (size_t)b * d_kv * rk * esz;
+    const char *bv = (const char *)Bvt + (size_t)b * d_kv * rv * esz;
+    int64_t tail0 = ((int64_t)b * Hkv + g) * T_max * hd;   /* element offset of row 0 */
+    double *z = malloc(sizeof(double) * nR * G);
+    double *row = malloc(sizeof(double) * hd);
+    double *acc = calloc((size_t)G * hd, sizeof(double));
+    double *qd = malloc(sizeof(double) * G * hd);
+    if (!z || !row || !acc || !qd) {
+        free(z); free(row); free(acc); free(qd);
+        return -2;
+    }
+    for (int hh = 0; hh < G; ++hh)
+        for (int d = 0; d < hd; ++d)
+            qd[hh * hd + d] = ora_load(q, dtype, ((int64_t)b * Hq + g * G + hh) * hd + d);
+    double scale = 1.0 / sqrt((double)hd);
+    int rc = 0;
+    /* logits: the reconstructed keys of the selected rows, then the tail's keys */
+    for (int64_t i = 0; i < nR; ++i) {
+        if (i < nT) {
+            int64_t t = i;
+            if (sel_bg) {
+                int64_t c = sel_bg[i / C];
+                if (c < 0 || c >= nC) {
+                    rc = -1;
+                    goto done;
+                }
+                t = c * C + i % C;
+            }
+            ora_recon_row(ak, bk, dtype, t, rk, g, hd, row);
+        } else {
+            for (int d = 0; d < hd; ++d)
+                row[d] = ora_load(Kt, dtype, tail0 + (i - nT) * hd + d);
+        }
+        for (int hh = 0; hh < G; ++hh) {
+            double s = 0.0;
+            for (int d = 0; d < hd; ++d)
+                s += qd[hh * hd + d] * row[d];
+            z[i * G + hh] = s * scale;
+        }
+    }
+    for (int hh = 0; hh < G; ++hh) {
+        double m = -INFINITY, l = 0.0;
+        for (int64_t i = 0; i < nR; ++i)
+            if (z[i * G + hh] > m)
+                m = z[i * G + hh];
+        for (int64_t i = 0; i < nR; ++i) {
+            z[i * G + hh] = exp(z[i * G + hh] - m);
+            l += z[i * G + hh];
+        }
+        for (int64_t i = 0; i < nR; ++i)
+            z[i * G + hh] /= l;
+    }
+    /* values: the reconstructed rows, then the tail's rows */
+    for (int64_t i = 0; i < nR; ++i) {
+        if (i < nT) {
+            int64_t t = sel_bg ? (int64_t)sel_bg[i / C] * C + i % C : i;
+            ora_recon_row(av, bv, dtype, t, rv, g, hd, row);
+        } else {
+            for (int d = 0; d < hd; ++d)
+                row[d] = ora_load(Vt, dtype, tail0 + (i - nT) * hd + d);
+        }
+        for (int hh = 0; hh < G; ++hh)
+            for (int d = 0; d < hd; ++d)
+                acc[hh * hd + d] += z[i * G + hh] * row[d];
+    }
+    for (int hh = 0; hh < G; ++hh)
+        for (int d = 0; d < hd; ++d)
+            out[((int64_t)b * Hq + g * G + hh) * hd + d] = (float)acc[hh * hd + d];
+done:
+    free(z); free(row); free(acc); free(qd);
+    return rc;
+}
+
 /* ------------------------------------------------------------ [R-CLA] sharing set */
 
 /* leader_of[l] = max{s in S : s <= l}; S must contain layer 0. */

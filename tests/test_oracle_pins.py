@@ -149,6 +149,47 @@ def test_selective_equals_sdpa_over_selected_rows(ora):
         assert np.max(np.abs(o[0, g * G:(g + 1) * G] - ref)) <= 1e-6 * np.max(np.abs(ref))
 
 
+@pytest.mark.parametrize("dense,n_tail", [(False, 5), (True, 3), (False, 0)])
+def test_tail_rows_join_the_selected_rows_in_one_softmax(ora, dense, n_tail):
+    """Generated tokens kept uncompressed: SDPA over the selected (or all) reconstructed
+    rows followed by the tail rows, in fp64."""
+    L, hd, C, Hq, Hkv, T_max = 128, 16, 8, 4, 2, 7
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 11)
+    sel = None if dense else np.array([[[0, 3, 7, 15], [1, 2, 9, 14]]], dtype=np.int32)
+    rng = np.random.default_rng(12)
+    Kt = (rng.standard_normal((1, Hkv, T_max, hd)) * 0.5).astype(np.float32)
+    Vt = rng.standard_normal((1, Hkv, T_max, hd)).astype(np.float32)
+    o = ora.reconstruct_attend_tail(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")],
+                                    _f32(q), sel, C, _f32(Kt), _f32(Vt), n_tail)
+    K, V = _khat(f, "k", Hkv, hd), _khat(f, "v", Hkv, hd)
+    G = Hq // Hkv
+    for g in range(Hkv):
+        rows = np.arange(L) if dense else \
+            np.concatenate([np.arange(c * C, (c + 1) * C) for c in sel[0, g]])
+        Kg = np.concatenate([K[g, rows], Kt[0, g, :n_tail]])[None]
+        Vg = np.concatenate([V[g, rows], Vt[0, g, :n_tail]])[None]
+        ref = _sdpa64(q[0, g * G:(g + 1) * G], Kg, Vg)
+        assert np.max(np.abs(o[0, g * G:(g + 1) * G] - ref)) <= 1e-6 * np.max(np.abs(ref))
+    if n_tail == 0:       # an empty tail is the plain call, operation for operation
+        plain = ora.reconstruct_attend(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")],
+                                       _f32(q), sel, C)
+        assert np.array_equal(o, plain)
+
+
+def test_a_dominant_tail_row_returns_its_value(ora):
+    """One tail key aligned with the query and far larger than every other logit: the
+    output is that row's value (closed form)."""
+    L, hd, C, Hq, Hkv = 64, 16, 8, 2, 1
+    _, _, f, q = _xkv_case(L, 1, Hq, Hkv, hd, 13)
+    Kt = np.zeros((1, Hkv, 4, hd), dtype=np.float32)
+    Vt = np.zeros((1, Hkv, 4, hd), dtype=np.float32)
+    Kt[0, 0, 2] = 200.0 * (q[0, 0] + q[0, 1])
+    Vt[0, 0, 2] = np.arange(hd)
+    o = ora.reconstruct_attend_tail(*[_f32(f[k]) for k in ("Ak", "Av", "Bkt", "Bvt")],
+                                    _f32(q), None, C, _f32(Kt), _f32(Vt), 3)
+    assert np.allclose(o[0], np.arange(hd)[None], atol=1e-6)
+
+
 def test_softmax_shift_invariance_through_an_extra_rank_term(ora):
     """Adding u to every key row (a rank-1 term: a ones column in A^K, u in B^K) shifts each
     head's logits by a constant, which softmax ignores.  Catches a dropped rank term or a
