@@ -254,11 +254,24 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
                                   (cudaStream_t)stream), who);
 }
 
-xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
-                                  const void *Bkt_layer, const void *Bvt_layer, const void *q,
-                                  const int32_t *sel, int32_t n_sel, float *out, void *ws,
-                                  size_t ws_bytes, void *stream) {
-    const char *who = "xkv_reconstruct_attend";
+}  // extern "C"
+
+namespace {
+
+// Splits the tail of generated tokens adds to an attention call (0 without a tail).
+int64_t tail_bound(const xkv_dims &d, int64_t T_max) {
+    return T_max > 0 ? plan_rcla(d, T_max).n_bound : 0;
+}
+
+// Reconstruct-then-attend over the selected (or all) rows of the window, plus, when
+// n_tail > 0, the first n_tail rows of an uncompressed tail K_tail / V_tail
+// [B][Hkv][T_max][hd]: the attention kernel writes its splits, the R-CLA kernel writes
+// the tail's splits after them, and one combine merges all of them.
+xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win,
+                       const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                       const void *q, const int32_t *sel, int32_t n_sel, const void *K_tail,
+                       const void *V_tail, int64_t T_max, int64_t n_tail, float *out, void *ws,
+                       size_t ws_bytes, void *stream) {
     xkv_status st;
     if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
     if (!Ak_win || !Av_win || !Bkt_layer || !Bvt_layer || !q || !out || !ws)
@@ -270,14 +283,20 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     const int64_t nC = dims->ctx_len / dims->chunk;
     if (sel && (n_sel <= 0 || n_sel > nC))
         return fail(XKV_ERR_INVALID_ARG, "%s: n_sel must be in [1, n_chunks]", who);
+    if (T_max < 0 || n_tail < 0 || n_tail > T_max)
+        return fail(XKV_ERR_INVALID_ARG, "%s: need 0 <= n_tail <= T_max", who);
+    if (n_tail > 0 && (!K_tail || !V_tail || !aligned16(K_tail) || !aligned16(V_tail)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: tail pointers must be 16-byte aligned", who);
     const int64_t rows = sel ? (int64_t)n_sel * dims->chunk : dims->ctx_len;
     const SplitPlan plan = plan_xkv(*dims, rows);
     const int n_tc = attend_tc_shape_ok(*dims) ? tc_splits(*dims, (int)(rows / dims->chunk)) : 0;
-    if (plan.n_split > 65535 || n_tc > 65535)
+    const int64_t n_att = n_tc > plan.n_bound ? n_tc : plan.n_bound;
+    const int64_t n_tail_bound = tail_bound(*dims, T_max);
+    if (plan.n_split > 65535 || n_tc > 65535 || n_att + n_tail_bound > 65535)
         return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    // the same amount xkv_workspace_bytes reports, whichever kernel runs
-    const size_t need = ws_header_bytes(*dims) +
-                        partial_bytes(*dims, (int)(n_tc > plan.n_bound ? n_tc : plan.n_bound));
+    // the same amount xkv_workspace_bytes / xkv_tail_workspace_bytes report, whichever
+    // kernel runs
+    const size_t need = ws_header_bytes(*dims) + partial_bytes(*dims, (int)(n_att + n_tail_bound));
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
@@ -292,18 +311,59 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
     // into the status word; the combine kernel turns a non-zero word into NaN outputs
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
     if (e != cudaSuccess) return launched(e, who);
+    int used = 0;
     if (use_tc) {
-        int used_split = n_tc;
+        used = n_tc;
         e = launch_attend_tc(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
                              sel ? n_sel : (int)(dims->ctx_len / dims->chunk), partials, status,
-                             &used_split, s);
-        if (e == cudaSuccess) e = launch_combine(*dims, used_split, partials, out, status, s);
+                             &used, s);
     } else {
+        used = plan.n_split;
         e = launch_attend_simt(*dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel, plan,
                                partials, status, s);
-        if (e == cudaSuccess) e = launch_combine(*dims, plan.n_split, partials, out, status, s);
     }
+    if (e == cudaSuccess && n_tail > 0) {
+        const SplitPlan tp = plan_rcla(*dims, n_tail);
+        float *tail_partials = partials + (size_t)used * dims->batch * dims->n_q_heads *
+                                              (dims->head_dim + 2);
+        e = launch_rcla(*dims, 0, T_max, n_tail, -1, const_cast<void *>(K_tail),
+                        const_cast<void *>(V_tail), nullptr, nullptr, q, tp, tail_partials, s);
+        used += tp.n_split;
+    }
+    if (e == cudaSuccess) e = launch_combine(*dims, used, partials, out, status, s);
     return launched(e, who);
+}
+
+}  // namespace
+
+extern "C" {
+
+xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
+                                  const void *Bkt_layer, const void *Bvt_layer, const void *q,
+                                  const int32_t *sel, int32_t n_sel, float *out, void *ws,
+                                  size_t ws_bytes, void *stream) {
+    return attend_impl("xkv_reconstruct_attend", dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
+                       sel, n_sel, nullptr, nullptr, 0, 0, out, ws, ws_bytes, stream);
+}
+
+xkv_status xkv_reconstruct_attend_tail(const xkv_dims *dims, const void *Ak_win,
+                                       const void *Av_win, const void *Bkt_layer,
+                                       const void *Bvt_layer, const void *q,
+                                       const int32_t *sel, int32_t n_sel, const void *K_tail,
+                                       const void *V_tail, int64_t T_max, int64_t n_tail,
+                                       float *out, void *ws, size_t ws_bytes, void *stream) {
+    if (T_max <= 0)
+        return fail(XKV_ERR_INVALID_ARG, "xkv_reconstruct_attend_tail: T_max must be positive");
+    return attend_impl("xkv_reconstruct_attend_tail", dims, Ak_win, Av_win, Bkt_layer, Bvt_layer,
+                       q, sel, n_sel, K_tail, V_tail, T_max, n_tail, out, ws, ws_bytes, stream);
+}
+
+size_t xkv_tail_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int64_t T_max) {
+    if (T_max <= 0) return 0;
+    const size_t base = xkv_workspace_bytes(dims, n_sel,
+                                            n_sel > 0 ? XKV_MODE_SELECTIVE : XKV_MODE_DENSE);
+    if (!base) return 0;
+    return base + partial_bytes(*dims, (int)tail_bound(*dims, T_max));
 }
 
 xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,

@@ -52,6 +52,9 @@ _sigs = {
                                ctypes.c_int),
     "rcla_decode_attend": ([_D, _i32, _vp, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                             _sz, _vp], ctypes.c_int),
+    "xkv_reconstruct_attend_tail": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i64,
+                                     _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "xkv_tail_workspace_bytes": ([_D, _i32, _i64], _sz),
     "xkv_reassociated_attend": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp],
                                 ctypes.c_int),
     "xkv_reconstruct_attend_noalloc": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp],
@@ -150,6 +153,25 @@ def xkv_reconstruct_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
     if check:
         _check(st)
     return st
+
+
+def xkv_reconstruct_attend_tail(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel,
+                                n_sel, K_tail, V_tail, T_max, n_tail, out, ws, ws_bytes=None,
+                                stream=None, check=True):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = _lib.xkv_reconstruct_attend_tail(ctypes.byref(d), _ptr(Ak_win), _ptr(Av_win),
+                                          _ptr(Bkt_layer), _ptr(Bvt_layer), _ptr(q), _ptr(sel),
+                                          int(n_sel), _ptr(K_tail), _ptr(V_tail), int(T_max),
+                                          int(n_tail), _ptr(out), _ptr(ws), int(ws_bytes),
+                                          _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_tail_workspace_bytes(d: xkv_dims, n_sel, T_max) -> int:
+    return int(_lib.xkv_tail_workspace_bytes(ctypes.byref(d), int(n_sel), int(T_max)))
 
 
 def xkv_reassociated_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel,

@@ -193,6 +193,26 @@ xkv_status xkv_reconstruct_attend_noalloc(const xkv_dims *dims, const void *Ak_w
                                           void *stream);
 
 /*
+ * xkv_reconstruct_attend plus a tail of tokens generated after the cache was compressed,
+ * kept uncompressed and always attended: for each (b, g) the softmax runs over the rows T
+ * of xkv_reconstruct_attend followed by rows [0, n_tail) of the tail.  The pages are
+ * silent on generated tokens; this is the reading taken (they are not refolded into
+ * the basis here).
+ *   K_tail, V_tail [B][Hkv][T_max][hd] in the storage type; 0 <= n_tail <= T_max,
+ *   T_max > 0; NULL tails are allowed when n_tail == 0.
+ *   ws, ws_bytes: at least xkv_tail_workspace_bytes(dims, sel ? n_sel : 0, T_max).
+ * Other arguments, layouts and failure signalling as for xkv_reconstruct_attend.
+ */
+xkv_status xkv_reconstruct_attend_tail(const xkv_dims *dims, const void *Ak_win,
+                                       const void *Av_win, const void *Bkt_layer,
+                                       const void *Bvt_layer, const void *q,
+                                       const int32_t *sel, int32_t n_sel, const void *K_tail,
+                                       const void *V_tail, int64_t T_max, int64_t n_tail,
+                                       float *out, void *ws, size_t ws_bytes, void *stream);
+/* Workspace bytes for xkv_reconstruct_attend_tail (0 on invalid arguments). */
+size_t xkv_tail_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int64_t T_max);
+
+/*
  * The same decode attention as xkv_reconstruct_attend, computed by associativity in the
  * rank space of the window's basis [xKV 2.2: K_hat = A^K B^K_l, V_hat = A^V B^V_l]:
  *   q~_h = B^K_g q_h,   z_h[t] = A^K[b][t] . q~_h / sqrt(hd),   p_h = softmax_t(z_h),

@@ -107,6 +107,28 @@ def test_workspace_bound_covers_every_smaller_call(xkv):
             assert xkv.xkv_workspace_bytes(dd, 0, xkv.XKV_MODE_RCLA) <= big_r
 
 
+def test_tail_call_arguments_rejected_without_launch(xkv):
+    """xkv_reconstruct_attend_tail: the tail's bounds, pointers and workspace are checked
+    before any CUDA call, and its workspace adds room for the tail's splits."""
+    d = _d(xkv)
+    base = xkv.xkv_workspace_bytes(d, 10, xkv.XKV_MODE_SELECTIVE)
+    ws = xkv.xkv_tail_workspace_bytes(d, 10, 64)
+    assert ws > base and xkv.xkv_tail_workspace_bytes(d, 10, 0) == 0
+    assert xkv.xkv_tail_workspace_bytes(d, 10, 128) >= ws   # bound grows with T_max
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10)
+
+    def call(Kt, Vt, T_max, n_tail, wsb=ws):
+        return xkv.xkv_reconstruct_attend_tail(d, *args, Kt, Vt, T_max, n_tail, FAKE, FAKE,
+                                               wsb, stream=0, check=False)
+    assert call(FAKE, FAKE, 64, 65) == 1                    # n_tail > T_max
+    assert call(FAKE, FAKE, 0, 0) == 1                      # T_max must be positive
+    assert call(FAKE, FAKE, 64, -1) == 1
+    assert call(0, FAKE, 64, 3) == 1                        # tail pointer missing
+    assert call(FAKE + 4, FAKE, 64, 3) == 1                 # misaligned
+    assert call(FAKE, FAKE, 64, 3, ws - 4) == 1             # workspace too small
+    assert "workspace" in xkv.last_error()
+
+
 def test_rcla_leader_rules(xkv):
     d = _d(xkv)
     ws = xkv.xkv_workspace_bytes(_d(xkv, ctx_len=64), 0, xkv.XKV_MODE_RCLA)

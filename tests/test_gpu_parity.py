@@ -303,6 +303,40 @@ def test_pipeline_end_to_end_tiny(xkv, ora):
         compare_outputs(out.cpu().numpy(), o_ref, w.dtype)
 
 
+# ------------------------------------------------------------- generated-token tail
+@pytest.mark.parametrize("w,dense,n_tail", [(LLAMA_R, False, 37), (LLAMA_R, False, 1),
+                                            (LLAMA_R, False, 0), (TINY, False, 5),
+                                            (DENSE_R, True, 17), (QWEN14_R, False, 300)],
+                         ids=lambda v: getattr(v, "name", str(v)))
+def test_reconstruct_attend_with_tail(xkv, ora, w, dense, n_tail):
+    """Selected (or all) reconstructed rows plus an uncompressed tail in one softmax."""
+    x = _layer_inputs(w)
+    T_max = max(n_tail, 1) + 3
+    rng = np.random.default_rng(n_tail + 7)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    Kt = torch.tensor(rng.standard_normal((w.batch, w.n_kv_heads, T_max, w.head_dim)) * 0.3,
+                      dtype=dt)
+    Vt = torch.tensor(rng.standard_normal((w.batch, w.n_kv_heads, T_max, w.head_dim)), dtype=dt)
+    sel = None
+    if not dense:
+        lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim,
+                                               w.chunk))
+        sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    ref = ora.reconstruct_attend_tail(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel,
+                                      w.chunk, Kt, Vt, n_tail)
+    d = xkv.dims_of(w)
+    n_sel = 0 if sel is None else sel.shape[2]
+    ws = torch.empty(xkv.xkv_tail_workspace_bytes(d, n_sel, T_max), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), device=DEV)
+    xkv.xkv_reconstruct_attend_tail(d, _dev(x["Ak"]), _dev(x["Av"]), _dev(x["Bkt"]),
+                                    _dev(x["Bvt"]), _dev(x["q"]),
+                                    None if sel is None else torch.from_numpy(sel).to(DEV),
+                                    n_sel, _dev(Kt), _dev(Vt), T_max, n_tail, out, ws)
+    torch.cuda.synchronize()
+    compare_outputs(out.cpu().numpy(), ref, w.dtype)
+
+
 # ------------------------------------------------------- reassociated (rank space)
 def _reassoc(xkv, w, x, sel):
     d = xkv.dims_of(w)
