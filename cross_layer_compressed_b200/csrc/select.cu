@@ -51,7 +51,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
                                                         int top_k, int n_sink, int n_recent,
                                                         int n_sel) {
     extern __shared__ unsigned long long keys[];  // [nC]
-    __shared__ unsigned hist[256];
+    __shared__ unsigned hist[2][256];             // passes alternate: one is zeroed while
+                                                  // the other is scanned
     __shared__ unsigned warp_tot[SEL_WARPS];
     __shared__ unsigned s_total;
     __shared__ unsigned long long s_prefix, s_mask;
@@ -63,31 +64,14 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     const double *s = scores + (size_t)unit * nC;
     auto forced = [&](int c) { return c < n_sink || c >= nC - n_recent; };
 
-    unsigned nf_local = 0;
-    bool nan_seen = false;
-    for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
-        const double v = s[c];
-        nan_seen |= isnan(v);
-        keys[c] = order_key(v);
-        nf_local += forced(c) ? 1u : 0u;
-    }
-    // a NaN score marks a failed scoring launch: the unit selects nothing (-1 entries),
-    // which makes the attention call that consumes it fail with NaN outputs
-    if (__syncthreads_or(nan_seen)) {
-        for (int i = threadIdx.x; i < n_sel; i += SEL_THREADS)
-            sel[(size_t)unit * n_sel + i] = -1;
-        return;
-    }
-    (void)block_exclusive_scan(nf_local, warp_tot, &s_total);  // also a barrier
-    const int n_forced = (int)s_total;
+    // forced chunks: [0, n_sink) and [nC - n_recent, nC), which may overlap
+    const int f_lo = min(n_sink, nC), f_hi = max(nC - n_recent, 0);
+    const int n_forced = f_lo + (nC - f_hi) - max(0, f_lo - f_hi);
     const int n_cand = nC - n_forced;
     const int k_eff = min(top_k, n_cand);
-
     // 0: take no candidate, 1: take every candidate, 2: threshold select with ties ranked
     // by index, 3: threshold select whose whole last bin is taken
     int mode = k_eff == 0 ? 0 : (k_eff == n_cand ? 1 : 2);
-    unsigned long long T = 0, M = 0;
-    unsigned krem = 0;
     if (mode == 2) {
         if (threadIdx.x == 0) {
             s_prefix = 0ull;
@@ -95,24 +79,44 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
             s_krem = (unsigned)k_eff;
             s_done = 0;
         }
+        for (int i = threadIdx.x; i < 256; i += SEL_THREADS) hist[0][i] = 0u;
+    }
+    bool nan_seen = false;
+    for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
+        const double v = s[c];
+        nan_seen |= isnan(v);
+        keys[c] = order_key(v);
+    }
+    // a NaN score marks a failed scoring launch: the unit selects nothing (-1 entries),
+    // which makes the attention call that consumes it fail with NaN outputs.  The same
+    // barrier publishes the keys and the first pass's state.
+    if (__syncthreads_or(nan_seen)) {
+        for (int i = threadIdx.x; i < n_sel; i += SEL_THREADS)
+            sel[(size_t)unit * n_sel + i] = -1;
+        return;
+    }
+    unsigned long long T = 0, M = 0;
+    unsigned krem = 0;
+    if (mode == 2) {
         unsigned long long mask = 0ull;
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int i = threadIdx.x; i < 256; i += SEL_THREADS) hist[i] = 0u;
-            __syncthreads();
+        int buf = 0;
+        for (int shift = 56; shift >= 0; shift -= 8, buf ^= 1) {
             const unsigned long long prefix = s_prefix;
             for (int c = threadIdx.x; c < nC; c += SEL_THREADS) {
                 const unsigned long long k = keys[c];
                 if (!forced(c) && (k & mask) == prefix)
-                    atomicAdd(&hist[(unsigned)(k >> shift) & 255u], 1u);
+                    atomicAdd(&hist[buf][(unsigned)(k >> shift) & 255u], 1u);
             }
             __syncthreads();
-            if (threadIdx.x < 32) {
+            if (threadIdx.x >= 32) {                   // the next pass's histogram
+                for (int i = threadIdx.x - 32; i < 256; i += SEL_THREADS - 32) hist[buf ^ 1][i] = 0u;
+            } else {
                 const int lane = threadIdx.x;
                 const unsigned need = s_krem;
                 unsigned cnt[8], tot = 0;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    cnt[i] = hist[255 - (lane * 8 + i)];  // lanes walk the digits downwards
+                    cnt[i] = hist[buf][255 - (lane * 8 + i)];  // lanes walk the digits downwards
                     tot += cnt[i];
                 }
                 unsigned inc = tot;
