@@ -178,3 +178,40 @@ def test_size_helpers_match_oracle(xkv, ora):
         assert xkv.xkv_n_selected(nC, k, s, r) == ora.n_selected(nC, k, s, r)
     d = xkv.dims(16, 32, 8, 128, 32832, dtype=1)
     assert xkv.rcla_cache_bytes(d, 9, 32832) == ora.rcla_cache_bytes(16, 8, 128, 32832, 1, 9)
+
+
+def test_plain_c_program_links_and_calls_the_host_entry_points(xkv, tmp_path):
+    """The boundary is a C ABI: a C99 program that includes include/xkv.h and links the
+    library calls the host-only entry points (no device needed) and gets the same
+    answers as the Python binding."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "xkv.h"
+int main(void) {
+    xkv_dims d = {8, 32, 8, 128, 32768, 8, 512, 768, XKV_BF16};
+    long long nsel = (long long)xkv_n_selected(4096, 256, 1, 4);
+    long long fp = (long long)xkv_footprint_bytes(&d, 32, 4, 1);
+    unsigned long long ws = (unsigned long long)xkv_workspace_bytes(&d, 261, XKV_MODE_SELECTIVE);
+    xkv_dims bad = d;
+    bad.head_dim = 96;
+    xkv_status st = xkv_score_landmarks(&bad, (void *)0, (void *)0, (double *)0, (void *)0);
+    printf("%lld %lld %llu %d %s\n", nsel, fp, ws, (int)st, xkv_last_error()[0] ? "msg" : "none");
+    return 0;
+}
+''')
+    lib_dir = os.path.dirname(xkv.LIB_PATH)
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", str(src), "-I",
+                    os.path.join(ROOT, "include"), "-L", lib_dir, "-lxkv",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    d = xkv.dims(8, 32, 8, 128, 32768, 8, 512, 768, xkv.XKV_BF16)
+    assert int(out[0]) == xkv.xkv_n_selected(4096, 256, 1, 4) == 261
+    assert int(out[1]) == xkv.xkv_footprint_bytes(d, 32, 4, 1)
+    assert int(out[2]) == xkv.xkv_workspace_bytes(d, 261, xkv.XKV_MODE_SELECTIVE)
+    assert int(out[3]) == xkv.XKV_ERR_UNSUPPORTED and out[4] == "msg"
