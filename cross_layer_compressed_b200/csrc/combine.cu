@@ -36,12 +36,71 @@ __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ parti
     if (j < hd) out[(size_t)bh * hd + j] = acc / l;
 }
 
+// Many splits (dense reconstruction: hundreds per sequence): one CTA per (b, h) of 8
+// warps; the splits' running max comes from a block reduction, then warp w sums splits
+// w, w + 8, ... with each lane holding 4 columns, so many loads are in flight, and the
+// warps' sums meet in shared memory.  Same merge as k_combine, in another order.
+constexpr int CW_THREADS = 256;
+__global__ void __launch_bounds__(CW_THREADS) k_combine_wide(const float *__restrict__ partials,
+                                                             float *__restrict__ out,
+                                                             int n_split, int BH, int hd,
+                                                             const unsigned *__restrict__ status) {
+    constexpr int NW = CW_THREADS / 32;
+    __shared__ float red[NW][128];
+    __shared__ float s_m[NW], s_l[NW];
+    const int bh = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (status && *(volatile const unsigned *)status) {  // the attention kernel gave up
+        if (threadIdx.x < hd) out[(size_t)bh * hd + threadIdx.x] = __int_as_float(0x7fc00000);
+        return;
+    }
+    const size_t stride = (size_t)BH * (hd + 2);
+    const float *p = partials + (size_t)bh * (hd + 2);
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < n_split; s += CW_THREADS) M = fmaxf(M, p[s * stride]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) s_m[warp] = M;
+    __syncthreads();
+    M = s_m[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) M = fmaxf(M, s_m[w]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+#pragma unroll 4
+    for (int s = warp; s < n_split; s += NW) {
+        const float *ps = p + s * stride;
+        const float w = expf(ps[0] - M);
+        l = fmaf(w, ps[1], l);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = lane + 32 * k;
+            if (j < hd) acc[k] = fmaf(w, ps[2 + j], acc[k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) red[warp][lane + 32 * k] = acc[k];
+    if (lane == 0) s_l[warp] = l;
+    __syncthreads();
+    if (threadIdx.x < hd) {
+        float sum = 0.f, ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            sum += red[w][threadIdx.x];
+            ls += s_l[w];
+        }
+        out[(size_t)bh * hd + threadIdx.x] = sum / ls;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
                            const unsigned *status, cudaStream_t s) {
     const int BH = d.batch * d.n_q_heads;
-    k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
+    if (n_split > 32)
+        k_combine_wide<<<BH, CW_THREADS, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
+    else
+        k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
     return cudaGetLastError();
 }
 
