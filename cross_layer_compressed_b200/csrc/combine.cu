@@ -36,8 +36,8 @@ __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ parti
     if (j < hd) out[(size_t)bh * hd + j] = acc / l;
 }
 
-// Many splits (dense reconstruction: hundreds per sequence): one CTA per (b, h) of 8
-// warps; the splits' running max comes from a block reduction, then warp w sums splits
+// More than a few splits (9 for a selective call at 32K, hundreds for dense 128K): one
+// CTA per (b, h) of 8 warps; the splits' running max comes from a block reduction, then warp w sums splits
 // w, w + 8, ... with each lane holding 4 columns, so many loads are in flight, and the
 // warps' sums meet in shared memory.  Same merge as k_combine, in another order.
 constexpr int CW_THREADS = 256;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(CW_THREADS) k_combine_wide(const float *__rest
 cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials, float *out,
                            const unsigned *status, cudaStream_t s) {
     const int BH = d.batch * d.n_q_heads;
-    if (n_split > 32)
+    if (n_split > 4)
         k_combine_wide<<<BH, CW_THREADS, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
     else
         k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
