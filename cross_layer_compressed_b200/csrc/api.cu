@@ -309,7 +309,7 @@ xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win
     float *partials = (float *)((char *)ws + hdr);
     // device-side errors of this call (timeouts, selections out of range) are OR-ed
     // into the status word; the combine kernel turns a non-zero word into NaN outputs
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
+    cudaError_t e = launch_clear_status(status, s);
     if (e != cudaSuccess) return launched(e, who);
     int used = 0;
     if (use_tc) {

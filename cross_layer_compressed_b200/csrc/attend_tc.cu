@@ -231,6 +231,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
+    grid_dep_wait();    // selection, query and status come from the kernels before
+    grid_dep_launch();
 
     if (warp >= W_LOAD && warp < W_LOAD + N_LOAD) {
         // ------------------------------------------------------------ TMA producers
@@ -495,8 +497,8 @@ cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s)
     cudaError_t e = set_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
-    k<<<grid, TC_THREADS, smem, s>>>(maps[0], maps[1], maps[2], maps[3], p);
-    return cudaGetLastError();
+    return launch_chained(k, dim3(grid), dim3(TC_THREADS), smem, s, maps[0], maps[1], maps[2],
+                          maps[3], p);
 }
 
 }  // namespace

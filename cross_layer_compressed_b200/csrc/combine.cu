@@ -1,6 +1,7 @@
 // Merge of split-K partial attention results (flash-decoding): each split s of a
 // (sequence, query head) left (m_s, l_s, acc_s) with acc_s = sum_t exp(z_t - m_s) v_t
 // over its rows.  out = sum_s exp(m_s - M) acc_s / sum_s exp(m_s - M) l_s, M = max m_s.
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -16,6 +17,7 @@ __global__ void __launch_bounds__(128) k_combine(const float *__restrict__ parti
                                                  const unsigned *__restrict__ status) {
     const int bh = blockIdx.x;
     const int j = threadIdx.x;
+    grid_dep_wait();  // the partials and the status word come from the kernels before
     if (status && *(volatile const unsigned *)status) {  // the attention kernel gave up
         if (j < hd) out[(size_t)bh * hd + j] = __int_as_float(0x7fc00000);
         return;
@@ -50,6 +52,7 @@ __global__ void __launch_bounds__(CW_THREADS) k_combine_wide(const float *__rest
     __shared__ float s_m[NW], s_l[NW];
     const int bh = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dep_wait();
     if (status && *(volatile const unsigned *)status) {  // the attention kernel gave up
         if (threadIdx.x < hd) out[(size_t)bh * hd + threadIdx.x] = __int_as_float(0x7fc00000);
         return;
@@ -98,11 +101,27 @@ cudaError_t launch_combine(const xkv_dims &d, int n_split, const float *partials
                            const unsigned *status, cudaStream_t s) {
     const int BH = d.batch * d.n_q_heads;
     if (n_split > 4)
-        k_combine_wide<<<BH, CW_THREADS, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
-    else
-        k_combine<<<BH, 128, 0, s>>>(partials, out, n_split, BH, d.head_dim, status);
-    return cudaGetLastError();
+        return launch_chained(k_combine_wide, dim3(BH), dim3(CW_THREADS), 0, s, partials, out,
+                              n_split, BH, d.head_dim, status);
+    return launch_chained(k_combine, dim3(BH), dim3(128), 0, s, partials, out, n_split, BH,
+                          d.head_dim, status);
 }
+
+namespace {
+// Lets the kernels after it be scheduled at once, then waits for the grid before it, so
+// that a grid waiting on this one also waits on that one.
+__global__ void k_clear_status(unsigned *status) {
+    grid_dep_launch();
+    grid_dep_wait();
+    *status = 0u;
+}
+}  // namespace
+
+cudaError_t launch_clear_status(unsigned *status, cudaStream_t s) {
+    return launch_chained(k_clear_status, dim3(1), dim3(1), 0, s, status);
+}
+
+bool chain_enabled() { return getenv("XKV_NO_PDL") == nullptr; }
 
 SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max_rows) {
     // Aim for about four CTAs per SM over the 148 SMs of a B200, with at least

@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     __syncthreads();
     tcgen05_after();
     const uint32_t tmem = sh->tmem_base;
+    grid_dep_launch();  // the split merge after this kernel may be scheduled
 
     if (warp == W_LOAD) {
         // ------------------------------------------------------------ TMA producer

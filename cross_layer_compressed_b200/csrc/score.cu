@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(SC_THREADS) k_score(const T *__restrict__ lm,
     constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
     constexpr int NG = G > 0 ? G : SC_MAXG;
     extern __shared__ __align__(16) double qs[];   // [hd][ng]
+    grid_dep_launch();  // the selection kernel after this one may be scheduled
     const int ng = G > 0 ? G : g_rt;
     const int b = blockIdx.z, g = blockIdx.y;
     const T *qb = q + ((size_t)b * Hq + (size_t)g * ng) * hd;

@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(const double *__restrict
     __shared__ unsigned s_krem;
     __shared__ int s_done;
 
+    grid_dep_wait();    // the scores come from the kernel before
+    grid_dep_launch();
     const int nC = (int)nC_;
     const int unit = blockIdx.x;
     const double *s = scores + (size_t)unit * nC;
@@ -205,9 +207,8 @@ cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, in
     const int64_t nC = d.ctx_len / d.chunk;
     const size_t smem = (size_t)nC * sizeof(unsigned long long);
     set_smem_limit((const void *)k_select, smem);
-    k_select<<<d.batch * d.n_kv_heads, SEL_THREADS, smem, s>>>(scores, sel, nC, top_k, n_sink,
-                                                               n_recent, n_sel);
-    return cudaGetLastError();
+    return launch_chained(k_select, dim3(d.batch * d.n_kv_heads), dim3(SEL_THREADS), smem, s,
+                          scores, sel, nC, top_k, n_sink, n_recent, n_sel);
 }
 
 }  // namespace xkv

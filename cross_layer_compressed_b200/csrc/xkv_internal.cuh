@@ -73,6 +73,37 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
                              float *partials, unsigned *status, int *n_split_out,
                              cudaStream_t s);
 
+// Clears the workspace status word of a call (a one-thread kernel launched with
+// launch_chained, so that it and the attention kernel after it are scheduled while the
+// previous kernel of the stream finishes).
+cudaError_t launch_clear_status(unsigned *status, cudaStream_t s);
+
+// ------------------------------------------------------------------ chained launches
+// Kernels that follow one another in a stream are launched with programmatic dependent
+// launch (CUDA 12): a grid so launched may be scheduled as soon as every CTA of the grid
+// before it has executed griddepcontrol.launch_dependents (or exited).  Each kernel
+// launched this way runs griddepcontrol.wait before it touches global memory that an
+// earlier grid writes or reads (setup of shared memory, mbarriers and TMEM may come
+// first), and that wait returns once the previous grid has completed and its writes are
+// visible; without the launch attribute the wait returns at once.  Setting XKV_NO_PDL in
+// the environment launches every kernel in plain stream order.
+bool chain_enabled();
+template <typename... P, typename... A>
+cudaError_t launch_chained(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = chain_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k, static_cast<A &&>(args)...);
+}
+
 // Sets the calling thread's xkv_last_error() message (defined with the C ABI layer).
 void set_last_error(const char *msg);
 
@@ -83,6 +114,14 @@ inline size_t ws_header_bytes(const xkv_dims &) { return 256; }
 // ------------------------------------------------------------------ device helpers
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Programmatic dependent launch, device side (see launch_chained).
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 template <typename T> struct Elem;
 template <> struct Elem<float> {

@@ -303,6 +303,47 @@ def test_pipeline_end_to_end_tiny(xkv, ora):
         compare_outputs(out.cpu().numpy(), o_ref, w.dtype)
 
 
+@pytest.mark.parametrize("plain_order", [False, True], ids=["chained", "plain_order"])
+def test_device_chain_back_to_back(xkv, ora, monkeypatch, plain_order):
+    """Score, select and attend of two bf16 layers issued back to back on one stream with
+    no host synchronisation in between, the kernels chained by programmatic dependent
+    launch (or, with XKV_NO_PDL, in plain stream order): scores and selections equal the
+    oracle's bit for bit and the outputs agree within tolerance."""
+    if plain_order:
+        monkeypatch.setenv("XKV_NO_PDL", "1")
+    w = LLAMA_R
+    d = xkv.dims_of(w)
+    refs, devs = [], []
+    for layer in range(2):
+        x = _layer_inputs(w, layer)
+        lm_np = ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk)
+        s_ref = ora.score_landmarks(_host_lm(ora, lm_np), x["q"])
+        sel_ref = ora.select_chunks(s_ref, w.top_k, w.n_sink, w.n_recent)
+        o_ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel_ref,
+                                       w.chunk)
+        refs.append((s_ref, sel_ref, o_ref))
+        devs.append(dict(lm=_dev(_host_lm(ora, lm_np)), q=_dev(x["q"]), Ak=_dev(x["Ak"]),
+                         Av=_dev(x["Av"]), Bkt=_dev(x["Bkt"]), Bvt=_dev(x["Bvt"])))
+    torch.cuda.synchronize()
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, w.n_sel, 0), dtype=torch.uint8, device=DEV)
+    got = []
+    for t in devs:
+        sc = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
+        sel = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
+        out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+        xkv.xkv_score_landmarks(d, t["lm"], t["q"], sc)
+        xkv.xkv_select_chunks(d, sc, w.top_k, w.n_sink, w.n_recent, sel)
+        xkv.xkv_reconstruct_attend(d, t["Ak"], t["Av"], t["Bkt"], t["Bvt"], t["q"], sel,
+                                   w.n_sel, out, ws)
+        got.append((sc, sel, out))
+    torch.cuda.synchronize()
+    for (sc, sel, out), (s_ref, sel_ref, o_ref) in zip(got, refs):
+        assert np.array_equal(sc.cpu().numpy().view(np.uint64), s_ref.view(np.uint64))
+        assert np.array_equal(sel.cpu().numpy(), sel_ref)
+        compare_outputs(out.cpu().numpy(), o_ref, w.dtype)
+    assert int(ws[:4].cpu().view(torch.int32).item()) == 0
+
+
 # ------------------------------------------------------------- generated-token tail
 @pytest.mark.parametrize("w,dense,n_tail", [(LLAMA_R, False, 37), (LLAMA_R, False, 1),
                                             (LLAMA_R, False, 0), (TINY, False, 5),
