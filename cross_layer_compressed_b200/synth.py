@@ -162,7 +162,7 @@ def reduced(w: Workload, **kw) -> Workload:
 # numpy generators (CPU, fp64 before the cast to the storage dtype): small workloads
 # ----------------------------------------------------------------------------------
 _TAGS = {"Ak": 1, "Av": 2, "Bk": 3, "Bv": 4, "q": 5, "needle": 6, "K": 7, "V": 8,
-         "knew": 9, "vnew": 10, "outlier": 11}
+         "knew": 9, "vnew": 10, "outlier": 11, "clfU": 12, "clfV": 13, "omega": 14}
 
 
 def _rng(seed: int, tag: str, *idx: int) -> np.random.Generator:
@@ -212,6 +212,41 @@ def np_plant_needles(w: Workload, q: np.ndarray, Ak_seq: np.ndarray, Bkt_seq: np
             u.append(d / np.linalg.norm(d))
         for j in range(G):
             q[seq, g * G + j, :] += lam * u[j % len(u)]
+
+
+def window_spectrum(n_modes: int, rank: int, tau: float, gap: float) -> np.ndarray:
+    """Singular values of a synthetic window concatenation: exp(-i/tau), times `gap`
+    from index `rank` on (gap < 1 puts a drop right after the kept rank)."""
+    i = np.arange(n_modes, dtype=np.float64)
+    s = np.exp(-i / tau)
+    s[rank:] *= gap
+    return s
+
+
+def np_window_caches(W: int, B: int, L: int, d_kv: int, n_modes: int, rank: int,
+                     tau: float, gap: float, seed: int):
+    """Caches of a window of W layers whose layers share one token subspace (the xKV
+    page's observation, section 2.1), with a known spectrum: per sequence the
+    concatenation [X_0 | ... | X_{W-1}] is exactly U diag(s) V^T, U (L x m) and V
+    (W·d_kv x m) with orthonormal columns (QR of Gaussian matrices), s from
+    window_spectrum, m = min(n_modes, L, W·d_kv); X_l = U diag(s) V_l^T with V_l the
+    l-th block of d_kv rows of V.  Returns (X [W][B][L][d_kv] fp64, s [m])."""
+    n = W * d_kv
+    m = min(n_modes, L, n)
+    s = window_spectrum(m, rank, tau, gap)
+    X = np.empty((W, B, L, d_kv))
+    for b in range(B):
+        U, _ = np.linalg.qr(_rng(seed, "clfU", b).standard_normal((L, m)))
+        V, _ = np.linalg.qr(_rng(seed, "clfV", b).standard_normal((n, m)))
+        US = U * s[None, :]
+        for l in range(W):
+            X[l, b] = US @ V[l * d_kv:(l + 1) * d_kv].T
+    return X, s
+
+
+def np_test_matrix(n: int, rank: int, seed: int) -> np.ndarray:
+    """The Gaussian test matrix of the randomized range finder, n x r, fp32."""
+    return _rng(seed, "omega", n, rank).standard_normal((n, rank)).astype(np.float32)
 
 
 def to_storage(x: np.ndarray, dtype: str):
@@ -416,3 +451,24 @@ def torch_rcla_cache(w: Workload, seed: int, device="cuda") -> dict:
     vn = torch.randn((nq, nl, B, H, hd), generator=_tgen(seed, "vnew", 0, device=device),
                      device=device).to(dt)
     return dict(K_lead=K, V_lead=V, k_new=kn, v_new=vn)
+
+
+def torch_window_caches(W: int, B: int, L: int, d_kv: int, n_modes: int, rank: int,
+                        tau: float, gap: float, dtype: str, seed: int, device="cuda"):
+    """np_window_caches at full size, built on the device (fp32 QR and products, then
+    the storage dtype).  Returns (X [W][B][L][d_kv], s [m] as fp64 numpy)."""
+    import torch
+    n = W * d_kv
+    m = min(n_modes, L, n)
+    s = window_spectrum(m, rank, tau, gap)
+    st = torch.tensor(s, dtype=torch.float32, device=device)
+    X = torch.empty((W, B, L, d_kv), dtype=_tdtype(dtype), device=device)
+    for b in range(B):
+        gu = _tgen(seed, "clfU", b, device=device)
+        gv = _tgen(seed, "clfV", b, device=device)
+        U, _ = torch.linalg.qr(torch.randn((L, m), generator=gu, device=device))
+        V, _ = torch.linalg.qr(torch.randn((n, m), generator=gv, device=device))
+        US = U * st[None, :]
+        for l in range(W):
+            X[l, b] = (US @ V[l * d_kv:(l + 1) * d_kv].T).to(X.dtype)
+    return X, s

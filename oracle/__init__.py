@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline leg may use it; the library itself never does.  The arithmetic lives in
 ``xkv_oracle.c`` (plain scalar C, fp64); this module compiles it with gcc and passes
-buffers to it.  Inputs are torch CPU tensors (fp32 or bf16) or numpy arrays.
+buffers to it.  Inputs are torch CPU tensors (fp32 or bf16) or numpy arrays.  The
+cross-layer factorization of a window (``clf.py``) is numpy fp64 around LAPACK's SVD.
 """
 from __future__ import annotations
 
@@ -19,6 +20,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 F32, BF16 = 0, 1
+
+from .clf import concatenate_window, factorize_window, reconstruct_window  # noqa: E402,F401
 
 
 def build(force: bool = False) -> str:

@@ -524,3 +524,95 @@ def test_needles_are_selected_by_the_oracle(ora):
     for b in range(w.batch):
         for g in range(w.n_kv_heads):
             assert set(x["needles"][b].tolist()) <= set(sel[b, g].tolist())
+
+
+# ------------------------------------------------- cross-layer factorization (CLF)
+# xKV page, section 2.2: concatenate the window's caches, rank-r SVD, shared A and per-
+# layer B_l.  The pins build caches whose SVD is known by construction.
+def _orthonormal(rng, rows, cols):
+    q, _ = np.linalg.qr(rng.standard_normal((rows, cols)))
+    return q
+
+
+def _window_from_modes(U, s, V, W, d):
+    """X_l = U diag(s) V_l^T, V_l the l-th block of d rows of V: [W][1][L][d]."""
+    return np.stack([(U * s) @ V[l * d:(l + 1) * d].T for l in range(W)])[:, None]
+
+
+def test_clf_tiny_closed_form(ora):
+    """One layer, X = [[3, 0], [0, 4], [0, 0]]: singular values (4, 3); the rank-1 part
+    is the 4 alone."""
+    X = np.array([[3.0, 0.0], [0.0, 4.0], [0.0, 0.0]])[None, None]
+    A, Bt, S = ora.factorize_window(X, 1)
+    assert np.allclose(S[0], [4.0, 3.0], atol=1e-14)
+    prod = ora.reconstruct_window(A, Bt)[0, 0]
+    assert np.allclose(prod, [[0.0, 0.0], [0.0, 4.0], [0.0, 0.0]], atol=1e-14)
+
+
+@pytest.mark.parametrize("W,L,d,m,r", [(2, 40, 8, 12, 5), (4, 64, 6, 20, 9), (3, 30, 4, 12, 12)])
+def test_clf_known_spectrum(ora, W, L, d, m, r):
+    """Caches built as U diag(s) V^T: the oracle returns s, its rank-r product is the
+    first r modes of the construction layer by layer, and the residual energy is the
+    sum of the dropped s_i^2 (Eckart-Young)."""
+    rng = np.random.default_rng(7)
+    U, V = _orthonormal(rng, L, m), _orthonormal(rng, W * d, m)
+    s = np.sort(rng.uniform(0.5, 3.0, m))[::-1]
+    X = _window_from_modes(U, s, V, W, d)
+    A, Bt, S = ora.factorize_window(X, r)
+    assert np.allclose(S[0, :m], s, atol=1e-12) and np.allclose(S[0, m:], 0.0, atol=1e-12)
+    want = _window_from_modes(U[:, :r], s[:r], V[:, :r], W, d)
+    got = ora.reconstruct_window(A, Bt)
+    assert np.abs(got - want).max() <= 1e-12 * s[0]
+    resid = np.sum((X - got) ** 2)
+    assert abs(resid - np.sum(s[r:] ** 2)) <= 1e-12 * np.sum(s ** 2)
+
+
+def test_clf_full_rank_is_exact(ora):
+    """r = min(L, W·d): the factorization reproduces every layer's cache."""
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((3, 2, 10, 4))            # L = 10 < W·d = 12
+    A, Bt, _ = ora.factorize_window(X, 10)
+    assert np.abs(ora.reconstruct_window(A, Bt) - X).max() <= 1e-12 * np.abs(X).max()
+
+
+def test_clf_basis_and_blocks(ora):
+    """A has orthonormal columns; B_l = A^T X_l block by block, so a layer that is
+    twice another gets twice its B, and a zero layer gets B_l = 0 -- a transposed or
+    misplaced concatenation block fails here."""
+    rng = np.random.default_rng(5)
+    X0 = rng.standard_normal((1, 2, 50, 6))
+    X = np.concatenate([X0, 2.0 * X0, np.zeros_like(X0)], axis=0)      # W = 3
+    A, Bt, _ = ora.factorize_window(X, 4)
+    for b in range(2):
+        assert np.allclose(A[b].T @ A[b], np.eye(4), atol=1e-12)
+        for l in range(3):
+            assert np.allclose(Bt[l, b], X[l, b].T @ A[b], atol=1e-12)
+        assert np.allclose(Bt[1, b], 2.0 * Bt[0, b], atol=1e-12)
+        assert np.abs(Bt[2, b]).max() == 0.0
+
+
+def test_clf_layer_order(ora):
+    """Reordering the window's layers reorders the B_l and leaves each A·B_l in place."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((3, 1, 30, 5))
+    r = 6
+    P = ora.reconstruct_window(*ora.factorize_window(X, r)[:2])
+    perm = [2, 0, 1]
+    Pp = ora.reconstruct_window(*ora.factorize_window(X[perm], r)[:2])
+    assert np.abs(Pp - P[perm]).max() <= 1e-12 * np.abs(X).max()
+
+
+def test_clf_rank_bounds(ora):
+    X = np.zeros((2, 1, 5, 3))
+    for r in (0, 7):
+        with pytest.raises(ValueError):
+            ora.factorize_window(X, r)
+
+
+def test_clf_generator_spectrum(ora):
+    """The input generator's caches have exactly the spectrum it states."""
+    X, s = synth.np_window_caches(2, 2, 120, 16, 40, 8, 6.0, 0.1, seed=0)
+    _, _, S = ora.factorize_window(X, 8)
+    for b in range(2):
+        assert np.allclose(S[b, :40], s, atol=1e-12)
+        assert np.allclose(S[b, 40:], 0.0, atol=1e-12)
