@@ -429,11 +429,209 @@ def aggregate_tokens_per_s(batch_per_rank: int, steps: int, world: int,
 
 
 # --------------------------------------------------------------------------- driver
+# ------------------------------------------------- cross-layer factorization (prefill)
+# One window of the Llama-3.1-8B-shaped 32K workload: W = 4 layers, 8 sequences, L =
+# 32768, d_kv = 8 x 128, ranks 512 (K) and 768 (V), 2 power passes.  A step factorizes
+# the window's K caches and its V caches for every sequence.
+CLF_WORKLOAD = "llama8b_clf_32k"
+CLF = dict(window=4, batch=8, ctx_len=32768, n_kv_heads=8, head_dim=128, rank_k=512,
+           rank_v=768, n_iter=2, tau=128.0, gap=0.1)
+CLF_METRIC = ("prefill cross-layer factorization tokens/s (window of 4 layers, K and V "
+              "caches, 32K ctx)")
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz (max clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def clf_flops(c, r):
+    """(fp32 GEMM flops, fp64 Gram flops) of one factorization call of rank r."""
+    B, L, q = c["batch"], c["ctx_len"], c["n_iter"]
+    n = c["window"] * c["n_kv_heads"] * c["head_dim"]
+    orth_rows = L * (1 + q) + n * q              # rows of every matrix orthonormalised
+    gemm = 2 * B * (L * r * n * (2 + 2 * q) + 2 * r * r * orth_rows)
+    gram = 2 * B * orth_rows * r * (r + 1)       # two CholeskyQR passes, r(r+1)/2 dots
+    return gemm, gram
+
+
+def clf_cpu_baseline(c, seed, rows=2048):
+    """The oracle (LAPACK SVD in fp64, one BLAS thread) on one sequence's K window cut
+    to `rows` tokens; tokens/s counts K and V (two factorizations per token)."""
+    import oracle
+    from cross_layer_compressed_b200 import synth
+    from threadpoolctl import threadpool_limits
+    dk = c["n_kv_heads"] * c["head_dim"]
+    X, _ = synth.np_window_caches(c["window"], 1, rows, dk, c["rank_k"] + 64, c["rank_k"],
+                                  c["tau"], c["gap"], seed)
+    Xq = synth.to_storage(X, "bf16").double().numpy()
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        oracle.factorize_window(Xq, c["rank_k"])
+        dt = time.perf_counter() - t0
+    return {"value": rows / (2 * dt), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"1 sequence x {rows} tokens of the K window (W = {c['window']}, "
+                      f"d_kv = {dk}, exact SVD), counted twice for K and V",
+            "sample_seconds": round(dt, 3)}
+
+
+def run_clf(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from cross_layer_compressed_b200 import build, synth
+    c = dict(CLF)
+    if args.batch:
+        c["batch"] = args.batch
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            clf_cpu_baseline(c, args.seed, rows=512)
+        vals = [clf_cpu_baseline(c, args.seed) for _ in range(args.steps)]
+        v = float(np.mean([x["value"] for x in vals]))
+        line = {"metric": CLF_METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * c["batch"] * c["ctx_len"] / v, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference", "config": {"workload": CLF_WORKLOAD, **c},
+                "cpu_baseline": {**vals[-1], "value": v},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    assert args.warmup >= 3 or os.environ.get("XKV_BENCH_ALLOW_SHORT"), "need >= 3 warm-up steps"
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    build.build()
+    from cross_layer_compressed_b200 import xkv
+    W, B, L = c["window"], c["batch"], c["ctx_len"]
+    dk = c["n_kv_heads"] * c["head_dim"]
+    n = W * dk
+    d = xkv.dims(B, c["n_kv_heads"], c["n_kv_heads"], c["head_dim"], L, dtype="bf16")
+    seed = args.seed + 1000 * rank
+    calls = []
+    for which, r in (("k", c["rank_k"]), ("v", c["rank_v"])):
+        X, _ = synth.torch_window_caches(W, B, L, dk, r + 64, r, c["tau"], c["gap"], "bf16",
+                                         seed + (0 if which == "k" else 1), device=dev)
+        om = torch.from_numpy(synth.np_test_matrix(n, r, seed)).to(dev)
+        A = torch.empty((B, L, r), dtype=torch.bfloat16, device=dev)
+        Bt = torch.empty((W, B, dk, r), dtype=torch.bfloat16, device=dev)
+        calls.append(dict(r=r, X=X, om=om, A=A, Bt=Bt))
+    ws = torch.empty(max(xkv.xkv_factorize_workspace_bytes(d, W, k["r"]) for k in calls),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        for i, k in enumerate(calls):
+            if events is not None:
+                events[i][0].record(stream)
+            xkv.xkv_factorize_window(d, W, k["r"], k["X"], k["om"], c["n_iter"], k["A"], k["Bt"],
+                                     ws)
+            if events is not None:
+                events[i][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    clocks = ClockSampler(dev.index)
+    barrier()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    # per call, CUDA events on the launching stream
+    per_call = [[], []]
+    for _ in range(args.steps):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in calls]
+        step(ev)
+        barrier()
+        for i in range(len(calls)):
+            per_call[i].append(ev[i][0].elapsed_time(ev[i][1]))
+    call_ms = [float(np.mean(p)) for p in per_call]
+    # end to end: the caches from pinned host memory, the factors back to the host
+    e2e = None
+    if not args.no_e2e:
+        hx = [torch.empty(k["X"].shape, dtype=k["X"].dtype, pin_memory=True) for k in calls]
+        for h, k in zip(hx, calls):
+            h.copy_(k["X"].cpu())
+        ha = [torch.empty(k["A"].shape, dtype=k["A"].dtype, pin_memory=True) for k in calls]
+        hb = [torch.empty(k["Bt"].shape, dtype=k["Bt"].dtype, pin_memory=True) for k in calls]
+
+        def e2e_step():
+            for h, k in zip(hx, calls):
+                k["X"].copy_(h, non_blocking=True)
+            step()
+            for a, b, k in zip(ha, hb, calls):
+                a.copy_(k["A"], non_blocking=True)
+                b.copy_(k["Bt"], non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        h2d = sum(h.numel() * h.element_size() for h in hx)
+        d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size()
+                  for a, b in zip(ha, hb))
+        e2e = {"value": B * L * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = clf_cpu_baseline(c, args.seed)
+    if rank == 0:
+        # the V call (rank 768) is the larger; its fp32 GEMM rate over the whole call
+        # (Gram and Cholesky kernels included) is a lower bound for the GEMM kernel's
+        g_flops, gram_flops = clf_flops(c, c["rank_v"])
+        tflops = g_flops / (call_ms[1] / 1e3) / 1e12
+        line = {
+            "metric": CLF_METRIC, "value": B * L * world * args.steps / (elapsed_ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": CLF_WORKLOAD, **c, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {2 * calls[0]['X'].numel() * 2 / 1e9:.1f} "
+                             "GB of caches per step"},
+            "roofline": {"bound": "alu", "kernel": "factorize_window (rank 768 call, whole)",
+                         "achieved": tflops, "peak": FP32_PEAK_TFLOPS,
+                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                         "unit": "TFLOP/s", "frac": tflops / FP32_PEAK_TFLOPS, "traffic": None,
+                         "flops_per_launch": g_flops, "fp64_gram_flops": gram_flops,
+                         "avg_launch_ms": call_ms[1], "rank_512_call_ms": call_ms[0]},
+            "gpu_launches": None, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        q = c["n_iter"]
+        orths = 1 + 2 * q
+        per_call_launches = (2 + 2 * q) + orths * 2 * 3 + 1     # GEMMs, Gram/Cholesky/apply, store
+        line["gpu_launches"] = per_call_launches * 2 * args.steps
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload == CLF_WORKLOAD:
+        run_clf(args, rank, world)
+        return
     from cross_layer_compressed_b200 import synth
     w = synth.WORKLOADS[args.workload]
     if args.batch:

@@ -257,6 +257,63 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
 }  // extern "C"
 
 namespace {
+xkv_status check_factorize(const xkv_dims *d, int32_t window, int32_t rank, const char *who) {
+    if (!d) return fail(XKV_ERR_INVALID_ARG, "%s: dims is NULL", who);
+    if (d->batch <= 0 || d->n_kv_heads <= 0 || d->ctx_len <= 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: batch, n_kv_heads and ctx_len must be positive",
+                    who);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: head_dim must be 64 or 128", who);
+    if (d->dtype != XKV_F32 && d->dtype != XKV_BF16)
+        return fail(XKV_ERR_INVALID_ARG, "%s: unknown dtype %d", who, d->dtype);
+    if (window < 1) return fail(XKV_ERR_INVALID_ARG, "%s: window must be >= 1", who);
+    const int64_t n = (int64_t)window * d->n_kv_heads * d->head_dim;
+    if (rank < 16 || rank % 16)
+        return fail(XKV_ERR_INVALID_ARG, "%s: rank must be a positive multiple of 16", who);
+    if (rank > 1024) return fail(XKV_ERR_UNSUPPORTED, "%s: rank above 1024", who);
+    if (rank > d->ctx_len || rank > n)
+        return fail(XKV_ERR_INVALID_ARG, "%s: rank above min(ctx_len, window * d_kv)", who);
+    if (d->ctx_len > (1 << 24) || n > (1 << 24) || d->batch > 65535)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: ctx_len, window * d_kv or batch too large", who);
+    return XKV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t xkv_factorize_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank) {
+    if (check_factorize(dims, window, rank, "xkv_factorize_workspace_bytes") != XKV_OK) return 0;
+    return factorize_ws_bytes(*dims, window, rank);
+}
+
+xkv_status xkv_factorize_window(const xkv_dims *dims, int32_t window, int32_t rank,
+                                const void *X, const float *omega, int32_t n_iter,
+                                void *A_out, void *Bt_out, void *ws, size_t ws_bytes,
+                                void *stream) {
+    const char *who = "xkv_factorize_window";
+    xkv_status st;
+    if ((st = check_factorize(dims, window, rank, who)) != XKV_OK) return st;
+    if (n_iter < 0 || n_iter > 16)
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_iter must be in [0, 16]", who);
+    if (!X || !omega || !A_out || !Bt_out || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL pointer", who);
+    if (!aligned16(X) || !aligned16(omega) || !aligned16(A_out) || !aligned16(Bt_out) ||
+        !aligned16(ws))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    const size_t need = factorize_ws_bytes(*dims, window, rank);
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_factorize(*dims, window, rank, X, omega, n_iter, A_out, Bt_out, ws,
+                                     (cudaStream_t)stream),
+                    who);
+}
+
+}  // extern "C"
+
+namespace {
 
 // Splits the tail of generated tokens adds to an attention call (0 without a tail).
 int64_t tail_bound(const xkv_dims &d, int64_t T_max) {

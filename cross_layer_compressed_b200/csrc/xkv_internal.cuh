@@ -73,6 +73,11 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
                              float *partials, unsigned *status, int *n_split_out,
                              cudaStream_t s);
 
+// cross-layer factorization of one window (clf.cu)
+size_t factorize_ws_bytes(const xkv_dims &d, int W, int r);
+cudaError_t launch_factorize(const xkv_dims &d, int W, int r, const void *X, const float *omega,
+                             int n_iter, void *A_out, void *Bt_out, void *ws, cudaStream_t s);
+
 // Clears the workspace status word of a call (a one-thread kernel launched with
 // launch_chained, so that it and the attention kernel after it are scheduled while the
 // previous kernel of the stream finishes).

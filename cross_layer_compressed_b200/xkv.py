@@ -60,6 +60,9 @@ _sigs = {
     "xkv_reconstruct_attend_noalloc": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp],
                                        ctypes.c_int),
     "xkv_workspace_bytes": ([_D, _i32, _i32], _sz),
+    "xkv_factorize_window": ([_D, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp],
+                             ctypes.c_int),
+    "xkv_factorize_workspace_bytes": ([_D, _i32, _i32], _sz),
     "xkv_n_selected": ([_i64, _i32, _i32, _i32], _i64),
     "xkv_footprint_bytes": ([_D, _i32, _i32, _i32], _i64),
     "rcla_cache_bytes": ([_D, _i32, _i64], _i64),
@@ -211,6 +214,22 @@ def rcla_decode_attend(d: xkv_dims, layer, leader_of, K_lead, V_lead, L_max, len
     if check:
         _check(st)
     return st
+
+
+def xkv_factorize_window(d: xkv_dims, window, rank, X, omega, n_iter, A_out, Bt_out, ws,
+                         ws_bytes=None, stream=None, check=True):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = _lib.xkv_factorize_window(ctypes.byref(d), int(window), int(rank), _ptr(X), _ptr(omega),
+                                   int(n_iter), _ptr(A_out), _ptr(Bt_out), _ptr(ws),
+                                   int(ws_bytes), _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_factorize_workspace_bytes(d: xkv_dims, window, rank) -> int:
+    return int(_lib.xkv_factorize_workspace_bytes(ctypes.byref(d), int(window), int(rank)))
 
 
 def xkv_workspace_bytes(d: xkv_dims, n_sel: int, mode: int) -> int:

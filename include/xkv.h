@@ -234,6 +234,44 @@ xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, con
 /* Scratch bytes the attention calls need (the split-K partial results). 0 on bad dims. */
 size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode);
 
+/*
+ * Cross-layer factorization of one window [xKV 2.2, steps 1-3: concatenate the W
+ * layers' caches side by side, rank-r SVD, one shared token basis A and one
+ * reconstruction matrix B_l per layer].  Per sequence b, with
+ * X_b = [X_0,b | ... | X_{W-1},b] (L x W*d_kv), it returns A_b (L x r, orthonormal
+ * columns spanning the dominant rank-r left singular subspace of X_b) and
+ * B_l,b = A_b^T X_l,b, so that A_b B_l,b is the rank-r truncated SVD of X_b restricted
+ * to layer l's columns once the iteration has converged.  Computed by randomized
+ * subspace iteration (Halko, Martinsson and Tropp 2011, Algorithm 4.4) with n_iter
+ * power passes and CholeskyQR2 orthonormalisation; the error against the exact
+ * truncated SVD shrinks like (s_{r+1} / s_r)^(2 n_iter + 1).  If rank(X_b) < r the
+ * surplus columns of A_b (and rows of B_l,b) are zero.
+ *
+ *   dims        batch, n_kv_heads, head_dim, ctx_len (= L) and dtype are used; the
+ *               query-head, chunk and rank fields are ignored
+ *   window      W >= 1 layers in the window
+ *   rank        r: a multiple of 16, 16 <= r <= min(1024, L, W*d_kv)
+ *   X           [W][B][L][d_kv] in dtype: layer l's cache, token-major, the KV heads of
+ *               a token side by side (d_kv = n_kv_heads * head_dim)
+ *   omega       [W*d_kv][r] fp32, device: the Gaussian test matrix (the caller draws it)
+ *   n_iter      power passes, 0..16
+ *   A_out       [B][L][r] in dtype (the window basis the decode calls take as Ak_win /
+ *               Av_win)
+ *   Bt_out      [W][B][d_kv][r] in dtype: B_l stored column-major per layer (what the
+ *               decode calls take as Bkt_layer / Bvt_layer)
+ *   ws          device scratch of xkv_factorize_workspace_bytes bytes
+ * All device pointers 16-byte aligned.  fp32 products, fp64 Gram matrices and Cholesky
+ * factors.  Asynchronous on `stream`; INVALID_ARG / UNSUPPORTED before any launch.
+ */
+xkv_status xkv_factorize_window(const xkv_dims *dims, int32_t window, int32_t rank,
+                                const void *X, const float *omega, int32_t n_iter,
+                                void *A_out, void *Bt_out, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* Scratch bytes of xkv_factorize_window for these dims, window and rank (0 on bad
+ * arguments). */
+size_t xkv_factorize_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank);
+
 /* Chunks selected per (b, g): min(top_k, nC - |F|) + |F|; -1 on bad arguments. */
 int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t n_recent);
 

@@ -215,3 +215,62 @@ int main(void) {
     assert int(out[1]) == xkv.xkv_footprint_bytes(d, 32, 4, 1)
     assert int(out[2]) == xkv.xkv_workspace_bytes(d, 261, xkv.XKV_MODE_SELECTIVE)
     assert int(out[3]) == xkv.XKV_ERR_UNSUPPORTED and out[4] == "msg"
+
+
+# ------------------------------------------------------- cross-layer factorization
+def _fd(xkv, **kw):
+    base = dict(batch=2, n_q_heads=2, n_kv_heads=2, head_dim=64, ctx_len=1000, chunk=8,
+                rank_k=0, rank_v=0, dtype=xkv.XKV_BF16)
+    base.update(kw)
+    return xkv.dims(**base)
+
+
+@pytest.mark.parametrize("kw,window,rank,n_iter,status", [
+    ({}, 0, 32, 1, 1),                              # window < 1
+    ({}, 2, 40, 1, 1),                              # rank not a multiple of 16
+    ({}, 2, 0, 1, 1),
+    ({}, 2, 2048, 1, 2),                            # rank above 1024
+    (dict(ctx_len=16), 2, 32, 1, 1),                # rank above L
+    (dict(n_kv_heads=1), 1, 80, 1, 1),              # rank above W * d_kv = 64
+    ({}, 2, 32, -1, 1),                             # n_iter out of range
+    ({}, 2, 32, 17, 1),
+    (dict(head_dim=96), 2, 32, 1, 2),
+    (dict(dtype=5), 2, 32, 1, 1),
+    (dict(batch=0), 2, 32, 1, 1),
+])
+def test_factorize_bad_arguments_rejected_without_launch(xkv, kw, window, rank, n_iter, status):
+    d = _fd(xkv, **kw)
+    st = xkv.xkv_factorize_window(d, window, rank, FAKE, FAKE, n_iter, FAKE, FAKE, FAKE,
+                                  1 << 40, stream=0, check=False)
+    assert st == status
+    assert xkv.last_error()
+
+
+def test_factorize_pointer_and_workspace_checks(xkv):
+    d = _fd(xkv)
+    need = xkv.xkv_factorize_workspace_bytes(d, 2, 32)
+    B, L, r, n = 2, 1000, 32, 2 * 128
+
+    def al(x):
+        return (x + 255) // 256 * 256
+    assert need == 2 * al(B * L * r * 4) + 2 * al(B * n * r * 4) + 2 * al(B * r * r * 8) + \
+        al(B * r * r * 4)
+    assert xkv.xkv_factorize_workspace_bytes(d, 2, 40) == 0
+    args = [FAKE] * 2
+    assert xkv.xkv_factorize_window(d, 2, 32, 0, FAKE, 1, FAKE, FAKE, FAKE, need, stream=0,
+                                    check=False) == 1
+    assert xkv.xkv_factorize_window(d, 2, 32, FAKE, FAKE + 4, 1, FAKE, FAKE, FAKE, need,
+                                    stream=0, check=False) == 1
+    assert "aligned" in xkv.last_error()
+    assert xkv.xkv_factorize_window(d, 2, 32, *args, 1, FAKE, FAKE, FAKE, need - 1, stream=0,
+                                    check=False) == 1
+    assert "workspace" in xkv.last_error()
+
+
+def test_factorize_fault_injection(xkv, monkeypatch):
+    monkeypatch.setenv("XKV_FAULT", "xkv_factorize_window:4")
+    d = _fd(xkv)
+    need = xkv.xkv_factorize_workspace_bytes(d, 2, 32)
+    assert xkv.xkv_factorize_window(d, 2, 32, FAKE, FAKE, 1, FAKE, FAKE, FAKE, need, stream=0,
+                                    check=False) == 4
+    assert "injected" in xkv.last_error()
