@@ -15,6 +15,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
+# cuBLAS serves the plain GEMMs of the prefill-side factorization only
+LIBS = ["-lcublas", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 
 
 def sources() -> list[str]:
@@ -32,7 +34,7 @@ def _stale() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if force or _stale():
         tmp = LIB + ".tmp"
-        cmd = [NVCC, *FLAGS, "-o", tmp, *sources()]
+        cmd = [NVCC, *FLAGS, "-o", tmp, *sources(), *LIBS]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.check_call(cmd)

@@ -4,7 +4,7 @@
 // layer, so that A·B_l stands in for layer l's cache).
 //
 // Per sequence the concatenation X = [X_0 | ... | X_{W-1}] (L x n, n = W·d_kv) is never
-// built: every product addresses layer l's block of columns in place.  The rank-r
+// built: every product runs layer by layer on the W cache buffers.  The rank-r
 // factorization comes from randomized subspace iteration (Halko, Martinsson and Tropp,
 // "Finding structure with randomness", SIAM Review 2011, Algorithm 4.4) with the
 // caller's Gaussian test matrix Omega (n x r):
@@ -17,128 +17,34 @@
 // SVD's product; A itself is one orthonormal basis of that subspace, not U_r (the two
 // differ by an r x r rotation that no product sees).
 //
-// orth() is CholeskyQR2 (two passes of: G = Y^T Y in fp64, G = R^T R by Cholesky in
-// fp64, Y <- Y R^-1).  A column whose Cholesky pivot is below 1e-12 of the largest
-// diagonal entry of G (a direction the data does not have: rank(X) < r) is zeroed
-// rather than normalised, so A keeps orthonormal columns and zero columns.
+// orth() is CholeskyQR2: twice G = Y^T Y (fp64), G = R^T R (blocked Cholesky, fp64),
+// Y <- Y R^-1 (R^-1 by blocked triangular inversion, fp64).  A column whose Cholesky
+// pivot is below 1e-12 of the largest diagonal entry of G (a direction the data does
+// not have: rank(X) < r) is zeroed rather than normalised.
 //
-// The products are fp32 CUDA-core GEMMs (fp32 accumulation); the Gram matrices,
-// Cholesky factors and triangular inverses are fp64.
+// The large products are plain GEMMs and run in cuBLAS on the tensor cores: for bf16
+// caches the fp32 operand (Q, Z) is split into bf16 hi + lo parts (about 16 significant
+// bits; the test matrix is used at bf16 precision, which only makes it another test
+// matrix) and the products with R^-1 use TF32; for fp32 caches every product is a plain
+// fp32 GEMM.  The Gram matrices, the Cholesky factorization and the inversion are this
+// file's own fp64 kernels.
+#include <cublas_v2.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "xkv_internal.cuh"
 
 namespace xkv {
 namespace {
 
-// A matrix operand of one sequence: element (row i, column j) of sequence b sits at
-// b*s_b + i*s_r + j*s_c, plus jump_r for every whole block of blk_r rows before i and
-// jump_c for every whole block of blk_c columns before j (blk = 0: no blocks).  The
-// blocks let one operand walk the W layer buffers of a window as one matrix.
-struct Mat {
-    const void *p;
-    int64_t s_r, s_c, s_b;
-    int32_t blk_r, blk_c;
-    int64_t jump_r, jump_c;
-};
-
-__device__ __forceinline__ int64_t row_part(const Mat &m, int i) {
-    int64_t o = (int64_t)i * m.s_r;
-    if (m.blk_r) o += (int64_t)(i / m.blk_r) * m.jump_r;
-    return o;
-}
-__device__ __forceinline__ int64_t col_part(const Mat &m, int j) {
-    int64_t o = (int64_t)j * m.s_c;
-    if (m.blk_c) o += (int64_t)(j / m.blk_c) * m.jump_c;
-    return o;
-}
-
-template <typename T> __device__ __forceinline__ float load_f32(const void *p, int64_t o) {
-    return Elem<T>::f32(reinterpret_cast<const T *>(p)[o]);
-}
-template <typename T> __device__ __forceinline__ void store_f32(void *p, int64_t o, float v);
-template <> __device__ __forceinline__ void store_f32<float>(void *p, int64_t o, float v) {
-    reinterpret_cast<float *>(p)[o] = v;
-}
-template <> __device__ __forceinline__ void store_f32<__nv_bfloat16>(void *p, int64_t o, float v) {
-    reinterpret_cast<__nv_bfloat16 *>(p)[o] = __float2bfloat16_rn(v);
-}
-
-// ------------------------------------------------------------------ fp32 GEMM
-// C (M x N) = A (M x K) · B (K x N) per sequence (blockIdx.z).  128 x 128 tile per CTA,
-// 16-deep slices of K staged in shared memory, 8 x 8 outputs per thread.  Loads follow
-// whichever index of the operand is contiguous, so X and X^T are both read coalesced.
-constexpr int GM = 128, GN = 128, GK = 16, G_THREADS = 256;
-
-template <typename TA, typename TC>
-__global__ void __launch_bounds__(G_THREADS) k_gemm(const Mat A, const Mat Bm, const Mat C,
-                                                    int M, int N, int K) {
-    __shared__ __align__(16) float As[GK][GM + 4];
-    __shared__ __align__(16) float Bs[GK][GN + 4];
-    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-    const int m0 = blockIdx.y * GM, n0 = blockIdx.x * GN, b = blockIdx.z;
-    const bool a_kc = A.s_c == 1 && A.s_r != 1;   // K is A's contiguous index
-    const bool b_nc = Bm.s_c == 1;                // N is B's contiguous index
-    const int64_t a_b = (int64_t)b * A.s_b, b_b = (int64_t)b * Bm.s_b;
-    float acc[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-
-    for (int k0 = 0; k0 < K; k0 += GK) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = tid + j * G_THREADS;
-            const int mm = a_kc ? e / GK : e % GM, kk = a_kc ? e % GK : e / GM;
-            const int gm = m0 + mm, gk = k0 + kk;
-            As[kk][mm] = (gm < M && gk < K)
-                             ? load_f32<TA>(A.p, a_b + row_part(A, gm) + col_part(A, gk))
-                             : 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = tid + j * G_THREADS;
-            const int nn = b_nc ? e % GN : e / GK, kk = b_nc ? e / GN : e % GK;
-            const int gn = n0 + nn, gk = k0 + kk;
-            Bs[kk][nn] = (gn < N && gk < K)
-                             ? load_f32<float>(Bm.p, b_b + row_part(Bm, gk) + col_part(Bm, gn))
-                             : 0.f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < GK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&As[kk][64 + ty * 4]);
-            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
-            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][64 + tx * 4]);
-            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-    const int64_t c_b = (int64_t)b * C.s_b;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-        if (gm >= M) continue;
-        const int64_t ro = c_b + row_part(C, gm);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-            if (gn < N) store_f32<TC>(const_cast<void *>(C.p), ro + col_part(C, gn), acc[i][j]);
-        }
-    }
-}
+constexpr int NB = 64;         // block size of the Cholesky factorization and inversion
+constexpr int NBP = NB + 1;    // padded shared-memory row
 
 // ------------------------------------------------------------------ fp64 Gram
 // G[b] += Y[b]^T Y[b] over one slice of rows, for the 64 x 64 tiles on or above the
-// diagonal (the Cholesky reads the upper triangle only).  fp32 x fp32 products are exact
-// in fp64; the slices meet through fp64 atomics.
+// diagonal (the factorization reads the upper triangle only).  fp32 x fp32 products are
+// exact in fp64; the slices meet through fp64 atomics.
 constexpr int GR_T = 64, GR_ROWS = 32;
 
 __global__ void __launch_bounds__(256) k_gram(const float *__restrict__ Y, int rows, int r,
@@ -191,214 +97,519 @@ __global__ void __launch_bounds__(256) k_gram(const float *__restrict__ Y, int r
     }
 }
 
-// ------------------------------------------------- fp64 Cholesky and R^-1 (one CTA)
-// G = R^T R with R upper triangular, in place on G's upper triangle (right-looking,
-// one pivot at a time), then R^-1 by back substitution, one column per thread.  A pivot
-// at or below `tol` marks a dependent column: its row of R and its column of R^-1 are
-// zero.  Requires r <= CH_THREADS.
-constexpr int CH_THREADS = 1024;
-
-__global__ void __launch_bounds__(CH_THREADS) k_chol_inv(double *__restrict__ G, int r,
-                                                         double *__restrict__ R64,
-                                                         float *__restrict__ R32) {
-    __shared__ double rowj[CH_THREADS];
-    __shared__ double red[CH_THREADS / 32];
-    __shared__ int s_dep;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    double *g = G + (int64_t)blockIdx.x * r * r;
-    double *ri = R64 + (int64_t)blockIdx.x * r * r;
-    float *ro = R32 + (int64_t)blockIdx.x * r * r;
-
+// ------------------------------------------- blocked Cholesky G = R^T R (fp64)
+// Per sequence the pivot tolerance: 1e-12 of the largest diagonal entry of G.
+__global__ void __launch_bounds__(256) k_maxdiag(const double *__restrict__ G, int r,
+                                                 double *__restrict__ tol) {
+    __shared__ double red[8];
+    const double *g = G + (int64_t)blockIdx.x * r * r;
     double mx = 0.0;
-    for (int i = tid; i < r; i += CH_THREADS) mx = fmax(mx, g[(int64_t)i * r + i]);
+    for (int i = threadIdx.x; i < r; i += 256) mx = fmax(mx, g[(int64_t)i * r + i]);
 #pragma unroll
     for (int off = 16; off; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if (lane == 0) red[warp] = mx;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
     __syncthreads();
-    mx = 0.0;
-    for (int w = 0; w < CH_THREADS / 32; ++w) mx = fmax(mx, red[w]);
-    const double tol = 1e-12 * mx;
+    if (threadIdx.x == 0) {
+        mx = red[0];
+        for (int w = 1; w < 8; ++w) mx = fmax(mx, red[w]);
+        tol[blockIdx.x] = 1e-12 * mx;
+    }
+}
 
-    for (int j = 0; j < r; ++j) {
-        if (tid == 0) {
-            const double p = g[(int64_t)j * r + j];
-            const int dep = !(p > tol);  // NaN counts as dependent too
+// Diagonal block k: unblocked right-looking Cholesky in shared memory (one thread per
+// column), then the block's inverse D_k = R_kk^-1 by back substitution.  A dependent
+// pivot gives a zero row of R and a zero row and column of D_k.
+__global__ void __launch_bounds__(NB) k_potrf_diag(double *__restrict__ G, int r, int k,
+                                                   const double *__restrict__ tol,
+                                                   double *__restrict__ D) {
+    extern __shared__ double sm[];
+    double (*a)[NBP] = reinterpret_cast<double (*)[NBP]>(sm);
+    double (*di)[NBP] = reinterpret_cast<double (*)[NBP]>(sm + NB * NBP);
+    __shared__ int s_dep;
+    const int b = blockIdx.x, c = threadIdx.x, o = k * NB;
+    const int bk = min(NB, r - o);
+    double *g = G + (int64_t)b * r * r;
+    for (int p = 0; p < NB; ++p)
+        a[p][c] = (p < bk && c < bk && p <= c) ? g[(int64_t)(o + p) * r + o + c] : 0.0;
+    const double t = tol[b];
+    __syncthreads();
+    for (int j = 0; j < bk; ++j) {
+        if (c == 0) {
+            const double pv = a[j][j];
+            const int dep = !(pv > t);  // NaN counts as dependent too
             s_dep = dep;
-            g[(int64_t)j * r + j] = dep ? 0.0 : sqrt(p);
+            a[j][j] = dep ? 0.0 : sqrt(pv);
         }
         __syncthreads();
         const int dep = s_dep;
-        const double rjj = g[(int64_t)j * r + j];
-        for (int c = j + 1 + tid; c < r; c += CH_THREADS) {
-            const double v = dep ? 0.0 : g[(int64_t)j * r + c] / rjj;
-            g[(int64_t)j * r + c] = v;
-            rowj[c] = v;
-        }
+        if (c > j && c < bk) a[j][c] = dep ? 0.0 : a[j][c] / a[j][j];
         __syncthreads();
-        if (!dep) {
-            const int n = r - j - 1;
-            for (int e = tid; e < n * n; e += CH_THREADS) {
-                const int i = j + 1 + e / n, c = j + 1 + e % n;
-                if (i <= c) g[(int64_t)i * r + c] -= rowj[i] * rowj[c];
-            }
-        }
+        if (!dep && c > j && c < bk)
+            for (int i = j + 1; i <= c; ++i) a[i][c] -= a[j][i] * a[j][c];
         __syncthreads();
     }
+    for (int i = NB - 1; i >= 0; --i) {
+        double x = 0.0;
+        if (i <= c && c < bk && a[i][i] != 0.0) {
+            double s = i == c ? 1.0 : 0.0;
+            for (int m = i + 1; m <= c; ++m) s -= a[i][m] * di[m][c];
+            x = s / a[i][i];
+        }
+        di[i][c] = x;
+    }
+    __syncthreads();
+    double *dk = D + ((int64_t)b * ((r + NB - 1) / NB) + k) * NB * NB;
+    for (int p = 0; p < NB; ++p) {
+        dk[p * NB + c] = di[p][c];
+        if (p < bk && c < bk && p <= c) g[(int64_t)(o + p) * r + o + c] = a[p][c];
+    }
+}
 
-    for (int c = tid; c < r; c += CH_THREADS) {
-        for (int i = r - 1; i >= 0; --i) {
-            double x = 0.0;
-            if (i <= c) {
-                const double rii = g[(int64_t)i * r + i];
-                if (rii != 0.0) {
-                    double s = i == c ? 1.0 : 0.0;
-                    for (int m = i + 1; m <= c; ++m)
-                        s -= g[(int64_t)i * r + m] * ri[(int64_t)m * r + c];
-                    x = s / rii;
-                }
-            }
-            ri[(int64_t)i * r + c] = x;
-            ro[(int64_t)i * r + c] = (float)x;
-        }
+// 64 x 64 block product: acc[i][j] += sum_q Lm[q][row_i] * Rm[q][col_j] (the left
+// operand stored transposed) over q < nq, for the thread's 4 x 4 outputs.
+__device__ __forceinline__ void mm_tn(const double (*Lm)[NBP], const double (*Rm)[NBP], int nq,
+                                      int ty, int tx, double acc[4][4]) {
+    for (int q = 0; q < nq; ++q) {
+        double a[4], c[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = Lm[q][ty * 4 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[j] = Rm[q][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
     }
+}
+
+__device__ __forceinline__ void load_block(double (*dst)[NBP], const double *src, int64_t ld,
+                                           int rows, int cols) {
+    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+        const int p = e / NB, c = e % NB;
+        dst[p][c] = (p < rows && c < cols) ? src[(int64_t)p * ld + c] : 0.0;
+    }
+}
+
+// Row panel of block row k: R_kj = D_k^T G_kj for every block column j > k.
+__global__ void __launch_bounds__(256) k_trsm_panel(double *__restrict__ G, int r, int k,
+                                                    const double *__restrict__ D) {
+    extern __shared__ double sm[];
+    double (*dv)[NBP] = reinterpret_cast<double (*)[NBP]>(sm);
+    double (*gb)[NBP] = reinterpret_cast<double (*)[NBP]>(sm + NB * NBP);
+    const int b = blockIdx.y, J = k + 1 + blockIdx.x;
+    const int KB = (r + NB - 1) / NB;
+    const int o = k * NB, oj = J * NB, bk = min(NB, r - o), bj = min(NB, r - oj);
+    double *g = G + (int64_t)b * r * r;
+    load_block(dv, D + ((int64_t)b * KB + k) * NB * NB, NB, NB, NB);
+    load_block(gb, g + (int64_t)o * r + oj, r, bk, bj);
+    __syncthreads();
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    double acc[4][4] = {};
+    mm_tn(dv, gb, bk, ty, tx, acc);  // out[p][c] = sum_q D[q][p] G[q][c]
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int p = ty * 4 + i, c = tx * 4 + j;
+            if (p < bk && c < bj) g[(int64_t)(o + p) * r + oj + c] = acc[i][j];
+        }
+}
+
+// Trailing update after block row k: G_IJ -= R_kI^T R_kJ for k < I <= J.
+__global__ void __launch_bounds__(256) k_syrk_update(double *__restrict__ G, int r, int k) {
+    extern __shared__ double sm[];
+    double (*ri)[NBP] = reinterpret_cast<double (*)[NBP]>(sm);
+    double (*rj)[NBP] = reinterpret_cast<double (*)[NBP]>(sm + NB * NBP);
+    const int b = blockIdx.y;
+    const int KB = (r + NB - 1) / NB, m = KB - k - 1;
+    int I = 0, rem = blockIdx.x;            // blockIdx.x -> (I, J), 0 <= I <= J < m
+    while (rem >= m - I) {
+        rem -= m - I;
+        ++I;
+    }
+    const int J = I + rem + k + 1;
+    I += k + 1;
+    const int o = k * NB, oi = I * NB, oj = J * NB;
+    const int bk = min(NB, r - o), bi = min(NB, r - oi), bj = min(NB, r - oj);
+    double *g = G + (int64_t)b * r * r;
+    load_block(ri, g + (int64_t)o * r + oi, r, bk, bi);
+    load_block(rj, g + (int64_t)o * r + oj, r, bk, bj);
+    __syncthreads();
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    double acc[4][4] = {};
+    mm_tn(ri, rj, bk, ty, tx, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int p = ty * 4 + i, c = tx * 4 + j;
+            if (p < bi && c < bj) g[(int64_t)(oi + p) * r + oj + c] -= acc[i][j];
+        }
+}
+
+// Block row i of R^-1 (the block rows below it are done):
+//   X_ii = D_i,  X_iJ = -D_i sum_{K=i+1..J} R_iK X_KJ  (J > i).
+__global__ void __launch_bounds__(256) k_trinv_row(const double *__restrict__ G, int r, int i,
+                                                   const double *__restrict__ D,
+                                                   double *__restrict__ X64,
+                                                   float *__restrict__ X32) {
+    extern __shared__ double sm[];
+    double (*s0)[NBP] = reinterpret_cast<double (*)[NBP]>(sm);
+    double (*s1)[NBP] = reinterpret_cast<double (*)[NBP]>(sm + NB * NBP);
+    const int b = blockIdx.y, J = i + blockIdx.x;
+    const int KB = (r + NB - 1) / NB;
+    const int oi = i * NB, oj = J * NB, bi = min(NB, r - oi), bj = min(NB, r - oj);
+    const double *g = G + (int64_t)b * r * r;
+    double *x = X64 + (int64_t)b * r * r;
+    float *x32 = X32 + (int64_t)b * r * r;
+    const double *di = D + ((int64_t)b * KB + i) * NB * NB;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    double acc[4][4] = {};
+    if (J == i) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = di[(ty * 4 + a) * NB + tx * 4 + c];
+    } else {
+        // T = sum_K R_iK X_KJ, R_iK loaded transposed so that mm_tn applies
+        for (int K = i + 1; K <= J; ++K) {
+            const int oK = K * NB, bK = min(NB, r - oK);
+            for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+                const int q = e / NB, p = e % NB;  // s0[q][p] = R[oi + p][oK + q]
+                s0[q][p] = (p < bi && q < bK) ? g[(int64_t)(oi + p) * r + oK + q] : 0.0;
+            }
+            load_block(s1, x + (int64_t)oK * r + oj, r, bK, bj);
+            __syncthreads();
+            mm_tn(s0, s1, bK, ty, tx, acc);
+            __syncthreads();
+        }
+        // X_iJ = -D_i T: T to shared memory, D_i transposed beside it
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s1[ty * 4 + a][tx * 4 + c] = acc[a][c];
+        for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+            const int q = e / NB, p = e % NB;  // s0[q][p] = D_i[p][q]
+            s0[q][p] = di[p * NB + q];
+        }
+        __syncthreads();
+        double out[4][4] = {};
+        mm_tn(s0, s1, NB, ty, tx, out);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = -out[a][c];
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int p = ty * 4 + a, q = tx * 4 + c;
+            if (p < bi && q < bj) {
+                x[(int64_t)(oi + p) * r + oj + q] = acc[a][c];
+                x32[(int64_t)(oi + p) * r + oj + q] = (float)acc[a][c];
+            }
+        }
+}
+
+// ------------------------------------------------------------ small elementwise kernels
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): about 16 significant bits.
+__global__ void k_split_hi_lo(const float *__restrict__ src, __nv_bfloat16 *__restrict__ hi,
+                              __nv_bfloat16 *__restrict__ lo, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float x = src[i];
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        hi[i] = h;
+        lo[i] = __float2bfloat16_rn(x - __bfloat162float(h));
+    }
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
 }
 
 template <typename T>
 __global__ void k_to_storage(const float *__restrict__ src, T *__restrict__ dst, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
-        store_f32<T>(dst, i, src[i]);
+        dst[i] = from_f32<T>(src[i]);
+}
+
+// Z [B][W·d_kv][r] (fp32) -> Bt [W][B][d_kv][r] (storage dtype)
+template <typename T>
+__global__ void k_store_bt(const float *__restrict__ Z, T *__restrict__ Bt, int B, int W,
+                           int64_t dk, int r) {
+    const int64_t total = (int64_t)B * W * dk * r;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e % r, j = (e / r) % dk, l = (e / (r * dk)) % W, b = e / (r * dk * W);
+        Bt[((l * B + b) * dk + j) * r + i] = from_f32<T>(Z[e]);
+    }
+}
+
+int grid_for(int64_t n) {
+    const int64_t g = (n + 255) / 256;
+    return (int)(g < 8192 ? (g > 0 ? g : 1) : 8192);
 }
 
 // ------------------------------------------------------------------ host side
-Mat dense(const void *p, int64_t rows, int64_t cols) {
-    Mat m{};
-    m.p = p;
-    m.s_r = cols;
-    m.s_c = 1;
-    m.s_b = rows * cols;
-    return m;
-}
+std::mutex g_blas_mu;
 
-template <typename TA, typename TC>
-cudaError_t gemm(const Mat &A, const Mat &B, const Mat &C, int M, int N, int K, int batch,
-                 cudaStream_t s) {
-    const dim3 grid((N + GN - 1) / GN, (M + GM - 1) / GM, batch);
-    k_gemm<TA, TC><<<grid, G_THREADS, 0, s>>>(A, B, C, M, N, K);
-    return cudaGetLastError();
+cublasHandle_t blas_handle() {  // one per device, created on first use (under g_blas_mu)
+    static cublasHandle_t handles[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS)
+        handles[dev] = nullptr;
+    return handles[dev];
 }
-
-struct Scratch {
-    float *y[2], *z[2];
-    double *g, *r64;
-    float *r32;
-};
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-Scratch carve(void *ws, int64_t B, int64_t L, int64_t n, int64_t r) {
-    char *p = (char *)ws;
-    Scratch s;
-    for (int i = 0; i < 2; ++i) {
-        s.y[i] = (float *)p;
-        p += align256((size_t)B * L * r * 4);
-    }
-    for (int i = 0; i < 2; ++i) {
-        s.z[i] = (float *)p;
-        p += align256((size_t)B * n * r * 4);
-    }
-    s.g = (double *)p;
-    p += align256((size_t)B * r * r * 8);
-    s.r64 = (double *)p;
-    p += align256((size_t)B * r * r * 8);
-    s.r32 = (float *)p;
+struct Scratch {
+    float *y[2], *z[2];
+    double *g, *d, *r64, *tol;
+    float *r32;
+    __nv_bfloat16 *hi, *lo, *om_hi;
+};
+
+struct Shape {
+    int B, W, r;
+    int64_t L, dk, n;
+    bool bf16;
+};
+
+Shape shape_of(const xkv_dims &d, int W, int r) {
+    Shape s;
+    s.B = d.batch;
+    s.W = W;
+    s.r = r;
+    s.L = d.ctx_len;
+    s.dk = (int64_t)d.n_kv_heads * d.head_dim;
+    s.n = W * s.dk;
+    s.bf16 = d.dtype == XKV_BF16;
     return s;
 }
 
-// CholeskyQR2 of the `rows` x r matrices of every sequence in buf[0]; buf[1] is the
-// other half of the ping-pong, and the result ends in buf[0].
-cudaError_t orth(float *const buf[2], int64_t rows, int r, int B, const Scratch &sc,
-                 cudaStream_t s) {
-    const int T = (r + GR_T - 1) / GR_T;
-    int n_split = (int)((rows + 1023) / 1024);
-    const int cap = 65535 / B;
-    if (n_split > cap) n_split = cap;
-    const int rps = (int)((rows + n_split - 1) / n_split);
-    for (int pass = 0; pass < 2; ++pass) {
-        float *src = buf[pass], *dst = buf[pass ^ 1];
-        cudaError_t e = cudaMemsetAsync(sc.g, 0, (size_t)B * r * r * sizeof(double), s);
-        if (e != cudaSuccess) return e;
-        k_gram<<<dim3(T, T, B * n_split), 256, 0, s>>>(src, (int)rows, r, rps, n_split, sc.g);
-        k_chol_inv<<<B, CH_THREADS, 0, s>>>(sc.g, r, sc.r64, sc.r32);
-        Mat Rm = dense(sc.r32, r, r);
-        e = gemm<float, float>(dense(src, rows, r), Rm, dense(dst, rows, r), (int)rows, r, r,
-                               B, s);
-        if (e != cudaSuccess) return e;
+// Lays the scratch out in ws (when given) and returns its size.
+size_t carve(const Shape &s, void *ws, Scratch *out) {
+    char *p = (char *)ws;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *q = p ? p + off : nullptr;
+        off += align256(bytes);
+        return q;
+    };
+    const int64_t B = s.B, r = s.r, KB = (r + NB - 1) / NB;
+    const int64_t rows_max = s.L > s.n ? s.L : s.n;
+    Scratch sc{};
+    for (int i = 0; i < 2; ++i) sc.y[i] = (float *)take((size_t)B * s.L * r * 4);
+    for (int i = 0; i < 2; ++i) sc.z[i] = (float *)take((size_t)B * s.n * r * 4);
+    sc.g = (double *)take((size_t)B * r * r * 8);
+    sc.d = (double *)take((size_t)B * KB * NB * NB * 8);
+    sc.r64 = (double *)take((size_t)B * r * r * 8);
+    sc.tol = (double *)take((size_t)B * 8);
+    sc.r32 = (float *)take((size_t)B * r * r * 4);
+    if (s.bf16) {
+        sc.hi = (__nv_bfloat16 *)take((size_t)B * rows_max * r * 2);
+        sc.lo = (__nv_bfloat16 *)take((size_t)B * rows_max * r * 2);
+        sc.om_hi = (__nv_bfloat16 *)take((size_t)s.n * r * 2);
     }
-    return cudaGetLastError();
+    if (out) *out = sc;
+    return off;
+}
+
+// Row-major C = op(A) op(B) (M x N, inner K) in fp32, batched over sequences.
+cublasStatus_t rm_gemm(cublasHandle_t h, bool tA, bool tB, int M, int N, int K, const void *A,
+                       cudaDataType ta, int lda, long long sA, const void *Bm, cudaDataType tb,
+                       int ldb, long long sB, void *C, int ldc, long long sC, int batch,
+                       float beta, cublasComputeType_t ct) {
+    const float alpha = 1.f;
+    return cublasGemmStridedBatchedEx(h, tB ? CUBLAS_OP_T : CUBLAS_OP_N,
+                                      tA ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, Bm, tb,
+                                      ldb, sB, A, ta, lda, sA, &beta, C, CUDA_R_32F, ldc, sC,
+                                      batch, ct, CUBLAS_GEMM_DEFAULT);
+}
+
+struct Run {
+    Shape s;
+    Scratch sc;
+    cublasHandle_t h;
+    cudaStream_t st;
+    const void *X;
+    cudaDataType xt;
+    cublasComputeType_t exact;   // the products with X
+    cublasComputeType_t apply;   // the products with R^-1
+    cudaError_t err = cudaSuccess;
+    bool blas_ok = true;
+
+    bool ok() const { return err == cudaSuccess && blas_ok; }
+    void check(cublasStatus_t b) {
+        if (b != CUBLAS_STATUS_SUCCESS) blas_ok = false;
+    }
+    void check(cudaError_t e) {
+        if (e != cudaSuccess && err == cudaSuccess) err = e;
+    }
+    const char *xl(int l) const {  // layer l's cache [B][L][d_kv]
+        return (const char *)X + (size_t)l * s.B * s.L * s.dk * (s.bf16 ? 2 : 4);
+    }
+
+    void split(const float *src, int64_t n) {
+        k_split_hi_lo<<<grid_for(n), 256, 0, st>>>(src, sc.hi, sc.lo, n);
+        check(cudaGetLastError());
+    }
+
+    // Y = sum_l X_l F_l, F [B][n][r] fp32; F == nullptr: the test matrix (shared by the
+    // sequences; bf16 caches read its bf16 copy)
+    void x_times(const float *F, const float *omega, float *Y) {
+        const int B = s.B, r = s.r;
+        for (int l = 0; l < s.W && ok(); ++l) {
+            if (s.bf16) {
+                if (F && l == 0) split(F, (int64_t)B * s.n * r);
+                const int parts = F ? 2 : 1;
+                for (int part = 0; part < parts && ok(); ++part) {
+                    const __nv_bfloat16 *f = F ? (part ? sc.lo : sc.hi) + (size_t)l * s.dk * r
+                                               : sc.om_hi + (size_t)l * s.dk * r;
+                    check(rm_gemm(h, false, false, (int)s.L, r, (int)s.dk, xl(l), xt, (int)s.dk,
+                                  s.L * s.dk, f, CUDA_R_16BF, r, F ? s.n * r : 0, Y, r, s.L * r,
+                                  B, (l || part) ? 1.f : 0.f, exact));
+                }
+            } else {
+                const float *f = (F ? F : omega) + (size_t)l * s.dk * r;
+                check(rm_gemm(h, false, false, (int)s.L, r, (int)s.dk, xl(l), xt, (int)s.dk,
+                              s.L * s.dk, f, CUDA_R_32F, r, F ? s.n * r : 0, Y, r, s.L * r, B,
+                              l ? 1.f : 0.f, exact));
+            }
+        }
+    }
+
+    // Z_l = X_l^T Q for every layer: Z [B][n][r] fp32
+    void xt_times(const float *Q, float *Z) {
+        const int B = s.B, r = s.r;
+        if (s.bf16) split(Q, (int64_t)B * s.L * r);
+        for (int l = 0; l < s.W && ok(); ++l) {
+            if (s.bf16) {
+                for (int part = 0; part < 2 && ok(); ++part)
+                    check(rm_gemm(h, true, false, (int)s.dk, r, (int)s.L, xl(l), xt, (int)s.dk,
+                                  s.L * s.dk, part ? sc.lo : sc.hi, CUDA_R_16BF, r, s.L * r,
+                                  Z + (size_t)l * s.dk * r, r, s.n * r, B, part ? 1.f : 0.f,
+                                  exact));
+            } else {
+                check(rm_gemm(h, true, false, (int)s.dk, r, (int)s.L, xl(l), xt, (int)s.dk,
+                              s.L * s.dk, Q, CUDA_R_32F, r, s.L * r, Z + (size_t)l * s.dk * r,
+                              r, s.n * r, B, 0.f, exact));
+            }
+        }
+    }
+
+    // CholeskyQR2 of the rows x r matrices in buf[0] (buf[1]: the other ping-pong half);
+    // the result ends in buf[0]
+    void orth(float *const buf[2], int64_t rows) {
+        const int B = s.B, r = s.r, KB = (r + NB - 1) / NB, T = (r + GR_T - 1) / GR_T;
+        int n_split = (int)((rows + 1023) / 1024);
+        const int cap = 65535 / B;
+        if (n_split > cap) n_split = cap;
+        const int rps = (int)((rows + n_split - 1) / n_split);
+        const size_t blk_smem = 2 * NB * NBP * sizeof(double);
+        for (int pass = 0; pass < 2 && ok(); ++pass) {
+            float *src = buf[pass], *dst = buf[pass ^ 1];
+            check(cudaMemsetAsync(sc.g, 0, (size_t)B * r * r * sizeof(double), st));
+            check(cudaMemsetAsync(sc.r64, 0, (size_t)B * r * r * sizeof(double), st));
+            check(cudaMemsetAsync(sc.r32, 0, (size_t)B * r * r * sizeof(float), st));
+            k_gram<<<dim3(T, T, B * n_split), 256, 0, st>>>(src, (int)rows, r, rps, n_split,
+                                                            sc.g);
+            k_maxdiag<<<B, 256, 0, st>>>(sc.g, r, sc.tol);
+            for (int k = 0; k < KB; ++k) {
+                k_potrf_diag<<<B, NB, blk_smem, st>>>(sc.g, r, k, sc.tol, sc.d);
+                const int m = KB - k - 1;
+                if (m > 0) {
+                    k_trsm_panel<<<dim3(m, B), 256, blk_smem, st>>>(sc.g, r, k, sc.d);
+                    k_syrk_update<<<dim3(m * (m + 1) / 2, B), 256, blk_smem, st>>>(sc.g, r, k);
+                }
+            }
+            for (int i = KB - 1; i >= 0; --i)
+                k_trinv_row<<<dim3(KB - i, B), 256, blk_smem, st>>>(sc.g, r, i, sc.d, sc.r64,
+                                                                    sc.r32);
+            check(cudaGetLastError());
+            if (!ok()) return;
+            check(rm_gemm(h, false, false, (int)rows, r, r, src, CUDA_R_32F, r, rows * r,
+                          sc.r32, CUDA_R_32F, r, (long long)r * r, dst, r, rows * r, B, 0.f,
+                          apply));
+        }
+    }
+};
+
+cudaError_t set_block_smem() {
+    const size_t bytes = 2 * NB * NBP * sizeof(double);
+    cudaError_t e = set_smem_limit((const void *)k_potrf_diag, bytes);
+    if (e == cudaSuccess) e = set_smem_limit((const void *)k_trsm_panel, bytes);
+    if (e == cudaSuccess) e = set_smem_limit((const void *)k_syrk_update, bytes);
+    if (e == cudaSuccess) e = set_smem_limit((const void *)k_trinv_row, bytes);
+    return e;
 }
 
 template <typename T>
-cudaError_t factorize_t(const xkv_dims &d, int W, int r, const void *X, const float *omega,
-                        int n_iter, void *A_out, void *Bt_out, void *ws, cudaStream_t s) {
-    const int B = d.batch;
-    const int64_t L = d.ctx_len, dk = (int64_t)d.n_kv_heads * d.head_dim, n = W * dk;
-    const Scratch sc = carve(ws, B, L, n, r);
-    // X as L x n (token rows, layer-major feature columns) and as its transpose
-    Mat Xr{};
-    Xr.p = X;
-    Xr.s_r = dk;
-    Xr.s_c = 1;
-    Xr.s_b = L * dk;
-    Xr.blk_c = (int32_t)dk;
-    Xr.jump_c = (int64_t)B * L * dk - dk;
-    Mat Xt{};
-    Xt.p = X;
-    Xt.s_r = 1;
-    Xt.s_c = dk;
-    Xt.s_b = L * dk;
-    Xt.blk_r = (int32_t)dk;
-    Xt.jump_r = (int64_t)B * L * dk - dk;
-    Mat Om = dense(omega, n, r);
-    Om.s_b = 0;
-    const Mat Y = dense(sc.y[0], L, r), Z = dense(sc.z[0], n, r);
-
-    cudaError_t e = gemm<T, float>(Xr, Om, Y, (int)L, r, (int)n, B, s);
-    if (e == cudaSuccess) e = orth(sc.y, L, r, B, sc, s);
-    for (int it = 0; it < n_iter && e == cudaSuccess; ++it) {
-        e = gemm<T, float>(Xt, Y, Z, (int)n, r, (int)L, B, s);
-        if (e == cudaSuccess) e = orth(sc.z, n, r, B, sc, s);
-        if (e == cudaSuccess) e = gemm<T, float>(Xr, Z, Y, (int)L, r, (int)n, B, s);
-        if (e == cudaSuccess) e = orth(sc.y, L, r, B, sc, s);
-    }
+cudaError_t factorize_t(const Shape &s, const void *X, const float *omega, int n_iter,
+                        void *A_out, void *Bt_out, void *ws, cudaStream_t st) {
+    cudaError_t e = set_block_smem();
     if (e != cudaSuccess) return e;
-    const int64_t na = (int64_t)B * L * r;
-    k_to_storage<T><<<(int)((na + 255) / 256 < 65535 ? (na + 255) / 256 : 65535), 256, 0, s>>>(
-        sc.y[0], (T *)A_out, na);
-    // B_l^T = X_l^T A, written as [W][B][d_kv][r]
-    Mat Bt{};
-    Bt.p = Bt_out;
-    Bt.s_r = r;
-    Bt.s_c = 1;
-    Bt.s_b = dk * r;
-    Bt.blk_r = (int32_t)dk;
-    Bt.jump_r = ((int64_t)B * dk - dk) * r;
-    return gemm<T, T>(Xt, Y, Bt, (int)n, r, (int)L, B, s);
+    std::lock_guard<std::mutex> lock(g_blas_mu);
+    cublasHandle_t h = blas_handle();
+    if (!h || cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return cudaErrorNotReady;
+    Run run;
+    run.s = s;
+    carve(s, ws, &run.sc);
+    run.h = h;
+    run.st = st;
+    run.X = X;
+    run.xt = s.bf16 ? CUDA_R_16BF : CUDA_R_32F;
+    // bf16 x bf16 products are exact in fp32, so the tensor cores lose nothing there;
+    // fp32 caches keep every product in plain fp32
+    run.exact = s.bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC;
+    run.apply = s.bf16 ? CUBLAS_COMPUTE_32F_FAST_TF32 : CUBLAS_COMPUTE_32F_PEDANTIC;
+    const int B = s.B, r = s.r;
+    const Scratch &sc = run.sc;
+
+    if (s.bf16) {
+        k_split_hi_lo<<<grid_for(s.n * r), 256, 0, st>>>(omega, sc.om_hi, sc.lo, s.n * r);
+        run.check(cudaGetLastError());
+    }
+    run.x_times(nullptr, omega, sc.y[0]);
+    if (run.ok()) run.orth(sc.y, s.L);
+    for (int it = 0; it < n_iter && run.ok(); ++it) {
+        run.xt_times(sc.y[0], sc.z[0]);
+        if (run.ok()) run.orth(sc.z, s.n);
+        if (run.ok()) run.x_times(sc.z[0], omega, sc.y[0]);
+        if (run.ok()) run.orth(sc.y, s.L);
+    }
+    if (run.ok()) {
+        const int64_t na = (int64_t)B * s.L * r;
+        k_to_storage<T><<<grid_for(na), 256, 0, st>>>(sc.y[0], (T *)A_out, na);
+        run.check(cudaGetLastError());
+        run.xt_times(sc.y[0], sc.z[0]);
+        const int64_t nb = (int64_t)B * s.n * r;
+        if (run.ok())
+            k_store_bt<T><<<grid_for(nb), 256, 0, st>>>(sc.z[0], (T *)Bt_out, B, s.W, s.dk, r);
+        run.check(cudaGetLastError());
+    }
+    if (run.err != cudaSuccess) return run.err;
+    return run.blas_ok ? cudaSuccess : cudaErrorUnknown;
 }
 
 }  // namespace
 
 size_t factorize_ws_bytes(const xkv_dims &d, int W, int r) {
-    const int64_t B = d.batch, L = d.ctx_len, n = (int64_t)W * d.n_kv_heads * d.head_dim;
-    return 2 * align256((size_t)B * L * r * 4) + 2 * align256((size_t)B * n * r * 4) +
-           2 * align256((size_t)B * r * r * 8) + align256((size_t)B * r * r * 4);
+    return carve(shape_of(d, W, r), nullptr, nullptr);
 }
 
 cudaError_t launch_factorize(const xkv_dims &d, int W, int r, const void *X, const float *omega,
                              int n_iter, void *A_out, void *Bt_out, void *ws, cudaStream_t s) {
-    return d.dtype == XKV_F32
-               ? factorize_t<float>(d, W, r, X, omega, n_iter, A_out, Bt_out, ws, s)
-               : factorize_t<__nv_bfloat16>(d, W, r, X, omega, n_iter, A_out, Bt_out, ws, s);
+    const Shape sh = shape_of(d, W, r);
+    return sh.bf16 ? factorize_t<__nv_bfloat16>(sh, X, omega, n_iter, A_out, Bt_out, ws, s)
+                   : factorize_t<float>(sh, X, omega, n_iter, A_out, Bt_out, ws, s);
 }
 
 }  // namespace xkv

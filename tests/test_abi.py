@@ -253,8 +253,11 @@ def test_factorize_pointer_and_workspace_checks(xkv):
 
     def al(x):
         return (x + 255) // 256 * 256
-    assert need == 2 * al(B * L * r * 4) + 2 * al(B * n * r * 4) + 2 * al(B * r * r * 8) + \
-        al(B * r * r * 4)
+    # Y and Z ping-pong (fp32); Gram, diagonal-block inverses, R^-1 (fp64); tolerances;
+    # R^-1 (fp32); bf16 hi / lo splits and the bf16 test matrix
+    assert need == (2 * al(B * L * r * 4) + 2 * al(B * n * r * 4) + al(B * r * r * 8)
+                    + al(B * 1 * 64 * 64 * 8) + al(B * r * r * 8) + al(B * 8) + al(B * r * r * 4)
+                    + 2 * al(B * max(L, n) * r * 2) + al(n * r * 2))
     assert xkv.xkv_factorize_workspace_bytes(d, 2, 40) == 0
     args = [FAKE] * 2
     assert xkv.xkv_factorize_window(d, 2, 32, 0, FAKE, 1, FAKE, FAKE, FAKE, need, stream=0,
