@@ -438,18 +438,29 @@ CLF = dict(window=4, batch=8, ctx_len=32768, n_kv_heads=8, head_dim=128, rank_k=
            rank_v=768, n_iter=2, tau=128.0, gap=0.1)
 CLF_METRIC = ("prefill cross-layer factorization tokens/s (window of 4 layers, K and V "
               "caches, 32K ctx)")
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz (max clock)
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# fp64 FMA peak of the CUDA cores: 148 SMs x 64 fp64 FMA per clock x 2 flop x 1.965 GHz
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+TF32_OVER_BF16 = 1.1 / 2.25                      # nominal dense tf32 : bf16 ratio
 
 
-def clf_flops(c, r):
-    """(fp32 GEMM flops, fp64 Gram flops) of one factorization call of rank r."""
-    B, L, q = c["batch"], c["ctx_len"], c["n_iter"]
-    n = c["window"] * c["n_kv_heads"] * c["head_dim"]
-    orth_rows = L * (1 + q) + n * q              # rows of every matrix orthonormalised
-    gemm = 2 * B * (L * r * n * (2 + 2 * q) + 2 * r * r * orth_rows)
-    gram = 2 * B * orth_rows * r * (r + 1)       # two CholeskyQR passes, r(r+1)/2 dots
-    return gemm, gram
+def clf_work(c, r):
+    """Work of one bf16 factorization call of rank r, by arithmetic unit, and its launch
+    counts.  Passes of CholeskyQR: the first and intermediate bases one each, the final
+    basis two; every pass is a Gram matrix (fp64), a blocked Cholesky and inverse, and a
+    product with R^-1 (TF32)."""
+    B, L, q, W = c["batch"], c["ctx_len"], c["n_iter"], c["window"]
+    n = W * c["n_kv_heads"] * c["head_dim"]
+    KB = (r + 63) // 64
+    y_pass = 2 if q == 0 else 1 + q + 1          # passes over L-row bases
+    z_pass = q                                   # passes over n-row bases
+    pass_rows = y_pass * L + z_pass * n
+    bf16 = 2 * B * L * r * n * (1 + 4 * q + 2)   # X products: test matrix 1 part, others hi+lo
+    tf32 = 2 * B * r * r * pass_rows
+    fp64 = B * r * (r + 1) * pass_rows           # Gram matrices: r(r+1)/2 dot products
+    own = (2 + 2 * q) + 2 + (y_pass + z_pass) * 4 * KB
+    blas = W + 4 * q * W + 2 * W + (y_pass + z_pass)
+    return {"bf16": bf16, "tf32": tf32, "fp64": fp64, "own_launches": own,
+            "blas_calls": blas}
 
 
 def clf_cpu_baseline(c, seed, rows=2048):
@@ -525,8 +536,10 @@ def run_clf(args, rank, world):
         for i, k in enumerate(calls):
             if events is not None:
                 events[i][0].record(stream)
+            torch.cuda.nvtx.range_push("xkv_factorize")    # lets a profiler skip the setup
             xkv.xkv_factorize_window(d, W, k["r"], k["X"], k["om"], c["n_iter"], k["A"], k["Bt"],
                                      ws)
+            torch.cuda.nvtx.range_pop()
             if events is not None:
                 events[i][1].record(stream)
 
@@ -594,30 +607,38 @@ def run_clf(args, rank, world):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = clf_cpu_baseline(c, args.seed)
     if rank == 0:
-        # the V call (rank 768) is the larger; its fp32 GEMM rate over the whole call
-        # (Gram and Cholesky kernels included) is a lower bound for the GEMM kernel's
-        g_flops, gram_flops = clf_flops(c, c["rank_v"])
-        tflops = g_flops / (call_ms[1] / 1e3) / 1e12
+        # Roofline of the whole V call (rank 768, the larger): the time its work needs on
+        # each unit at that unit's peak -- bf16 products at the measured sustained bf16
+        # rate, TF32 products at the nominal fraction of it, the fp64 Gram matrices at the
+        # fp64 peak derived from unit counts and clock -- against the measured time.
+        wv = clf_work(c, c["rank_v"])
+        bf16_peak, bf16_kind = measured_tflops_sustained()
+        t_ideal = (wv["bf16"] / (bf16_peak * 1e12) + wv["tf32"] / (bf16_peak * TF32_OVER_BF16 * 1e12)
+                   + wv["fp64"] / (FP64_PEAK_TFLOPS * 1e12))
+        flops = wv["bf16"] + wv["tf32"] + wv["fp64"]
+        t_call = call_ms[1] / 1e3
         line = {
             "metric": CLF_METRIC, "value": B * L * world * args.steps / (elapsed_ms / 1e3),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": CLF_WORKLOAD, **c, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {2 * calls[0]['X'].numel() * 2 / 1e9:.1f} "
                              "GB of caches per step"},
             "roofline": {"bound": "alu", "kernel": "factorize_window (rank 768 call, whole)",
-                         "achieved": tflops, "peak": FP32_PEAK_TFLOPS,
-                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
-                         "unit": "TFLOP/s", "frac": tflops / FP32_PEAK_TFLOPS, "traffic": None,
-                         "flops_per_launch": g_flops, "fp64_gram_flops": gram_flops,
-                         "avg_launch_ms": call_ms[1], "rank_512_call_ms": call_ms[0]},
-            "gpu_launches": None, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+                         "achieved": flops / t_call / 1e12, "peak": flops / t_ideal / 1e12,
+                         "peak_kind": f"composite: bf16 {bf16_kind} {bf16_peak}, tf32 x"
+                                      f"{TF32_OVER_BF16:.2f} of it, fp64 derived "
+                                      f"{FP64_PEAK_TFLOPS:.1f} (148 SMs x 64 FMA x 2 x 1.965 GHz)",
+                         "unit": "TFLOP/s", "frac": t_ideal / t_call, "traffic": None,
+                         "flops_bf16": wv["bf16"], "flops_tf32": wv["tf32"],
+                         "flops_fp64": wv["fp64"], "avg_launch_ms": call_ms[1],
+                         "rank_512_call_ms": call_ms[0]},
+            "gpu_launches": sum(clf_work(c, k["r"])["own_launches"] for k in calls) * args.steps,
+            "library_gemm_calls": sum(clf_work(c, k["r"])["blas_calls"] for k in calls)
+                                  * args.steps,
+            "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }
-        q = c["n_iter"]
-        orths = 1 + 2 * q
-        per_call_launches = (2 + 2 * q) + orths * 2 * 3 + 1     # GEMMs, Gram/Cholesky/apply, store
-        line["gpu_launches"] = per_call_launches * 2 * args.steps
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

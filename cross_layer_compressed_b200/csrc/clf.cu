@@ -17,8 +17,9 @@
 // SVD's product; A itself is one orthonormal basis of that subspace, not U_r (the two
 // differ by an r x r rotation that no product sees).
 //
-// orth() is CholeskyQR2: twice G = Y^T Y (fp64), G = R^T R (blocked Cholesky, fp64),
-// Y <- Y R^-1 (R^-1 by blocked triangular inversion, fp64).  A column whose Cholesky
+// orth() is CholeskyQR: G = Y^T Y (fp64), G = R^T R (blocked Cholesky, fp64), Y <- Y R^-1
+// (R^-1 by blocked triangular inversion, fp64); twice (CholeskyQR2) for the returned
+// basis, once for the intermediate ones, which only have to stay well conditioned.  A column whose Cholesky
 // pivot is below 1e-12 of the largest diagonal entry of G (a direction the data does
 // not have: rank(X) < r) is zeroed rather than normalised.
 //
@@ -42,56 +43,76 @@ constexpr int NB = 64;         // block size of the Cholesky factorization and i
 constexpr int NBP = NB + 1;    // padded shared-memory row
 
 // ------------------------------------------------------------------ fp64 Gram
-// G[b] += Y[b]^T Y[b] over one slice of rows, for the 64 x 64 tiles on or above the
-// diagonal (the factorization reads the upper triangle only).  fp32 x fp32 products are
-// exact in fp64; the slices meet through fp64 atomics.
-constexpr int GR_T = 64, GR_ROWS = 32;
+// G[b] += Y[b]^T Y[b] over one slice of rows, for the 128 x 128 tiles on or above the
+// diagonal (the factorization reads the upper triangle only).  Rows are staged in
+// shared memory already widened to fp64 (fp32 x fp32 products are exact in fp64); each
+// thread owns 8 x 8 outputs (rows and columns 16 apart), so a row step costs 16
+// conflict-free shared loads per 64 fp64 FMAs.  The slices meet through fp64 atomics.
+constexpr int GR_T = 128, GR_ROWS = 16, GR_THREADS = 256;
 
-__global__ void __launch_bounds__(256) k_gram(const float *__restrict__ Y, int rows, int r,
-                                              int rows_per_split, int n_split,
-                                              double *__restrict__ G) {
+__global__ void __launch_bounds__(GR_THREADS) k_gram(const float *__restrict__ Y, int rows, int r,
+                                                     int rows_per_split, int n_split,
+                                                     double *__restrict__ G) {
     const int ti = blockIdx.y, tj = blockIdx.x;
     if (tj < ti) return;
     const int b = blockIdx.z / n_split, sp = blockIdx.z % n_split;
-    __shared__ float Yi[GR_ROWS][GR_T + 1], Yj[GR_ROWS][GR_T + 1];
+    __shared__ __align__(16) double Yi[GR_ROWS][GR_T], Yj[GR_ROWS][GR_T];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const float *y = Y + (int64_t)b * rows * r;
     const int t_lo = sp * rows_per_split;
     const int t_hi = min(rows, t_lo + rows_per_split);
-    double acc[4][4];
+    double acc[8][8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int t0 = t_lo; t0 < t_hi; t0 += GR_ROWS) {
-        for (int e = tid; e < GR_ROWS * GR_T; e += 256) {
-            const int tt = e / GR_T, c = e % GR_T, t = t0 + tt;
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    // the next slice's values wait in registers while this one is multiplied (one CTA
+    // per SM: nothing else would hide the loads)
+    constexpr int PER = GR_ROWS * GR_T / GR_THREADS;
+    float ni[PER], nj[PER];
+    auto fetch = [&](int t0) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * GR_THREADS, tt = e / GR_T, c = e % GR_T, t = t0 + tt;
             const int ci = ti * GR_T + c, cj = tj * GR_T + c;
-            Yi[tt][c] = (t < t_hi && ci < r) ? y[(int64_t)t * r + ci] : 0.f;
-            Yj[tt][c] = (t < t_hi && cj < r) ? y[(int64_t)t * r + cj] : 0.f;
+            ni[u] = (t < t_hi && ci < r) ? y[(int64_t)t * r + ci] : 0.f;
+            nj[u] = (t < t_hi && cj < r) ? y[(int64_t)t * r + cj] : 0.f;
+        }
+    };
+    fetch(t_lo);
+    for (int t0 = t_lo; t0 < t_hi; t0 += GR_ROWS) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * GR_THREADS, tt = e / GR_T, c = e % GR_T;
+            Yi[tt][c] = (double)ni[u];
+            Yj[tt][c] = (double)nj[u];
         }
         __syncthreads();
-#pragma unroll 4
+        if (t0 + GR_ROWS < t_hi) fetch(t0 + GR_ROWS);
+#pragma unroll 2
         for (int tt = 0; tt < GR_ROWS; ++tt) {
-            double a[4], c[4];
+            // rows ty + 16 i and columns tx + 16 j: a warp's loads are 128 contiguous
+            // bytes (columns) or broadcasts (rows), one shared-memory wavefront each
+            double a[8], c[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = (double)Yi[tt][ty * 4 + i];
+            for (int i = 0; i < 8; ++i) {
+                a[i] = Yi[tt][ty + 16 * i];
+                c[i] = Yj[tt][tx + 16 * i];
+            }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) c[j] = (double)Yj[tt][tx * 4 + j];
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
         }
         __syncthreads();
     }
     double *g = G + (int64_t)b * r * r;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int gi = ti * GR_T + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int gi = ti * GR_T + ty + 16 * i;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int gj = tj * GR_T + tx * 4 + j;
+        for (int j = 0; j < 8; ++j) {
+            const int gj = tj * GR_T + tx + 16 * j;
             if (gi < r && gj < r && gi <= gj) atomicAdd(&g[(int64_t)gi * r + gj], acc[i][j]);
         }
     }
@@ -119,22 +140,25 @@ __global__ void __launch_bounds__(256) k_maxdiag(const double *__restrict__ G, i
 // Diagonal block k: unblocked right-looking Cholesky in shared memory (one thread per
 // column), then the block's inverse D_k = R_kk^-1 by back substitution.  A dependent
 // pivot gives a zero row of R and a zero row and column of D_k.
-__global__ void __launch_bounds__(NB) k_potrf_diag(double *__restrict__ G, int r, int k,
-                                                   const double *__restrict__ tol,
-                                                   double *__restrict__ D) {
+__global__ void __launch_bounds__(256) k_potrf_diag(double *__restrict__ G, int r, int k,
+                                                    const double *__restrict__ tol,
+                                                    double *__restrict__ D) {
     extern __shared__ double sm[];
     double (*a)[NBP] = reinterpret_cast<double (*)[NBP]>(sm);
     double (*di)[NBP] = reinterpret_cast<double (*)[NBP]>(sm + NB * NBP);
     __shared__ int s_dep;
-    const int b = blockIdx.x, c = threadIdx.x, o = k * NB;
+    const int b = blockIdx.x, tid = threadIdx.x, o = k * NB;
     const int bk = min(NB, r - o);
     double *g = G + (int64_t)b * r * r;
-    for (int p = 0; p < NB; ++p)
+    for (int e = tid; e < NB * NB; e += blockDim.x) {       // coalesced block copy
+        const int p = e / NB, c = e % NB;
         a[p][c] = (p < bk && c < bk && p <= c) ? g[(int64_t)(o + p) * r + o + c] : 0.0;
+    }
     const double t = tol[b];
     __syncthreads();
+    const int c = tid;                                      // threads 0..63: one column each
     for (int j = 0; j < bk; ++j) {
-        if (c == 0) {
+        if (tid == 0) {
             const double pv = a[j][j];
             const int dep = !(pv > t);  // NaN counts as dependent too
             s_dep = dep;
@@ -148,20 +172,28 @@ __global__ void __launch_bounds__(NB) k_potrf_diag(double *__restrict__ G, int r
             for (int i = j + 1; i <= c; ++i) a[i][c] -= a[j][i] * a[j][c];
         __syncthreads();
     }
-    for (int i = NB - 1; i >= 0; --i) {
-        double x = 0.0;
-        if (i <= c && c < bk && a[i][i] != 0.0) {
-            double s = i == c ? 1.0 : 0.0;
-            for (int m = i + 1; m <= c; ++m) s -= a[i][m] * di[m][c];
-            x = s / a[i][i];
+    // D = R_kk^-1 by back substitution, all 64 columns at once: four adjacent lanes per
+    // column split each dot product
+    {
+        const int cc = tid >> 2, q = tid & 3;
+        for (int i = NB - 1; i >= 0; --i) {
+            double part = 0.0;
+            if (i < cc)
+                for (int m = i + 1 + q; m <= cc; m += 4) part += a[i][m] * di[m][cc];
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            double x = 0.0;
+            if (i <= cc && cc < bk && a[i][i] != 0.0) x = ((i == cc ? 1.0 : 0.0) - part) / a[i][i];
+            if (q == 0) di[i][cc] = x;
+            __syncwarp();
         }
-        di[i][c] = x;
     }
     __syncthreads();
     double *dk = D + ((int64_t)b * ((r + NB - 1) / NB) + k) * NB * NB;
-    for (int p = 0; p < NB; ++p) {
-        dk[p * NB + c] = di[p][c];
-        if (p < bk && c < bk && p <= c) g[(int64_t)(o + p) * r + o + c] = a[p][c];
+    for (int e = tid; e < NB * NB; e += blockDim.x) {
+        const int p = e / NB, q = e % NB;
+        dk[e] = di[p][q];
+        if (p < bk && q < bk && p <= q) g[(int64_t)(o + p) * r + o + q] = a[p][q];
     }
 }
 
@@ -505,25 +537,25 @@ struct Run {
         }
     }
 
-    // CholeskyQR2 of the rows x r matrices in buf[0] (buf[1]: the other ping-pong half);
-    // the result ends in buf[0]
-    void orth(float *const buf[2], int64_t rows) {
+    // CholeskyQR of the rows x r matrices in buf[0] (buf[1]: the other ping-pong half),
+    // `passes` times (2: CholeskyQR2); the result ends in buf[0]
+    void orth(float *buf[2], int64_t rows, int passes) {
         const int B = s.B, r = s.r, KB = (r + NB - 1) / NB, T = (r + GR_T - 1) / GR_T;
         int n_split = (int)((rows + 1023) / 1024);
         const int cap = 65535 / B;
         if (n_split > cap) n_split = cap;
         const int rps = (int)((rows + n_split - 1) / n_split);
         const size_t blk_smem = 2 * NB * NBP * sizeof(double);
-        for (int pass = 0; pass < 2 && ok(); ++pass) {
-            float *src = buf[pass], *dst = buf[pass ^ 1];
+        for (int pass = 0; pass < passes && ok(); ++pass) {
+            float *src = buf[0], *dst = buf[1];
             check(cudaMemsetAsync(sc.g, 0, (size_t)B * r * r * sizeof(double), st));
             check(cudaMemsetAsync(sc.r64, 0, (size_t)B * r * r * sizeof(double), st));
             check(cudaMemsetAsync(sc.r32, 0, (size_t)B * r * r * sizeof(float), st));
-            k_gram<<<dim3(T, T, B * n_split), 256, 0, st>>>(src, (int)rows, r, rps, n_split,
-                                                            sc.g);
+            k_gram<<<dim3(T, T, B * n_split), GR_THREADS, 0, st>>>(src, (int)rows, r, rps,
+                                                                   n_split, sc.g);
             k_maxdiag<<<B, 256, 0, st>>>(sc.g, r, sc.tol);
             for (int k = 0; k < KB; ++k) {
-                k_potrf_diag<<<B, NB, blk_smem, st>>>(sc.g, r, k, sc.tol, sc.d);
+                k_potrf_diag<<<B, 256, blk_smem, st>>>(sc.g, r, k, sc.tol, sc.d);
                 const int m = KB - k - 1;
                 if (m > 0) {
                     k_trsm_panel<<<dim3(m, B), 256, blk_smem, st>>>(sc.g, r, k, sc.d);
@@ -538,6 +570,8 @@ struct Run {
             check(rm_gemm(h, false, false, (int)rows, r, r, src, CUDA_R_32F, r, rows * r,
                           sc.r32, CUDA_R_32F, r, (long long)r * r, dst, r, rows * r, B, 0.f,
                           apply));
+            buf[0] = dst;
+            buf[1] = src;
         }
     }
 };
@@ -571,19 +605,22 @@ cudaError_t factorize_t(const Shape &s, const void *X, const float *omega, int n
     run.exact = s.bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC;
     run.apply = s.bf16 ? CUBLAS_COMPUTE_32F_FAST_TF32 : CUBLAS_COMPUTE_32F_PEDANTIC;
     const int B = s.B, r = s.r;
-    const Scratch &sc = run.sc;
+    const Scratch &sc = run.sc;  // y[0] / z[0] follow the ping-pong of orth()
 
     if (s.bf16) {
         k_split_hi_lo<<<grid_for(s.n * r), 256, 0, st>>>(omega, sc.om_hi, sc.lo, s.n * r);
         run.check(cudaGetLastError());
     }
-    run.x_times(nullptr, omega, sc.y[0]);
-    if (run.ok()) run.orth(sc.y, s.L);
+    // The intermediate bases only have to stay well conditioned: one CholeskyQR pass
+    // each; the final basis (the returned A) gets two.
+    Scratch &sw = run.sc;
+    run.x_times(nullptr, omega, sw.y[0]);
+    if (run.ok()) run.orth(sw.y, s.L, n_iter == 0 ? 2 : 1);
     for (int it = 0; it < n_iter && run.ok(); ++it) {
-        run.xt_times(sc.y[0], sc.z[0]);
-        if (run.ok()) run.orth(sc.z, s.n);
-        if (run.ok()) run.x_times(sc.z[0], omega, sc.y[0]);
-        if (run.ok()) run.orth(sc.y, s.L);
+        run.xt_times(sw.y[0], sw.z[0]);
+        if (run.ok()) run.orth(sw.z, s.n, 1);
+        if (run.ok()) run.x_times(sw.z[0], omega, sw.y[0]);
+        if (run.ok()) run.orth(sw.y, s.L, it == n_iter - 1 ? 2 : 1);
     }
     if (run.ok()) {
         const int64_t na = (int64_t)B * s.L * r;
