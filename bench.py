@@ -438,6 +438,11 @@ CLF = dict(window=4, batch=8, ctx_len=32768, n_kv_heads=8, head_dim=128, rank_k=
            rank_v=768, n_iter=2, tau=128.0, gap=0.1)
 CLF_METRIC = ("prefill cross-layer factorization tokens/s (window of 4 layers, K and V "
               "caches, 32K ctx)")
+# The same window after 256 generated tokens: the tail folded back into the factors.
+REFOLD_WORKLOAD = "llama8b_refold_32k"
+REFOLD_TAIL = 256
+REFOLD_METRIC = ("tail refold tokens/s (window of 4 layers, K and V caches, 32K compressed "
+                 "+ 256 generated rows)")
 # fp64 FMA peak of the CUDA cores: 148 SMs x 64 fp64 FMA per clock x 2 flop x 1.965 GHz
 FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
 TF32_OVER_BF16 = 1.1 / 2.25                      # nominal dense tf32 : bf16 ratio
@@ -490,6 +495,9 @@ def run_clf(args, rank, world):
     c = dict(CLF)
     if args.batch:
         c["batch"] = args.batch
+    refold = args.workload == REFOLD_WORKLOAD
+    T = REFOLD_TAIL if refold else 0
+    name, metric = (REFOLD_WORKLOAD, REFOLD_METRIC) if refold else (CLF_WORKLOAD, CLF_METRIC)
     if args.impl == "reference":
         if rank != 0:
             return
@@ -497,11 +505,11 @@ def run_clf(args, rank, world):
             clf_cpu_baseline(c, args.seed, rows=512)
         vals = [clf_cpu_baseline(c, args.seed) for _ in range(args.steps)]
         v = float(np.mean([x["value"] for x in vals]))
-        line = {"metric": CLF_METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        line = {"metric": metric, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * c["batch"] * c["ctx_len"] / v, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "impl": "reference", "config": {"workload": CLF_WORKLOAD, **c},
+                "impl": "reference", "config": {"workload": name, **c, "n_tail": T},
                 "cpu_baseline": {**vals[-1], "value": v},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -522,13 +530,27 @@ def run_clf(args, rank, world):
     seed = args.seed + 1000 * rank
     calls = []
     for which, r in (("k", c["rank_k"]), ("v", c["rank_v"])):
-        X, _ = synth.torch_window_caches(W, B, L, dk, r + 64, r, c["tau"], c["gap"], "bf16",
+        X, _ = synth.torch_window_caches(W, B, L + T, dk, r + 64, r, c["tau"], c["gap"], "bf16",
                                          seed + (0 if which == "k" else 1), device=dev)
         om = torch.from_numpy(synth.np_test_matrix(n, r, seed)).to(dev)
-        A = torch.empty((B, L, r), dtype=torch.bfloat16, device=dev)
+        A = torch.empty((B, L + T, r), dtype=torch.bfloat16, device=dev)
         Bt = torch.empty((W, B, dk, r), dtype=torch.bfloat16, device=dev)
-        calls.append(dict(r=r, X=X, om=om, A=A, Bt=Bt))
-    ws = torch.empty(max(xkv.xkv_factorize_workspace_bytes(d, W, k["r"]) for k in calls),
+        k = dict(r=r, X=X, om=om, A=A, Bt=Bt)
+        if refold:
+            # the window as the decode loop holds it: L rows in factors, T generated rows
+            k["X"] = X[:, :, :L].contiguous()
+            k["tail"] = X[:, :, L:].contiguous()
+            del X
+            k["A0"] = torch.empty((B, L, r), dtype=torch.bfloat16, device=dev)
+            k["Bt0"] = torch.empty((W, B, dk, r), dtype=torch.bfloat16, device=dev)
+            wsf = torch.empty(xkv.xkv_factorize_workspace_bytes(d, W, r), dtype=torch.uint8,
+                              device=dev)
+            xkv.xkv_factorize_window(d, W, r, k["X"], om, c["n_iter"], k["A0"], k["Bt0"], wsf)
+            torch.cuda.synchronize(dev)
+            del wsf
+        calls.append(k)
+    ws = torch.empty(max(xkv.xkv_refold_workspace_bytes(d, W, k["r"], T) if refold else
+                         xkv.xkv_factorize_workspace_bytes(d, W, k["r"]) for k in calls),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -537,8 +559,12 @@ def run_clf(args, rank, world):
             if events is not None:
                 events[i][0].record(stream)
             torch.cuda.nvtx.range_push("xkv_factorize")    # lets a profiler skip the setup
-            xkv.xkv_factorize_window(d, W, k["r"], k["X"], k["om"], c["n_iter"], k["A"], k["Bt"],
-                                     ws)
+            if refold:
+                xkv.xkv_refold_window(d, W, k["r"], k["A0"], k["Bt0"], k["tail"], T, k["om"],
+                                      c["n_iter"], k["A"], k["Bt"], ws)
+            else:
+                xkv.xkv_factorize_window(d, W, k["r"], k["X"], k["om"], c["n_iter"], k["A"],
+                                         k["Bt"], ws)
             torch.cuda.nvtx.range_pop()
             if events is not None:
                 events[i][1].record(stream)
@@ -571,18 +597,20 @@ def run_clf(args, rank, world):
         for i in range(len(calls)):
             per_call[i].append(ev[i][0].elapsed_time(ev[i][1]))
     call_ms = [float(np.mean(p)) for p in per_call]
-    # end to end: the caches from pinned host memory, the factors back to the host
+    # end to end: the caches (refold: the generated rows) from pinned host memory, the
+    # factors back to the host
     e2e = None
+    src = "tail" if refold else "X"
     if not args.no_e2e:
-        hx = [torch.empty(k["X"].shape, dtype=k["X"].dtype, pin_memory=True) for k in calls]
+        hx = [torch.empty(k[src].shape, dtype=k[src].dtype, pin_memory=True) for k in calls]
         for h, k in zip(hx, calls):
-            h.copy_(k["X"].cpu())
+            h.copy_(k[src].cpu())
         ha = [torch.empty(k["A"].shape, dtype=k["A"].dtype, pin_memory=True) for k in calls]
         hb = [torch.empty(k["Bt"].shape, dtype=k["Bt"].dtype, pin_memory=True) for k in calls]
 
         def e2e_step():
             for h, k in zip(hx, calls):
-                k["X"].copy_(h, non_blocking=True)
+                k[src].copy_(h, non_blocking=True)
             step()
             for a, b, k in zip(ha, hb, calls):
                 a.copy_(k["A"], non_blocking=True)
@@ -601,7 +629,7 @@ def run_clf(args, rank, world):
         h2d = sum(h.numel() * h.element_size() for h in hx)
         d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size()
                   for a, b in zip(ha, hb))
-        e2e = {"value": B * L * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": B * (L + T) * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -611,18 +639,18 @@ def run_clf(args, rank, world):
         # each unit at that unit's peak -- bf16 products at the measured sustained bf16
         # rate, TF32 products at the nominal fraction of it, the fp64 Gram matrices at the
         # fp64 peak derived from unit counts and clock -- against the measured time.
-        wv = clf_work(c, c["rank_v"])
+        wv = clf_work({**c, "ctx_len": L + T}, c["rank_v"])
         bf16_peak, bf16_kind = measured_tflops_sustained()
         t_ideal = (wv["bf16"] / (bf16_peak * 1e12) + wv["tf32"] / (bf16_peak * TF32_OVER_BF16 * 1e12)
                    + wv["fp64"] / (FP64_PEAK_TFLOPS * 1e12))
         flops = wv["bf16"] + wv["tf32"] + wv["fp64"]
         t_call = call_ms[1] / 1e3
         line = {
-            "metric": CLF_METRIC, "value": B * L * world * args.steps / (elapsed_ms / 1e3),
+            "metric": metric, "value": B * (L + T) * world * args.steps / (elapsed_ms / 1e3),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": CLF_WORKLOAD, **c, "parallelism": f"replicas x{world}",
+            "config": {"workload": name, **c, "n_tail": T, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {2 * calls[0]['X'].numel() * 2 / 1e9:.1f} "
                              "GB of caches per step"},
             "roofline": {"bound": "alu", "kernel": "factorize_window (rank 768 call, whole)",
@@ -635,6 +663,7 @@ def run_clf(args, rank, world):
                          "flops_fp64": wv["fp64"], "avg_launch_ms": call_ms[1],
                          "rank_512_call_ms": call_ms[0]},
             "gpu_launches": sum(clf_work(c, k["r"])["own_launches"] for k in calls) * args.steps,
+            "refold_reconstruct_flops": (2 * B * L * c["rank_v"] * n) if refold else 0,
             "library_gemm_calls": sum(clf_work(c, k["r"])["blas_calls"] for k in calls)
                                   * args.steps,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
@@ -650,7 +679,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.workload == CLF_WORKLOAD:
+    if args.workload in (CLF_WORKLOAD, REFOLD_WORKLOAD):
         run_clf(args, rank, world)
         return
     from cross_layer_compressed_b200 import synth

@@ -281,6 +281,42 @@ xkv_status check_factorize(const xkv_dims *d, int32_t window, int32_t rank, cons
 
 extern "C" {
 
+size_t xkv_refold_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank,
+                                  int64_t n_tail) {
+    if (check_factorize(dims, window, rank, "xkv_refold_workspace_bytes") != XKV_OK ||
+        n_tail < 0 || dims->ctx_len + n_tail > (1 << 24))
+        return 0;
+    return refold_ws_bytes(*dims, window, rank, n_tail);
+}
+
+xkv_status xkv_refold_window(const xkv_dims *dims, int32_t window, int32_t rank,
+                             const void *A_win, const void *Bt_win, const void *tail,
+                             int64_t n_tail, const float *omega, int32_t n_iter, void *A_out,
+                             void *Bt_out, void *ws, size_t ws_bytes, void *stream) {
+    const char *who = "xkv_refold_window";
+    xkv_status st;
+    if ((st = check_factorize(dims, window, rank, who)) != XKV_OK) return st;
+    if (n_tail < 0 || dims->ctx_len + n_tail > (1 << 24))
+        return fail(XKV_ERR_INVALID_ARG, "%s: need 0 <= n_tail and ctx_len + n_tail <= 2^24",
+                    who);
+    if (n_iter < 0 || n_iter > 16)
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_iter must be in [0, 16]", who);
+    if (!A_win || !Bt_win || (n_tail > 0 && !tail) || !omega || !A_out || !Bt_out || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL pointer", who);
+    if (!aligned16(A_win) || !aligned16(Bt_win) || (n_tail > 0 && !aligned16(tail)) ||
+        !aligned16(omega) || !aligned16(A_out) || !aligned16(Bt_out) || !aligned16(ws))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    const size_t need = refold_ws_bytes(*dims, window, rank, n_tail);
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_refold(*dims, window, rank, A_win, Bt_win, tail, n_tail, omega,
+                                  n_iter, A_out, Bt_out, ws, (cudaStream_t)stream),
+                    who);
+}
+
 size_t xkv_factorize_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank) {
     if (check_factorize(dims, window, rank, "xkv_factorize_workspace_bytes") != XKV_OK) return 0;
     return factorize_ws_bytes(*dims, window, rank);

@@ -454,16 +454,17 @@ size_t carve(const Shape &s, void *ws, Scratch *out) {
     return off;
 }
 
-// Row-major C = op(A) op(B) (M x N, inner K) in fp32, batched over sequences.
+// Row-major C = op(A) op(B) (M x N, inner K), batched over sequences; C in fp32 unless
+// `tc` says otherwise.
 cublasStatus_t rm_gemm(cublasHandle_t h, bool tA, bool tB, int M, int N, int K, const void *A,
                        cudaDataType ta, int lda, long long sA, const void *Bm, cudaDataType tb,
                        int ldb, long long sB, void *C, int ldc, long long sC, int batch,
-                       float beta, cublasComputeType_t ct) {
+                       float beta, cublasComputeType_t ct, cudaDataType tc = CUDA_R_32F) {
     const float alpha = 1.f;
     return cublasGemmStridedBatchedEx(h, tB ? CUBLAS_OP_T : CUBLAS_OP_N,
                                       tA ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, Bm, tb,
-                                      ldb, sB, A, ta, lda, sA, &beta, C, CUDA_R_32F, ldc, sC,
-                                      batch, ct, CUBLAS_GEMM_DEFAULT);
+                                      ldb, sB, A, ta, lda, sA, &beta, C, tc, ldc, sC, batch, ct,
+                                      CUBLAS_GEMM_DEFAULT);
 }
 
 struct Run {
@@ -636,7 +637,67 @@ cudaError_t factorize_t(const Shape &s, const void *X, const float *omega, int n
     return run.blas_ok ? cudaSuccess : cudaErrorUnknown;
 }
 
+// Refold (the decode loop's tail of generated rows folded back into the factors): the
+// extended caches [A·B_l ; tail_l] are built in the workspace -- the reconstruction in
+// the storage type, as the decode calls would see it -- and factored again.
+template <typename T>
+cudaError_t refold_t(const Shape &s, int64_t n_tail, const void *A, const void *Bt,
+                     const void *tail, const float *omega, int n_iter, void *A_out,
+                     void *Bt_out, void *ws, size_t x_bytes, cudaStream_t st) {
+    const int64_t L = s.L - n_tail, e = sizeof(T);
+    char *xbuf = (char *)ws;
+    {
+        std::lock_guard<std::mutex> lock(g_blas_mu);
+        cublasHandle_t h = blas_handle();
+        if (!h || cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return cudaErrorNotReady;
+        const cudaDataType dt = s.bf16 ? CUDA_R_16BF : CUDA_R_32F;
+        const cublasComputeType_t ct = s.bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC;
+        for (int l = 0; l < s.W; ++l) {
+            // X'_l[b][0:L] = A_b B_l,b (B_l stored column-major: Bt_l,b is d_kv x r)
+            const cublasStatus_t bs =
+                rm_gemm(h, false, true, (int)L, (int)s.dk, s.r, A, dt, s.r, L * s.r,
+                        (const char *)Bt + (size_t)l * s.B * s.dk * s.r * e, dt, s.r,
+                        s.dk * s.r, xbuf + (size_t)l * s.B * s.L * s.dk * e, (int)s.dk,
+                        s.L * s.dk, s.B, 0.f, ct, dt);
+            if (bs != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
+            if (n_tail > 0) {
+                cudaError_t c = cudaMemcpy2DAsync(
+                    xbuf + ((size_t)l * s.B * s.L + L) * s.dk * e, (size_t)s.L * s.dk * e,
+                    (const char *)tail + (size_t)l * s.B * n_tail * s.dk * e,
+                    (size_t)n_tail * s.dk * e, (size_t)n_tail * s.dk * e, (size_t)s.B,
+                    cudaMemcpyDeviceToDevice, st);
+                if (c != cudaSuccess) return c;
+            }
+        }
+    }
+    return factorize_t<T>(s, xbuf, omega, n_iter, A_out, Bt_out, xbuf + x_bytes, st);
+}
+
+size_t refold_x_bytes(const Shape &s) {
+    return align256((size_t)s.W * s.B * s.L * s.dk * (s.bf16 ? 2 : 4));
+}
+
 }  // namespace
+
+size_t refold_ws_bytes(const xkv_dims &d, int W, int r, int64_t n_tail) {
+    xkv_dims e = d;
+    e.ctx_len = d.ctx_len + n_tail;
+    const Shape s = shape_of(e, W, r);
+    return refold_x_bytes(s) + carve(s, nullptr, nullptr);
+}
+
+cudaError_t launch_refold(const xkv_dims &d, int W, int r, const void *A, const void *Bt,
+                          const void *tail, int64_t n_tail, const float *omega, int n_iter,
+                          void *A_out, void *Bt_out, void *ws, cudaStream_t s) {
+    xkv_dims e = d;
+    e.ctx_len = d.ctx_len + n_tail;
+    const Shape sh = shape_of(e, W, r);
+    const size_t xb = refold_x_bytes(sh);
+    return sh.bf16 ? refold_t<__nv_bfloat16>(sh, n_tail, A, Bt, tail, omega, n_iter, A_out,
+                                             Bt_out, ws, xb, s)
+                   : refold_t<float>(sh, n_tail, A, Bt, tail, omega, n_iter, A_out, Bt_out, ws,
+                                     xb, s);
+}
 
 size_t factorize_ws_bytes(const xkv_dims &d, int W, int r) {
     return carve(shape_of(d, W, r), nullptr, nullptr);

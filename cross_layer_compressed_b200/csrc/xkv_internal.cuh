@@ -77,6 +77,11 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
 size_t factorize_ws_bytes(const xkv_dims &d, int W, int r);
 cudaError_t launch_factorize(const xkv_dims &d, int W, int r, const void *X, const float *omega,
                              int n_iter, void *A_out, void *Bt_out, void *ws, cudaStream_t s);
+// the tail of generated rows folded back: factorization of [A·B_l ; tail_l]
+size_t refold_ws_bytes(const xkv_dims &d, int W, int r, int64_t n_tail);
+cudaError_t launch_refold(const xkv_dims &d, int W, int r, const void *A, const void *Bt,
+                          const void *tail, int64_t n_tail, const float *omega, int n_iter,
+                          void *A_out, void *Bt_out, void *ws, cudaStream_t s);
 
 // Clears the workspace status word of a call (a one-thread kernel launched with
 // launch_chained, so that it and the attention kernel after it are scheduled while the

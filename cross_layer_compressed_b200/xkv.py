@@ -63,6 +63,9 @@ _sigs = {
     "xkv_factorize_window": ([_D, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp],
                              ctypes.c_int),
     "xkv_factorize_workspace_bytes": ([_D, _i32, _i32], _sz),
+    "xkv_refold_window": ([_D, _i32, _i32, _vp, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _sz,
+                           _vp], ctypes.c_int),
+    "xkv_refold_workspace_bytes": ([_D, _i32, _i32, _i64], _sz),
     "xkv_n_selected": ([_i64, _i32, _i32, _i32], _i64),
     "xkv_footprint_bytes": ([_D, _i32, _i32, _i32], _i64),
     "rcla_cache_bytes": ([_D, _i32, _i64], _i64),
@@ -230,6 +233,24 @@ def xkv_factorize_window(d: xkv_dims, window, rank, X, omega, n_iter, A_out, Bt_
 
 def xkv_factorize_workspace_bytes(d: xkv_dims, window, rank) -> int:
     return int(_lib.xkv_factorize_workspace_bytes(ctypes.byref(d), int(window), int(rank)))
+
+
+def xkv_refold_window(d: xkv_dims, window, rank, A_win, Bt_win, tail, n_tail, omega, n_iter,
+                      A_out, Bt_out, ws, ws_bytes=None, stream=None, check=True):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    st = _lib.xkv_refold_window(ctypes.byref(d), int(window), int(rank), _ptr(A_win),
+                                _ptr(Bt_win), _ptr(tail) if tail is not None else None,
+                                int(n_tail), _ptr(omega), int(n_iter), _ptr(A_out),
+                                _ptr(Bt_out), _ptr(ws), int(ws_bytes), _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_refold_workspace_bytes(d: xkv_dims, window, rank, n_tail) -> int:
+    return int(_lib.xkv_refold_workspace_bytes(ctypes.byref(d), int(window), int(rank),
+                                               int(n_tail)))
 
 
 def xkv_workspace_bytes(d: xkv_dims, n_sel: int, mode: int) -> int:

@@ -272,6 +272,33 @@ xkv_status xkv_factorize_window(const xkv_dims *dims, int32_t window, int32_t ra
  * arguments). */
 size_t xkv_factorize_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank);
 
+/*
+ * Refold the tail of generated rows into a window's factors [xKV 2.2 applied again at
+ * decode time; the pages give no schedule]: per layer the cache the decode calls see,
+ * X'_l = [A·B_l ; tail_l] ((L + T) x d_kv, the reconstructed part rounded to dtype),
+ * is factored at rank r exactly as xkv_factorize_window does, so the next decode steps
+ * read L + T compressed rows and an empty tail.
+ *
+ *   dims        as for xkv_factorize_window; ctx_len = L, the rows already compressed
+ *   A_win       [B][L][r], Bt_win [W][B][d_kv][r]: the current factors (dtype)
+ *   tail        [W][B][T][d_kv] (dtype): the generated rows of each layer; may be NULL
+ *               when n_tail = T = 0
+ *   omega, n_iter, Bt_out   as for xkv_factorize_window
+ *   A_out       [B][L + T][r]
+ *   ws          device scratch of xkv_refold_workspace_bytes bytes (the extended caches
+ *               plus the factorization's scratch)
+ * Bt_out may be Bt_win (it is read before it is written, in stream order).  Asynchronous;
+ * INVALID_ARG / UNSUPPORTED before any launch.
+ */
+xkv_status xkv_refold_window(const xkv_dims *dims, int32_t window, int32_t rank,
+                             const void *A_win, const void *Bt_win, const void *tail,
+                             int64_t n_tail, const float *omega, int32_t n_iter, void *A_out,
+                             void *Bt_out, void *ws, size_t ws_bytes, void *stream);
+
+/* Scratch bytes of xkv_refold_window (0 on bad arguments). */
+size_t xkv_refold_workspace_bytes(const xkv_dims *dims, int32_t window, int32_t rank,
+                                  int64_t n_tail);
+
 /* Chunks selected per (b, g): min(top_k, nC - |F|) + |F|; -1 on bad arguments. */
 int64_t xkv_n_selected(int64_t n_chunks, int32_t top_k, int32_t n_sink, int32_t n_recent);
 

@@ -21,7 +21,8 @@ _lib = None
 
 F32, BF16 = 0, 1
 
-from .clf import concatenate_window, factorize_window, reconstruct_window  # noqa: E402,F401
+from .clf import (concatenate_window, factorize_window, reconstruct_window,  # noqa: E402,F401
+                  refold_window)
 
 
 def build(force: bool = False) -> str:

@@ -59,3 +59,16 @@ def reconstruct_window(A, Bt) -> np.ndarray:
         for b in range(B):
             out[l, b] = A[b] @ Bt[l, b].T
     return out
+
+
+def refold_window(A, Bt, tail, rank: int, to_storage=None):
+    """Refold a tail of generated, uncompressed rows into the window's factors (the dense
+    tail buffer of the decode loop, emptied periodically): per layer the cache the decode
+    calls see, [A·B_l ; tail_l] ((L + T) x d_kv, the reconstructed part rounded to the
+    storage type by `to_storage` when given), is factored again at rank r exactly as
+    factorize_window does.  tail: [W][B][T][d_kv].  Returns factorize_window's triple."""
+    P = reconstruct_window(A, Bt)
+    if to_storage is not None:
+        P = to_storage(P)
+    X = np.concatenate([P, np.asarray(tail, dtype=np.float64)], axis=2)
+    return factorize_window(X, rank)

@@ -277,3 +277,32 @@ def test_factorize_fault_injection(xkv, monkeypatch):
     assert xkv.xkv_factorize_window(d, 2, 32, FAKE, FAKE, 1, FAKE, FAKE, FAKE, need, stream=0,
                                     check=False) == 4
     assert "injected" in xkv.last_error()
+
+
+def test_refold_argument_checks(xkv, monkeypatch):
+    d = _fd(xkv)
+    need = xkv.xkv_refold_workspace_bytes(d, 2, 32, 100)
+    assert need > xkv.xkv_factorize_workspace_bytes(d, 2, 32)
+    # the extended caches (W x B x (L + T) x d_kv in bf16) come first
+    assert need == (2 * 2 * 1100 * 128 * 2 + 255) // 256 * 256 + \
+        xkv.xkv_factorize_workspace_bytes(_fd(xkv, ctx_len=1100), 2, 32)
+    assert xkv.xkv_refold_workspace_bytes(d, 2, 32, -1) == 0
+    args = dict(A_win=FAKE, Bt_win=FAKE, tail=FAKE, omega=FAKE, A_out=FAKE, Bt_out=FAKE, ws=FAKE)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return xkv.xkv_refold_window(kw.pop("d", d), 2, kw.pop("rank", 32), a["A_win"],
+                                     a["Bt_win"], a["tail"], kw.get("n_tail", 100), a["omega"],
+                                     kw.get("n_iter", 1), a["A_out"], a["Bt_out"], a["ws"],
+                                     kw.get("ws_bytes", need), stream=0, check=False)
+    assert call(n_tail=-1) == 1
+    assert call(tail=0) == 1                       # a tail is needed when n_tail > 0
+    assert call(A_win=FAKE + 8) == 1 and "aligned" in xkv.last_error()
+    assert call(ws_bytes=need - 1) == 1 and "workspace" in xkv.last_error()
+    assert call(n_iter=17) == 1
+    assert call(rank=40) == 1
+    monkeypatch.setenv("XKV_FAULT", "xkv_refold_window:3")
+    assert call() == 3
+    # no tail: NULL is accepted and only the factorization's scratch is added
+    need0 = xkv.xkv_refold_workspace_bytes(d, 2, 32, 0)
+    assert call(tail=0, n_tail=0, ws_bytes=need0) == 3

@@ -165,3 +165,51 @@ def test_factorize_full_size_properties(xkv):
             assert abs(Bt[l, b, j, i] - want) <= 2e-2 * np.linalg.norm(col)
     del X
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------------ refold
+def _refold(xkv, A, Bt, tail, W, B, L, T, Hkv, hd, r, n_iter, dtype, seed=0):
+    d = xkv.dims(B, Hkv, Hkv, hd, L, chunk=8, rank_k=0, rank_v=0, dtype=dtype)
+    dk = Hkv * hd
+    A2 = torch.empty((B, L + T, r), dtype=_tdt(dtype), device=DEV)
+    Bt2 = torch.empty((W, B, dk, r), dtype=_tdt(dtype), device=DEV)
+    ws = torch.empty(xkv.xkv_refold_workspace_bytes(d, W, r, T), dtype=torch.uint8, device=DEV)
+    om = torch.from_numpy(synth.np_test_matrix(W * dk, r, seed)).to(DEV)
+    xkv.xkv_refold_window(d, W, r, A.to(DEV), Bt.to(DEV), tail.to(DEV) if T else None, T, om,
+                          n_iter, A2, Bt2, ws)
+    torch.cuda.synchronize()
+    return A2.double().cpu().numpy(), Bt2.double().cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_refold_matches_oracle(xkv, ora, dtype):
+    """Caches of L = 512 compressed rows (factors from the oracle, in the storage type)
+    plus T = 100 generated rows: the refolded factors' product equals the oracle's
+    refactorization of [A·B_l ; tail_l] (reconstruction rounded to the storage type)."""
+    W, B, L, T, Hkv, hd, r = 2, 2, 512, 100, 2, 64, 32
+    X, _ = synth.np_window_caches(W, B, L + T, Hkv * hd, 96, r, 16.0, 0.05, seed=3)
+    A, Bt, _ = ora.factorize_window(X[:, :, :L], r)
+    As, Bts = synth.to_storage(A, dtype), synth.to_storage(Bt, dtype)
+    tail = synth.to_storage(X[:, :, L:], dtype)
+    A2, Bt2 = _refold(xkv, As, Bts, tail, W, B, L, T, Hkv, hd, r, 3, dtype)
+    round_to = (lambda P: synth.to_storage(P, dtype).double().numpy())
+    Ar, Btr, S = ora.refold_window(As.double().numpy(), Bts.double().numpy(),
+                                   tail.double().numpy(), r, to_storage=round_to)
+    P_ref = ora.reconstruct_window(Ar, Btr)
+    P = ora.reconstruct_window(A2, Bt2)
+    assert A2.shape == (B, L + T, r)
+    assert np.abs(P - P_ref).max() <= TOL[dtype] * np.abs(P_ref).max()
+    for b in range(B):
+        assert np.abs(A2[b].T @ A2[b] - np.eye(r)).max() <= ORTH_TOL[dtype]
+
+
+def test_refold_without_tail_keeps_the_product(xkv, ora):
+    """T = 0 (NULL tail): a rank-r product refactored at rank r is unchanged."""
+    W, B, L, Hkv, hd, r = 3, 2, 700, 1, 64, 48
+    X, _ = synth.np_window_caches(W, B, L, Hkv * hd, 80, r, 24.0, 0.05, seed=4)
+    A, Bt, _ = ora.factorize_window(X, r)
+    As, Bts = synth.to_storage(A, "f32"), synth.to_storage(Bt, "f32")
+    A2, Bt2 = _refold(xkv, As, Bts, None, W, B, L, 0, Hkv, hd, r, 1, "f32")
+    P0 = ora.reconstruct_window(As.double().numpy(), Bts.double().numpy())
+    P = ora.reconstruct_window(A2, Bt2)
+    assert np.abs(P - P0).max() <= 1e-4 * np.abs(P0).max()

@@ -616,3 +616,43 @@ def test_clf_generator_spectrum(ora):
     for b in range(2):
         assert np.allclose(S[b, :40], s, atol=1e-12)
         assert np.allclose(S[b, 40:], 0.0, atol=1e-12)
+
+
+def test_clf_refold_empty_tail_keeps_the_product(ora):
+    """Refolding no rows refactors a rank-r product at rank r: the product is unchanged
+    (the rank-r matrix is its own truncated SVD)."""
+    rng = np.random.default_rng(21)
+    X = rng.standard_normal((2, 2, 60, 5))
+    A, Bt, _ = ora.factorize_window(X, 4)
+    A2, Bt2, _ = ora.refold_window(A, Bt, np.zeros((2, 2, 0, 5)), 4)
+    assert np.abs(ora.reconstruct_window(A2, Bt2) - ora.reconstruct_window(A, Bt)).max() <= 1e-12
+
+
+def test_clf_refold_tail_in_span_is_exact(ora):
+    """Tail rows that are combinations of the basis' rows' directions (each tail row a
+    mix of rows of A·B_l with one set of weights across layers) add nothing new: the
+    refolded product is [A·B_l ; tail_l] exactly, and the tail rows are rebuilt."""
+    rng = np.random.default_rng(22)
+    X = rng.standard_normal((3, 1, 40, 4))
+    A, Bt, _ = ora.factorize_window(X, 5)
+    P = ora.reconstruct_window(A, Bt)                         # rank 5 per sequence
+    w = rng.standard_normal((7, 40))
+    tail = np.stack([w @ P[l, 0] for l in range(3)])[:, None]  # [3][1][7][4], same rows mixed
+    A2, Bt2, _ = ora.refold_window(A, Bt, tail, 5)
+    want = np.concatenate([P, tail], axis=2)
+    assert np.abs(ora.reconstruct_window(A2, Bt2) - want).max() <= 1e-10 * np.abs(want).max()
+
+
+def test_clf_refold_is_the_factorization_of_the_extended_cache(ora):
+    """A general tail: refolding equals factorizing the extended caches directly (the
+    composition the refold is defined by), and the new basis covers L + T rows."""
+    rng = np.random.default_rng(23)
+    X = rng.standard_normal((2, 2, 30, 6))
+    A, Bt, _ = ora.factorize_window(X, 6)
+    tail = rng.standard_normal((2, 2, 9, 6))
+    A2, Bt2, S2 = ora.refold_window(A, Bt, tail, 6)
+    ext = np.concatenate([ora.reconstruct_window(A, Bt), tail], axis=2)
+    A3, Bt3, S3 = ora.factorize_window(ext, 6)
+    assert A2.shape == (2, 39, 6)
+    assert np.allclose(S2, S3, atol=1e-12)
+    assert np.abs(ora.reconstruct_window(A2, Bt2) - ora.reconstruct_window(A3, Bt3)).max() <= 1e-12
