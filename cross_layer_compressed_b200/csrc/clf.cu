@@ -156,7 +156,8 @@ __global__ void __launch_bounds__(256) k_potrf_diag(double *__restrict__ G, int 
     }
     const double t = tol[b];
     __syncthreads();
-    const int c = tid;                                      // threads 0..63: one column each
+    // four threads per column: thread 4c + q updates rows i = q (mod 4) of column c
+    const int c = tid >> 2, q = tid & 3;
     for (int j = 0; j < bk; ++j) {
         if (tid == 0) {
             const double pv = a[j][j];
@@ -166,10 +167,10 @@ __global__ void __launch_bounds__(256) k_potrf_diag(double *__restrict__ G, int 
         }
         __syncthreads();
         const int dep = s_dep;
-        if (c > j && c < bk) a[j][c] = dep ? 0.0 : a[j][c] / a[j][j];
+        if (q == 0 && c > j && c < bk) a[j][c] = dep ? 0.0 : a[j][c] / a[j][j];
         __syncthreads();
         if (!dep && c > j && c < bk)
-            for (int i = j + 1; i <= c; ++i) a[i][c] -= a[j][i] * a[j][c];
+            for (int i = j + 1 + q; i <= c; i += 4) a[i][c] -= a[j][i] * a[j][c];
         __syncthreads();
     }
     // D = R_kk^-1 by back substitution, all 64 columns at once: four adjacent lanes per
