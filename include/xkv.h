@@ -9,7 +9,10 @@
  *          one small reconstruction matrix B_l (r x d_kv) per layer.  Section 2.3,
  *          selective reconstruction (SR): landmark-based chunk selection, then only
  *          the selected rows of K = A B_l (and V) are rebuilt.  Section 4, dense
- *          reconstruction (all rows).
+ *          reconstruction (all rows).  The prefill side of section 2.2 -- the
+ *          concatenation, the rank-r factorization, A and the B_l -- is here too
+ *          (xkv_factorize_window), and so is folding generated rows back into the
+ *          factors (xkv_refold_window).
  *  [R-CLA] "Stochastic KV Routing: adaptive depth-wise cache sharing".  Inference
  *          with a fixed sharing set S: a layer outside S reuses the KV cache of the
  *          nearest previous layer in S and skips its own K/V load and update

@@ -200,7 +200,10 @@ int main(void) {
     xkv_dims bad = d;
     bad.head_dim = 96;
     xkv_status st = xkv_score_landmarks(&bad, (void *)0, (void *)0, (double *)0, (void *)0);
-    printf("%lld %lld %llu %d %s\n", nsel, fp, ws, (int)st, xkv_last_error()[0] ? "msg" : "none");
+    unsigned long long fws = (unsigned long long)xkv_factorize_workspace_bytes(&d, 4, 512);
+    unsigned long long rws = (unsigned long long)xkv_refold_workspace_bytes(&d, 4, 512, 256);
+    printf("%lld %lld %llu %d %s %llu %llu\n", nsel, fp, ws, (int)st,
+           xkv_last_error()[0] ? "msg" : "none", fws, rws);
     return 0;
 }
 ''')
@@ -215,6 +218,8 @@ int main(void) {
     assert int(out[1]) == xkv.xkv_footprint_bytes(d, 32, 4, 1)
     assert int(out[2]) == xkv.xkv_workspace_bytes(d, 261, xkv.XKV_MODE_SELECTIVE)
     assert int(out[3]) == xkv.XKV_ERR_UNSUPPORTED and out[4] == "msg"
+    assert int(out[5]) == xkv.xkv_factorize_workspace_bytes(d, 4, 512) > 0
+    assert int(out[6]) == xkv.xkv_refold_workspace_bytes(d, 4, 512, 256) > int(out[5])
 
 
 # ------------------------------------------------------- cross-layer factorization
