@@ -22,7 +22,9 @@
  *  - All tensor arguments are DEVICE pointers to dense row-major arrays (last index
  *    fastest) in the layouts stated below, unless marked "host".  The caller owns
  *    every buffer; the library never allocates, frees or keeps a pointer after the
- *    call returns.
+ *    call returns.  One exception: the factorization calls (xkv_factorize_window,
+ *    xkv_refold_window) run their plain GEMMs in cuBLAS, whose handle -- created once
+ *    per device on first use and kept until exit -- holds cuBLAS's own resources.
  *  - Storage type (dims->dtype): XKV_F32 or XKV_BF16, shared by the factors,
  *    landmarks, queries and caches of a call.  Outputs are fp32; scores are fp64.
  *  - Every pointer the kernels read or write must be 16-byte aligned.
