@@ -168,10 +168,11 @@ class XkvStep:
         self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
                                dtype=torch.float32, device=dev)
         self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
-        # our kernels per layer: score + select (selective only), then attention + split
-        # combine (explicit) or q~ + attention + merge + projection (reassociated)
+        # our kernels per layer: score + select (selective only), then status clear +
+        # attention + split merge (explicit) or q~ + attention + merge + projection
+        # (reassociated; q~ clears the status word)
         self.launches_per_step = w.n_layers * ((0 if self.dense else 2) +
-                                               (4 if path == "reassociated" else 2))
+                                               (4 if path == "reassociated" else 3))
         torch.cuda.synchronize()
 
     def resident_bytes(self):
