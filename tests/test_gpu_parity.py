@@ -563,3 +563,55 @@ def test_unsupported_device_paths_fail_loudly(xkv):
     d = xkv.dims(1, 4, 2, 64, 64, 8, 16, 16, xkv.XKV_BF16)
     with pytest.raises(xkv.XkvError):
         xkv.xkv_score_landmarks(d, None, None, None)
+
+
+# ------------------------------------------------------------ repeat-run determinism
+def test_repeat_runs_are_bit_identical(xkv, ora):
+    """With no race checker on this pool, repeat runs stand in for one: every stage of
+    the decode path (scores, selection, explicit and rank-space attention, R-CLA with its
+    cache update) has a fixed reduction order and no atomics on data, so five runs on the
+    same inputs must agree bit for bit.  A race in the selection, the split merge or a
+    shared-memory ring shows up as a difference."""
+    w = QWEN14_R
+    d = xkv.dims_of(w)
+    x = _layer_inputs(w)
+    lm = _dev(_host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim,
+                                                w.chunk)))
+    g = {k: _dev(x[k]) for k in ("Ak", "Av", "Bkt", "Bvt", "q")}
+    runs = []
+    for _ in range(5):
+        sc = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
+        sel = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
+        xkv.xkv_score_landmarks(d, lm, g["q"], sc)
+        xkv.xkv_select_chunks(d, sc, w.top_k, w.n_sink, w.n_recent, sel)
+        outs = []
+        for fn, mode in ((xkv.xkv_reconstruct_attend, xkv.XKV_MODE_SELECTIVE),
+                         (xkv.xkv_reassociated_attend, xkv.XKV_MODE_REASSOC)):
+            ws = torch.empty(xkv.xkv_workspace_bytes(d, w.n_sel, mode), dtype=torch.uint8,
+                             device=DEV)
+            out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+            fn(d, g["Ak"], g["Av"], g["Bkt"], g["Bvt"], g["q"], sel, w.n_sel, out, ws)
+            outs.append(out)
+        torch.cuda.synchronize()
+        runs.append([t.cpu().numpy().copy() for t in (sc, sel, *outs)])
+    for r in runs[1:]:
+        for a, b in zip(runs[0], r):
+            assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+    wr = RCLA_R
+    xr = synth.np_rcla_inputs(wr, seed=0, len_rows=wr.ctx_len)
+    dr = xkv.dims(wr.batch, wr.n_q_heads, wr.n_kv_heads, wr.head_dim, wr.L_max, dtype=wr.dtype)
+    wsr = torch.empty(xkv.xkv_workspace_bytes(dr, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                      device=DEV)
+    lo = [0] * wr.n_layers
+    res = []
+    for _ in range(3):
+        K, V = _dev(xr["K_lead"]), _dev(xr["V_lead"])
+        o = torch.empty((wr.batch, wr.n_q_heads, wr.head_dim), device=DEV)
+        xkv.rcla_decode_attend(dr, 0, lo, K, V, wr.L_max, wr.ctx_len, _dev(xr["k_new"][0]),
+                               _dev(xr["v_new"][0]), _dev(xr["q"][0]), o, wsr)
+        torch.cuda.synchronize()
+        res.append((o.cpu().numpy().copy(), K.cpu().view(torch.int16).numpy().copy()))
+    for o, k in res[1:]:
+        assert np.array_equal(o.view(np.uint8), res[0][0].view(np.uint8))
+        assert np.array_equal(k, res[0][1])
