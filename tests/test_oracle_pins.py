@@ -656,3 +656,36 @@ def test_clf_refold_is_the_factorization_of_the_extended_cache(ora):
     assert A2.shape == (2, 39, 6)
     assert np.allclose(S2, S3, atol=1e-12)
     assert np.abs(ora.reconstruct_window(A2, Bt2) - ora.reconstruct_window(A3, Bt3)).max() <= 1e-12
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis is part of the test environment
+    given = None
+
+if given is not None:
+    @settings(max_examples=30, deadline=None)
+    @given(W=st.integers(1, 3), L=st.integers(3, 24), d=st.integers(1, 5),
+           frac=st.floats(0.1, 1.0), seed=st.integers(0, 2 ** 31 - 1))
+    def test_clf_random_windows_are_optimal_projections(ora, W, L, d, frac, seed):
+        """Random windows and ranks: A is orthonormal, B_l = A^T X_l, the product is an
+        orthogonal projection (||X||^2 = ||AB||^2 + ||X - AB||^2), and no random rank-r
+        orthonormal basis leaves a smaller residual (Eckart-Young optimality checked
+        against competitors, not against the SVD's own numbers)."""
+        n = W * d
+        r = max(1, min(L, n, int(round(frac * min(L, n)))))
+        rng = np.random.default_rng(seed)
+        X = rng.standard_normal((W, 1, L, d))
+        A, Bt, _ = ora.factorize_window(X, r)
+        a = A[0]
+        assert np.allclose(a.T @ a, np.eye(r), atol=1e-10)
+        for l in range(W):
+            assert np.allclose(Bt[l, 0], X[l, 0].T @ a, atol=1e-10)
+        P = ora.reconstruct_window(A, Bt)
+        tot, kept, res = np.sum(X ** 2), np.sum(P ** 2), np.sum((X - P) ** 2)
+        assert abs(tot - kept - res) <= 1e-9 * tot
+        Xc = ora.concatenate_window(X, 0)
+        for _ in range(5):
+            q, _ = np.linalg.qr(rng.standard_normal((L, r)))
+            other = np.sum((Xc - q @ (q.T @ Xc)) ** 2)
+            assert other >= res - 1e-9 * tot
