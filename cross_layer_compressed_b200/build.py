@@ -1,19 +1,24 @@
-"""Build the CUDA library (libxkv.so) in-tree for sm_100a with nvcc."""
+"""Build the CUDA library (libxkv.so) in-tree for sm_100a with nvcc.
+
+Each .cu file is compiled to an object of its own (in parallel, under _build/), then the
+objects are linked into libxkv.so."""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libxkv.so")
+OBJ = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-         "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
+         "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
 # cuBLAS serves the plain GEMMs of the prefill-side factorization only
 LIBS = ["-lcublas", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
@@ -23,22 +28,48 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _headers() -> list[str]:
+    return glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "xkv.h")]
+
+
+def _obj(src: str) -> str:
+    return os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+
+
+def _stale(target: str, deps: list[str]) -> bool:
+    if not os.path.exists(target):
         return True
-    t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "xkv.h")]
+    t = os.path.getmtime(target)
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+def _compile(src: str, verbose: bool) -> str:
+    obj = _obj(src)
+    tmp = obj + ".tmp.o"
+    cmd = [NVCC, *FLAGS, "-c", "-o", tmp, src]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, obj)
+    return obj
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    if force or _stale():
-        tmp = LIB + ".tmp"
-        cmd = [NVCC, *FLAGS, "-o", tmp, *sources(), *LIBS]
-        if verbose:
-            print(" ".join(cmd), file=sys.stderr)
-        subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
+    srcs = sources()
+    hdrs = _headers()
+    if not force and not _stale(LIB, srcs + hdrs):
+        return LIB
+    os.makedirs(OBJ, exist_ok=True)
+    todo = [s for s in srcs if force or _stale(_obj(s), [s] + hdrs)]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(todo), os.cpu_count() or 4))) as ex:
+        list(ex.map(lambda s: _compile(s, verbose), todo))
+    tmp = LIB + ".tmp"
+    cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp,
+           *[_obj(s) for s in srcs], *LIBS]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
     return LIB
 
 

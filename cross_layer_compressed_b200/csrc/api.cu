@@ -149,6 +149,14 @@ SplitPlan plan_rcla(const xkv_dims &d, int64_t rows) {
 
 void xkv::set_last_error(const char *msg) { g_last_error = msg; }
 
+// The switches are read once, on first use, and hold for the life of the process.
+bool xkv::env_flag(EnvFlag f) {
+    static const bool flags[3] = {getenv("XKV_FORCE_SIMT") != nullptr,
+                                  getenv("XKV_NO_TC") != nullptr,
+                                  getenv("XKV_NO_PDL") != nullptr};
+    return flags[(int)f];
+}
+
 extern "C" {
 
 const char *xkv_last_error(void) { return g_last_error.c_str(); }
@@ -268,6 +276,43 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
                                   (cudaStream_t)stream), who);
 }
 
+size_t xkv_score_select_workspace_bytes(const xkv_dims *dims) {
+    if (check_dims(dims, true, "xkv_score_select_workspace_bytes") != XKV_OK) return 0;
+    return score_select_ws_bytes(*dims);
+}
+
+xkv_status xkv_score_select(const xkv_dims *dims, const void *lm_layer, const void *q,
+                            int32_t top_k, int32_t n_sink, int32_t n_recent, int32_t *sel,
+                            int32_t *n_sel_out, void *ws, size_t ws_bytes, void *stream) {
+    Range nvtx_range("xkv_score_select");
+    const char *who = "xkv_score_select";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!lm_layer || !q || !sel || !ws)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(lm_layer) || !aligned16(q) || !aligned16(sel) || !aligned16(ws))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (top_k < 0 || n_sink < 0 || n_recent < 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: top_k, n_sink, n_recent must be >= 0", who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (nC > 16384)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: more than 16384 chunks per unit", who);
+    if (!score_select_shape_ok(*dims))
+        return fail(XKV_ERR_UNSUPPORTED, "%s: G = n_q_heads / n_kv_heads must be 1..8 or 16",
+                    who);
+    const size_t need = score_select_ws_bytes(*dims);
+    if (ws_bytes < need)
+        return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
+                    need);
+    const int64_t n_sel = xkv_n_selected(nC, top_k, n_sink, n_recent);
+    if (n_sel_out) *n_sel_out = (int32_t)n_sel;
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    return launched(launch_score_select(*dims, lm_layer, q, top_k, n_sink, n_recent, sel,
+                                        (int)n_sel, ws, (cudaStream_t)stream),
+                    who);
+}
+
 }  // extern "C"
 
 namespace {
@@ -372,22 +417,26 @@ int64_t tail_bound(const xkv_dims &d, int64_t T_max) {
     return T_max > 0 ? plan_rcla(d, T_max).n_bound : 0;
 }
 
-// Reconstruct-then-attend over the selected (or all) rows of the window, plus, when
-// n_tail > 0, the first n_tail rows of an uncompressed tail K_tail / V_tail
-// [B][Hkv][T_max][hd]: the attention kernel writes its splits, the R-CLA kernel writes
-// the tail's splits after them, and one combine merges all of them.
-xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win,
-                       const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
-                       const void *q, const int32_t *sel, int32_t n_sel, const void *K_tail,
-                       const void *V_tail, int64_t T_max, int64_t n_tail, float *out, void *ws,
-                       size_t ws_bytes, void *stream) {
+}  // namespace
+
+// Host-side checks of a reconstruct-then-attend call: every argument rule, then the
+// scratch the call needs (*need_out) against ws_bytes -- the caller's workspace when
+// check_ws is set, else the size of the library's own fixed array (the allocation-free
+// entry point: ws is not checked, a larger need is XKV_ERR_UNSUPPORTED).  Then the
+// injected fault of `who`, then the device.  Nothing here launches.
+xkv_status xkv::attend_validate(const char *who, const xkv_dims *dims, const void *Ak_win,
+                           const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                           const void *q, const int32_t *sel, int32_t n_sel,
+                           const void *K_tail, const void *V_tail, int64_t T_max,
+                           int64_t n_tail, const float *out, const void *ws, size_t ws_bytes,
+                           bool check_ws, size_t *need_out) {
     xkv_status st;
     if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
-    if (!Ak_win || !Av_win || !Bkt_layer || !Bvt_layer || !q || !out || !ws)
+    if (!Ak_win || !Av_win || !Bkt_layer || !Bvt_layer || !q || !out || (check_ws && !ws))
         return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
     if (!aligned16(Ak_win) || !aligned16(Av_win) || !aligned16(Bkt_layer) ||
-        !aligned16(Bvt_layer) || !aligned16(q) || !aligned16(out) || !aligned16(ws) ||
-        (sel && !aligned16(sel)))
+        !aligned16(Bvt_layer) || !aligned16(q) || !aligned16(out) ||
+        (check_ws && !aligned16(ws)) || (sel && !aligned16(sel)))
         return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
     const int64_t nC = dims->ctx_len / dims->chunk;
     if (sel && (n_sel <= 0 || n_sel > nC))
@@ -406,12 +455,33 @@ xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win
     // the same amount xkv_workspace_bytes / xkv_tail_workspace_bytes report, whichever
     // kernel runs
     const size_t need = ws_header_bytes(*dims) + partial_bytes(*dims, (int)(n_att + n_tail_bound));
-    if (ws_bytes < need)
+    if (need_out) *need_out = need;
+    if (check_ws && ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
+    if (!check_ws && need > ws_bytes)
+        return fail(XKV_ERR_UNSUPPORTED,
+                    "%s: this call needs %zu bytes of scratch, above the fixed %zu-byte array; "
+                    "use xkv_reconstruct_attend with a caller-provided workspace",
+                    who, need, ws_bytes);
     if (injected(who, &st)) return st;
-    if ((st = check_device(who)) != XKV_OK) return st;
-    const bool use_tc = n_tc > 0 && attend_tc_supported(*dims) && !getenv("XKV_FORCE_SIMT");
+    return check_device(who);
+}
+
+// Reconstruct-then-attend over the selected (or all) rows of the window, plus, when
+// n_tail > 0, the first n_tail rows of an uncompressed tail K_tail / V_tail
+// [B][Hkv][T_max][hd]: the attention kernel writes its splits, the R-CLA kernel writes
+// the tail's splits after them, and one combine merges all of them.  The arguments were
+// checked by attend_validate; ws holds at least the scratch it reported.
+xkv_status xkv::attend_launch(const char *who, const xkv_dims *dims, const void *Ak_win,
+                         const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                         const void *q, const int32_t *sel, int32_t n_sel, const void *K_tail,
+                         const void *V_tail, int64_t T_max, int64_t n_tail, float *out,
+                         void *ws, void *stream) {
+    const int64_t rows = sel ? (int64_t)n_sel * dims->chunk : dims->ctx_len;
+    const SplitPlan plan = plan_xkv(*dims, rows);
+    const int n_tc = attend_tc_shape_ok(*dims) ? tc_splits(*dims, (int)(rows / dims->chunk)) : 0;
+    const bool use_tc = n_tc > 0 && attend_tc_supported(*dims) && !env_flag(ENV_FORCE_SIMT);
     cudaStream_t s = (cudaStream_t)stream;
     const size_t hdr = ws_header_bytes(*dims);
     unsigned *status = (unsigned *)ws;
@@ -441,6 +511,21 @@ xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win
     }
     if (e == cudaSuccess) e = launch_combine(*dims, used, partials, out, status, s);
     return launched(e, who);
+}
+
+namespace {
+
+xkv_status attend_impl(const char *who, const xkv_dims *dims, const void *Ak_win,
+                       const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                       const void *q, const int32_t *sel, int32_t n_sel, const void *K_tail,
+                       const void *V_tail, int64_t T_max, int64_t n_tail, float *out, void *ws,
+                       size_t ws_bytes, void *stream) {
+    const xkv_status st = attend_validate(who, dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
+                                          sel, n_sel, K_tail, V_tail, T_max, n_tail, out, ws,
+                                          ws_bytes, true, nullptr);
+    if (st != XKV_OK) return st;
+    return attend_launch(who, dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel, K_tail,
+                         V_tail, T_max, n_tail, out, ws, stream);
 }
 
 }  // namespace

@@ -121,7 +121,7 @@ cudaError_t launch_clear_status(unsigned *status, cudaStream_t s) {
     return launch_chained(k_clear_status, dim3(1), dim3(1), 0, s, status);
 }
 
-bool chain_enabled() { return getenv("XKV_NO_PDL") == nullptr; }
+bool chain_enabled() { return !env_flag(ENV_NO_PDL); }
 
 SplitPlan plan_splits(int64_t rows, int64_t units, int64_t min_rows, int64_t max_rows) {
     // Aim for about four CTAs per SM over the 148 SMs of a B200, with at least

@@ -11,7 +11,9 @@
 // The array is a file-scope __device__ variable of XKV_NOALLOC_SCRATCH_BYTES (16 MiB).
 // Every GPU that loads the library holds it until the process exits.  Host code cannot
 // use the variable's name as a device address, so the first call on each device (with
-// that device current) asks the runtime for its address once and keeps it.
+// that device current) asks the runtime for its address once and keeps it.  The kept
+// address belongs to the device's current context: a cudaDeviceReset would replace it,
+// so the entry point must not be used after one.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -38,17 +40,13 @@ extern "C" xkv_status xkv_reconstruct_attend_noalloc(const xkv_dims *dims, const
                                                      const int32_t *sel, int32_t n_sel,
                                                      float *out, void *stream) {
     const char *who = "xkv_reconstruct_attend_noalloc";
-    char msg[256];
-    const int32_t mode = sel ? XKV_MODE_SELECTIVE : XKV_MODE_DENSE;
-    const size_t need = xkv_workspace_bytes(dims, sel ? n_sel : 0, mode);
-    if (need > XKV_NOALLOC_SCRATCH_BYTES) {
-        snprintf(msg, sizeof msg,
-                 "%s: this call needs %zu bytes of scratch, above the fixed %zu-byte array; "
-                 "use xkv_reconstruct_attend with a caller-provided workspace",
-                 who, need, XKV_NOALLOC_SCRATCH_BYTES);
-        xkv::set_last_error(msg);
-        return XKV_ERR_UNSUPPORTED;
-    }
+    char msg[320];
+    // Every argument rule first, on the host, under this entry point's name (and its
+    // XKV_FAULT injection); no CUDA call happens before they pass.
+    xkv_status st = xkv::attend_validate(who, dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q,
+                                         sel, n_sel, nullptr, nullptr, 0, 0, out, nullptr,
+                                         XKV_NOALLOC_SCRATCH_BYTES, false, nullptr);
+    if (st != XKV_OK) return st;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -73,9 +71,8 @@ extern "C" xkv_status xkv_reconstruct_attend_noalloc(const xkv_dims *dims, const
         }
         scratch = g_noalloc_ptr[dev];
     }
-    // Arguments are validated (and the launches made) by the workspace entry point; the
-    // partials need no clearing (every one is written before it is read) and the status
-    // word is reset by the kernel that may set it.
-    return xkv_reconstruct_attend(dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel, out,
-                                  scratch, XKV_NOALLOC_SCRATCH_BYTES, stream);
+    // The partials need no clearing (every one is written before it is read) and the
+    // status word is reset by the call's first kernel.
+    return xkv::attend_launch(who, dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel,
+                              nullptr, nullptr, 0, 0, out, scratch, stream);
 }

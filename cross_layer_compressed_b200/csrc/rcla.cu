@@ -490,7 +490,7 @@ bool rcla_tma_ok(const xkv_dims &d, int slot, int64_t L_max, const SplitPlan &pl
     return d.dtype == XKV_BF16 && d.head_dim == 128 && (G == 1 || G == 2 || G == 4 ||
            G == 5 || G == 8) && (int64_t)plan.rows_per_split * G <= 4096 &&
            rows + R3_ROWS < ((int64_t)1 << 31) &&
-           tma_available() && !getenv("XKV_FORCE_SIMT");
+           tma_available() && !env_flag(ENV_FORCE_SIMT);
 }
 
 cudaError_t launch_rcla(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,

@@ -473,8 +473,8 @@ bool rcla_tc_ok(const xkv_dims &d, int slot, int64_t L_max, const SplitPlan &pla
     return d.dtype == XKV_BF16 && d.head_dim == RT_HD &&
            (G == 1 || G == 2 || G == 4 || G == 5 || G == 8) &&
            plan.rows_per_split <= RT_MAX_TILES * RT_ROWS &&
-           rows + RT_ROWS < ((int64_t)1 << 31) && tma_available() && !getenv("XKV_FORCE_SIMT") &&
-           !getenv("XKV_NO_TC");
+           rows + RT_ROWS < ((int64_t)1 << 31) && tma_available() && !env_flag(ENV_FORCE_SIMT) &&
+           !env_flag(ENV_NO_TC);
 }
 
 cudaError_t launch_rcla_tc(const xkv_dims &d, int slot, int64_t L_max, int64_t n_rows,

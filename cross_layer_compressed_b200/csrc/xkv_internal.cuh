@@ -38,6 +38,13 @@ cudaError_t launch_score(const xkv_dims &d, const void *lm, const void *q, doubl
                          cudaStream_t s);
 cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, int n_sink,
                           int n_recent, int32_t *sel, int n_sel, cudaStream_t s);
+// fused scoring + selection (score_select.cu): the selection xkv_select_chunks makes from
+// xkv_score_landmarks' scores, with fp32 scores and an fp64 rescore of the uncertain band
+bool score_select_shape_ok(const xkv_dims &d);   // G in 1..8 or 16
+size_t score_select_ws_bytes(const xkv_dims &d);
+cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q, int top_k,
+                                int n_sink, int n_recent, int32_t *sel, int n_sel, void *ws,
+                                cudaStream_t s);
 cudaError_t launch_attend_simt(const xkv_dims &d, const void *Ak, const void *Av,
                                const void *Bkt, const void *Bvt, const void *q,
                                const int32_t *sel, int n_sel, const SplitPlan &plan,
@@ -116,6 +123,32 @@ cudaError_t launch_chained(void (*k)(P...), dim3 grid, dim3 block, size_t smem, 
 
 // Sets the calling thread's xkv_last_error() message (defined with the C ABI layer).
 void set_last_error(const char *msg);
+
+// Environment switches (documented in include/xkv.h), read once per process:
+// XKV_FORCE_SIMT takes the CUDA-core kernels for both attentions, XKV_NO_TC the TMA +
+// CUDA-core R-CLA kernel, XKV_NO_PDL plain stream order for every launch.
+enum EnvFlag { ENV_FORCE_SIMT = 0, ENV_NO_TC = 1, ENV_NO_PDL = 2 };
+bool env_flag(EnvFlag f);
+
+// Host-side checks of xkv_reconstruct_attend(_tail) and its launches, shared with the
+// allocation-free entry point.  attend_validate checks every argument rule, reports the
+// scratch the call needs in *need_out and checks it against ws_bytes (with check_ws: the
+// caller's workspace ws, too small = XKV_ERR_INVALID_ARG; without: a fixed array of
+// ws_bytes, too small = XKV_ERR_UNSUPPORTED), applies the injected fault of `who` and
+// checks the device; it launches nothing.
+// attend_launch queues the kernels of a validated call on `stream`, with `ws` holding at
+// least that scratch.
+xkv_status attend_validate(const char *who, const xkv_dims *dims, const void *Ak_win,
+                           const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                           const void *q, const int32_t *sel, int32_t n_sel,
+                           const void *K_tail, const void *V_tail, int64_t T_max,
+                           int64_t n_tail, const float *out, const void *ws, size_t ws_bytes,
+                           bool check_ws, size_t *need_out);
+xkv_status attend_launch(const char *who, const xkv_dims *dims, const void *Ak_win,
+                         const void *Av_win, const void *Bkt_layer, const void *Bvt_layer,
+                         const void *q, const int32_t *sel, int32_t n_sel, const void *K_tail,
+                         const void *V_tail, int64_t T_max, int64_t n_tail, float *out,
+                         void *ws, void *stream);
 
 // Workspace layout: a 256-byte header (word 0: device status bits, 1 << xkv_status) and
 // then the partials.

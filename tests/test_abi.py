@@ -311,3 +311,33 @@ def test_refold_argument_checks(xkv, monkeypatch):
     # no tail: NULL is accepted and only the factorization's scratch is added
     need0 = xkv.xkv_refold_workspace_bytes(d, 2, 32, 0)
     assert call(tail=0, n_tail=0, ws_bytes=need0) == 3
+
+
+# --------------------------------------------------- allocation-free reconstruct+attend
+def test_noalloc_arguments_rejected_before_any_cuda_call(xkv, monkeypatch):
+    """xkv_reconstruct_attend_noalloc checks every argument on the host under its own
+    name before it asks CUDA for anything, so these fail the same way with no GPU."""
+    d = _d(xkv)
+
+    def call(dd=d, ptrs=(FAKE,) * 6, n_sel=10, out=FAKE):
+        return xkv.xkv_reconstruct_attend_noalloc(dd, *ptrs, n_sel, out, stream=0, check=False)
+    assert call(dd=_d(xkv, head_dim=96)) == xkv.XKV_ERR_UNSUPPORTED
+    assert call(dd=_d(xkv, chunk=12)) == xkv.XKV_ERR_INVALID_ARG
+    assert "xkv_reconstruct_attend_noalloc" in xkv.last_error()
+    assert call(ptrs=(0,) + (FAKE,) * 5) == xkv.XKV_ERR_INVALID_ARG          # NULL basis
+    assert call(out=0) == xkv.XKV_ERR_INVALID_ARG                           # NULL output
+    assert call(ptrs=(FAKE, FAKE + 8) + (FAKE,) * 4) == xkv.XKV_ERR_INVALID_ARG
+    assert "aligned" in xkv.last_error()
+    assert call(ptrs=(FAKE,) * 5 + (FAKE + 4,)) == xkv.XKV_ERR_INVALID_ARG   # misaligned sel
+    assert call(n_sel=0) == xkv.XKV_ERR_INVALID_ARG                          # n_sel out of range
+    assert call(n_sel=129) == xkv.XKV_ERR_INVALID_ARG
+    # a call whose scratch exceeds the fixed array is refused before any CUDA call
+    big = xkv.dims(64, 512, 32, 128, 1 << 20, 8, 512, 768, xkv.XKV_BF16)
+    assert call(dd=big, ptrs=(FAKE,) * 5 + (None,), n_sel=0) == xkv.XKV_ERR_UNSUPPORTED
+    assert "scratch" in xkv.last_error()
+    # fault injection under this entry point's own name, after the checks
+    monkeypatch.setenv("XKV_FAULT", "xkv_reconstruct_attend_noalloc:4")
+    assert call() == 4 and "injected" in xkv.last_error()
+    assert call(n_sel=0) == xkv.XKV_ERR_INVALID_ARG          # argument errors come first
+    monkeypatch.setenv("XKV_FAULT", "xkv_reconstruct_attend:4")
+    assert call(out=0) == xkv.XKV_ERR_INVALID_ARG
