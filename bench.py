@@ -47,6 +47,12 @@ def parse():
     p.add_argument("--path", choices=["explicit", "reassociated"], default="explicit",
                    help="xKV attention: explicit reconstruction (the method as the pages "
                         "state it) or its rank-space reassociation")
+    p.add_argument("--scoring", choices=["fused", "separate"], default="fused",
+                   help="selective xKV: one fused scoring + selection call per layer "
+                        "(xkv_score_select) or xkv_score_landmarks + xkv_select_chunks")
+    p.add_argument("--layers", type=int, default=0,
+                   help="run only the first N layers of the workload (small cases for "
+                        "profiling; the reported config says so)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call directly instead of replaying a captured step")
@@ -135,12 +141,13 @@ class ClockSampler:
 class XkvStep:
     """Device-resident xKV workload (selective or dense) and its decode step."""
 
-    def __init__(self, w, seed, dev, path="explicit"):
+    def __init__(self, w, seed, dev, path="explicit", scoring="fused"):
         import torch
         from cross_layer_compressed_b200 import synth
         from cross_layer_compressed_b200 import xkv
         self.w, self.dev, self.xkv = w, dev, xkv
         self.path = path
+        self.scoring = scoring
         self.d = xkv.dims_of(w)
         self.cache = synth.torch_xkv_cache(w, seed, device=dev)
         dt = self.cache["Ak"].dtype
@@ -163,15 +170,20 @@ class XkvStep:
                        else xkv.xkv_reconstruct_attend)
         self.scores = torch.empty((w.batch, w.n_kv_heads, max(w.n_chunks, 1)),
                                   dtype=torch.float64, device=dev)
+        self.ws_select = None
+        if not self.dense and scoring == "fused":
+            self.ws_select = torch.empty(xkv.xkv_score_select_workspace_bytes(self.d),
+                                         dtype=torch.uint8, device=dev)
         self.sel = torch.empty((w.n_layers, w.batch, w.n_kv_heads, max(self.n_sel, 1)),
                                dtype=torch.int32, device=dev)
         self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
                                dtype=torch.float32, device=dev)
         self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
-        # our kernels per layer: score + select (selective only), then status clear +
-        # attention + split merge (explicit) or q~ + attention + merge + projection
+        # our kernels per layer: the fused score + select (or score, select), then status
+        # clear + attention + split merge (explicit) or q~ + attention + merge + projection
         # (reassociated; q~ clears the status word)
-        self.launches_per_step = w.n_layers * ((0 if self.dense else 2) +
+        n_sel_kernels = 0 if self.dense else (1 if scoring == "fused" else 2)
+        self.launches_per_step = w.n_layers * (n_sel_kernels +
                                                (4 if path == "reassociated" else 3))
         torch.cuda.synchronize()
 
@@ -181,14 +193,23 @@ class XkvStep:
             n += self.lm.numel() * self.lm.element_size()
         return n
 
-    def step(self, slot=None, q=None, attend_events=None):
+    def step(self, slot=None, q=None, attend_events=None, select_events=None):
         w, xkv, d = self.w, self.xkv, self.d
         qq = self.qpool[slot] if q is None else q
         for l in range(w.n_layers):
             win = l // w.window
             if not self.dense:
-                xkv.xkv_score_landmarks(d, self.lm[l], qq[l], self.scores)
-                xkv.xkv_select_chunks(d, self.scores, w.top_k, w.n_sink, w.n_recent, self.sel[l])
+                if select_events is not None:
+                    select_events[l][0].record()
+                if self.scoring == "fused":
+                    xkv.xkv_score_select(d, self.lm[l], qq[l], w.top_k, w.n_sink, w.n_recent,
+                                         self.sel[l], self.ws_select)
+                else:
+                    xkv.xkv_score_landmarks(d, self.lm[l], qq[l], self.scores)
+                    xkv.xkv_select_chunks(d, self.scores, w.top_k, w.n_sink, w.n_recent,
+                                          self.sel[l])
+                if select_events is not None:
+                    select_events[l][1].record()
             if attend_events is not None:
                 attend_events[l][0].record()
             self.attend(d, self.cache["Ak"][win], self.cache["Av"][win], self.cache["Bkt"][l],
@@ -270,7 +291,7 @@ class RclaStep:
     def resident_bytes(self):
         return 2 * self.K.numel() * self.K.element_size()
 
-    def step(self, slot=None, q=None, attend_events=None):
+    def step(self, slot=None, q=None, attend_events=None, select_events=None):
         w, xkv = self.w, self.xkv
         qq = self.qpool[slot] if q is None else q
         # cache length cycles within the capacity so every step does the same work
@@ -312,25 +333,59 @@ class RclaStep:
 
 
 # --------------------------------------------------------------------- CPU baseline
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _run_units(fn, n_units, threads):
+    """Runs fn(i) for i < n_units on `threads` host threads (the oracle's C calls release
+    the interpreter lock, so the threads run on separate cores); returns the wall time."""
+    from concurrent.futures import ThreadPoolExecutor
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(fn, range(n_units)))
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(w, seed, budget_s=20.0):
-    """The oracle, as it stands, on a bounded sample of one decode step, extrapolated."""
+    """The oracle, as it stands, on a bounded sample of one decode step, run on every host
+    core: independent (sequence, KV head) units of one layer go to a pool of one thread
+    per core, and the step time is extrapolated from the units finished per second."""
     import torch
     import oracle
     from cross_layer_compressed_b200 import synth
     oracle.build()
+    cores = host_cores()
+    G = w.n_q_heads // w.n_kv_heads
     if w.mode == "rcla":
         wl = synth.reduced(w, batch=1, n_layers=1, ctx_len=w.ctx_len, extra_rows=1)
         x = synth.np_rcla_inputs(wl, seed, len_rows=w.ctx_len)
-        K = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
-        V = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
-        t0 = time.perf_counter()
-        oracle.rcla_decode_attend(0, [0], K, V, w.ctx_len, x["k_new"][0], x["v_new"][0],
-                                  x["q"][0])
-        dt = time.perf_counter() - t0
-        scale = w.batch * w.n_layers
-        sample = f"1 sequence x 1 layer (all {w.n_kv_heads} KV heads) of the {w.batch}-sequence x {w.n_layers}-layer step, extrapolated x{scale}"
+        K = x["K_lead"].view(torch.int16).numpy().view(np.uint16)
+        V = x["V_lead"].view(torch.int16).numpy().view(np.uint16)
+        heads = [(np.ascontiguousarray(K[:, :, g:g + 1]), np.ascontiguousarray(V[:, :, g:g + 1]),
+                  x["k_new"][0][:, g:g + 1].contiguous(), x["v_new"][0][:, g:g + 1].contiguous(),
+                  x["q"][0][:, g * G:(g + 1) * G].contiguous()) for g in range(w.n_kv_heads)]
+
+        def unit(i):
+            Kg, Vg, kn, vn, qg = heads[i % w.n_kv_heads]
+            oracle.rcla_decode_attend(0, [0], Kg.copy(), Vg.copy(), w.ctx_len, kn, vn, qg)
+        what = "leader update + attention of one (sequence, KV head)"
     else:
-        # one sequence, one layer, `heads` KV heads: scores, selection, reconstruct+attend
         rng = np.random.default_rng(seed)
         wl = synth.reduced(w, batch=1, n_layers=1, ctx_len=w.ctx_len, n_needles=0)
         Ak = synth.to_storage(synth.np_basis(wl, seed, 0, 0, "k")[None], w.dtype)
@@ -340,25 +395,37 @@ def cpu_baseline(w, seed, budget_s=20.0):
         q = synth.to_storage(synth.np_queries(wl, seed, 0, 0), w.dtype)
         lm = synth.to_storage(rng.standard_normal((1, w.n_kv_heads, w.n_chunks, w.head_dim))
                               * 1e-2, w.dtype) if w.mode != "dense" else None
-        t0 = time.perf_counter()
-        if lm is not None:
-            s = oracle.score_landmarks(lm, q)
-            sel = oracle.select_chunks(s, w.top_k, w.n_sink, w.n_recent)
-        else:
+
+        def unit(i):
+            g = i % w.n_kv_heads
             sel = None
-        heads = 0
-        for g in range(w.n_kv_heads):
+            if lm is not None:
+                s = oracle.score_landmarks(lm[:, g:g + 1].contiguous(),
+                                           q[:, g * G:(g + 1) * G].contiguous())
+                sel = np.zeros((1, w.n_kv_heads, w.n_sel), dtype=np.int32)
+                sel[:, g:g + 1] = oracle.select_chunks(s, w.top_k, w.n_sink, w.n_recent)
             oracle.reconstruct_attend(Ak, Av, Bkt, Bvt, q, sel, w.chunk, units=[(0, g)])
-            heads += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
-        dt = (time.perf_counter() - t0) * w.n_kv_heads / heads
-        scale = w.batch * w.n_layers
-        sample = (f"1 sequence x 1 layer ({heads} of {w.n_kv_heads} KV heads timed, scaled to "
-                  f"all) of the {w.batch}-sequence x {w.n_layers}-layer step, extrapolated x{scale}")
-    step_s = dt * scale
-    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": sample, "sample_seconds": round(dt, 3)}
+        what = ("scoring + selection + reconstruct-attend of one (sequence, KV head)"
+                if w.mode != "dense" else "dense reconstruct-attend of one (sequence, KV head)")
+    # one unit alone sizes the sample: as many units per core as fit the budget
+    t1 = _run_units(unit, 1, 1)
+    per_core = max(1, min(8, int(budget_s / max(t1, 1e-3) / 2)))
+    n_units = cores * per_core
+    wall = _run_units(unit, n_units, cores) if t1 < budget_s else t1
+    if t1 >= budget_s:
+        n_units, used = 1, 1
+    else:
+        used = cores
+    units_per_s = n_units / wall
+    step_units = w.batch * w.n_layers * w.n_kv_heads
+    step_s = step_units / units_per_s
+    sample = (f"{n_units} units ({what}; full-size rows, one layer's factors) on {used} host "
+              f"threads of {cores} cores ({host_cpu_model()}): {units_per_s:.3g} units/s, "
+              f"extrapolated to the {step_units} units of a {w.batch}-sequence x "
+              f"{w.n_layers}-layer step")
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": sample, "sample_seconds": round(wall, 3), "host_cores": cores,
+            "cpu_model": host_cpu_model()}
 
 
 def reference_arm(args, w, rank, world):
@@ -382,8 +449,9 @@ def reference_arm(args, w, rank, world):
             "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "batch": w.batch, "ctx_len": w.ctx_len,
                        "n_layers": w.n_layers},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": r["sample"]},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": r["sample"],
+                             "cpu_model": r["cpu_model"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -685,9 +753,11 @@ def main():
         return
     from cross_layer_compressed_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    import dataclasses
     if args.batch:
-        import dataclasses
         w = dataclasses.replace(w, batch=args.batch)
+    if args.layers:
+        w = dataclasses.replace(w, n_layers=min(args.layers, w.n_layers))
     if args.impl == "reference":
         reference_arm(args, w, rank, world)
         return
@@ -704,7 +774,7 @@ def main():
     from cross_layer_compressed_b200 import build
     build.build()
     wl = RclaStep(w, args.seed + rank, dev) if w.mode == "rcla" else \
-        XkvStep(w, args.seed + rank, dev, args.path)
+        XkvStep(w, args.seed + rank, dev, args.path, args.scoring)
     nq = wl.qpool.shape[0]
     stream = torch.cuda.current_stream(dev)
 
@@ -763,16 +833,22 @@ def main():
 
     # ---------------- per-launch time of the attention kernel: the same steps launched
     # directly, CUDA events around every attention call on the launching stream
-    ev_steps = []
+    def events():
+        return [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                for _ in range(w.n_layers)]
+    ev_steps, sel_steps = [], []
     barrier()
     for s in range(args.steps):
-        ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-              for _ in range(w.n_layers)]
-        wl.step(s % nq, attend_events=ev)
+        ev, sv = events(), events()
+        wl.step(s % nq, attend_events=ev,
+                select_events=sv if w.mode == "sr" else None)
         ev_steps.append(ev)
+        sel_steps.append(sv)
     barrier()
     per_launch = [a.elapsed_time(b) for step in ev_steps for a, b in step]
     attend_avg_ms = float(np.mean(per_launch))
+    select_avg_ms = (float(np.mean([a.elapsed_time(b) for step in sel_steps for a, b in step]))
+                     if w.mode == "sr" else None)
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -797,7 +873,22 @@ def main():
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d, d2h = wl.io_bytes()
         e2e = {"value": aggregate_tokens_per_s(w.batch, args.steps, world, e2e_ms),
-               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "launch": "cuda graph" if e2e_graph is not None else "direct calls"}
+        if e2e_graph is not None:
+            # the same loop with every C-ABI call made directly from the host (argument
+            # checks, tensor-map encoding and the ctypes calls inside the timed region)
+            barrier()
+            e0.record(stream)
+            for s in range(args.steps):
+                wl.q_in.copy_(q_host[s % nq], non_blocking=True)
+                wl.step(q=wl.q_in)
+                out_host.copy_(wl.out, non_blocking=True)
+            e1.record(stream)
+            barrier()
+            direct_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+            e2e["direct_calls_value"] = aggregate_tokens_per_s(w.batch, args.steps, world,
+                                                               direct_ms)
 
     # ---------------- algorithmic bytes (untimed: selections recomputed per slot)
     slots = sorted({s % nq for s in range(args.steps)})[:4]
@@ -851,7 +942,9 @@ def main():
                         "mode": w.mode, "path": args.path})
         if w.mode == "sr":
             cfg.update({"top_k": w.top_k, "n_sink": w.n_sink, "n_recent": w.n_recent,
-                        "n_sel": w.n_sel})
+                        "n_sel": w.n_sel, "scoring": args.scoring})
+        if args.layers:
+            cfg["layers_run"] = f"first {w.n_layers} layers only (profiling case)"
         if w.mode == "rcla":
             cfg.update({"leaders": len(wl.S), "ctx_rows": f"{w.ctx_len}..{w.L_max}"})
         line = {
@@ -863,6 +956,7 @@ def main():
             "step_gbs": step_bytes / (ms_step / 1e3) / 1e9,
             "roofline": roofline,
             "gpu_launches": wl.launches_per_step * args.steps,
+            "score_select_avg_ms": select_avg_ms,
             "cuda_graph": use_graph,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }

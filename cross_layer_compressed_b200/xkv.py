@@ -48,6 +48,9 @@ _sigs = {
     "xkv_score_landmarks": ([_D, _vp, _vp, _vp, _vp], ctypes.c_int),
     "xkv_select_chunks": ([_D, _vp, _i32, _i32, _i32, _vp, ctypes.POINTER(_i32), _vp],
                           ctypes.c_int),
+    "xkv_score_select": ([_D, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.POINTER(_i32), _vp, _sz,
+                          _vp], ctypes.c_int),
+    "xkv_score_select_workspace_bytes": ([_D], _sz),
     "xkv_reconstruct_attend": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp],
                                ctypes.c_int),
     "rcla_decode_attend": ([_D, _i32, _vp, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
@@ -146,6 +149,25 @@ def xkv_select_chunks(d: xkv_dims, scores, top_k, n_sink, n_recent, sel, stream=
         _check(st)
         return n.value
     return st
+
+
+def xkv_score_select(d: xkv_dims, lm_layer, q, top_k, n_sink, n_recent, sel, ws,
+                     ws_bytes=None, stream=None, check=True):
+    """Returns n_sel (or the status when check=False)."""
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    n = _i32(0)
+    st = _lib.xkv_score_select(ctypes.byref(d), _ptr(lm_layer), _ptr(q), int(top_k),
+                               int(n_sink), int(n_recent), _ptr(sel), ctypes.byref(n), _ptr(ws),
+                               int(ws_bytes), _stream(stream))
+    if check:
+        _check(st)
+        return n.value
+    return st
+
+
+def xkv_score_select_workspace_bytes(d: xkv_dims) -> int:
+    return int(_lib.xkv_score_select_workspace_bytes(ctypes.byref(d)))
 
 
 def xkv_reconstruct_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel,

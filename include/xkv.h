@@ -37,6 +37,15 @@
  *  - Inputs holding NaN or Inf are outside the contract.
  *  - The library runs on compute capability 10.0 devices only (XKV_ERR_UNSUPPORTED
  *    otherwise).
+ *  - Environment switches, read once per process on first use:
+ *      XKV_FORCE_SIMT  take the CUDA-core kernels for both attention paths instead of
+ *                      the tensor-core ones (same results within the output tolerance)
+ *      XKV_NO_TC       take the TMA + CUDA-core R-CLA kernel instead of the tensor-core one
+ *      XKV_NO_PDL      launch every kernel in plain stream order (no programmatic
+ *                      dependent launch between the kernels of a call)
+ *      XKV_FAULT       "<entry point>:<status>": that entry point returns the status after
+ *                      its argument checks, launching nothing (fault injection for tests;
+ *                      read on every call)
  */
 #ifndef XKV_H
 #define XKV_H
@@ -131,6 +140,28 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
                              int32_t *n_sel_out, void *stream);
 
 /*
+ * Scoring and selection in one call [xKV 2.3]: sel is bit for bit what
+ * xkv_select_chunks(xkv_score_landmarks(lm_layer, q), top_k, n_sink, n_recent) gives --
+ * the canonical fp64 scores, the forced chunks, the top_k by (score descending, chunk
+ * index ascending), ascending order -- without writing the scores.  The landmarks are
+ * scored in fp32 with a certified error bound; only the chunks whose membership that
+ * bound leaves open (the band around the k-th score) are scored again in fp64, exactly as
+ * xkv_score_landmarks scores them.  Arguments as for those two calls, plus
+ *   ws, ws_bytes: scratch of at least xkv_score_select_workspace_bytes(dims) bytes.  On
+ *       return (in stream order) its first B * Hkv 32-bit words hold, per (b, g), the
+ *       number of chunks rescored in fp64, or 0xFFFFFFFF when the unit was scored wholly
+ *       in fp64 (a band wider than 512 chunks, e.g. many equal scores, or fp32 scores out
+ *       of range); the rest is the fp64 scores of such units.
+ * G = n_q_heads / n_kv_heads in 1..8 or 16; nC <= 16384.  A unit whose fp64 scores hold a
+ * NaN (inputs outside the contract) gets every entry -1.
+ */
+xkv_status xkv_score_select(const xkv_dims *dims, const void *lm_layer, const void *q,
+                            int32_t top_k, int32_t n_sink, int32_t n_recent, int32_t *sel,
+                            int32_t *n_sel_out, void *ws, size_t ws_bytes, void *stream);
+/* Scratch bytes of xkv_score_select (0 on bad dims). */
+size_t xkv_score_select_workspace_bytes(const xkv_dims *dims);
+
+/*
  * Selective (or dense) reconstruction followed by GQA attention
  * [xKV 2.3 "only the rows of the selected tokens are reconstructed from the shared
  * basis and the per-layer matrices"; xKV 4, dense reconstruction].
@@ -186,7 +217,10 @@ xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t
  *   GPU that loads the library until the process exits.  A call whose scratch need
  *   (xkv_workspace_bytes) exceeds 16 MiB returns XKV_ERR_UNSUPPORTED.
  *   The first call on a device (with that device current) looks up the array's device
- *   address once; make that first call before any stream capture.
+ *   address once and keeps it; make that first call before any stream capture, and do
+ *   not use this entry point after cudaDeviceReset (the kept address would be stale).
+ *   Argument errors are reported as by xkv_reconstruct_attend, before any CUDA call;
+ *   XKV_FAULT injection uses this entry point's own name.
  *   Every call on a device shares the one array: calls whose kernels overlap on the GPU
  *   (different streams, or graphs replayed concurrently) race and give wrong results.
  *   Calls queued on one stream are safe.  The function calls no allocator.

@@ -37,3 +37,45 @@ def bf16_ulp_diff(a_u16: np.ndarray, b_u16: np.ndarray) -> np.ndarray:
     a = np.where(a & 0x8000, -(a & 0x7FFF), a)
     b = np.where(b & 0x8000, -(b & 0x7FFF), b)
     return np.abs(a - b)
+
+
+def _gamma(n, u):
+    return n * u / (1 - n * u)
+
+
+def certify_near_ties(lm_gpu, lm_ora, q, sel_gpu, sel_ora, s_ora, G, top_k, n_sink, n_recent):
+    """Checks that every chunk selected on one side only is a certified near-tie and
+    returns the number of units whose selections differ.
+
+    lm_* [B][Hkv][nC][hd] and q [B][Hq][hd] as fp64; s_ora the oracle's scores of lm_ora;
+    sel_gpu is the selection made from lm_gpu, sel_ora the oracle's from lm_ora.
+    beta_c = max_h sum_d |lm_gpu - lm_ora|[c][d] |q_h[d]|
+             + gamma_hd(2^-53) max_h sum_d (|lm_gpu| + |lm_ora|)[c][d] |q_h[d]|
+    bounds |s_gpu(c) - s_ora(c)| (the first term the change of the exact sums, the second
+    the fp64 rounding of both canonical sums).  The k-th candidate score moves by at most
+    beta = max_c beta_c, so a chunk selected on one side only scores within 2 beta of the
+    oracle's k-th score, at or below it if only the GPU side took it, at or above it if
+    only the oracle did."""
+    B, Hkv, nC, hd = lm_ora.shape
+    forced = np.zeros(nC, dtype=bool)
+    forced[:min(n_sink, nC)] = True
+    forced[max(nC - n_recent, 0):] = True
+    k_eff = min(top_k, int((~forced).sum()))
+    n_diff = 0
+    for b in range(B):
+        for g in range(Hkv):
+            a, o = set(sel_gpu[b, g].tolist()), set(sel_ora[b, g].tolist())
+            if a == o:
+                continue
+            n_diff += 1
+            qg = np.abs(q[b, g * G:(g + 1) * G])                       # [G][hd]
+            dl = np.abs(lm_gpu[b, g] - lm_ora[b, g])                    # [nC][hd]
+            mag = (np.abs(lm_ora[b, g]) + np.abs(lm_gpu[b, g])) @ qg.T
+            beta_c = (dl @ qg.T).max(axis=1) + _gamma(hd, 2.0 ** -53) * mag.max(axis=1)
+            beta = beta_c.max() * (1 + 1e-9)
+            tau = np.sort(s_ora[b, g][~forced])[::-1][k_eff - 1]
+            for c in a ^ o:
+                sc = s_ora[b, g, c]
+                assert abs(sc - tau) <= 2 * beta, (b, g, c, sc, tau, beta)
+                assert (sc <= tau) if c in a else (sc >= tau), (b, g, c, sc, tau)
+    return n_diff
