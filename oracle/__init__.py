@@ -48,6 +48,12 @@ def lib():
         L.oracle_n_selected.argtypes = [i64, i32, i32, i32]
         L.oracle_n_selected.restype = i64
         L.oracle_select_chunks.argtypes = [i32, i32, i64, vp, i32, i32, i32, vp, vp]
+        L.oracle_value_ranges.argtypes = [i32, i32, i32, i64, i32, i32, i32, vp, vp, vp]
+        L.oracle_n_reserved.argtypes = [i64, i32, i32, i32]
+        L.oracle_n_reserved.restype = i64
+        L.oracle_reserve_value_chunks.argtypes = [i32, i32, i64, vp, i32, i32, i32, vp, vp]
+        L.oracle_select_chunks_reserved.argtypes = [i32, i32, i64, vp, vp, i32, i32, i32, i32,
+                                                    vp, vp]
         L.oracle_attend_unit.argtypes = [i32, i32, i32, i32, i32, i32, i64, i32, i32, i32,
                                          i32, vp, vp, vp, vp, vp, vp, i64, vp]
         L.oracle_reconstruct_attend.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32, i32,
@@ -169,6 +175,50 @@ def select_chunks(scores: np.ndarray, top_k: int, n_sink: int, n_recent: int) ->
     ns = ctypes.c_int64(0)
     _check(lib().oracle_select_chunks(B, Hkv, nC, _p(s), top_k, n_sink, n_recent, _p(sel),
                                       ctypes.byref(ns)), "select_chunks")
+    return sel
+
+
+def value_ranges(Av, Bvt, n_kv_heads: int, head_dim: int, chunk: int) -> np.ndarray:
+    """rho [B][Hkv][nC] fp64: per chunk, the largest max - min of a reconstructed value row
+    (one KV head's slice) among the chunk's rows."""
+    a, dt = _buf(Av)
+    bt, dt2 = _buf(Bvt)
+    assert dt == dt2
+    B, L, rv = a.shape
+    rho = np.empty((B, n_kv_heads, L // chunk), dtype=np.float64)
+    _check(lib().oracle_value_ranges(B, n_kv_heads, head_dim, L, chunk, rv, dt, _p(a), _p(bt),
+                                     _p(rho)), "value_ranges")
+    return rho
+
+
+def n_reserved(n_chunks: int, n_value: int, n_sink: int, n_recent: int) -> int:
+    return int(lib().oracle_n_reserved(n_chunks, n_value, n_sink, n_recent))
+
+
+def reserve_value_chunks(rho: np.ndarray, n_value: int, n_sink: int, n_recent: int):
+    """reserved [B][Hkv][n_res] int32: the n_res candidates of largest rho, ascending."""
+    r = np.ascontiguousarray(rho, dtype=np.float64)
+    B, Hkv, nC = r.shape
+    n_res = n_reserved(nC, n_value, n_sink, n_recent)
+    out = np.empty((B, Hkv, max(n_res, 0)), dtype=np.int32)
+    _check(lib().oracle_reserve_value_chunks(B, Hkv, nC, _p(r), n_value, n_sink, n_recent,
+                                             _p(out), None), "reserve_value_chunks")
+    return out
+
+
+def select_chunks_reserved(scores: np.ndarray, reserved: np.ndarray, top_k: int, n_sink: int,
+                           n_recent: int) -> np.ndarray:
+    """Selection whose forced chunks also include reserved [B][Hkv][n_res]."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    B, Hkv, nC = s.shape
+    res = np.ascontiguousarray(reserved, dtype=np.int32)
+    n_res = res.shape[2]
+    rest = nC - n_selected(nC, 0, n_sink, n_recent) - n_res
+    n_sel = n_selected(nC, 0, n_sink, n_recent) + n_res + min(top_k, rest)
+    sel = np.empty((B, Hkv, n_sel), dtype=np.int32)
+    _check(lib().oracle_select_chunks_reserved(B, Hkv, nC, _p(s), _p(res) if n_res else None,
+                                               n_res, top_k, n_sink, n_recent, _p(sel), None),
+           "select_chunks_reserved")
     return sel
 
 

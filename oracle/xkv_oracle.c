@@ -14,6 +14,9 @@
  *          O(L*r + W*r*d).  Section 2.3, selective reconstruction: landmark-based
  *          chunk selection, then only the selected rows are rebuilt from A and B_l.
  *          Section 4: dense reconstruction mode.
+ *  [VASE]  "Value-Aware Stochastic KV cache Eviction" technical summary page.  Section
+ *          2.A: the N_v tokens whose value vector has the largest range max(v) - min(v)
+ *          are always kept.
  *  [R-CLA] "Stochastic KV Routing: adaptive depth-wise cache sharing" page.  Inference
  *          uses a fixed sharing set S; a layer outside S reuses the nearest previous
  *          cached layer's KV and skips its own K/V load and update (its Algorithm 2).
@@ -33,6 +36,10 @@
  *  - attention: z = (q . K_hat) / sqrt(hd), softmax over the selected rows,
  *    o = sum p * V_hat; no mask, no positional rotation (the factors represent the
  *    keys as attended);
+ *  - value-range reservation (after the VASE page, section 2.A, applied to chunks): a
+ *    chunk's statistic is the largest max(v) - min(v) over the reconstructed value rows
+ *    of its tokens (one KV head's slice); the n_value largest chunks outside the sink
+ *    and recent windows are kept whatever the scores, in addition to the top-k;
  *  - R-CLA: lead(l) = max{s in S : s <= l}; the cache slot of a leader is its rank
  *    in S; a leader call with a new row writes it at row len and attends len+1 rows;
  *    any other call attends the len rows present.
@@ -276,6 +283,164 @@ int oracle_select_chunks(int B, int Hkv, int64_t nC, const double *scores, int t
         }
     free(cand);
     free(pick);
+    if (n_sel_out)
+        *n_sel_out = n_sel;
+    return 0;
+}
+
+/* ------------------------- [VASE] 2.A value-range reservation, applied to the chunks */
+
+/*
+ * The VASE page keeps, whatever the scores, the N_v tokens whose value vector has the
+ * largest range Range(v) = max(v) - min(v).  Applied to this path's chunk selection:
+ *   rho[b][g][c] = max over the C rows t of chunk c of Range(V_hat[t][g*hd .. g*hd+hd-1]),
+ * V_hat = A^V B^V_l reconstructed exactly in fp64 (one KV head's slice of each row).
+ */
+int oracle_value_ranges(int B, int Hkv, int hd, int64_t L, int C, int rv, int dtype,
+                        const void *Av, const void *Bvt, double *rho)
+{
+    if (B <= 0 || Hkv <= 0 || hd <= 0 || L <= 0 || C <= 0 || L % C || rv <= 0 || !Av ||
+        !Bvt || !rho)
+        return -1;
+    const int64_t nC = L / C, d_kv = (int64_t)Hkv * hd, es = dtype == 1 ? 2 : 4;
+    double *v = malloc(sizeof(double) * hd);
+    if (!v)
+        return -2;
+    for (int b = 0; b < B; ++b) {
+        const char *A = (const char *)Av + (size_t)b * L * rv * es;
+        const char *Bt = (const char *)Bvt + (size_t)b * d_kv * rv * es;
+        for (int g = 0; g < Hkv; ++g)
+            for (int64_t c = 0; c < nC; ++c) {
+                double best = 0.0;
+                for (int64_t t = c * C; t < (c + 1) * C; ++t) {
+                    ora_recon_row(A, Bt, dtype, t, rv, g, hd, v);
+                    double lo = v[0], hi = v[0];
+                    for (int j = 1; j < hd; ++j) {
+                        if (v[j] < lo) lo = v[j];
+                        if (v[j] > hi) hi = v[j];
+                    }
+                    if (hi - lo > best)
+                        best = hi - lo;
+                }
+                rho[((int64_t)b * Hkv + g) * nC + c] = best;
+            }
+    }
+    free(v);
+    return 0;
+}
+
+/* Chunks reserved per (sequence, KV head): min(n_value, chunks outside sink and recent). */
+int64_t oracle_n_reserved(int64_t nC, int n_value, int n_sink, int n_recent)
+{
+    int64_t base = oracle_n_selected(nC, 0, n_sink, n_recent);
+    if (base < 0 || n_value < 0)
+        return -1;
+    int64_t cand = nC - base;
+    return n_value < cand ? n_value : cand;
+}
+
+/*
+ * reserved[b][g][0..n_res) = the n_res chunks outside the sink and recent windows with
+ * the largest rho under (rho descending, index ascending), written in ascending order.
+ */
+int oracle_reserve_value_chunks(int B, int Hkv, int64_t nC, const double *rho, int n_value,
+                                int n_sink, int n_recent, int32_t *reserved,
+                                int64_t *n_res_out)
+{
+    int64_t n_res = oracle_n_reserved(nC, n_value, n_sink, n_recent);
+    if (!rho || B <= 0 || Hkv <= 0 || n_res < 0 || (n_res > 0 && !reserved))
+        return -1;
+    ora_cand *cand = malloc(sizeof(ora_cand) * (nC ? nC : 1));
+    int32_t *pick = malloc(sizeof(int32_t) * (nC ? nC : 1));
+    if (!cand || !pick) {
+        free(cand);
+        free(pick);
+        return -2;
+    }
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hkv; ++g) {
+            const double *r = rho + ((int64_t)b * Hkv + g) * nC;
+            int64_t nc = 0;
+            for (int64_t c = 0; c < nC; ++c) {
+                if ((c < n_sink) || (c >= nC - n_recent))
+                    continue;
+                cand[nc].key = ora_order_key(r[c]);
+                cand[nc].idx = (int32_t)c;
+                ++nc;
+            }
+            qsort(cand, nc, sizeof(ora_cand), ora_cmp_rank);
+            for (int64_t i = 0; i < n_res; ++i)
+                pick[i] = cand[i].idx;
+            qsort(pick, n_res, sizeof(int32_t), ora_cmp_int);
+            if (n_res)
+                memcpy(reserved + ((int64_t)b * Hkv + g) * n_res, pick, sizeof(int32_t) * n_res);
+        }
+    free(cand);
+    free(pick);
+    if (n_res_out)
+        *n_res_out = n_res;
+    return 0;
+}
+
+/*
+ * Selection with value-reserved chunks: the forced chunks are the sink and recent
+ * windows plus reserved[b][g][0..n_res) (chunks outside those windows, no repeats);
+ * then the top_k of the other chunks under (score descending, index ascending); the
+ * union sorted ascending.  n_sel = |sink U recent| + n_res + min(top_k, rest).
+ */
+int oracle_select_chunks_reserved(int B, int Hkv, int64_t nC, const double *scores,
+                                  const int32_t *reserved, int n_res, int top_k, int n_sink,
+                                  int n_recent, int32_t *sel, int64_t *n_sel_out)
+{
+    int64_t base = oracle_n_selected(nC, 0, n_sink, n_recent);
+    if (!scores || !sel || B <= 0 || Hkv <= 0 || base < 0 || n_res < 0 || top_k < 0 ||
+        (n_res > 0 && !reserved) || n_res > nC - base)
+        return -1;
+    const int64_t rest = nC - base - n_res;
+    const int64_t n_sel = base + n_res + (top_k < rest ? top_k : rest);
+    ora_cand *cand = malloc(sizeof(ora_cand) * (nC ? nC : 1));
+    int32_t *pick = malloc(sizeof(int32_t) * (nC ? nC : 1));
+    unsigned char *held = calloc(nC ? nC : 1, 1);
+    if (!cand || !pick || !held) {
+        free(cand);
+        free(pick);
+        free(held);
+        return -2;
+    }
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hkv; ++g) {
+            const double *s = scores + ((int64_t)b * Hkv + g) * nC;
+            const int32_t *res = reserved ? reserved + ((int64_t)b * Hkv + g) * n_res : NULL;
+            memset(held, 0, nC);
+            for (int i = 0; i < n_res; ++i) {
+                int32_t c = res[i];
+                if (c < 0 || c >= nC || held[c] || c < n_sink || c >= nC - n_recent) {
+                    free(cand);
+                    free(pick);
+                    free(held);
+                    return -3;       /* a reserved chunk must be a distinct candidate */
+                }
+                held[c] = 1;
+            }
+            int64_t nc = 0, np = 0;
+            for (int64_t c = 0; c < nC; ++c) {
+                if ((c < n_sink) || (c >= nC - n_recent) || held[c]) {
+                    pick[np++] = (int32_t)c;
+                } else {
+                    cand[nc].key = ora_order_key(s[c]);
+                    cand[nc].idx = (int32_t)c;
+                    ++nc;
+                }
+            }
+            qsort(cand, nc, sizeof(ora_cand), ora_cmp_rank);
+            for (int64_t i = 0; i < nc && i < top_k; ++i)
+                pick[np++] = cand[i].idx;
+            qsort(pick, np, sizeof(int32_t), ora_cmp_int);
+            memcpy(sel + ((int64_t)b * Hkv + g) * n_sel, pick, sizeof(int32_t) * np);
+        }
+    free(cand);
+    free(pick);
+    free(held);
     if (n_sel_out)
         *n_sel_out = n_sel;
     return 0;

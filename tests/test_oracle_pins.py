@@ -689,3 +689,104 @@ if given is not None:
             q, _ = np.linalg.qr(rng.standard_normal((L, r)))
             other = np.sum((Xc - q @ (q.T @ Xc)) ** 2)
             assert other >= res - 1e-9 * tot
+
+
+# -------------------------------------- value-range reservation pins (VASE page, 2.A)
+def test_value_ranges_with_identity_basis_are_row_ranges(ora):
+    """With A^V = I (L = r) the reconstruction is exact and V_hat is B^V_l^T itself, so the
+    statistic is numpy's peak-to-peak of each row's head slice, maxed over the chunk."""
+    rng = np.random.default_rng(7)
+    B, Hkv, hd, C, L = 2, 3, 8, 4, 16
+    d_kv = Hkv * hd
+    V = rng.standard_normal((B, L, d_kv))
+    V[1, 9, 2 * hd + 5] = 40.0                  # one large value: chunk 2 of head 2
+    Av = np.stack([np.eye(L)] * B)              # [B][L][r], r = L
+    Bvt = np.ascontiguousarray(V.transpose(0, 2, 1))   # [B][d_kv][r]: Bvt[j][i] = V[i][j]
+    rho = ora.value_ranges(_f32(Av), _f32(Bvt), Hkv, hd, C)
+    Vf = _f32(V).double().numpy()
+    want = np.ptp(Vf.reshape(B, L // C, C, Hkv, hd), axis=4).max(axis=2).transpose(0, 2, 1)
+    assert np.array_equal(rho, want)
+    assert int(np.argmax(rho[1, 2])) == 2 and rho[1, 2, 2] > 40.0
+
+
+def test_value_ranges_scale_and_shift(ora):
+    """Range is translation invariant per row and scales with |alpha| (a sign flip swaps
+    max and min); a constant row has range 0."""
+    rng = np.random.default_rng(8)
+    B, Hkv, hd, C, L, r = 1, 2, 16, 8, 32, 12
+    Av = rng.standard_normal((B, L, r))
+    Bvt = rng.standard_normal((B, Hkv * hd, r))
+    rho = ora.value_ranges(_f32(Av), _f32(Bvt), Hkv, hd, C)
+    rho_neg = ora.value_ranges(_f32(-2.0 * Av), _f32(Bvt), Hkv, hd, C)
+    assert np.allclose(rho_neg, 2.0 * rho, rtol=1e-12, atol=0)
+    const = np.zeros((B, Hkv * hd, r))
+    const[:, :, 0] = 1.0                        # every head slice of a row is constant
+    assert np.all(ora.value_ranges(_f32(Av), _f32(const), Hkv, hd, C) == 0.0)
+
+
+def _brute_force_reserve(rho, n_value, forced):
+    """Exhaustive: the unique n_res-subset of candidates preceding every other candidate
+    under (rho descending, index ascending)."""
+    return _brute_force_select(rho, n_value, []) if not forced else \
+        [c for c in _brute_force_select(rho, n_value, forced) if c not in forced]
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_reserve_matches_brute_force_with_ties(ora, seed):
+    rng = np.random.default_rng(200 + seed)
+    n = 11
+    rho = rng.integers(0, 4, size=n).astype(np.float64)       # many exact ties
+    for nv, sink, recent in [(3, 1, 1), (0, 1, 2), (2, 0, 0), (20, 1, 1), (4, 2, 3)]:
+        forced = sorted(set(range(sink)) | set(range(n - recent, n)))
+        want = _brute_force_reserve(rho, nv, forced)
+        got = ora.reserve_value_chunks(rho[None, None, :], nv, sink, recent)[0, 0]
+        assert list(got) == want
+        assert ora.n_reserved(n, nv, sink, recent) == len(want)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_select_with_reserved_chunks_matches_brute_force(ora, seed):
+    """The reserved chunks join the forced set; the top-k of the others by score follow."""
+    rng = np.random.default_rng(300 + seed)
+    n = 12
+    scores = rng.integers(-2, 3, size=n).astype(np.float64)
+    for k, sink, recent, res in [(3, 1, 1, [4, 7]), (2, 0, 0, [0]), (4, 1, 2, []),
+                                 (50, 1, 1, [3, 5]), (0, 2, 2, [6])]:
+        forced = sorted(set(range(sink)) | set(range(n - recent, n)) | set(res))
+        want = _brute_force_select(scores, k, forced)
+        resv = np.array(res, dtype=np.int32).reshape(1, 1, -1)
+        got = ora.select_chunks_reserved(scores[None, None, :], resv, k, sink, recent)[0, 0]
+        assert list(got) == want
+
+
+def test_select_with_no_reserved_chunks_is_plain_selection(ora):
+    rng = np.random.default_rng(9)
+    s = rng.standard_normal((2, 3, 200))
+    empty = np.zeros((2, 3, 0), dtype=np.int32)
+    assert np.array_equal(ora.select_chunks_reserved(s, empty, 17, 1, 4),
+                          ora.select_chunks(s, 17, 1, 4))
+
+
+def test_select_with_reserved_rejects_forced_or_repeated_chunks(ora):
+    s = np.zeros((1, 1, 10))
+    with pytest.raises(ValueError):
+        ora.select_chunks_reserved(s, np.array([[[0, 5]]], dtype=np.int32), 2, 1, 1)   # sink
+    with pytest.raises(ValueError):
+        ora.select_chunks_reserved(s, np.array([[[5, 5]]], dtype=np.int32), 2, 1, 1)   # repeat
+
+
+def test_large_range_chunk_is_kept_whatever_its_score(ora):
+    """A chunk whose values span a large range is reserved even when its score is the
+    lowest of all (the point of the VASE reservation)."""
+    rng = np.random.default_rng(10)
+    B, Hkv, hd, C, L, r = 1, 1, 16, 8, 128, 16
+    Av = rng.standard_normal((B, L, r)) * 0.1
+    Av[0, 5 * C + 3] *= 200.0                  # token in chunk 5: a large-range value row
+    Bvt = rng.standard_normal((B, Hkv * hd, r))
+    rho = ora.value_ranges(_f32(Av), _f32(Bvt), Hkv, hd, C)
+    res = ora.reserve_value_chunks(rho, 1, 1, 1)
+    assert list(res[0, 0]) == [5]
+    scores = np.arange(L // C, dtype=np.float64)[None, None, :].copy()
+    scores[0, 0, 5] = -1e9                     # the worst score
+    sel = ora.select_chunks_reserved(scores, res, 3, 1, 1)[0, 0]
+    assert 5 in sel and list(sel) == [0, 5, 12, 13, 14, 15]
