@@ -50,6 +50,10 @@ def parse():
     p.add_argument("--scoring", choices=["fused", "separate"], default="fused",
                    help="selective xKV: one fused scoring + selection call per layer "
                         "(xkv_score_select) or xkv_score_landmarks + xkv_select_chunks")
+    p.add_argument("--value-reserve", type=int, default=0,
+                   help="selective xKV: also keep the N chunks of largest value range per "
+                        "(sequence, KV head) (value-range-aware selection; the statistic and "
+                        "the reserved chunks are built once, at setup)")
     p.add_argument("--layers", type=int, default=0,
                    help="run only the first N layers of the workload (small cases for "
                         "profiling; the reported config says so)")
@@ -141,7 +145,7 @@ class ClockSampler:
 class XkvStep:
     """Device-resident xKV workload (selective or dense) and its decode step."""
 
-    def __init__(self, w, seed, dev, path="explicit", scoring="fused"):
+    def __init__(self, w, seed, dev, path="explicit", scoring="fused", value_reserve=0):
         import torch
         from cross_layer_compressed_b200 import synth
         from cross_layer_compressed_b200 import xkv
@@ -161,6 +165,28 @@ class XkvStep:
                                         self.cache["Bkt"][l], self.lm[l])
         self.qpool = synth.torch_queries(w, seed, self.cache, device=dev)   # [nq][N][B][Hq][hd]
         self.n_sel = 0 if self.dense else w.n_sel
+        # value-range-aware selection: per layer the statistic and the reserved chunks,
+        # built once (setup, timed apart from the step)
+        self.reserved, self.n_res, self.setup_value_ms = None, 0, None
+        if value_reserve and not self.dense:
+            assert scoring == "fused", "reserved chunks go through the fused selection"
+            self.n_res = xkv.xkv_n_reserved(w.n_chunks, value_reserve, w.n_sink, w.n_recent)
+            rho = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float32,
+                              device=dev)
+            self.reserved = torch.empty((w.n_layers, w.batch, w.n_kv_heads, self.n_res),
+                                        dtype=torch.int32, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for l in range(w.n_layers):
+                xkv.xkv_build_value_ranges(self.d, self.cache["Av"][l // w.window],
+                                           self.cache["Bvt"][l], rho)
+                xkv.xkv_reserve_value_chunks(self.d, rho, value_reserve, w.n_sink, w.n_recent,
+                                             self.reserved[l])
+            e1.record()
+            torch.cuda.synchronize()
+            self.setup_value_ms = e0.elapsed_time(e1)
+            base = xkv.xkv_n_selected(w.n_chunks, 0, w.n_sink, w.n_recent)
+            self.n_sel = base + self.n_res + min(w.top_k, w.n_chunks - base - self.n_res)
         mode = xkv.XKV_MODE_DENSE if self.dense else xkv.XKV_MODE_SELECTIVE
         if path == "reassociated":
             mode = xkv.XKV_MODE_REASSOC
@@ -203,7 +229,9 @@ class XkvStep:
                     select_events[l][0].record()
                 if self.scoring == "fused":
                     xkv.xkv_score_select(d, self.lm[l], qq[l], w.top_k, w.n_sink, w.n_recent,
-                                         self.sel[l], self.ws_select)
+                                         self.sel[l], self.ws_select,
+                                         reserved=None if self.reserved is None
+                                         else self.reserved[l], n_reserved=self.n_res)
                 else:
                     xkv.xkv_score_landmarks(d, self.lm[l], qq[l], self.scores)
                     xkv.xkv_select_chunks(d, self.scores, w.top_k, w.n_sink, w.n_recent,
@@ -247,7 +275,7 @@ class XkvStep:
         """Tensor-core flops of one explicit attention launch: the two reconstruction
         GEMMs over the attended rows plus q.K_hat and p.V_hat (dense mode: every row)."""
         w = self.w
-        rows = w.ctx_len if self.dense else w.n_sel * w.chunk
+        rows = w.ctx_len if self.dense else self.n_sel * w.chunk
         return (2.0 * w.batch * w.n_kv_heads * rows * w.head_dim * (w.rank_k + w.rank_v)
                 + 4.0 * w.batch * w.n_q_heads * rows * w.head_dim)
 
@@ -531,10 +559,12 @@ def clf_work(c, r):
     bf16 = 2 * B * L * r * n * (1 + 4 * q + 2)   # X products: test matrix 1 part, others hi+lo
     tf32 = 2 * B * r * r * pass_rows
     fp64 = B * r * (r + 1) * pass_rows           # Gram matrices: r(r+1)/2 dot products
-    own = (2 + 2 * q) + 2 + (y_pass + z_pass) * 4 * KB
-    blas = W + 4 * q * W + 2 * W + (y_pass + z_pass)
+    # products (the library's own GEMM kernel): X Omega, per iteration X^T Q and X Z, the
+    # final X^T Q, and one product with R^-1 per CholeskyQR pass
+    gemm = 1 + 2 * q + 1 + (y_pass + z_pass)
+    own = (2 + 2 * q) + 2 + (y_pass + z_pass) * 4 * KB + gemm
     return {"bf16": bf16, "tf32": tf32, "fp64": fp64, "own_launches": own,
-            "blas_calls": blas}
+            "gemm_launches": gemm}
 
 
 def clf_cpu_baseline(c, seed, rows=2048):
@@ -733,8 +763,7 @@ def run_clf(args, rank, world):
                          "rank_512_call_ms": call_ms[0]},
             "gpu_launches": sum(clf_work(c, k["r"])["own_launches"] for k in calls) * args.steps,
             "refold_reconstruct_flops": (2 * B * L * c["rank_v"] * n) if refold else 0,
-            "library_gemm_calls": sum(clf_work(c, k["r"])["blas_calls"] for k in calls)
-                                  * args.steps,
+            "library_gemm_calls": 0,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -774,7 +803,7 @@ def main():
     from cross_layer_compressed_b200 import build
     build.build()
     wl = RclaStep(w, args.seed + rank, dev) if w.mode == "rcla" else \
-        XkvStep(w, args.seed + rank, dev, args.path, args.scoring)
+        XkvStep(w, args.seed + rank, dev, args.path, args.scoring, args.value_reserve)
     nq = wl.qpool.shape[0]
     stream = torch.cuda.current_stream(dev)
 
@@ -942,7 +971,10 @@ def main():
                         "mode": w.mode, "path": args.path})
         if w.mode == "sr":
             cfg.update({"top_k": w.top_k, "n_sink": w.n_sink, "n_recent": w.n_recent,
-                        "n_sel": w.n_sel, "scoring": args.scoring})
+                        "n_sel": wl.n_sel, "scoring": args.scoring})
+            if args.value_reserve:
+                cfg.update({"value_reserve": args.value_reserve, "n_reserved": wl.n_res,
+                            "setup_value_ranges_ms": wl.setup_value_ms})
         if args.layers:
             cfg["layers_run"] = f"first {w.n_layers} layers only (profiling case)"
         if w.mode == "rcla":

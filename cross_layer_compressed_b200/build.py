@@ -20,8 +20,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
-# cuBLAS serves the plain GEMMs of the prefill-side factorization only
-LIBS = ["-lcublas", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
+LIBS = ["-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 
 
 def sources() -> list[str]:

@@ -281,22 +281,112 @@ size_t xkv_score_select_workspace_bytes(const xkv_dims *dims) {
     return score_select_ws_bytes(*dims);
 }
 
+int64_t xkv_n_reserved(int64_t n_chunks, int32_t n_value, int32_t n_sink, int32_t n_recent) {
+    if (n_chunks < 0 || n_value < 0 || n_sink < 0 || n_recent < 0) return -1;
+    const int64_t cand = n_chunks - n_forced(n_chunks, n_sink, n_recent);
+    return n_value < cand ? n_value : cand;
+}
+
+xkv_status xkv_build_value_ranges(const xkv_dims *dims, const void *Av_win,
+                                  const void *Bvt_layer, float *rho_layer, unsigned *status,
+                                  void *stream) {
+    Range nvtx_range("xkv_build_value_ranges");
+    const char *who = "xkv_build_value_ranges";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (!Av_win || !Bvt_layer || !rho_layer)
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(Av_win) || !aligned16(Bvt_layer) || !aligned16(rho_layer) ||
+        (status && ((uintptr_t)status & 3u)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned (status: 4)",
+                    who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (nC > (int64_t)1 << 31 || (int64_t)dims->batch * dims->ctx_len >= ((int64_t)1 << 31))
+        return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool tc = dims->dtype == XKV_BF16 && tma_available();
+    cudaError_t e = cudaSuccess;
+    if (status) e = cudaMemsetAsync(status, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess && tc)   // the tensor-core epilogue folds chunks in with atomicMax
+        e = cudaMemsetAsync(rho_layer, 0, (size_t)dims->batch * dims->n_kv_heads * nC * 4, s);
+    if (e != cudaSuccess) return launched(e, who);
+    GemmDesc g{};
+    g.mode = GM_VRANGE;
+    g.tc = tc;
+    g.M = (int)dims->ctx_len;
+    g.N = dims->n_kv_heads * dims->head_dim;
+    g.nb = dims->batch;
+    g.nl = 1;
+    g.n_seg = 1;
+    g.P = 1;
+    g.K_seg = dims->rank_v;
+    g.A = Av_win;
+    g.B0 = Bvt_layer;
+    g.L = dims->ctx_len;
+    g.dk = g.N;
+    g.r = dims->rank_v;
+    g.n_rows = g.N;
+    g.W = 1;
+    g.status = status;
+    g.rho = rho_layer;
+    g.hd = dims->head_dim;
+    g.chunk = dims->chunk;
+    g.Hkv = dims->n_kv_heads;
+    g.nC = nC;
+    return launched(launch_gemm(g, s), who);
+}
+
+xkv_status xkv_reserve_value_chunks(const xkv_dims *dims, const float *rho_layer,
+                                    int32_t n_value, int32_t n_sink, int32_t n_recent,
+                                    int32_t *reserved, int32_t *n_res_out, void *stream) {
+    Range nvtx_range("xkv_reserve_value_chunks");
+    const char *who = "xkv_reserve_value_chunks";
+    xkv_status st;
+    if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
+    if (n_value < 0 || n_sink < 0 || n_recent < 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: n_value, n_sink, n_recent must be >= 0", who);
+    const int64_t nC = dims->ctx_len / dims->chunk;
+    if (nC > 16384)
+        return fail(XKV_ERR_UNSUPPORTED, "%s: more than 16384 chunks per unit", who);
+    const int64_t n_res = xkv_n_reserved(nC, n_value, n_sink, n_recent);
+    if (!rho_layer || (n_res > 0 && !reserved))
+        return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+    if (!aligned16(rho_layer) || (reserved && !aligned16(reserved)))
+        return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (n_res_out) *n_res_out = (int32_t)n_res;
+    if (injected(who, &st)) return st;
+    if ((st = check_device(who)) != XKV_OK) return st;
+    if (n_res == 0) return ok();
+    return launched(launch_reserve(*dims, rho_layer, (int)n_res, n_sink, n_recent, reserved,
+                                   (cudaStream_t)stream),
+                    who);
+}
+
 xkv_status xkv_score_select(const xkv_dims *dims, const void *lm_layer, const void *q,
-                            int32_t top_k, int32_t n_sink, int32_t n_recent, int32_t *sel,
+                            int32_t top_k, int32_t n_sink, int32_t n_recent,
+                            const int32_t *reserved, int32_t n_reserved, int32_t *sel,
                             int32_t *n_sel_out, void *ws, size_t ws_bytes, void *stream) {
     Range nvtx_range("xkv_score_select");
     const char *who = "xkv_score_select";
     xkv_status st;
     if ((st = check_dims(dims, true, who)) != XKV_OK) return st;
-    if (!lm_layer || !q || !sel || !ws)
+    if (!lm_layer || !q || !sel || !ws || (n_reserved > 0 && !reserved))
         return fail(XKV_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
-    if (!aligned16(lm_layer) || !aligned16(q) || !aligned16(sel) || !aligned16(ws))
+    if (!aligned16(lm_layer) || !aligned16(q) || !aligned16(sel) || !aligned16(ws) ||
+        (n_reserved > 0 && !aligned16(reserved)))
         return fail(XKV_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
-    if (top_k < 0 || n_sink < 0 || n_recent < 0)
-        return fail(XKV_ERR_INVALID_ARG, "%s: top_k, n_sink, n_recent must be >= 0", who);
+    if (top_k < 0 || n_sink < 0 || n_recent < 0 || n_reserved < 0)
+        return fail(XKV_ERR_INVALID_ARG, "%s: top_k, n_sink, n_recent, n_reserved must be >= 0",
+                    who);
     const int64_t nC = dims->ctx_len / dims->chunk;
     if (nC > 16384)
         return fail(XKV_ERR_UNSUPPORTED, "%s: more than 16384 chunks per unit", who);
+    const int64_t n_base = n_forced(nC, n_sink, n_recent);
+    if (n_reserved > nC - n_base)
+        return fail(XKV_ERR_INVALID_ARG, "%s: more reserved chunks than chunks outside the sink "
+                    "and recent windows", who);
     if (!score_select_shape_ok(*dims))
         return fail(XKV_ERR_UNSUPPORTED, "%s: G = n_q_heads / n_kv_heads must be 1..8 or 16",
                     who);
@@ -304,11 +394,13 @@ xkv_status xkv_score_select(const xkv_dims *dims, const void *lm_layer, const vo
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);
-    const int64_t n_sel = xkv_n_selected(nC, top_k, n_sink, n_recent);
+    const int64_t rest = nC - n_base - n_reserved;
+    const int64_t n_sel = n_base + n_reserved + (top_k < rest ? top_k : rest);
     if (n_sel_out) *n_sel_out = (int32_t)n_sel;
     if (injected(who, &st)) return st;
     if ((st = check_device(who)) != XKV_OK) return st;
-    return launched(launch_score_select(*dims, lm_layer, q, top_k, n_sink, n_recent, sel,
+    return launched(launch_score_select(*dims, lm_layer, q, top_k, n_sink, n_recent,
+                                        n_reserved > 0 ? reserved : nullptr, n_reserved, sel,
                                         (int)n_sel, ws, (cudaStream_t)stream),
                     who);
 }

@@ -86,55 +86,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared
     }
     return false;
 }
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (leading offset unused for this layout; version 1).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) |
-           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                     uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            su32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
-        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, "
-        "%26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
-          "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
-          "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
+// Shared-memory descriptor of a K-major 128-byte-swizzled operand: 8-row groups 1 KB apart.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) { return smem_desc_sw128(saddr, 16, 1024); }
 // Named barrier 1: the epilogue threads.
 __device__ __forceinline__ void epi_bar() {
     asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
@@ -227,9 +180,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    tc_fence_before();
+    tcgen05_before();
     __syncthreads();
-    tc_fence_after();
+    tcgen05_after();
     const uint32_t tmem = sh->tmem_base;
     grid_dep_wait();    // selection, query and status come from the kernels before
     grid_dep_launch();
@@ -292,49 +245,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++ic) {
                 const Item w = decode(p, item);
                 const int nr16 = (w.nr + 15) & ~15;
-                const uint32_t idK = idesc_bf16(128, TC_HD);
-                const uint32_t idV = idesc_bf16(128, nr16);
+                const uint32_t idK = idesc_f16(128, TC_HD, false, false);
+                const uint32_t idV = idesc_f16(128, nr16, false, false);
                 // key phase into columns [0, 256)
                 if (!mbar_wait(&sh->kfree, (ic & 1) ^ 1, sh)) { abort_cta(sh, p); ok = false; break; }
-                tc_fence_after();
+                tcgen05_after();
                 const int nk = p.rk / TC_KS;
                 for (int ks = 0; ks < nk && ok; ++ks, ++it) {
                     const int s = it % TC_STAGES, n = it / TC_STAGES;
                     if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
-                    tc_fence_after();
+                    tcgen05_after();
                     const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
 #pragma unroll
                     for (int kk = 0; kk < TC_KS / 16; ++kk) {
                         const uint32_t acc = (ks | kk) ? 1u : 0u;
-                        umma(tmem, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), idK, acc);
+                        umma_f16(tmem, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), idK, acc);
                         if (w.nr > 128)
-                            umma(tmem + 128, sdesc(a0 + 16384 + kk * 32), sdesc(b0 + kk * 32), idK,
+                            umma_f16(tmem + 128, sdesc(a0 + 16384 + kk * 32), sdesc(b0 + kk * 32), idK,
                                  acc);
                     }
-                    umma_commit(&sh->empty[s]);
+                    umma_arrive(&sh->empty[s]);
                 }
                 if (!ok) break;
-                umma_commit(&sh->kdone);
+                umma_arrive(&sh->kdone);
                 // value phase into columns [256, 512)
                 if (!mbar_wait(&sh->vfree, (ic & 1) ^ 1, sh)) { abort_cta(sh, p); ok = false; break; }
-                tc_fence_after();
+                tcgen05_after();
                 const int nv = p.rv / TC_KS;
                 for (int ks = 0; ks < nv && ok; ++ks, ++it) {
                     const int s = it % TC_STAGES, n = it / TC_STAGES;
                     if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
-                    tc_fence_after();
+                    tcgen05_after();
                     const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
 #pragma unroll
                     for (int kk = 0; kk < TC_KS / 16; ++kk)
-                        umma(tmem + 256, sdesc(b0 + kk * 32), sdesc(a0 + kk * 32), idV,
+                        umma_f16(tmem + 256, sdesc(b0 + kk * 32), sdesc(a0 + kk * 32), idV,
                              (ks | kk) ? 1u : 0u);
-                    umma_commit(&sh->empty[s]);
+                    umma_arrive(&sh->empty[s]);
                 }
                 if (!ok) break;
-                umma_commit(&sh->vdone);
+                umma_arrive(&sh->vdone);
             }
             // all MMAs issued by this thread have completed once `idle` fires
-            umma_commit(&sh->idle);
+            umma_arrive(&sh->idle);
             for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
                 if (mbar_test(&sh->idle, 0)) break;
         }
@@ -360,7 +313,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (fail) abort_cta(sh, p);
                 if (epi_bar_any(fail)) break;     // also publishes qs
             }
-            tc_fence_after();
+            tcgen05_after();
             // key epilogue: thread = token grp*128 + quad*32 + lane
             if (grp * 128 < w.nr) {
                 float acc[G];
@@ -369,7 +322,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll 1
                 for (int c0 = 0; c0 < TC_HD; c0 += 32) {
                     float v[32];
-                    tmem_ld32(tmem + lane_base + grp * 128 + c0, v);
+                    tmem_load32(tmem + lane_base + grp * 128 + c0, v);
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const float *qd = qs + (c0 + c) * G;
@@ -383,7 +336,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     for (int h = 0; h < G; ++h) zs[t * G + h] = acc[h];
                 }
             }
-            tc_fence_before();
+            tcgen05_before();
             epi_bar();
             if (et == 0) mbar_arrive(&sh->kfree);
             // exact softmax statistics of the item's rows (log2 domain)
@@ -436,7 +389,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int k = 0; k < N_EPI; ++k) ll += sh->red[k][h];
                 l[h] = ll;
             }
-            tc_fence_after();
+            tcgen05_after();
             // value epilogue: thread = output column j; tokens [128 grp, 128 grp + 128)
             float o[G];
 #pragma unroll
@@ -445,7 +398,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll 1
             for (int c0 = grp * 128; c0 < tend; c0 += 32) {
                 float v[32];
-                tmem_ld32(tmem + lane_base + 256 + c0, v);
+                tmem_load32(tmem + lane_base + 256 + c0, v);
                 const int nc = tend - c0;      // >= 1; columns past it are not attended
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -456,7 +409,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                 }
             }
-            tc_fence_before();
+            tcgen05_before();
             const int j = quad * 32 + lane;
             if (grp == 1) {
 #pragma unroll
@@ -479,9 +432,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
     }
-    tc_fence_before();
+    tcgen05_before();
     __syncthreads();
-    tc_fence_after();
+    tcgen05_after();
     if (warp == W_MMA)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
                      : "memory");

@@ -23,16 +23,16 @@
 // pivot is below 1e-12 of the largest diagonal entry of G (a direction the data does
 // not have: rank(X) < r) is zeroed rather than normalised.
 //
-// The large products are plain GEMMs and run in cuBLAS on the tensor cores: for bf16
-// caches the fp32 operand (Q, Z) is split into bf16 hi + lo parts (about 16 significant
-// bits; the test matrix is used at bf16 precision, which only makes it another test
-// matrix) and the products with R^-1 use TF32; for fp32 caches every product is a plain
-// fp32 GEMM.  The Gram matrices, the Cholesky factorization and the inversion are this
-// file's own fp64 kernels.
-#include <cublas_v2.h>
+// The large products run in gemm.cu on the tensor cores: for bf16 caches the fp32
+// operand (Q, Z) is split into bf16 hi + lo parts (about 16 significant bits; the test
+// matrix is used at bf16 precision, which only makes it another test matrix) and the
+// products with R^-1 use TF32; for fp32 caches every product is a plain fp32 product on
+// the CUDA cores.  The Gram matrices, the Cholesky factorization and the inversion are
+// this file's own fp64 kernels.
+//
+// Device-side failures (a bounded wait of a product kernel that gave up) set bits in the
+// status word at the start of the workspace; the factors are then written as NaN.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "xkv_internal.cuh"
 
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(256) k_trinv_row(const double *__restrict__ G,
             const int p = ty * 4 + a, q = tx * 4 + c;
             if (p < bi && q < bj) {
                 x[(int64_t)(oi + p) * r + oj + q] = acc[a][c];
-                x32[(int64_t)(oi + p) * r + oj + q] = (float)acc[a][c];
+                x32[(int64_t)(oj + q) * r + oi + p] = (float)acc[a][c];   // transposed
             }
         }
 }
@@ -365,21 +365,24 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 template <typename T>
-__global__ void k_to_storage(const float *__restrict__ src, T *__restrict__ dst, int64_t n) {
+__global__ void k_to_storage(const float *__restrict__ src, T *__restrict__ dst, int64_t n,
+                             const unsigned *__restrict__ status) {
+    const bool failed = *status != 0u;           // a failed call leaves NaN factors
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
-        dst[i] = from_f32<T>(src[i]);
+        dst[i] = from_f32<T>(failed ? __int_as_float(0x7fc00000) : src[i]);
 }
 
 // Z [B][W·d_kv][r] (fp32) -> Bt [W][B][d_kv][r] (storage dtype)
 template <typename T>
 __global__ void k_store_bt(const float *__restrict__ Z, T *__restrict__ Bt, int B, int W,
-                           int64_t dk, int r) {
+                           int64_t dk, int r, const unsigned *__restrict__ status) {
+    const bool failed = *status != 0u;
     const int64_t total = (int64_t)B * W * dk * r;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t i = e % r, j = (e / r) % dk, l = (e / (r * dk)) % W, b = e / (r * dk * W);
-        Bt[((l * B + b) * dk + j) * r + i] = from_f32<T>(Z[e]);
+        Bt[((l * B + b) * dk + j) * r + i] = from_f32<T>(failed ? __int_as_float(0x7fc00000) : Z[e]);
     }
 }
 
@@ -389,23 +392,13 @@ int grid_for(int64_t n) {
 }
 
 // ------------------------------------------------------------------ host side
-std::mutex g_blas_mu;
-
-cublasHandle_t blas_handle() {  // one per device, created on first use (under g_blas_mu)
-    static cublasHandle_t handles[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS)
-        handles[dev] = nullptr;
-    return handles[dev];
-}
-
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Scratch {
+    unsigned *status;       // device-side failures of the call (bits 1 << xkv_status)
     float *y[2], *z[2];
     double *g, *d, *r64, *tol;
-    float *r32;
+    float *r32;             // R^-1 transposed, fp32
     __nv_bfloat16 *hi, *lo, *om_hi;
 };
 
@@ -427,7 +420,8 @@ Shape shape_of(const xkv_dims &d, int W, int r) {
     return s;
 }
 
-// Lays the scratch out in ws (when given) and returns its size.
+// Lays the scratch out in ws (when given) and returns its size: a 256-byte header holding
+// the status word, then the bases and the small factors.
 size_t carve(const Shape &s, void *ws, Scratch *out) {
     char *p = (char *)ws;
     size_t off = 0;
@@ -439,6 +433,7 @@ size_t carve(const Shape &s, void *ws, Scratch *out) {
     const int64_t B = s.B, r = s.r, KB = (r + NB - 1) / NB;
     const int64_t rows_max = s.L > s.n ? s.L : s.n;
     Scratch sc{};
+    sc.status = (unsigned *)take(256);
     for (int i = 0; i < 2; ++i) sc.y[i] = (float *)take((size_t)B * s.L * r * 4);
     for (int i = 0; i < 2; ++i) sc.z[i] = (float *)take((size_t)B * s.n * r * 4);
     sc.g = (double *)take((size_t)B * r * r * 8);
@@ -455,40 +450,16 @@ size_t carve(const Shape &s, void *ws, Scratch *out) {
     return off;
 }
 
-// Row-major C = op(A) op(B) (M x N, inner K), batched over sequences; C in fp32 unless
-// `tc` says otherwise.
-cublasStatus_t rm_gemm(cublasHandle_t h, bool tA, bool tB, int M, int N, int K, const void *A,
-                       cudaDataType ta, int lda, long long sA, const void *Bm, cudaDataType tb,
-                       int ldb, long long sB, void *C, int ldc, long long sC, int batch,
-                       float beta, cublasComputeType_t ct, cudaDataType tc = CUDA_R_32F) {
-    const float alpha = 1.f;
-    return cublasGemmStridedBatchedEx(h, tB ? CUBLAS_OP_T : CUBLAS_OP_N,
-                                      tA ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, Bm, tb,
-                                      ldb, sB, A, ta, lda, sA, &beta, C, tc, ldc, sC, batch, ct,
-                                      CUBLAS_GEMM_DEFAULT);
-}
-
 struct Run {
     Shape s;
     Scratch sc;
-    cublasHandle_t h;
     cudaStream_t st;
     const void *X;
-    cudaDataType xt;
-    cublasComputeType_t exact;   // the products with X
-    cublasComputeType_t apply;   // the products with R^-1
     cudaError_t err = cudaSuccess;
-    bool blas_ok = true;
 
-    bool ok() const { return err == cudaSuccess && blas_ok; }
-    void check(cublasStatus_t b) {
-        if (b != CUBLAS_STATUS_SUCCESS) blas_ok = false;
-    }
+    bool ok() const { return err == cudaSuccess; }
     void check(cudaError_t e) {
         if (e != cudaSuccess && err == cudaSuccess) err = e;
-    }
-    const char *xl(int l) const {  // layer l's cache [B][L][d_kv]
-        return (const char *)X + (size_t)l * s.B * s.L * s.dk * (s.bf16 ? 2 : 4);
     }
 
     void split(const float *src, int64_t n) {
@@ -496,47 +467,76 @@ struct Run {
         check(cudaGetLastError());
     }
 
-    // Y = sum_l X_l F_l, F [B][n][r] fp32; F == nullptr: the test matrix (shared by the
-    // sequences; bf16 caches read its bf16 copy)
-    void x_times(const float *F, const float *omega, float *Y) {
-        const int B = s.B, r = s.r;
-        for (int l = 0; l < s.W && ok(); ++l) {
-            if (s.bf16) {
-                if (F && l == 0) split(F, (int64_t)B * s.n * r);
-                const int parts = F ? 2 : 1;
-                for (int part = 0; part < parts && ok(); ++part) {
-                    const __nv_bfloat16 *f = F ? (part ? sc.lo : sc.hi) + (size_t)l * s.dk * r
-                                               : sc.om_hi + (size_t)l * s.dk * r;
-                    check(rm_gemm(h, false, false, (int)s.L, r, (int)s.dk, xl(l), xt, (int)s.dk,
-                                  s.L * s.dk, f, CUDA_R_16BF, r, F ? s.n * r : 0, Y, r, s.L * r,
-                                  B, (l || part) ? 1.f : 0.f, exact));
-                }
-            } else {
-                const float *f = (F ? F : omega) + (size_t)l * s.dk * r;
-                check(rm_gemm(h, false, false, (int)s.L, r, (int)s.dk, xl(l), xt, (int)s.dk,
-                              s.L * s.dk, f, CUDA_R_32F, r, F ? s.n * r : 0, Y, r, s.L * r, B,
-                              l ? 1.f : 0.f, exact));
-            }
-        }
+    GemmDesc base(int mode) const {
+        GemmDesc g{};
+        g.mode = mode;
+        g.tc = s.bf16;
+        g.nb = s.B;
+        g.nl = 1;
+        g.P = 1;
+        g.n_seg = 1;
+        g.L = s.L;
+        g.dk = s.dk;
+        g.r = s.r;
+        g.n_rows = s.n;
+        g.W = s.W;
+        g.status = sc.status;
+        return g;
     }
 
-    // Z_l = X_l^T Q for every layer: Z [B][n][r] fp32
-    void xt_times(const float *Q, float *Z) {
-        const int B = s.B, r = s.r;
-        if (s.bf16) split(Q, (int64_t)B * s.L * r);
-        for (int l = 0; l < s.W && ok(); ++l) {
-            if (s.bf16) {
-                for (int part = 0; part < 2 && ok(); ++part)
-                    check(rm_gemm(h, true, false, (int)s.dk, r, (int)s.L, xl(l), xt, (int)s.dk,
-                                  s.L * s.dk, part ? sc.lo : sc.hi, CUDA_R_16BF, r, s.L * r,
-                                  Z + (size_t)l * s.dk * r, r, s.n * r, B, part ? 1.f : 0.f,
-                                  exact));
+    // Y = sum_l X_l F_l, F [B][n][r] fp32; F == nullptr: the test matrix (shared by the
+    // sequences; bf16 caches read its bf16 copy).  One product: the layers (and the hi /
+    // lo parts of F) are consecutive K segments of one accumulation.
+    void x_times(const float *F, const float *omega, float *Y) {
+        GemmDesc g = base(GM_XF);
+        g.M = (int)s.L;
+        g.N = s.r;
+        g.K_seg = s.dk;
+        g.A = X;
+        if (s.bf16) {
+            if (F) {
+                split(F, (int64_t)s.B * s.n * s.r);
+                g.P = 2;
+                g.B0 = sc.hi;
+                g.B1 = sc.lo;
             } else {
-                check(rm_gemm(h, true, false, (int)s.dk, r, (int)s.L, xl(l), xt, (int)s.dk,
-                              s.L * s.dk, Q, CUDA_R_32F, r, s.L * r, Z + (size_t)l * s.dk * r,
-                              r, s.n * r, B, 0.f, exact));
+                g.B0 = sc.om_hi;
+                g.b_shared = 1;
             }
+        } else {
+            g.B0 = F ? F : omega;
+            g.b_shared = F ? 0 : 1;
         }
+        g.n_seg = s.W * g.P;
+        g.C = Y;
+        g.ldc = s.r;
+        g.c_b = s.L * s.r;
+        if (ok()) check(launch_gemm(g, st));
+    }
+
+    // Z_l = X_l^T Q for every layer: Z [B][n][r] fp32 (the hi and lo parts of Q are two K
+    // segments of one accumulation)
+    void xt_times(const float *Q, float *Z) {
+        GemmDesc g = base(GM_XT);
+        g.M = (int)s.dk;
+        g.N = s.r;
+        g.nl = s.W;
+        g.K_seg = s.L;
+        g.A = X;
+        if (s.bf16) {
+            split(Q, (int64_t)s.B * s.L * s.r);
+            g.P = 2;
+            g.B0 = sc.hi;
+            g.B1 = sc.lo;
+        } else {
+            g.B0 = Q;
+        }
+        g.n_seg = g.P;
+        g.C = Z;
+        g.ldc = s.r;
+        g.c_b = s.n * s.r;
+        g.c_l = s.dk * s.r;
+        if (ok()) check(launch_gemm(g, st));
     }
 
     // CholeskyQR of the rows x r matrices in buf[0] (buf[1]: the other ping-pong half),
@@ -569,9 +569,18 @@ struct Run {
                                                                     sc.r32);
             check(cudaGetLastError());
             if (!ok()) return;
-            check(rm_gemm(h, false, false, (int)rows, r, r, src, CUDA_R_32F, r, rows * r,
-                          sc.r32, CUDA_R_32F, r, (long long)r * r, dst, r, rows * r, B, 0.f,
-                          apply));
+            // dst = src R^-1 (TF32 on the tensor cores for bf16 caches)
+            GemmDesc g = base(GM_APPLY);
+            g.M = (int)rows;
+            g.N = r;
+            g.K_seg = r;
+            g.L = rows;
+            g.A = src;
+            g.B0 = sc.r32;
+            g.C = dst;
+            g.ldc = r;
+            g.c_b = rows * r;
+            check(launch_gemm(g, st));
             buf[0] = dst;
             buf[1] = src;
         }
@@ -587,27 +596,20 @@ cudaError_t set_block_smem() {
     return e;
 }
 
+// clear_status: false when the caller (the refold) already cleared the call's status word
 template <typename T>
 cudaError_t factorize_t(const Shape &s, const void *X, const float *omega, int n_iter,
-                        void *A_out, void *Bt_out, void *ws, cudaStream_t st) {
+                        void *A_out, void *Bt_out, void *ws, cudaStream_t st, bool clear_status) {
     cudaError_t e = set_block_smem();
     if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> lock(g_blas_mu);
-    cublasHandle_t h = blas_handle();
-    if (!h || cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return cudaErrorNotReady;
     Run run;
     run.s = s;
     carve(s, ws, &run.sc);
-    run.h = h;
     run.st = st;
     run.X = X;
-    run.xt = s.bf16 ? CUDA_R_16BF : CUDA_R_32F;
-    // bf16 x bf16 products are exact in fp32, so the tensor cores lose nothing there;
-    // fp32 caches keep every product in plain fp32
-    run.exact = s.bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC;
-    run.apply = s.bf16 ? CUBLAS_COMPUTE_32F_FAST_TF32 : CUBLAS_COMPUTE_32F_PEDANTIC;
     const int B = s.B, r = s.r;
     const Scratch &sc = run.sc;  // y[0] / z[0] follow the ping-pong of orth()
+    if (clear_status) run.check(cudaMemsetAsync(sc.status, 0, sizeof(unsigned), st));
 
     if (s.bf16) {
         k_split_hi_lo<<<grid_for(s.n * r), 256, 0, st>>>(omega, sc.om_hi, sc.lo, s.n * r);
@@ -626,52 +628,69 @@ cudaError_t factorize_t(const Shape &s, const void *X, const float *omega, int n
     }
     if (run.ok()) {
         const int64_t na = (int64_t)B * s.L * r;
-        k_to_storage<T><<<grid_for(na), 256, 0, st>>>(sc.y[0], (T *)A_out, na);
+        k_to_storage<T><<<grid_for(na), 256, 0, st>>>(sc.y[0], (T *)A_out, na, sc.status);
         run.check(cudaGetLastError());
         run.xt_times(sc.y[0], sc.z[0]);
         const int64_t nb = (int64_t)B * s.n * r;
         if (run.ok())
-            k_store_bt<T><<<grid_for(nb), 256, 0, st>>>(sc.z[0], (T *)Bt_out, B, s.W, s.dk, r);
+            k_store_bt<T><<<grid_for(nb), 256, 0, st>>>(sc.z[0], (T *)Bt_out, B, s.W, s.dk, r,
+                                                         sc.status);
         run.check(cudaGetLastError());
     }
-    if (run.err != cudaSuccess) return run.err;
-    return run.blas_ok ? cudaSuccess : cudaErrorUnknown;
+    return run.err;
 }
 
 // Refold (the decode loop's tail of generated rows folded back into the factors): the
-// extended caches [A·B_l ; tail_l] are built in the workspace -- the reconstruction in
-// the storage type, as the decode calls would see it -- and factored again.
+// extended caches [A·B_l ; tail_l] are built in the workspace after the factorization's
+// scratch -- the reconstruction in the storage type, as the decode calls would see it --
+// and factored again.
 template <typename T>
 cudaError_t refold_t(const Shape &s, int64_t n_tail, const void *A, const void *Bt,
                      const void *tail, const float *omega, int n_iter, void *A_out,
-                     void *Bt_out, void *ws, size_t x_bytes, cudaStream_t st) {
+                     void *Bt_out, void *ws, cudaStream_t st) {
     const int64_t L = s.L - n_tail, e = sizeof(T);
-    char *xbuf = (char *)ws;
-    {
-        std::lock_guard<std::mutex> lock(g_blas_mu);
-        cublasHandle_t h = blas_handle();
-        if (!h || cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return cudaErrorNotReady;
-        const cudaDataType dt = s.bf16 ? CUDA_R_16BF : CUDA_R_32F;
-        const cublasComputeType_t ct = s.bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC;
+    Scratch sc{};
+    const size_t fac_bytes = carve(s, ws, &sc);
+    char *xbuf = (char *)ws + fac_bytes;
+    cudaError_t c = cudaMemsetAsync(sc.status, 0, sizeof(unsigned), st);
+    if (c != cudaSuccess) return c;
+    // X'_l[b][0:L] = A_b B_l,b for every layer (B_l stored column-major: Bt_l,b d_kv x r)
+    GemmDesc g{};
+    g.mode = GM_REFOLD;
+    g.tc = s.bf16;
+    g.M = (int)L;
+    g.N = (int)s.dk;
+    g.nb = s.B;
+    g.nl = s.W;
+    g.n_seg = 1;
+    g.P = 1;
+    g.K_seg = s.r;
+    g.A = A;
+    g.B0 = Bt;
+    g.L = L;
+    g.dk = s.dk;
+    g.r = s.r;
+    g.n_rows = s.n;
+    g.W = s.W;
+    g.C = xbuf;
+    g.c_bf16 = s.bf16;
+    g.ldc = s.dk;
+    g.c_b = s.L * s.dk;
+    g.c_l = (int64_t)s.B * s.L * s.dk;
+    g.status = sc.status;
+    c = launch_gemm(g, st);
+    if (c != cudaSuccess) return c;
+    if (n_tail > 0) {
         for (int l = 0; l < s.W; ++l) {
-            // X'_l[b][0:L] = A_b B_l,b (B_l stored column-major: Bt_l,b is d_kv x r)
-            const cublasStatus_t bs =
-                rm_gemm(h, false, true, (int)L, (int)s.dk, s.r, A, dt, s.r, L * s.r,
-                        (const char *)Bt + (size_t)l * s.B * s.dk * s.r * e, dt, s.r,
-                        s.dk * s.r, xbuf + (size_t)l * s.B * s.L * s.dk * e, (int)s.dk,
-                        s.L * s.dk, s.B, 0.f, ct, dt);
-            if (bs != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
-            if (n_tail > 0) {
-                cudaError_t c = cudaMemcpy2DAsync(
-                    xbuf + ((size_t)l * s.B * s.L + L) * s.dk * e, (size_t)s.L * s.dk * e,
-                    (const char *)tail + (size_t)l * s.B * n_tail * s.dk * e,
-                    (size_t)n_tail * s.dk * e, (size_t)n_tail * s.dk * e, (size_t)s.B,
-                    cudaMemcpyDeviceToDevice, st);
-                if (c != cudaSuccess) return c;
-            }
+            c = cudaMemcpy2DAsync(
+                xbuf + ((size_t)l * s.B * s.L + L) * s.dk * e, (size_t)s.L * s.dk * e,
+                (const char *)tail + (size_t)l * s.B * n_tail * s.dk * e,
+                (size_t)n_tail * s.dk * e, (size_t)n_tail * s.dk * e, (size_t)s.B,
+                cudaMemcpyDeviceToDevice, st);
+            if (c != cudaSuccess) return c;
         }
     }
-    return factorize_t<T>(s, xbuf, omega, n_iter, A_out, Bt_out, xbuf + x_bytes, st);
+    return factorize_t<T>(s, xbuf, omega, n_iter, A_out, Bt_out, ws, st, false);
 }
 
 size_t refold_x_bytes(const Shape &s) {
@@ -693,11 +712,10 @@ cudaError_t launch_refold(const xkv_dims &d, int W, int r, const void *A, const 
     xkv_dims e = d;
     e.ctx_len = d.ctx_len + n_tail;
     const Shape sh = shape_of(e, W, r);
-    const size_t xb = refold_x_bytes(sh);
     return sh.bf16 ? refold_t<__nv_bfloat16>(sh, n_tail, A, Bt, tail, omega, n_iter, A_out,
-                                             Bt_out, ws, xb, s)
+                                             Bt_out, ws, s)
                    : refold_t<float>(sh, n_tail, A, Bt, tail, omega, n_iter, A_out, Bt_out, ws,
-                                     xb, s);
+                                     s);
 }
 
 size_t factorize_ws_bytes(const xkv_dims &d, int W, int r) {
@@ -707,8 +725,8 @@ size_t factorize_ws_bytes(const xkv_dims &d, int W, int r) {
 cudaError_t launch_factorize(const xkv_dims &d, int W, int r, const void *X, const float *omega,
                              int n_iter, void *A_out, void *Bt_out, void *ws, cudaStream_t s) {
     const Shape sh = shape_of(d, W, r);
-    return sh.bf16 ? factorize_t<__nv_bfloat16>(sh, X, omega, n_iter, A_out, Bt_out, ws, s)
-                   : factorize_t<float>(sh, X, omega, n_iter, A_out, Bt_out, ws, s);
+    return sh.bf16 ? factorize_t<__nv_bfloat16>(sh, X, omega, n_iter, A_out, Bt_out, ws, s, true)
+                   : factorize_t<float>(sh, X, omega, n_iter, A_out, Bt_out, ws, s, true);
 }
 
 }  // namespace xkv

@@ -24,8 +24,9 @@
 // cluster streams its slice of the unit's landmark rows (one row per thread, 16-byte
 // loads, the group's query in shared memory) and sends its fp32 keys to CTA 0's shared
 // memory; CTA 0 then runs steps 2-3 and writes the selection in ascending chunk order.
-// Units whose fp32 scores are not all finite or whose band is wider than BAND_CAP chunks
-// take the exact path for the whole unit: every chunk is
+// Optionally a per-unit list of reserved chunks (the value-range reservation) joins the
+// sink and recent chunks as forced.  Units whose fp32 scores are not all finite or whose
+// band is wider than BAND_CAP chunks take the exact path for the whole unit: every chunk is
 // scored in fp64 into the workspace and the full radix select runs on those keys.  The
 // workspace also records, per unit, the band size (or ~0 for the exact path).
 //
@@ -50,6 +51,7 @@ constexpr int HIST_BINS = 2048;                   // radix digits of 11, 11 and 
 constexpr int RANK_CAP = 256;                     // keys of a bin ranked directly
 constexpr int BAND_CAP = 512;                     // band chunks rescored in fp64
 constexpr uint32_t EXACT_PATH = 0xFFFFFFFFu;
+constexpr uint32_t BAD_RESERVED = 0xFFFFFFFEu;   // a reserved list broke its rules
 
 struct SsParams {
     const void *lm;       // [B][Hkv][nC][hd]
@@ -61,6 +63,8 @@ struct SsParams {
     int Hq, Hkv, hd;
     int top_k, n_sink, n_recent, n_sel;
     int cpc;              // chunks per CTA (a multiple of 4)
+    const int32_t *reserved;   // [B][Hkv][n_res] chunks forced in as well, or null
+    int n_res;
     double err_rel;       // (gamma_hd(2^-24) + gamma_hd(2^-53)) (1 + 2^-20)
     double err_abs;       // hd 2^-150 (1 + 2^-20)
 };
@@ -276,10 +280,11 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     uint32_t *keys = reinterpret_cast<uint32_t *>(ss_smem + 4 * hd * G);   // [nC] fp32 keys
     uint32_t *r1 = keys + ((nC + 3) & ~3);                                  // [HIST_BINS]
     uint32_t *bits = r1 + HIST_BINS;                                        // [nC / 32]
+    uint32_t *rbits = bits + (nC + 31) / 32;                                // [nC / 32]
     __shared__ float s_mx[SS_MAX_CLUSTER];
     __shared__ int s_bad[SS_MAX_CLUSTER];
     __shared__ RadixShared rs;
-    __shared__ int s_bad_cta, s_exact;
+    __shared__ int s_bad_cta, s_exact, s_bad_res;
     __shared__ unsigned s_cnt, s_nin, s_bin, s_above, s_tkey;
     __shared__ float s_mx_cta;
 
@@ -298,13 +303,24 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     }
     if (rank == 0) {
         for (int i = threadIdx.x; i < HIST_BINS; i += SS_THREADS) r1[i] = 0u;
-        for (int i = threadIdx.x; i < (nC + 31) / 32; i += SS_THREADS) bits[i] = 0u;
+        for (int i = threadIdx.x; i < (nC + 31) / 32; i += SS_THREADS) bits[i] = rbits[i] = 0u;
     }
     if (threadIdx.x == 0) {
         s_bad_cta = 0;
         s_mx_cta = 0.f;
+        s_bad_res = 0;
     }
     __syncthreads();
+    if (rank == 0 && p.n_res > 0) {
+        // the reserved chunks join the forced set: distinct chunks outside sink and recent
+        const int32_t *res = p.reserved + (size_t)unit * p.n_res;
+        for (int i = threadIdx.x; i < p.n_res; i += SS_THREADS) {
+            const int c = res[i];
+            bool bad = c < 0 || c >= nC || c < p.n_sink || c >= nC - p.n_recent;
+            if (!bad) bad = (atomicOr(&rbits[c >> 5], 1u << (c & 31)) >> (c & 31)) & 1u;
+            if (bad) s_bad_res = 1;
+        }
+    }
 
     // ---------------------------------------------------------------- fp32 pass
     constexpr int EPV = Vec<T>::N;
@@ -389,8 +405,17 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     // ---------------------------------------------------------------- CTA 0: selection
     const int ncl = (int)((nC + p.cpc - 1) / p.cpc);
     const int f_lo = min(p.n_sink, nC), f_hi = max(nC - p.n_recent, 0);
-    auto forced = [&](int c) { return c < p.n_sink || c >= nC - p.n_recent; };
-    const int n_forced = f_lo + (nC - f_hi) - max(0, f_lo - f_hi);
+    auto forced = [&](int c) {
+        return c < p.n_sink || c >= nC - p.n_recent || ((rbits[c >> 5] >> (c & 31)) & 1u);
+    };
+    if (s_bad_res) {
+        // a reserved list that is not a set of distinct candidates: the unit selects nothing
+        for (int i = threadIdx.x; i < p.n_sel; i += SS_THREADS)
+            p.sel[(size_t)unit * p.n_sel + i] = -1;
+        if (threadIdx.x == 0) p.band[unit] = BAD_RESERVED;
+        return;
+    }
+    const int n_forced = f_lo + (nC - f_hi) - max(0, f_lo - f_hi) + p.n_res;
     const int n_cand = nC - n_forced;
     const int k_eff = min(p.top_k, n_cand);
     const bool all_cand = k_eff == n_cand;         // every candidate is taken
@@ -575,11 +600,43 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     if (threadIdx.x == 0) p.band[unit] = band_size;
 }
 
+// The value-range reservation (VASE page, section 2.A, applied to chunks): per (b, g) the
+// n_res chunks outside the sink and recent windows with the largest rho, under (rho
+// descending, index ascending), written in ascending order.  rho is fp32; its keys are
+// those of the value widened to fp64, so the order is exactly the oracle's on the same
+// statistics.
+__global__ void __launch_bounds__(SS_THREADS) k_reserve(const float *__restrict__ rho,
+                                                        int32_t *__restrict__ reserved,
+                                                        int nC, int n_res, int n_sink,
+                                                        int n_recent) {
+    __shared__ RadixShared rs;
+    __shared__ uint32_t bits[16384 / 32];
+    const int unit = blockIdx.x;
+    const float *r = rho + (size_t)unit * nC;
+    for (int i = threadIdx.x; i < (nC + 31) / 32; i += SS_THREADS) bits[i] = 0u;
+    __syncthreads();
+    auto forced = [&](int c) { return c < n_sink || c >= nC - n_recent; };
+    radix_select(nC, (unsigned)n_res, [&](int c) { return order_key((double)r[c]); },
+                 [&](int c) { return !forced(c); },
+                 [&](int c) { atomicOr(&bits[c >> 5], 1u << (c & 31)); }, rs);
+    const int ipt = (nC + SS_THREADS - 1) / SS_THREADS;
+    const int lo = min(nC, (int)threadIdx.x * ipt), hi = min(nC, lo + ipt);
+    unsigned n_local = 0;
+    for (int c = lo; c < hi; ++c) n_local += (bits[c >> 5] >> (c & 31)) & 1u;
+    unsigned pos = block_scan(n_local, rs);
+    int32_t *out = reserved + (size_t)unit * n_res;
+    for (int c = lo; c < hi; ++c)
+        if ((bits[c >> 5] >> (c & 31)) & 1u) {
+            if (pos < (unsigned)n_res) out[pos] = c;
+            ++pos;
+        }
+}
+
 size_t ss_smem_bytes(const xkv_dims &d) {
     const int G = d.n_q_heads / d.n_kv_heads;
     const int64_t nC = d.ctx_len / d.chunk;
     return (size_t)4 * d.head_dim * G + 4 * (size_t)((nC + 3) & ~3) + 4 * HIST_BINS +
-           4 * (size_t)((nC + 31) / 32);
+           8 * (size_t)((nC + 31) / 32);
 }
 
 double gamma_n(int n, double u) { return n * u / (1.0 - n * u); }
@@ -675,9 +732,16 @@ size_t score_select_ws_bytes(const xkv_dims &d) {
 
 size_t score_select_smem_bytes(const xkv_dims &d) { return ss_smem_bytes(d); }
 
+cudaError_t launch_reserve(const xkv_dims &d, const float *rho, int n_res, int n_sink,
+                           int n_recent, int32_t *reserved, cudaStream_t s) {
+    k_reserve<<<d.batch * d.n_kv_heads, SS_THREADS, 0, s>>>(
+        rho, reserved, (int)(d.ctx_len / d.chunk), n_res, n_sink, n_recent);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q, int top_k,
-                                int n_sink, int n_recent, int32_t *sel, int n_sel, void *ws,
-                                cudaStream_t s) {
+                                int n_sink, int n_recent, const int32_t *reserved, int n_res,
+                                int32_t *sel, int n_sel, void *ws, cudaStream_t s) {
     const size_t units = (size_t)d.batch * d.n_kv_heads;
     SsParams p;
     p.lm = lm;
@@ -694,6 +758,8 @@ cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q
     p.n_recent = n_recent;
     p.n_sel = n_sel;
     p.cpc = 0;
+    p.reserved = reserved;
+    p.n_res = reserved ? n_res : 0;
     const double slack = 1.0 + 0x1p-20;
     p.err_rel = (gamma_n(d.head_dim, 0x1p-24) + gamma_n(d.head_dim, 0x1p-53)) * slack;
     p.err_abs = d.head_dim * 0x1p-150 * slack;

@@ -50,6 +50,14 @@ static __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint6
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(su32(bar))
         : "memory");
 }
+static __device__ __forceinline__ void tma_load_4d(const CUtensorMap *map, uint64_t *bar, void *dst,
+                                            int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(su32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(su32(bar))
+        : "memory");
+}
 static __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -80,6 +88,19 @@ static __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint3
 static __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
            ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Instruction descriptor, kind::tf32: tf32 x tf32 -> fp32 (both formats code 2).
+static __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+static __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 static __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
                                                 uint32_t idesc, uint32_t accumulate) {
@@ -132,8 +153,32 @@ static __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+static __device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, "
+        "%26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+          "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // ---------------------------------------------------------------- host side
 bool tma_available();
+// Tensor map of rank 1..5 over bf16 (f32 = false) or fp32 elements with the 128-byte
+// swizzle: dims[0] innermost, strides[i] = bytes between consecutive indices of dimension
+// i + 1, box[i] elements per dimension (box[0] * element size <= 128).
+bool make_map_sw128(CUtensorMap *m, const void *base, bool f32, int rank, const uint64_t *dims,
+                    const uint64_t *strides, const uint32_t *box);
 // 2D bf16 tensor map over a row-major [rows][cols] array, boxes of box_rows x 64 elements
 // (128 bytes) written to shared memory with the 128-byte swizzle.
 bool make_map_bf16_sw128(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,

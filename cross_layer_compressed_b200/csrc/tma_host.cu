@@ -66,6 +66,24 @@ int sm_count_impl() {
 }  // namespace
 
 bool tma_available() { return encode_fn() != nullptr; }
+bool make_map_sw128(CUtensorMap *m, const void *base, bool f32, int rank, const uint64_t *dims,
+                    const uint64_t *strides, const uint32_t *box) {
+    auto fn = encode_fn();
+    if (!fn || rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], estr[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        estr[i] = 1;
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+              (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 bool make_map_bf16_sw128(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                          uint32_t box_rows) {
     return make_map_impl(m, base, rows, cols, box_rows);

@@ -43,8 +43,11 @@ cudaError_t launch_select(const xkv_dims &d, const double *scores, int top_k, in
 bool score_select_shape_ok(const xkv_dims &d);   // G in 1..8 or 16
 size_t score_select_ws_bytes(const xkv_dims &d);
 cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q, int top_k,
-                                int n_sink, int n_recent, int32_t *sel, int n_sel, void *ws,
-                                cudaStream_t s);
+                                int n_sink, int n_recent, const int32_t *reserved, int n_res,
+                                int32_t *sel, int n_sel, void *ws, cudaStream_t s);
+// value-range reservation: per (b, g) the n_res candidates of largest rho, ascending
+cudaError_t launch_reserve(const xkv_dims &d, const float *rho, int n_res, int n_sink,
+                           int n_recent, int32_t *reserved, cudaStream_t s);
 cudaError_t launch_attend_simt(const xkv_dims &d, const void *Ak, const void *Av,
                                const void *Bkt, const void *Bvt, const void *q,
                                const int32_t *sel, int n_sel, const SplitPlan &plan,
@@ -79,6 +82,34 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
                              const void *Bvt, const void *q, const int32_t *sel, int n_sel,
                              float *partials, unsigned *status, int *n_split_out,
                              cudaStream_t s);
+
+// The dense products of the factorization (gemm.cu), batched over sequences (nb) and an
+// outer index (nl), each a sum over n_seg K segments of K_seg:
+//   GM_XF      C[b]    = sum_s X[s / P][b] F_{s % P}[b][(s / P) d_kv ...]   (Y = X Omega / X Z)
+//   GM_XT      C[l][b] = sum_s X[l][b]^T Q_s[b]                             (Z_l = X_l^T Q)
+//   GM_APPLY   C[b]    = A[b] (R^-1)[b], B0 holding (R^-1)^T                (Y R^-1)
+//   GM_REFOLD  C[l][b] = A[b] Bt[l][b]^T                                    (A B_l)
+// tc: bf16 operands (TF32 for GM_APPLY) on the tensor cores; else fp32 on the CUDA cores.
+//   GM_VRANGE  rho[b][g][c] = max over chunk c's rows of max - min of A[b] Bt[b]^T's
+//              head-g columns (atomicMax into rho, which the caller zeroes)
+enum GemmMode { GM_XF = 0, GM_XT = 1, GM_APPLY = 2, GM_REFOLD = 3, GM_VRANGE = 4 };
+struct GemmDesc {
+    int mode;
+    bool tc;
+    int M, N, nb, nl, n_seg, P;
+    int64_t K_seg;
+    const void *A, *B0, *B1;
+    int b_shared;                 // GM_XF: F has no batch dimension
+    int64_t L, dk, r, n_rows, W;  // rows of X (or of A), d_kv, rank, rows of F, layers
+    void *C;
+    int c_bf16;                   // C in bf16 (else fp32)
+    int64_t ldc, c_b, c_l;        // C strides of a row, a sequence, an outer index
+    unsigned *status;             // bits of device-side failures (bounded waits)
+    float *rho;                   // GM_VRANGE output [nb][Hkv][nC]
+    int hd, chunk, Hkv;
+    int64_t nC;
+};
+cudaError_t launch_gemm(const GemmDesc &g, cudaStream_t s);
 
 // cross-layer factorization of one window (clf.cu)
 size_t factorize_ws_bytes(const xkv_dims &d, int W, int r);

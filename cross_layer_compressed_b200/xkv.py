@@ -48,9 +48,13 @@ _sigs = {
     "xkv_score_landmarks": ([_D, _vp, _vp, _vp, _vp], ctypes.c_int),
     "xkv_select_chunks": ([_D, _vp, _i32, _i32, _i32, _vp, ctypes.POINTER(_i32), _vp],
                           ctypes.c_int),
-    "xkv_score_select": ([_D, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.POINTER(_i32), _vp, _sz,
-                          _vp], ctypes.c_int),
+    "xkv_score_select": ([_D, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp, ctypes.POINTER(_i32),
+                          _vp, _sz, _vp], ctypes.c_int),
     "xkv_score_select_workspace_bytes": ([_D], _sz),
+    "xkv_build_value_ranges": ([_D, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "xkv_reserve_value_chunks": ([_D, _vp, _i32, _i32, _i32, _vp, ctypes.POINTER(_i32), _vp],
+                                 ctypes.c_int),
+    "xkv_n_reserved": ([_i64, _i32, _i32, _i32], _i64),
     "xkv_reconstruct_attend": ([_D, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp],
                                ctypes.c_int),
     "rcla_decode_attend": ([_D, _i32, _vp, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
@@ -152,14 +156,15 @@ def xkv_select_chunks(d: xkv_dims, scores, top_k, n_sink, n_recent, sel, stream=
 
 
 def xkv_score_select(d: xkv_dims, lm_layer, q, top_k, n_sink, n_recent, sel, ws,
-                     ws_bytes=None, stream=None, check=True):
+                     ws_bytes=None, stream=None, check=True, reserved=None, n_reserved=0):
     """Returns n_sel (or the status when check=False)."""
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size()
     n = _i32(0)
     st = _lib.xkv_score_select(ctypes.byref(d), _ptr(lm_layer), _ptr(q), int(top_k),
-                               int(n_sink), int(n_recent), _ptr(sel), ctypes.byref(n), _ptr(ws),
-                               int(ws_bytes), _stream(stream))
+                               int(n_sink), int(n_recent), _ptr(reserved), int(n_reserved),
+                               _ptr(sel), ctypes.byref(n), _ptr(ws), int(ws_bytes),
+                               _stream(stream))
     if check:
         _check(st)
         return n.value
@@ -168,6 +173,32 @@ def xkv_score_select(d: xkv_dims, lm_layer, q, top_k, n_sink, n_recent, sel, ws,
 
 def xkv_score_select_workspace_bytes(d: xkv_dims) -> int:
     return int(_lib.xkv_score_select_workspace_bytes(ctypes.byref(d)))
+
+
+def xkv_build_value_ranges(d: xkv_dims, Av_win, Bvt_layer, rho_layer, status=None, stream=None,
+                           check=True):
+    st = _lib.xkv_build_value_ranges(ctypes.byref(d), _ptr(Av_win), _ptr(Bvt_layer),
+                                     _ptr(rho_layer), _ptr(status), _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def xkv_reserve_value_chunks(d: xkv_dims, rho_layer, n_value, n_sink, n_recent, reserved,
+                             stream=None, check=True):
+    """Returns n_res (or the status when check=False)."""
+    n = _i32(0)
+    st = _lib.xkv_reserve_value_chunks(ctypes.byref(d), _ptr(rho_layer), int(n_value),
+                                       int(n_sink), int(n_recent), _ptr(reserved),
+                                       ctypes.byref(n), _stream(stream))
+    if check:
+        _check(st)
+        return n.value
+    return st
+
+
+def xkv_n_reserved(n_chunks, n_value, n_sink, n_recent) -> int:
+    return int(_lib.xkv_n_reserved(int(n_chunks), int(n_value), int(n_sink), int(n_recent)))
 
 
 def xkv_reconstruct_attend(d: xkv_dims, Ak_win, Av_win, Bkt_layer, Bvt_layer, q, sel, n_sel,

@@ -22,9 +22,7 @@
  *  - All tensor arguments are DEVICE pointers to dense row-major arrays (last index
  *    fastest) in the layouts stated below, unless marked "host".  The caller owns
  *    every buffer; the library never allocates, frees or keeps a pointer after the
- *    call returns.  One exception: the factorization calls (xkv_factorize_window,
- *    xkv_refold_window) run their plain GEMMs in cuBLAS, whose handle -- created once
- *    per device on first use and kept until exit -- holds cuBLAS's own resources.
+ *    call returns.
  *  - Storage type (dims->dtype): XKV_F32 or XKV_BF16, shared by the factors,
  *    landmarks, queries and caches of a call.  Outputs are fp32; scores are fp64.
  *  - Every pointer the kernels read or write must be 16-byte aligned.
@@ -140,8 +138,9 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
                              int32_t *n_sel_out, void *stream);
 
 /*
- * Scoring and selection in one call [xKV 2.3]: sel is bit for bit what
- * xkv_select_chunks(xkv_score_landmarks(lm_layer, q), top_k, n_sink, n_recent) gives --
+ * Scoring and selection in one call [xKV 2.3]: with no reserved chunks, sel is bit for
+ * bit what xkv_select_chunks(xkv_score_landmarks(lm_layer, q), top_k, n_sink, n_recent)
+ * gives --
  * the canonical fp64 scores, the forced chunks, the top_k by (score descending, chunk
  * index ascending), ascending order -- without writing the scores.  The landmarks are
  * scored in fp32 with a certified error bound; only the chunks whose membership that
@@ -153,13 +152,51 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
  *       in fp64 (a band wider than 512 chunks, e.g. many equal scores, or fp32 scores out
  *       of range); the rest is the fp64 scores of such units.
  * G = n_q_heads / n_kv_heads in 1..8 or 16; nC <= 16384.  A unit whose fp64 scores hold a
- * NaN (inputs outside the contract) gets every entry -1.
+ * NaN (inputs outside the contract) gets every entry -1.  reserved [B][Hkv][n_reserved]
+ * (or NULL with n_reserved = 0): chunks forced in as well, see the value-range-aware
+ * selection below.
  */
 xkv_status xkv_score_select(const xkv_dims *dims, const void *lm_layer, const void *q,
-                            int32_t top_k, int32_t n_sink, int32_t n_recent, int32_t *sel,
+                            int32_t top_k, int32_t n_sink, int32_t n_recent,
+                            const int32_t *reserved, int32_t n_reserved, int32_t *sel,
                             int32_t *n_sel_out, void *ws, size_t ws_bytes, void *stream);
 /* Scratch bytes of xkv_score_select (0 on bad dims). */
 size_t xkv_score_select_workspace_bytes(const xkv_dims *dims);
+
+/*
+ * Value-range-aware selection [VASE, "Value-Aware Stochastic KV cache Eviction" page,
+ * section 2.A: the tokens whose value vector has the largest range max(v) - min(v) are
+ * always kept], applied to this path's chunks.  Setup, once per cache and layer:
+ *
+ * xkv_build_value_ranges: rho[b][g][c] = the largest max_j V_hat[t][g*hd + j] -
+ *   min_j V_hat[t][g*hd + j] over the rows t of chunk c, V_hat = A^V B^V_l (the
+ *   reconstructed values, never written to memory; bf16 caches on the tensor cores with
+ *   fp32 accumulation, fp32 caches on the CUDA cores).
+ *   Av_win [B][L][r_V], Bvt_layer [B][d_kv][r_V], rho_layer [B][Hkv][nC] fp32 (output).
+ *   status: optional device word (4-byte aligned, may be NULL) that receives 0 or the OR
+ *   of (1 << xkv_status) over device-side failures (a bounded wait that gave up).
+ *
+ * xkv_reserve_value_chunks: reserved[b][g][0..n_res) = the n_res chunks outside the sink
+ *   and recent windows with the largest rho under (rho descending, chunk index
+ *   ascending), in ascending order; n_res = xkv_n_reserved(nC, n_value, n_sink,
+ *   n_recent) = min(n_value, nC - |sink U recent|), also written to *n_res_out (host,
+ *   may be NULL).  nC <= 16384.
+ *
+ * Each decode step then passes reserved / n_res to xkv_score_select: the reserved chunks
+ * join the forced ones and top_k more are chosen by score among the rest, so
+ *   n_sel = |sink U recent| + n_res + min(top_k, nC - |sink U recent| - n_res).
+ * A reserved list that is not a set of distinct chunks outside the sink and recent
+ * windows makes its unit's entries -1 (and its band word 0xFFFFFFFE).  reserved = NULL
+ * with n_reserved = 0 is the plain selection.
+ */
+xkv_status xkv_build_value_ranges(const xkv_dims *dims, const void *Av_win,
+                                  const void *Bvt_layer, float *rho_layer, unsigned *status,
+                                  void *stream);
+xkv_status xkv_reserve_value_chunks(const xkv_dims *dims, const float *rho_layer,
+                                    int32_t n_value, int32_t n_sink, int32_t n_recent,
+                                    int32_t *reserved, int32_t *n_res_out, void *stream);
+/* min(n_value, n_chunks - |sink U recent|); -1 on bad arguments. */
+int64_t xkv_n_reserved(int64_t n_chunks, int32_t n_value, int32_t n_sink, int32_t n_recent);
 
 /*
  * Selective (or dense) reconstruction followed by GQA attention
@@ -298,9 +335,15 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode);
  *               Av_win)
  *   Bt_out      [W][B][d_kv][r] in dtype: B_l stored column-major per layer (what the
  *               decode calls take as Bkt_layer / Bvt_layer)
- *   ws          device scratch of xkv_factorize_workspace_bytes bytes
- * All device pointers 16-byte aligned.  fp32 products, fp64 Gram matrices and Cholesky
- * factors.  Asynchronous on `stream`; INVALID_ARG / UNSUPPORTED before any launch.
+ *   ws          device scratch of xkv_factorize_workspace_bytes bytes.  Its first 4 bytes
+ *               hold, after the call (in stream order), the OR of (1 << xkv_status) over
+ *               device-side failures (a bounded wait that gave up); A_out and Bt_out are
+ *               then NaN.
+ * All device pointers 16-byte aligned.  The products run on the library's own kernels:
+ * bf16 caches on the tensor cores (the fp32 bases split into bf16 hi + lo parts, the
+ * products with R^-1 in TF32), fp32 caches in plain fp32 on the CUDA cores; fp64 Gram
+ * matrices and Cholesky factors.  Asynchronous on `stream`; INVALID_ARG / UNSUPPORTED
+ * before any launch.
  */
 xkv_status xkv_factorize_window(const xkv_dims *dims, int32_t window, int32_t rank,
                                 const void *X, const float *omega, int32_t n_iter,
@@ -324,8 +367,9 @@ size_t xkv_factorize_workspace_bytes(const xkv_dims *dims, int32_t window, int32
  *               when n_tail = T = 0
  *   omega, n_iter, Bt_out   as for xkv_factorize_window
  *   A_out       [B][L + T][r]
- *   ws          device scratch of xkv_refold_workspace_bytes bytes (the extended caches
- *               plus the factorization's scratch)
+ *   ws          device scratch of xkv_refold_workspace_bytes bytes (the factorization's
+ *               scratch, then the extended caches); status word as for
+ *               xkv_factorize_window
  * Bt_out may be Bt_win (it is read before it is written, in stream order).  Asynchronous;
  * INVALID_ARG / UNSUPPORTED before any launch.
  */

@@ -258,9 +258,9 @@ def test_factorize_pointer_and_workspace_checks(xkv):
 
     def al(x):
         return (x + 255) // 256 * 256
-    # Y and Z ping-pong (fp32); Gram, diagonal-block inverses, R^-1 (fp64); tolerances;
-    # R^-1 (fp32); bf16 hi / lo splits and the bf16 test matrix
-    assert need == (2 * al(B * L * r * 4) + 2 * al(B * n * r * 4) + al(B * r * r * 8)
+    # status header; Y and Z ping-pong (fp32); Gram, diagonal-block inverses, R^-1 (fp64);
+    # tolerances; R^-1 (fp32); bf16 hi / lo splits and the bf16 test matrix
+    assert need == (256 + 2 * al(B * L * r * 4) + 2 * al(B * n * r * 4) + al(B * r * r * 8)
                     + al(B * 1 * 64 * 64 * 8) + al(B * r * r * 8) + al(B * 8) + al(B * r * r * 4)
                     + 2 * al(B * max(L, n) * r * 2) + al(n * r * 2))
     assert xkv.xkv_factorize_workspace_bytes(d, 2, 40) == 0
@@ -288,7 +288,7 @@ def test_refold_argument_checks(xkv, monkeypatch):
     d = _fd(xkv)
     need = xkv.xkv_refold_workspace_bytes(d, 2, 32, 100)
     assert need > xkv.xkv_factorize_workspace_bytes(d, 2, 32)
-    # the extended caches (W x B x (L + T) x d_kv in bf16) come first
+    # the factorization's scratch and the extended caches (W x B x (L + T) x d_kv, bf16)
     assert need == (2 * 2 * 1100 * 128 * 2 + 255) // 256 * 256 + \
         xkv.xkv_factorize_workspace_bytes(_fd(xkv, ctx_len=1100), 2, 32)
     assert xkv.xkv_refold_workspace_bytes(d, 2, 32, -1) == 0
