@@ -35,6 +35,8 @@
 // Every wait on an mbarrier is bounded; on expiry the CTA records XKV_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs (again bounded), frees TMEM and
 // returns; the combine kernel then writes NaN outputs.
+#include <cstdlib>
+
 #include "sm100_util.cuh"
 
 namespace xkv {
@@ -75,12 +77,14 @@ struct TcParams {
     int n_split;
     int n_items;
     float qscale;             // log2(e) / sqrt(hd)
+    uint32_t mma_spin;        // poll limit of the MMA issuer's waits for staged data
 };
 
 // ----------------------------------------------------------------- PTX wrappers
 // Bounded wait for the phase of parity `parity`; false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared *sh) {
-    for (uint32_t i = 0; i < SPIN_LIMIT; ++i) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, TcShared *sh,
+                                          uint32_t limit = SPIN_LIMIT) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_test(b, parity)) return true;
         if (*(volatile int *)&sh->abort) return false;
     }
@@ -231,10 +235,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
             }
         }
-        if (!ok && pi == 0 && lane == 0) {  // give this CTA's copies time to land
-            for (int s = 0; s < TC_STAGES; ++s)
+        if (!ok && pi == 0 && lane == 0) {
+            // Every stage the four warps issued lands before the CTA may leave: the last
+            // TC_STAGES fills (each issued whole: a warp checks for abort only in its wait
+            // on `empty`, which completes for all four warps alike) complete their phase.
+            for (int j = it - TC_STAGES > 0 ? it - TC_STAGES : 0; j < it; ++j)
                 for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
-                    if (mbar_test(&sh->full[s], 0) || mbar_test(&sh->full[s], 1)) break;
+                    if (mbar_test(&sh->full[j % TC_STAGES], (uint32_t)(j / TC_STAGES) & 1)) break;
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
@@ -253,7 +260,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int nk = p.rk / TC_KS;
                 for (int ks = 0; ks < nk && ok; ++ks, ++it) {
                     const int s = it % TC_STAGES, n = it / TC_STAGES;
-                    if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                    if (!mbar_wait(&sh->full[s], n & 1, sh, p.mma_spin)) { abort_cta(sh, p); ok = false; break; }
                     tcgen05_after();
                     const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
 #pragma unroll
@@ -274,7 +281,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int nv = p.rv / TC_KS;
                 for (int ks = 0; ks < nv && ok; ++ks, ++it) {
                     const int s = it % TC_STAGES, n = it / TC_STAGES;
-                    if (!mbar_wait(&sh->full[s], n & 1, sh)) { abort_cta(sh, p); ok = false; break; }
+                    if (!mbar_wait(&sh->full[s], n & 1, sh, p.mma_spin)) { abort_cta(sh, p); ok = false; break; }
                     tcgen05_after();
                     const uint32_t a0 = smem_base + s * STAGE_BYTES, b0 = a0 + A_TILE;
 #pragma unroll
@@ -499,6 +506,14 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
     p.n_split = (n_sel + p.chunks_per_item - 1) / p.chunks_per_item;
     p.n_items = d.batch * d.n_kv_heads * p.n_split;
     p.qscale = 1.4426950408889634f / sqrtf((float)d.head_dim);
+    // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the MMA
+    // issuer's waits on staged data, so a test can make them give up; every other wait,
+    // and the drain that follows, keeps its full bound
+    p.mma_spin = SPIN_LIMIT;
+    if (const char *e = getenv("XKV_TEST_MMA_SPIN")) {
+        const long v = atol(e);
+        if (v > 0 && v < (long)SPIN_LIMIT) p.mma_spin = (uint32_t)v;
+    }
     *n_split_out = p.n_split;
     switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_G(GG) \

@@ -1,0 +1,58 @@
+"""The device-side timeout path of the tensor-core attention kernel, exercised without
+faulting anything: a test-only variable shortens the poll limit of the MMA issuer's waits
+for staged data so that they give up; every other wait (and the drain of the copies and
+MMAs in flight) keeps its full bound.  The call must report XKV_ERR_TIMEOUT in its status
+word and NaN outputs, and the next call, with the normal limit, must be clean."""
+import numpy as np
+import pytest
+import torch
+
+from cross_layer_compressed_b200 import synth
+from parity_util import compare_outputs
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+
+
+@pytest.fixture(scope="module")
+def xkv():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from cross_layer_compressed_b200 import build
+    build.build()
+    from cross_layer_compressed_b200 import xkv as m
+    return m
+
+
+def test_attention_wait_timeout_is_reported_then_the_next_call_is_clean(xkv, ora, monkeypatch):
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=4096, top_k=60, n_needles=0)
+    x = synth.np_xkv_layer_inputs(w, seed=5, layer=0)
+    g = {k: x[k].to(DEV) for k in ("Ak", "Av", "Bkt", "Bvt", "q")}
+    rng = np.random.default_rng(5)
+    sel = np.stack([np.sort(rng.choice(w.n_chunks, w.n_sel, replace=False))
+                    for _ in range(w.batch * w.n_kv_heads)]).reshape(
+        w.batch, w.n_kv_heads, w.n_sel).astype(np.int32)
+    sel_d = torch.from_numpy(sel).to(DEV)
+    d = xkv.dims_of(w)
+    ws = torch.zeros(xkv.xkv_workspace_bytes(d, w.n_sel, xkv.XKV_MODE_SELECTIVE),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+
+    def call():
+        xkv.xkv_reconstruct_attend(d, g["Ak"], g["Av"], g["Bkt"], g["Bvt"], g["q"], sel_d,
+                                   w.n_sel, out, ws)
+        torch.cuda.synchronize()
+        return int(ws[:4].cpu().view(torch.int32).item()), out.cpu().numpy()
+
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "1")
+    status, o = call()
+    assert status & (1 << xkv.XKV_ERR_TIMEOUT), status
+    assert np.all(np.isnan(o))
+    monkeypatch.delenv("XKV_TEST_MMA_SPIN")
+    status, o = call()
+    assert status == 0
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk,
+                                 units=[(0, 1), (1, 6)])
+    for b, gg in ((0, 1), (1, 6)):
+        G = w.group
+        compare_outputs(o[b, gg * G:(gg + 1) * G], ref[b, gg * G:(gg + 1) * G], w.dtype)
