@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from cross_layer_compressed_b200 import synth
-from parity_util import bf16_ulp_diff, compare_outputs
+from parity_util import bf16_ulp_diff, certify_near_ties, compare_outputs
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -47,16 +47,40 @@ def _xkv_layer_check(xkv, ora, w, layer, units, dense=False, reassociated=False)
         return
     lm = torch.empty((w.batch, w.n_kv_heads, w.n_chunks, hd), dtype=torch.bfloat16, device=DEV)
     xkv.xkv_build_landmarks(d, c["Ak"], c["Bkt"], lm)
+    # the product pipeline on the GPU's own landmarks: the fused selection of every unit,
+    # which must equal the two-call path (score, select) bit for bit
+    sel_f = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
+    wss = torch.empty(xkv.xkv_score_select_workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    xkv.xkv_score_select(d, lm, q, w.top_k, w.n_sink, w.n_recent, sel_f, wss)
+    sc2 = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
+    sel2 = torch.empty_like(sel_f)
+    xkv.xkv_score_landmarks(d, lm, q, sc2)
+    xkv.xkv_select_chunks(d, sc2, w.top_k, w.n_sink, w.n_recent, sel2)
     torch.cuda.synchronize()
+    sel_f_h = sel_f.cpu().numpy()
+    assert np.array_equal(sel_f_h, sel2.cpu().numpy())
+    band = wss[:4 * w.batch * w.n_kv_heads].cpu().view(torch.int32).numpy().view(np.uint32)
+    assert np.all(band != 0xFFFFFFFF), "a unit left the fp32 + band path"
     host = {}
+    n_diff = 0
     for b, g in units:
         Ak = c["Ak"][b:b + 1].cpu()
         Bkt_g = c["Bkt"][b:b + 1, g * hd:(g + 1) * hd].contiguous().cpu()
         lm_ref = ora.build_landmarks(Ak, Bkt_g, 1, hd, w.chunk)          # oracle landmarks
         diff = bf16_ulp_diff(_u16(lm[b, g]), lm_ref[0, 0])
         assert diff.max() <= 1 and (diff > 0).mean() < 1e-4
+        # GPU landmarks against the oracle's: equal selections or certified near-ties
+        qg = q[b:b + 1, g * G:(g + 1) * G].cpu()
+        s_ref = ora.score_landmarks(ora.to_torch(lm_ref), qg)
+        sel_o = ora.select_chunks(s_ref, w.top_k, w.n_sink, w.n_recent)
+        n_diff += certify_near_ties(ora.as_float64(lm[b:b + 1, g:g + 1].cpu()),
+                                    ora.as_float64(ora.to_torch(lm_ref)), ora.as_float64(qg),
+                                    sel_f_h[b:b + 1, g:g + 1], sel_o, s_ref, G, w.top_k,
+                                    w.n_sink, w.n_recent)
         lm[b, g] = ora.to_torch(lm_ref)[0, 0].to(DEV)                   # score what the oracle scores
         host[(b, g)] = (Ak, Bkt_g, lm_ref)
+    print(f"{w.name}: {n_diff} of {len(units)} sampled units select differently from GPU "
+          "landmarks, all certified near-ties")
     scores = torch.empty((w.batch, w.n_kv_heads, w.n_chunks), dtype=torch.float64, device=DEV)
     sel = torch.empty((w.batch, w.n_kv_heads, w.n_sel), dtype=torch.int32, device=DEV)
     mode = xkv.XKV_MODE_REASSOC if reassociated else xkv.XKV_MODE_SELECTIVE
