@@ -20,10 +20,13 @@
 //  3. the rest (the band) is scored in fp64 exactly as the oracle scores it, and the
 //     top (k - #selected) of the band under (score desc, index asc) complete the set.
 //
-// Work split: one thread-block cluster per (sequence, KV head) unit.  Every CTA of the
-// cluster streams its slice of the unit's landmark rows (one row per thread, 16-byte
-// loads, the group's query in shared memory) and sends its fp32 keys to CTA 0's shared
-// memory; CTA 0 then runs steps 2-3 and writes the selection in ascending chunk order.
+// Work split: one thread-block cluster per (sequence, KV head) unit, a CTA of 256 threads
+// per 512 chunks (at most 8, the portable cluster size).  Every CTA of the cluster
+// streams its slice of the unit's landmark rows (two rows per thread, 16-byte loads, the
+// group's query in shared memory) and sends its fp32 keys to CTA 0's shared memory; CTA 0
+// then runs steps 2-3 and writes the selection in ascending chunk order.  The steps of
+// CTA 0 are written for latency: strided (bank-conflict-free) passes over the keys, the
+// band ranked by counting (no ordering needed), the output placed by ballots.
 // Optionally a per-unit list of reserved chunks (the value-range reservation) joins the
 // sink and recent chunks as forced.  Units whose fp32 scores are not all finite or whose
 // band is wider than BAND_CAP chunks take the exact path for the whole unit: every chunk is
@@ -33,22 +36,18 @@
 // Chosen for B200: 67 MB of landmarks per layer at the bench workload need ~10 us at the
 // copy bandwidth, while the fp64 pass spent ~30 us on conversions and fp64 FMAs; fp32
 // FMAs and shift-only bf16 widening keep the stream HBM-bound.
-#include <map>
-#include <mutex>
-#include <tuple>
-
 #include "xkv_internal.cuh"
 
 namespace xkv {
 namespace {
 
-constexpr int SS_THREADS = 128;
+constexpr int SS_THREADS = 256;
 constexpr int SS_WARPS = SS_THREADS / 32;
 constexpr int SS_RPT = 2;                         // rows per thread per pass
 constexpr int SS_ROWS = SS_THREADS * SS_RPT;      // rows per CTA pass
-constexpr int SS_MAX_CLUSTER = 16;
+constexpr int SS_MAX_CLUSTER = 8;                 // portable cluster size
 constexpr int HIST_BINS = 2048;                   // radix digits of 11, 11 and 10 bits
-constexpr int RANK_CAP = 256;                     // keys of a bin ranked directly
+constexpr int RANK_CAP = 32;                      // keys of a bin ranked directly
 constexpr int BAND_CAP = 512;                     // band chunks rescored in fp64
 constexpr uint32_t EXACT_PATH = 0xFFFFFFFFu;
 constexpr uint32_t BAD_RESERVED = 0xFFFFFFFEu;   // a reserved list broke its rules
@@ -285,7 +284,7 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     __shared__ int s_bad[SS_MAX_CLUSTER];
     __shared__ RadixShared rs;
     __shared__ int s_bad_cta, s_exact, s_bad_res;
-    __shared__ unsigned s_cnt, s_nin, s_bin, s_above, s_tkey;
+    __shared__ unsigned s_cnt, s_nin, s_bin, s_above, s_tkey, s_q1;
     __shared__ float s_mx_cta;
 
     // announce this CTA; the matching wait comes before the first remote store
@@ -403,6 +402,7 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
     if (rank != 0) return;
 
     // ---------------------------------------------------------------- CTA 0: selection
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ncl = (int)((nC + p.cpc - 1) / p.cpc);
     const int f_lo = min(p.n_sink, nC), f_hi = max(nC - p.n_recent, 0);
     auto forced = [&](int c) {
@@ -429,20 +429,24 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
         s_exact = ubad;
         s_cnt = 0u;
         s_nin = 0u;
+        s_q1 = 0u;
+    }
+    __syncthreads();
+    // max_h ||q_h||_1: a warp per head, fp32 partial sums of exact values (rounded up below)
+    for (int h = warp; h < G; h += SS_WARPS) {
+        float sum = 0.f;
+        for (int d = lane; d < hd; d += 32) sum += fabsf(qf[d * G + h]);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0) atomicMax(&s_q1, __float_as_uint(sum));
     }
     __syncthreads();
     unsigned band_size = 0;
-    const int ipt = (nC + SS_THREADS - 1) / SS_THREADS;
-    const int lo = min(nC, (int)threadIdx.x * ipt), hi = min(nC, lo + ipt);
     auto set_bit = [&](int c) { atomicOr(&bits[c >> 5], 1u << (c & 31)); };
     if (!s_exact && k_eff > 0 && !all_cand) {
-        // the certified error of every fp32 score of the unit
-        double q1 = 0.0;
-        for (int h = 0; h < G; ++h) {
-            double s1 = 0.0;
-            for (int d = 0; d < hd; ++d) s1 += fabs((double)qf[d * G + h]);
-            q1 = fmax(q1, s1);
-        }
+        // the certified error of every fp32 score of the unit; the fp32 sum of hd
+        // non-negative terms is within gamma_hd(2^-24) < 2^-14 of its exact value
+        const double q1 = (double)__uint_as_float(s_q1) * (1.0 + 0x1p-14);
         const double E = (p.err_rel * (double)umx * q1 * (1.0 + 0x1p-40)) + p.err_abs;
         // (a) t = the k-th largest candidate key: MSB-first radix descent over 11, 11 and
         //     10 bits of the 32-bit keys; once the bin holding t has at most RANK_CAP
@@ -515,48 +519,54 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
             __syncthreads();
             t_lo = fkey_inv(s_tkey);
         }
-        const float t_hi = t_lo;
         const double lo_b = __dsub_rd((double)t_lo, 2.0 * E);
-        const double hi_b = __dadd_ru((double)t_hi, 2.0 * E);
+        const double hi_b = __dadd_ru((double)t_lo, 2.0 * E);
+        if (threadIdx.x == 0) s_cnt = 0u;
         if (!(fabs(lo_b) <= 1.7e308) || !(fabs(hi_b) <= 1.7e308)) {
             if (threadIdx.x == 0) s_exact = 1;
         }
         __syncthreads();
         if (!s_exact) {
-            // (c) certain chunks into the bit set, the band into r1 in ascending order
-            unsigned nb = 0, nin = 0;
-            for (int c = lo; c < hi; ++c) {
+            // (c) certain chunks into the bit set, the band's chunk indices into r1
+            uint32_t *bidx = r1;
+            unsigned long long *bkey = reinterpret_cast<unsigned long long *>(r1 + BAND_CAP);
+            unsigned nin = 0;
+            for (int c = threadIdx.x; c < nC; c += SS_THREADS) {
                 if (forced(c)) continue;
-                const double s = (double)fkey_inv(keys[c]);
-                if (s > hi_b) {
+                const double sc = (double)fkey_inv(keys[c]);
+                if (sc > hi_b) {
                     set_bit(c);
                     ++nin;
-                } else if (s >= lo_b) {
-                    ++nb;
+                } else if (sc >= lo_b) {
+                    const unsigned pos = atomicAdd(&s_cnt, 1u);
+                    if (pos < (unsigned)BAND_CAP) bidx[pos] = (uint32_t)c;
                 }
             }
-            if (nin) atomicAdd(&s_nin, nin);
-            unsigned pos = block_scan(nb, rs);
-            const unsigned m = rs.total;
-            const unsigned n_in = s_nin;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) nin += __shfl_xor_sync(0xffffffffu, nin, off);
+            if (lane == 0 && nin) atomicAdd(&s_nin, nin);
+            __syncthreads();
+            const unsigned m = s_cnt, n_in = s_nin;
             const unsigned need2 = (unsigned)k_eff - n_in;
             if (m > (unsigned)BAND_CAP || need2 < 1u || need2 > m) {
                 if (threadIdx.x == 0) s_exact = 1;   // (need2 outside [1, m] cannot happen)
             } else {
-                uint32_t *bidx = r1;
-                unsigned long long *bkey = reinterpret_cast<unsigned long long *>(r1 + BAND_CAP);
-                for (int c = lo; c < hi && nb; ++c) {
-                    if (forced(c)) continue;
-                    const double s = (double)fkey_inv(keys[c]);
-                    if (s <= hi_b && s >= lo_b) bidx[pos++] = (uint32_t)c;
-                }
-                __syncthreads();
                 // (d) the band in fp64, as the oracle scores it
                 for (unsigned i = threadIdx.x; i < m; i += SS_THREADS)
                     bkey[i] = order_key(exact_score<T, G>(lmu + (size_t)bidx[i] * hd, qf, hd));
                 __syncthreads();
-                radix_select((int)m, need2, [&](int i) { return bkey[i]; },
-                             [](int) { return true; }, [&](int i) { set_bit((int)bidx[i]); }, rs);
+                // (e) the need2 first of the band under (score desc, chunk index asc): a
+                //     chunk's rank counts the band chunks that precede it
+                for (unsigned i = threadIdx.x; i < m; i += SS_THREADS) {
+                    const unsigned long long ki = bkey[i];
+                    const uint32_t ci = bidx[i];
+                    unsigned rank_i = 0;
+                    for (unsigned j = 0; j < m; ++j) {
+                        const unsigned long long kj = bkey[j];
+                        rank_i += (kj > ki || (kj == ki && bidx[j] < ci)) ? 1u : 0u;
+                    }
+                    if (rank_i < need2) set_bit((int)ci);
+                }
                 band_size = m;
             }
             __syncthreads();
@@ -569,9 +579,9 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
         double *sc = p.scratch + (size_t)unit * nC;
         bool nan_seen = false;
         for (int c = threadIdx.x; c < nC; c += SS_THREADS) {
-            const double s = exact_score<T, G>(lmu + (size_t)c * hd, qf, hd);
-            sc[c] = s;
-            nan_seen |= isnan(s);
+            const double v = exact_score<T, G>(lmu + (size_t)c * hd, qf, hd);
+            sc[c] = v;
+            nan_seen |= isnan(v);
         }
         if (__syncthreads_or(nan_seen)) {
             // NaN scores (inputs outside the contract): the unit selects nothing
@@ -586,16 +596,37 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
         band_size = EXACT_PATH;
     }
     // ------------------------------------------------------------ output
-    unsigned n_local = 0;
-    for (int c = lo; c < hi; ++c)
-        n_local += (forced(c) || all_cand || ((bits[c >> 5] >> (c & 31)) & 1u)) ? 1u : 0u;
-    unsigned pos = block_scan(n_local, rs);
-    int32_t *out = p.sel + (size_t)unit * p.n_sel;
-    for (int c = lo; c < hi; ++c) {
-        if (forced(c) || all_cand || ((bits[c >> 5] >> (c & 31)) & 1u)) {
-            if (pos < (unsigned)p.n_sel) out[pos] = c;
-            ++pos;
+    // ascending order: 32-chunk groups, a ballot per group, a scan over the group counts
+    const int n_groups = (nC + 31) / 32;
+    uint32_t *gcount = r1, *gbase = r1 + HIST_BINS / 2;
+    auto taken = [&](int c) {
+        return c < nC && (forced(c) || all_cand || ((bits[c >> 5] >> (c & 31)) & 1u));
+    };
+    __syncthreads();
+    for (int gi = warp; gi < n_groups; gi += SS_WARPS) {
+        const unsigned bal = __ballot_sync(0xffffffffu, taken(gi * 32 + lane));
+        if (lane == 0) gcount[gi] = __popc(bal);
+    }
+    __syncthreads();
+    {
+        const int gpt = (n_groups + SS_THREADS - 1) / SS_THREADS;   // groups per thread
+        const int g0 = min(n_groups, (int)threadIdx.x * gpt), g1 = min(n_groups, g0 + gpt);
+        unsigned cnt = 0;
+        for (int gi = g0; gi < g1; ++gi) cnt += gcount[gi];
+        unsigned run = block_scan(cnt, rs);
+        for (int gi = g0; gi < g1; ++gi) {
+            gbase[gi] = run;
+            run += gcount[gi];
         }
+    }
+    __syncthreads();
+    int32_t *out = p.sel + (size_t)unit * p.n_sel;
+    for (int gi = warp; gi < n_groups; gi += SS_WARPS) {
+        const int c = gi * 32 + lane;
+        const bool tk = taken(c);
+        const unsigned bal = __ballot_sync(0xffffffffu, tk);
+        const unsigned pos = gbase[gi] + __popc(bal & ((1u << lane) - 1u));
+        if (tk && pos < (unsigned)p.n_sel) out[pos] = c;
     }
     if (threadIdx.x == 0) p.band[unit] = band_size;
 }
@@ -641,38 +672,6 @@ size_t ss_smem_bytes(const xkv_dims &d) {
 
 double gamma_n(int n, double u) { return n * u / (1.0 - n * u); }
 
-// Cluster size of a launch: one CTA per SS_ROWS chunks, at most 16 (a non-portable size,
-// taken when the occupancy calculator says a 16-CTA cluster of this kernel fits), else 8.
-// Decided once per (kernel, device, shared-memory size).
-int cluster_size(const void *k, size_t smem, int want, cudaLaunchConfig_t cfg) {
-    if (want <= 8) return want;
-    static std::mutex mu;
-    static std::map<std::tuple<const void *, int, size_t>, int> chosen;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 8;
-    std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_tuple(k, dev, smem);
-    auto it = chosen.find(key);
-    if (it != chosen.end()) return it->second;
-    int cs = 8;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-        cudaSuccess) {
-        cudaLaunchAttribute at;
-        at.id = cudaLaunchAttributeClusterDimension;
-        at.val.clusterDim.x = SS_MAX_CLUSTER;
-        at.val.clusterDim.y = 1;
-        at.val.clusterDim.z = 1;
-        cfg.gridDim = dim3(SS_MAX_CLUSTER, 1, 1);
-        cfg.attrs = &at;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) == cudaSuccess && n > 0) cs = SS_MAX_CLUSTER;
-    }
-    (void)cudaGetLastError();
-    chosen[key] = cs;
-    return cs;
-}
-
 template <typename T, int G>
 cudaError_t launch_tg(const xkv_dims &d, const SsParams &p0, cudaStream_t s) {
     auto k = k_score_select<T, G>;
@@ -686,7 +685,6 @@ cudaError_t launch_tg(const xkv_dims &d, const SsParams &p0, cudaStream_t s) {
     cfg.blockDim = dim3(SS_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cs = cluster_size((const void *)k, smem, cs, cfg);
     SsParams p = p0;
     p.cpc = (int)(((nC + cs - 1) / cs + 3) & ~3);
     cudaLaunchAttribute at[2];
