@@ -44,31 +44,34 @@ constexpr int NBP = NB + 1;    // padded shared-memory row
 
 // ------------------------------------------------------------------ fp64 Gram
 // G[b] += Y[b]^T Y[b] over one slice of rows, for the 128 x 128 tiles on or above the
-// diagonal (the factorization reads the upper triangle only).  Rows are staged in
-// shared memory already widened to fp64 (fp32 x fp32 products are exact in fp64); each
-// thread owns 8 x 8 outputs (rows and columns 16 apart), so a row step costs 16
-// conflict-free shared loads per 64 fp64 FMAs.  The slices meet through fp64 atomics.
-constexpr int GR_T = 128, GR_ROWS = 16, GR_THREADS = 256;
+// diagonal (the factorization reads the upper triangle only), on the fp64 tensor cores:
+// mma.sync m8n8k4 f64 (exact fp32 x fp32 products, fp64 accumulation; the order of the
+// fp64 sums is the tensor core's, which only rounding sees).  16 warps, each owning a
+// 32 x 32 block of the tile as 4 x 4 fragments of 8 x 8; 16-row slices of the tile's two
+// column blocks are staged in shared memory already widened to fp64 (rows padded by 4
+// doubles), the next slice waiting in registers.  The slices of rows meet through fp64
+// atomics.
+constexpr int GR_T = 128, GR_ROWS = 16, GR_THREADS = 512, GR_PAD = GR_T + 4;
 
-__global__ void __launch_bounds__(GR_THREADS) k_gram(const float *__restrict__ Y, int rows, int r,
-                                                     int rows_per_split, int n_split,
-                                                     double *__restrict__ G) {
+__global__ void __launch_bounds__(GR_THREADS, 1) k_gram(const float *__restrict__ Y, int rows,
+                                                        int r, int rows_per_split, int n_split,
+                                                        double *__restrict__ G) {
     const int ti = blockIdx.y, tj = blockIdx.x;
     if (tj < ti) return;
     const int b = blockIdx.z / n_split, sp = blockIdx.z % n_split;
-    __shared__ __align__(16) double Yi[GR_ROWS][GR_T], Yj[GR_ROWS][GR_T];
-    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+    __shared__ __align__(16) double Yi[GR_ROWS][GR_PAD], Yj[GR_ROWS][GR_PAD];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wi = (warp >> 2) * 32, wj = (warp & 3) * 32;   // the warp's 32 x 32 block
+    const int fr = lane >> 2, fk = lane & 3;                 // fragment row / k of this lane
     const float *y = Y + (int64_t)b * rows * r;
     const int t_lo = sp * rows_per_split;
     const int t_hi = min(rows, t_lo + rows_per_split);
-    double acc[8][8];
+    double acc[4][4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-    // the next slice's values wait in registers while this one is multiplied (one CTA
-    // per SM: nothing else would hide the loads)
-    constexpr int PER = GR_ROWS * GR_T / GR_THREADS;
+        for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+    constexpr int PER = GR_ROWS * GR_T / GR_THREADS;   // 4
     float ni[PER], nj[PER];
     auto fetch = [&](int t0) {
 #pragma unroll
@@ -89,32 +92,39 @@ __global__ void __launch_bounds__(GR_THREADS) k_gram(const float *__restrict__ Y
         }
         __syncthreads();
         if (t0 + GR_ROWS < t_hi) fetch(t0 + GR_ROWS);
-#pragma unroll 2
-        for (int tt = 0; tt < GR_ROWS; ++tt) {
-            // rows ty + 16 i and columns tx + 16 j: a warp's loads are 128 contiguous
-            // bytes (columns) or broadcasts (rows), one shared-memory wavefront each
-            double a[8], c[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                a[i] = Yi[tt][ty + 16 * i];
-                c[i] = Yj[tt][tx + 16 * i];
-            }
+        for (int k0 = 0; k0 < GR_ROWS; k0 += 4) {
+            // A[i][k] = Y[t0 + k][i], B[k][j] = Y[t0 + k][j]: lane (fr, fk) holds
+            // A[fr][fk] and B[fk][fr] of each 8-wide fragment
+            double a[4], c[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 4; ++i) a[i] = Yi[k0 + fk][wi + 8 * i + fr];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
+            for (int j = 0; j < 4; ++j) c[j] = Yj[k0 + fk][wj + 8 * j + fr];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    asm volatile(
+                        "mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, "
+                        "{%0, %1};"
+                        : "+d"(acc[i][j][0]), "+d"(acc[i][j][1])
+                        : "d"(a[i]), "d"(c[j]));
         }
         __syncthreads();
     }
     double *g = G + (int64_t)b * r * r;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int gi = ti * GR_T + ty + 16 * i;
+    for (int i = 0; i < 4; ++i) {
+        const int gi = ti * GR_T + wi + 8 * i + fr;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int gj = tj * GR_T + tx + 16 * j;
-            if (gi < r && gj < r && gi <= gj) atomicAdd(&g[(int64_t)gi * r + gj], acc[i][j]);
-        }
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // accumulator (row fr, column 2 fk + h) of fragment (i, j)
+                const int gj = tj * GR_T + wj + 8 * j + 2 * fk + h;
+                if (gi < r && gj < r && gi <= gj) atomicAdd(&g[(int64_t)gi * r + gj], acc[i][j][h]);
+            }
     }
 }
 
