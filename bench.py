@@ -47,7 +47,7 @@ def parse():
     p.add_argument("--path", choices=["explicit", "reassociated"], default="explicit",
                    help="xKV attention: explicit reconstruction (the method as the pages "
                         "state it) or its rank-space reassociation")
-    p.add_argument("--scoring", choices=["fused", "separate"], default="fused",
+    p.add_argument("--scoring", choices=["fused", "separate"], default="separate",
                    help="selective xKV: one fused scoring + selection call per layer "
                         "(xkv_score_select) or xkv_score_landmarks + xkv_select_chunks")
     p.add_argument("--value-reserve", type=int, default=0,

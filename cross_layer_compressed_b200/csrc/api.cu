@@ -178,8 +178,8 @@ size_t xkv_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int32_t mode) {
     if (mode == XKV_MODE_REASSOC) {
         const int64_t nC = dims->ctx_len / dims->chunk;
         if (n_sel < 0 || n_sel > nC || !attend_ra_shape_ok(*dims)) return 0;
-        const int n = ra_splits(*dims, n_sel ? n_sel : (int)nC);
-        return ws_header_bytes(*dims) + ra_scratch_bytes(*dims, n);
+        return ws_header_bytes(*dims) +
+               ra_call_scratch_bytes(*dims, n_sel == 0, n_sel ? n_sel : (int)nC);
     }
     int64_t rows;
     if (mode == XKV_MODE_SELECTIVE) {
@@ -678,7 +678,7 @@ xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, con
     const int ns = sel ? n_sel : (int)nC;
     if (ra_splits(*dims, ns) > 65535 || (int64_t)dims->batch * dims->ctx_len >= (1ll << 31))
         return fail(XKV_ERR_UNSUPPORTED, "%s: too many rows", who);
-    const size_t need = ws_header_bytes(*dims) + ra_scratch_bytes(*dims, ra_splits(*dims, ns));
+    const size_t need = ws_header_bytes(*dims) + ra_call_scratch_bytes(*dims, !sel, ns);
     if (ws_bytes < need)
         return fail(XKV_ERR_INVALID_ARG, "%s: workspace %zu bytes, need %zu", who, ws_bytes,
                     need);

@@ -415,6 +415,409 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                      : "memory");
 }
 
+// ------------------------------------------------------------------ dense, all heads
+// Dense mode (every head attends every row): the rows of A are the same for all Hq heads
+// of a sequence, so the per-(b, g) items above would stream the window once per KV head.
+// k_xkv_ra_dense instead gives one CTA a span of the sequence's rows and all of its
+// heads, so A^K and A^V each cross HBM once per layer:
+//   pass 1, per 128-token tile: D_z[t][n] = A^K[t][:] . Q~[n][:]  (M = 128 tokens,
+//           N = NO = the hi and lo rows of the Hq heads), the logits z_h = D_z[t][h] +
+//           D_z[t][Hq + h] go to a global scratch (L2-resident: the same thread reads
+//           them back in pass 2) and the span's max per head is kept;
+//   pass 2, per tile: P[n][t] = exp2(z - m) as hi + lo bf16 rows, then
+//           D_u[r][n] += A^V[t][r] P[n][t]  (M = 128 rank columns per block, N = NO,
+//           K = tokens), accumulated in tensor memory over the whole span;
+//   end:    the span's (m, l, u) partial in rank space, merged across spans by k_merge_ra.
+// A stage is 128 tokens x 128 rank columns in one copy of the 3D view (64, rows, column
+// blocks) of A: two 64-column atoms of 128 rows, 16 KB apart.  Logits use A K-major
+// (8-row groups 1 KB apart), the value product reads the same stage MN-major (64-column
+// atoms 16 KB apart, 8-token groups 1 KB apart).  TMEM: two logit buffers, then the
+// r_V / 128 accumulator blocks, NO columns each.  Warp roles: warp 0 TMEM + MMA issue,
+// warp 1 the copies, warps 2-5 the epilogue (thread = TMEM lane = token, or rank column
+// at the end).
+constexpr int DN_TILE = 128;                     // tokens per tile
+constexpr int DN_STAGE = DN_TILE * 128 * 2;      // 128 tokens x 128 rank columns: 32 KB
+constexpr int DN_STAGES = 4;
+constexpr int DN_SPANS = 148;                    // spans per batch: one per SM of a B200
+constexpr int DW_MMA = 0, DW_LOAD = 1, DW_EPI = 2, DN_EPI = 4;
+constexpr int DN_THREADS = 32 * (DW_EPI + DN_EPI);   // 192
+constexpr int DN_EPI_THREADS = 32 * DN_EPI;           // 128
+
+struct DnShared {
+    uint64_t full[DN_STAGES], empty[DN_STAGES];
+    uint64_t q_full, zfull[2], zfree[2], pfull[2], pfree[2], ufull, ufree, idle;
+    uint32_t tmem_base;
+    int abort;
+    float red[DN_EPI][32];
+};
+
+struct DnParams {
+    const __nv_bfloat16 *qt_hi, *qt_lo;   // [B][Hq][r_K]
+    float *partials;                      // [n_span][B][Hq][r_V + 2]
+    float *z;                             // [B][Hq][tiles * 128] logits, log2 domain
+    unsigned *status;
+    int64_t L;
+    int rk, rv, B;
+    int tiles, tps, n_span, n_items;
+    float qscale;                         // log2(e) / sqrt(hd)
+};
+
+template <int HQ> struct DnCfg {
+    static constexpr int NO = (2 * HQ + 15) / 16 * 16;   // MMA N: hi and lo rows, padded
+    static constexpr int ATOM = NO / 8 * 1024;           // bytes per 64-wide K atom
+    static constexpr int PBUF = 2 * ATOM;                 // P: NO rows x 128 tokens
+};
+
+__device__ __forceinline__ void dn_epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(DN_EPI_THREADS) : "memory");
+}
+__device__ __forceinline__ bool dn_epi_bar_any(bool flag) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pin, pout;\n\t"
+        "setp.ne.u32 pin, %1, 0;\n\t"
+        "bar.red.or.pred pout, 1, %2, pin;\n\t"
+        "selp.u32 %0, 1, 0, pout;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag), "n"(DN_EPI_THREADS)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool dn_wait(uint64_t *b, uint32_t parity, DnShared *sh,
+                                        unsigned *status) {
+    if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
+    if (!*(volatile int *)&sh->abort) {
+        *(volatile int *)&sh->abort = 1;
+        if (status) atomicOr(status, 1u << XKV_ERR_TIMEOUT);
+    }
+    return false;
+}
+// N consecutive fp32 TMEM columns of this thread's lane, N a multiple of 16
+template <int N>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float *v) {
+    if constexpr (N >= 32) {
+        tmem_load32(taddr, *reinterpret_cast<float(*)[32]>(v));
+        tmem_load_cols<N - 32>(taddr + 32, v + 32);
+    } else if constexpr (N >= 16) {
+        tmem_load16(taddr, *reinterpret_cast<float(*)[16]>(v));
+    }
+}
+
+struct DnItem {
+    int b, span, t0, nt;   // sequence, span, first tile, tiles
+};
+__device__ __forceinline__ DnItem dn_decode(const DnParams &p, int item) {
+    DnItem it;
+    it.b = item / p.n_span;
+    it.span = item % p.n_span;
+    it.t0 = it.span * p.tps;
+    it.nt = min(p.tps, p.tiles - it.t0);
+    return it;
+}
+
+template <int HQ>
+__global__ void __launch_bounds__(DN_THREADS, 1)
+    k_xkv_ra_dense(const __grid_constant__ CUtensorMap tmAk,
+                   const __grid_constant__ CUtensorMap tmAv, const DnParams p) {
+    using Cfg = DnCfg<HQ>;
+    constexpr int NO = Cfg::NO, ATOM = Cfg::ATOM, PBUF = Cfg::PBUF;
+    constexpr uint32_t TM_Z = 0, TM_U = 2 * NO;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    unsigned char *qbuf = smem + DN_STAGES * DN_STAGE;
+    unsigned char *pbuf = qbuf + (p.rk / 64) * ATOM;      // two P buffers
+    DnShared *sh = reinterpret_cast<DnShared *>(pbuf + 2 * PBUF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t Lp = (int64_t)p.tiles * DN_TILE;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < DN_STAGES; ++s) {
+            mbar_init(&sh->full[s], 1);
+            mbar_init(&sh->empty[s], 1);
+        }
+        mbar_init(&sh->q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sh->zfull[i], 1);
+            mbar_init(&sh->zfree[i], 1);
+            mbar_init(&sh->pfull[i], 1);
+            mbar_init(&sh->pfree[i], 1);
+        }
+        mbar_init(&sh->ufull, 1);
+        mbar_init(&sh->ufree, 1);
+        mbar_init(&sh->idle, 1);
+        sh->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_tmap(&tmAk);
+        prefetch_tmap(&tmAv);
+    }
+    if (warp == DW_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         su32(&sh->tmem_base))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tcgen05_before();
+    __syncthreads();
+    tcgen05_after();
+    const uint32_t tmem = sh->tmem_base;
+
+    if (warp == DW_LOAD) {
+        // ------------------------------------------------------------ copies (one thread)
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+                const DnItem w = dn_decode(p, item);
+                const int row0 = (int)((int64_t)w.b * p.L + (int64_t)w.t0 * DN_TILE);
+                for (int phase = 0; phase < 2 && ok; ++phase) {
+                    const int nst = (phase == 0 ? p.rk : p.rv) / 128;
+                    const CUtensorMap *m = phase == 0 ? &tmAk : &tmAv;
+                    for (int i = 0; i < w.nt && ok; ++i)
+                        for (int st = 0; st < nst; ++st, ++it) {
+                            const int s = it % DN_STAGES, n = it / DN_STAGES;
+                            if (!dn_wait(&sh->empty[s], (n & 1) ^ 1, sh, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_expect_tx(&sh->full[s], (uint32_t)DN_STAGE);
+                            // rows past the batch's last row read as zeros (full box bytes)
+                            tma_load_3d(m, &sh->full[s], smem + s * DN_STAGE, 0,
+                                        row0 + i * DN_TILE, st * 2);
+                        }
+                }
+            }
+            if (!ok) {
+                // the copies issued into the last DN_STAGES stages land before the CTA leaves
+                for (int j = it - DN_STAGES > 0 ? it - DN_STAGES : 0; j < it; ++j)
+                    for (uint32_t i = 0; i < RA_SPIN; ++i)
+                        if (mbar_test(&sh->full[j % DN_STAGES], (uint32_t)(j / DN_STAGES) & 1))
+                            break;
+            }
+        }
+        __syncwarp();
+    } else if (warp == DW_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sbase = su32(smem), qb = su32(qbuf), pb = su32(pbuf);
+            constexpr uint32_t idZ = idesc_f16(128, NO, false, false);
+            constexpr uint32_t idU = idesc_f16(128, NO, true, false);   // A^V read MN-major
+            int it = 0, zt = 0, pt = 0, ic = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++ic) {
+                const DnItem w = dn_decode(p, item);
+                if (!dn_wait(&sh->q_full, ic & 1, sh, p.status)) break;
+                tcgen05_after();
+                // pass 1: logits of each tile into TMEM buffer zt & 1
+                for (int i = 0; i < w.nt && ok; ++i, ++zt) {
+                    const int zb = zt & 1;
+                    if (!dn_wait(&sh->zfree[zb], ((zt >> 1) & 1) ^ 1, sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_after();
+                    for (int st = 0; st < p.rk / 128; ++st, ++it) {
+                        const int s = it % DN_STAGES, n = it / DN_STAGES;
+                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tcgen05_after();
+                        const uint32_t a0 = sbase + s * DN_STAGE;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int k0 = st * 128 + kk * 16;
+                            umma_f16(tmem + TM_Z + zb * NO,
+                                     smem_desc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                     smem_desc_sw128(qb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32, 16, 1024),
+                                     idZ, (st | kk) ? 1u : 0u);
+                        }
+                        umma_arrive(&sh->empty[s]);
+                    }
+                    if (ok) umma_arrive(&sh->zfull[zb]);
+                }
+                if (!ok) break;
+                // pass 2: the span's value products, accumulated over its tiles
+                if (!dn_wait(&sh->ufree, (ic & 1) ^ 1, sh, p.status)) break;
+                tcgen05_after();
+                for (int i = 0; i < w.nt && ok; ++i, ++pt) {
+                    const int pbi = pt & 1;
+                    if (!dn_wait(&sh->pfull[pbi], (pt >> 1) & 1, sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_after();
+                    for (int st = 0; st < p.rv / 128; ++st, ++it) {
+                        const int s = it % DN_STAGES, n = it / DN_STAGES;
+                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tcgen05_after();
+                        const uint32_t a0 = sbase + s * DN_STAGE;
+#pragma unroll
+                        for (int kt = 0; kt < 8; ++kt)
+                            umma_f16(tmem + TM_U + st * NO,
+                                     smem_desc_sw128(a0 + kt * 2048, 16384, 1024),
+                                     smem_desc_sw128(pb + pbi * PBUF + (kt >> 2) * ATOM + (kt & 3) * 32, 16, 1024),
+                                     idU, (i | kt) ? 1u : 0u);
+                        umma_arrive(&sh->empty[s]);
+                    }
+                    if (ok) umma_arrive(&sh->pfree[pbi]);
+                }
+                if (!ok) break;
+                umma_arrive(&sh->ufull);
+            }
+            // every MMA this thread issued has completed once `idle` fires
+            umma_arrive(&sh->idle);
+            for (uint32_t i = 0; i < RA_SPIN; ++i)
+                if (mbar_test(&sh->idle, 0)) break;
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 32 * DW_EPI;   // 0..127
+        const int ew = warp - DW_EPI;
+        const int quad = warp & 3;                  // TMEM lane quadrant of this warp
+        const int lrow = quad * 32 + lane;          // token of a tile / rank column of a block
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        // zero Q~ and both P buffers: the padding rows n >= 2 Hq stay zero
+        for (int i = et; i < ((p.rk / 64) * ATOM + 2 * PBUF) / 16; i += DN_EPI_THREADS)
+            reinterpret_cast<uint4 *>(qbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+        dn_epi_bar();
+        auto write_q = [&](int b) {                 // Q~ rows: hi of the Hq heads, then lo
+            const size_t base = (size_t)b * HQ * p.rk;
+            const int per = p.rk / 8;               // 16-byte pieces per row
+            for (int e = et; e < 2 * HQ * per; e += DN_EPI_THREADS) {
+                const int n = e / per, c16 = e % per;
+                const __nv_bfloat16 *src =
+                    (n < HQ ? p.qt_hi : p.qt_lo) + base + (size_t)(n % HQ) * p.rk + c16 * 8;
+                *reinterpret_cast<uint4 *>(qbuf + kmaj_off(n, c16 * 8, ATOM)) =
+                    *reinterpret_cast<const uint4 *>(src);
+            }
+        };
+        if (blockIdx.x < p.n_items) write_q(dn_decode(p, blockIdx.x).b);
+        fence_async_smem();
+        dn_epi_bar();
+        if (et == 0) mbar_arrive(&sh->q_full);
+        int zt = 0, pt = 0, ic = 0;
+        bool dead = false;
+        for (int item = blockIdx.x; item < p.n_items && !dead; item += gridDim.x, ++ic) {
+            const DnItem w = dn_decode(p, item);
+            float m[HQ];
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) m[h] = -INFINITY;
+            float *zrow = p.z + (size_t)w.b * HQ * Lp;
+            // pass 1: logits to the scratch, running max
+            for (int i = 0; i < w.nt; ++i, ++zt) {
+                const int zb = zt & 1;
+                {
+                    const bool fail = !dn_wait(&sh->zfull[zb], (zt >> 1) & 1, sh, p.status);
+                    if (dn_epi_bar_any(fail)) { dead = true; break; }
+                }
+                tcgen05_after();
+                float v[NO];
+                tmem_load_cols<NO>(tmem + lane_base + TM_Z + zb * NO, v);
+                tcgen05_before();
+                const int64_t t = (int64_t)(w.t0 + i) * DN_TILE + lrow;
+                const bool valid = t < p.L;
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                    const float zh = valid ? (v[h] + v[HQ + h]) * p.qscale : -INFINITY;
+                    m[h] = fmaxf(m[h], zh);
+                    zrow[(size_t)h * Lp + t] = zh;
+                }
+                dn_epi_bar();
+                if (et == 0) mbar_arrive(&sh->zfree[zb]);
+            }
+            if (dead) break;
+            // the span's max per head
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1)
+                    m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
+                if (lane == 0) sh->red[ew][h] = m[h];
+            }
+            dn_epi_bar();
+#pragma unroll
+            for (int h = 0; h < HQ; ++h)
+                m[h] = fmaxf(fmaxf(sh->red[0][h], sh->red[1][h]), fmaxf(sh->red[2][h], sh->red[3][h]));
+            dn_epi_bar();
+            // every logit MMA of this item has completed: Q~ takes the next item's rows
+            if (item + (int)gridDim.x < p.n_items) {
+                write_q(dn_decode(p, item + gridDim.x).b);
+                fence_async_smem();
+                dn_epi_bar();
+                if (et == 0) mbar_arrive(&sh->q_full);
+            }
+            // pass 2: probabilities of each tile into P buffer pt & 1
+            float l[HQ];
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) l[h] = 0.f;
+            for (int i = 0; i < w.nt; ++i, ++pt) {
+                const int pbi = pt & 1;
+                {
+                    const bool fail = !dn_wait(&sh->pfree[pbi], ((pt >> 1) & 1) ^ 1, sh, p.status);
+                    if (dn_epi_bar_any(fail)) { dead = true; break; }
+                }
+                const int64_t t = (int64_t)(w.t0 + i) * DN_TILE + lrow;
+                unsigned char *pdst = pbuf + pbi * PBUF;
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                    const float pv = exp2f(zrow[(size_t)h * Lp + t] - m[h]);   // 0 past L
+                    l[h] += pv;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(pv - __bfloat162float(hi));
+                    *reinterpret_cast<__nv_bfloat16 *>(pdst + kmaj_off(h, lrow, ATOM)) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(pdst + kmaj_off(HQ + h, lrow, ATOM)) = lo;
+                }
+                fence_async_smem();
+                dn_epi_bar();
+                if (et == 0) mbar_arrive(&sh->pfull[pbi]);
+            }
+            if (dead) break;
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+                if (lane == 0) sh->red[ew][h] = l[h];
+            }
+            {
+                const bool fail = !dn_wait(&sh->ufull, ic & 1, sh, p.status);
+                if (dn_epi_bar_any(fail)) break;       // also publishes red
+            }
+#pragma unroll
+            for (int h = 0; h < HQ; ++h)
+                l[h] = (sh->red[0][h] + sh->red[1][h]) + (sh->red[2][h] + sh->red[3][h]);
+            tcgen05_after();
+            float *dst = p.partials + ((size_t)w.span * p.B + w.b) * HQ * (p.rv + 2);
+            for (int sb = 0; sb < p.rv / 128; ++sb) {
+                float v[NO];
+                tmem_load_cols<NO>(tmem + lane_base + TM_U + sb * NO, v);
+#pragma unroll
+                for (int h = 0; h < HQ; ++h)
+                    dst[(size_t)h * (p.rv + 2) + 2 + sb * 128 + lrow] = v[h] + v[HQ + h];
+            }
+            tcgen05_before();
+            if (et == 0) {
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                    dst[(size_t)h * (p.rv + 2)] = m[h] * 0.6931471805599453f;   // natural log
+                    dst[(size_t)h * (p.rv + 2) + 1] = l[h];
+                }
+            }
+            dn_epi_bar();                            // red is rewritten by the next item
+            if (et == 0) mbar_arrive(&sh->ufree);
+        }
+    }
+    tcgen05_before();
+    __syncthreads();
+    tcgen05_after();
+    if (warp == DW_MMA)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
+                     : "memory");
+}
+
 // q~[b][h][i] = sum_j q[b][h][j] B^K[b][i][g*hd + j]  (Bkt row g*hd + j holds column j of
 // the group's slice), fp32, then split into the bf16 nearest and the bf16 of the rest.
 // One CTA per (b, g, 128 columns i): warp w takes rows j = w, w + 8, ... of the slice, each
@@ -582,24 +985,86 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
     }
 }
 
+// Dense-mode plan: spans of whole 128-token tiles, about one span per SM over the batch.
+struct DnPlan {
+    int tiles, tps, n_span;
+};
+DnPlan dense_plan(const xkv_dims &d) {
+    DnPlan q;
+    q.tiles = (int)((d.ctx_len + DN_TILE - 1) / DN_TILE);
+    int ns = DN_SPANS / d.batch;
+    ns = ns < 1 ? 1 : (ns > q.tiles ? q.tiles : ns);
+    q.tps = (q.tiles + ns - 1) / ns;
+    q.n_span = (q.tiles + q.tps - 1) / q.tps;
+    return q;
+}
+template <int HQ>
+size_t dn_smem(const xkv_dims &d) {
+    return 1024 + (size_t)DN_STAGES * DN_STAGE + (size_t)(d.rank_k / 64) * DnCfg<HQ>::ATOM +
+           2 * (size_t)DnCfg<HQ>::PBUF + sizeof(DnShared);
+}
+template <int HQ>
+bool dn_fits(const xkv_dims &d) {
+    return (2 + d.rank_v / 128) * DnCfg<HQ>::NO <= 512 && dn_smem<HQ>(d) <= 232448;
+}
+bool dense_heads_ok(const xkv_dims &d) {
+    if ((int64_t)d.batch * d.ctx_len < DN_TILE) return false;   // a copy box fits the rows
+    switch (d.n_q_heads) {
+        case 8: return dn_fits<8>(d);
+        case 16: return dn_fits<16>(d);
+        case 24: return dn_fits<24>(d);
+        case 32: return dn_fits<32>(d);
+        default: return false;
+    }
+}
+template <int HQ>
+cudaError_t launch_dense_hq(const xkv_dims &d, const CUtensorMap *maps, const DnParams &dp,
+                            cudaStream_t s) {
+    const size_t smem = dn_smem<HQ>(d);
+    auto k = k_xkv_ra_dense<HQ>;
+    cudaError_t e = set_smem_limit((const void *)k, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = dp.n_items < sm_count() ? dp.n_items : sm_count();
+    k<<<grid, DN_THREADS, smem, s>>>(maps[0], maps[1], dp);
+    return cudaGetLastError();
+}
+cudaError_t launch_dense(const xkv_dims &d, const CUtensorMap *maps, const DnParams &dp,
+                         cudaStream_t s) {
+    switch (d.n_q_heads) {
+        case 8: return launch_dense_hq<8>(d, maps, dp, s);
+        case 16: return launch_dense_hq<16>(d, maps, dp, s);
+        case 24: return launch_dense_hq<24>(d, maps, dp, s);
+        case 32: return launch_dense_hq<32>(d, maps, dp, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int G>
 cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams &p,
-                     const void *q, const void *Bkt, const void *Bvt, __nv_bfloat16 *qt_hi,
-                     __nv_bfloat16 *qt_lo, float *U, float *Lsum, float *out, cudaStream_t s) {
+                     const DnParams *dp, const void *q, const void *Bkt, const void *Bvt,
+                     __nv_bfloat16 *qt_hi, __nv_bfloat16 *qt_lo, float *U, float *Lsum,
+                     float *out, cudaStream_t s) {
     k_qtilde<G><<<dim3(d.n_kv_heads, d.batch, d.rank_k / QT_COLS), 256, 0, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
         d.n_kv_heads, d.head_dim, d.rank_k, p.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem = 1024 + (size_t)RA_STAGES * RA_STAGE + RA_QBUF + RA_PBUF + sizeof(RaShared);
-    auto k = k_xkv_ra<G>;
-    if ((e = set_smem_limit((const void *)k, smem)) != cudaSuccess) return e;
-    const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
-    k<<<grid, RA_THREADS, smem, s>>>(maps[0], maps[1], p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    int n_split = p.n_split;
+    if (dp) {
+        if ((e = launch_dense(d, maps, *dp, s)) != cudaSuccess) return e;
+        n_split = dp->n_span;
+    } else {
+        const size_t smem =
+            1024 + (size_t)RA_STAGES * RA_STAGE + RA_QBUF + RA_PBUF + sizeof(RaShared);
+        auto k = k_xkv_ra<G>;
+        if ((e = set_smem_limit((const void *)k, smem)) != cudaSuccess) return e;
+        const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
+        k<<<grid, RA_THREADS, smem, s>>>(maps[0], maps[1], p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     const int BH = d.batch * d.n_q_heads;
     k_merge_ra<<<dim3(BH, (d.rank_v + MG_COLS - 1) / MG_COLS), MG_THREADS, 0, s>>>(
-        p.partials, U, Lsum, p.n_split, BH, d.rank_v, p.status);
+        p.partials, U, Lsum, n_split, BH, d.rank_v, p.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t psmem = sizeof(float) * (size_t)G * d.rank_v;
     auto kp = k_project_ra<G>;
@@ -636,6 +1101,20 @@ size_t ra_scratch_bytes(const xkv_dims &d, int n_split) {
            al256(bh * sizeof(float)) + (size_t)n_split * bh * (d.rank_v + 2) * sizeof(float);
 }
 
+// Dense calls with a supported head count run the head-batched kernel: partials per span,
+// then the logit scratch [B][Hq][tiles * 128] fp32 on a 256-byte boundary.
+bool attend_ra_dense_heads(const xkv_dims &d) { return attend_ra_shape_ok(d) && dense_heads_ok(d); }
+
+size_t ra_call_scratch_bytes(const xkv_dims &d, bool dense, int n_sel) {
+    if (dense && attend_ra_dense_heads(d)) {
+        const DnPlan pl = dense_plan(d);
+        const size_t bh = (size_t)d.batch * d.n_q_heads;
+        return al256(ra_scratch_bytes(d, pl.n_span)) +
+               bh * (size_t)pl.tiles * DN_TILE * sizeof(float);
+    }
+    return ra_scratch_bytes(d, ra_splits(d, n_sel));
+}
+
 cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
                              const void *Bvt, const void *q, const int32_t *sel, int n_sel,
                              void *scratch, unsigned *status, float *out, cudaStream_t s) {
@@ -670,12 +1149,36 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
     p.n_split = (n_sel + p.chunks_per_item - 1) / p.chunks_per_item;
     p.n_items = d.batch * d.n_kv_heads * p.n_split;
     p.qscale = 1.4426950408889634f / sqrtf((float)d.head_dim);
+    DnParams dp;
+    const DnParams *dpp = nullptr;
+    if (!sel && attend_ra_dense_heads(d)) {
+        const DnPlan pl = dense_plan(d);
+        dp.qt_hi = qt_hi;
+        dp.qt_lo = qt_lo;
+        dp.partials = p.partials;
+        dp.z = (float *)((char *)p.partials + al256((size_t)pl.n_span * bh * (d.rank_v + 2) *
+                                                    sizeof(float)));
+        dp.status = status;
+        dp.L = d.ctx_len;
+        dp.rk = d.rank_k;
+        dp.rv = d.rank_v;
+        dp.B = d.batch;
+        dp.tiles = pl.tiles;
+        dp.tps = pl.tps;
+        dp.n_span = pl.n_span;
+        dp.n_items = d.batch * pl.n_span;
+        dp.qscale = p.qscale;
+        dpp = &dp;
+        // the 3D views with 128-row boxes: one copy per 128 x 128 stage
+        if (!make_map_bf16_sw128_cb(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 128, 2) ||
+            !make_map_bf16_sw128_cb(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 128, 2))
+            return cudaErrorInvalidValue;
+    }
     switch (d.n_q_heads / d.n_kv_heads) {
-        case 1: return launch_g<1>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
-        case 2: return launch_g<2>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
-        case 4: return launch_g<4>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
-        case 5: return launch_g<5>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
-        case 8: return launch_g<8>(d, maps, p, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+#define XKV_RA_G(GG) \
+    case GG: return launch_g<GG>(d, maps, p, dpp, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+        XKV_RA_G(1) XKV_RA_G(2) XKV_RA_G(4) XKV_RA_G(5) XKV_RA_G(8)
+#undef XKV_RA_G
         default: return cudaErrorInvalidValue;
     }
 }

@@ -340,27 +340,33 @@ __global__ void __launch_bounds__(SS_THREADS) k_score_select(const SsParams p) {
         for (int i = 0; i < SS_RPT; ++i)
 #pragma unroll
             for (int h = 0; h < G; ++h) acc[i][h] = 0.f;
-#pragma unroll 2
-        for (int v = 0; v < vpr; ++v) {
-            uint4 w[SS_RPT];
+        // a row is read a 128-byte line at a time: the eight 16-byte loads of a line go
+        // out back to back and merge in flight (shared memory leaves L1 too small to keep
+        // a line between loads spread over the arithmetic)
+        for (int v0 = 0; v0 < vpr; v0 += 8) {
+            uint4 w[SS_RPT][8];
 #pragma unroll
-            for (int i = 0; i < SS_RPT; ++i) w[i] = __ldg(rp[i] + v);
+            for (int i = 0; i < SS_RPT; ++i)
 #pragma unroll
-            for (int k = 0; k < EPV; ++k) {
-                float x[SS_RPT];
+                for (int v = 0; v < 8; ++v) w[i][v] = __ldg(rp[i] + v0 + v);
 #pragma unroll
-                for (int i = 0; i < SS_RPT; ++i) {
-                    x[i] = Vec<T>::get(w[i], k);
-                    mx = fmaxf(mx, fabsf(x[i]));
+            for (int v = 0; v < 8; ++v)
+#pragma unroll
+                for (int k = 0; k < EPV; ++k) {
+                    float x[SS_RPT];
+#pragma unroll
+                    for (int i = 0; i < SS_RPT; ++i) {
+                        x[i] = Vec<T>::get(w[i][v], k);
+                        mx = fmaxf(mx, fabsf(x[i]));
+                    }
+                    const float *qd = qf + ((v0 + v) * EPV + k) * G;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float qv = qd[h];
+#pragma unroll
+                        for (int i = 0; i < SS_RPT; ++i) acc[i][h] = fmaf(x[i], qv, acc[i][h]);
+                    }
                 }
-                const float *qd = qf + (v * EPV + k) * G;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float qv = qd[h];
-#pragma unroll
-                    for (int i = 0; i < SS_RPT; ++i) acc[i][h] = fmaf(x[i], qv, acc[i][h]);
-                }
-            }
         }
 #pragma unroll
         for (int i = 0; i < SS_RPT; ++i) {

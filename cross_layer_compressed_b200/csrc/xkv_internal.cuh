@@ -69,6 +69,9 @@ bool tma_available();   // the driver exposes the tensor-map encoder
 bool attend_ra_shape_ok(const xkv_dims &d);
 int ra_splits(const xkv_dims &d, int n_sel);
 size_t ra_scratch_bytes(const xkv_dims &d, int n_split);
+// scratch of one reassociated call: dense (no selection) or n_sel selected chunks
+size_t ra_call_scratch_bytes(const xkv_dims &d, bool dense, int n_sel);
+bool attend_ra_dense_heads(const xkv_dims &d);
 cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, const void *Bkt,
                              const void *Bvt, const void *q, const int32_t *sel, int n_sel,
                              void *scratch, unsigned *status, float *out, cudaStream_t s);

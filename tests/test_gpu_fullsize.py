@@ -34,9 +34,10 @@ def _xkv_layer_check(xkv, ora, w, layer, units, dense=False, reassociated=False)
     out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
     hd, G = w.head_dim, w.group
     if dense:
-        ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_DENSE), dtype=torch.uint8,
-                         device=DEV)
-        xkv.xkv_reconstruct_attend(d, c["Ak"], c["Av"], c["Bkt"], c["Bvt"], q, None, 0, out, ws)
+        mode = xkv.XKV_MODE_REASSOC if reassociated else xkv.XKV_MODE_DENSE
+        attend = xkv.xkv_reassociated_attend if reassociated else xkv.xkv_reconstruct_attend
+        ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, mode), dtype=torch.uint8, device=DEV)
+        attend(d, c["Ak"], c["Av"], c["Bkt"], c["Bvt"], q, None, 0, out, ws)
         torch.cuda.synchronize()
         for b, g in units:
             ref = ora.reconstruct_attend(c["Ak"][b:b + 1].cpu(), c["Av"][b:b + 1].cpu(),
@@ -147,6 +148,14 @@ def test_qwen14b_selective_16k_full_layer_reassociated(xkv, ora):
 def test_llama8b_dense_128k_full_layer(xkv, ora):
     w = synth.LLAMA8B_DENSE_128K
     _xkv_layer_check(xkv, ora, w, layer=2, units=[(0, 3)], dense=True)
+    torch.cuda.empty_cache()
+
+
+def test_llama8b_dense_128k_full_layer_reassociated(xkv, ora):
+    """The head-batched rank-space kernel on the full 128K window: 147 spans of 7 tiles."""
+    w = synth.LLAMA8B_DENSE_128K
+    _xkv_layer_check(xkv, ora, w, layer=2, units=[(0, 0), (0, 6)], dense=True,
+                     reassociated=True)
     torch.cuda.empty_cache()
 
 

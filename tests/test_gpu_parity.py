@@ -409,6 +409,35 @@ def test_reassociated_attend_dense(xkv, ora):
     compare_outputs(_reassoc(xkv, w, x, None)[0], ref, w.dtype)
 
 
+# Dense mode runs the head-batched kernel (one pass over A for all heads of a sequence,
+# spans of 128-token tiles): ragged last tiles, several spans per sequence and several
+# tiles per span, batches whose spans do not fill the GPU evenly, 8 / 16 / 24 / 32 heads
+# and smaller ranks.
+DENSE_CASES = [
+    synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=1000, name="dense_ragged"),
+    synth.reduced(synth.LLAMA8B_DENSE_128K, batch=3, ctx_len=2056, name="dense_b3"),
+    synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=40960, name="dense_40k_spans"),
+    dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=2, ctx_len=1536),
+                        n_q_heads=16, n_kv_heads=8, name="dense_hq16_g2"),
+    dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=2, ctx_len=1152),
+                        n_q_heads=8, n_kv_heads=8, rank_k=256, rank_v=384, name="dense_hq8_g1"),
+    dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=2048),
+                        n_q_heads=24, n_kv_heads=6, rank_k=384, rank_v=640, name="dense_hq24"),
+]
+
+
+@pytest.mark.parametrize("w", DENSE_CASES, ids=lambda w: w.name)
+def test_reassociated_attend_dense_all_heads(xkv, ora, w):
+    x = _layer_inputs(w)
+    units = None if w.ctx_len <= 4096 else [(0, 0), (0, w.n_kv_heads - 1)]
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], None, w.chunk,
+                                 units=units)
+    got = _reassoc(xkv, w, x, None)[0]
+    G = w.n_q_heads // w.n_kv_heads
+    for b, g in units or [(b, g) for b in range(w.batch) for g in range(w.n_kv_heads)]:
+        compare_outputs(got[b, g * G:(g + 1) * G], ref[b, g * G:(g + 1) * G], w.dtype)
+
+
 @pytest.mark.parametrize("n_sel", [1, 3, 17, 33, 128])
 def test_reassociated_selection_sizes(xkv, ora, n_sel):
     """Items of one chunk, odd 8-row group counts (padded MMA steps), several splits."""
