@@ -762,9 +762,14 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                 }
                 const int64_t t = (int64_t)(w.t0 + i) * DN_TILE + lrow;
                 unsigned char *pdst = pbuf + pbi * PBUF;
+                // every logit load in flight before the first shared-memory store (the
+                // stores could otherwise order each load after the previous head's)
+                float zl[HQ];
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) zl[h] = __ldcg(zrow + (size_t)h * Lp + t);
 #pragma unroll
                 for (int h = 0; h < HQ; ++h) {
-                    const float pv = exp2f(zrow[(size_t)h * Lp + t] - m[h]);   // 0 past L
+                    const float pv = exp2f(zl[h] - m[h]);   // 0 past L
                     l[h] += pv;
                     const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
                     const __nv_bfloat16 lo = __float2bfloat16_rn(pv - __bfloat162float(hi));
@@ -820,11 +825,11 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
 
 // q~[b][h][i] = sum_j q[b][h][j] B^K[b][i][g*hd + j]  (Bkt row g*hd + j holds column j of
 // the group's slice), fp32, then split into the bf16 nearest and the bf16 of the rest.
-// One CTA per (b, g, 128 columns i): warp w takes rows j = w, w + 8, ... of the slice, each
-// lane 4 columns (one 8-byte load per row, all rows' loads in flight), and the 8 warps'
-// sums meet in shared memory.
-constexpr int QT_COLS = 128;
-template <int G>
+// One CTA per (b, g, 32 CPL columns i): warp w takes rows j = w, w + 8, ... of the slice,
+// each lane CPL columns (all 16 rows' loads in flight), and the 8 warps' sums meet in
+// shared memory.  The host takes CPL = 1 when the CPL = 4 grid would leave SMs idle
+// (batch 1: 16 slices per KV head at rank 512), else CPL = 4.
+template <int G, int CPL>
 __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict__ q,
                                                 const __nv_bfloat16 *__restrict__ Bkt,
                                                 __nv_bfloat16 *__restrict__ qt_hi,
@@ -835,33 +840,43 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
     // the call's device-side error word starts clean: this kernel runs first in the call,
     // so the clear is ordered before every kernel that may set it
     if (status && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *status = 0u;
+    constexpr int QT_COLS = 32 * CPL;
     __shared__ float red[8][G][QT_COLS];
     const int g = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * QT_COLS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < G * hd; e += blockDim.x)
         qs[e] = __bfloat162float(q[((size_t)b * Hq + (size_t)g * G) * hd + e]);
     __syncthreads();
-    const __nv_bfloat16 *Bg = Bkt + ((size_t)b * Hkv * hd + (size_t)g * hd) * rk + i0 + lane * 4;
-    float acc[G][4];
+    const __nv_bfloat16 *Bg =
+        Bkt + ((size_t)b * Hkv * hd + (size_t)g * hd) * rk + i0 + lane * CPL;
+    float acc[G][CPL];
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[h][c] = 0.f;
+        for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
 #pragma unroll 16
     for (int j = warp; j < hd; j += 8) {            // every row's load in flight at once
-        const uint2 w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
-        const float bv[4] = {bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y)};
+        float bv[CPL];
+        if constexpr (CPL == 4) {
+            const uint2 w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
+            bv[0] = bf16lo(w2.x);
+            bv[1] = bf16hi(w2.x);
+            bv[2] = bf16lo(w2.y);
+            bv[3] = bf16hi(w2.y);
+        } else {
+            bv[0] = __bfloat162float(Bg[(size_t)j * rk]);
+        }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             const float qv = qs[h * hd + j];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(qv, bv[c], acc[h][c]);
+            for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(qv, bv[c], acc[h][c]);
         }
     }
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) red[warp][h][lane * 4 + c] = acc[h][c];
+        for (int c = 0; c < CPL; ++c) red[warp][h][lane * CPL + c] = acc[h][c];
     __syncthreads();
     for (int e = threadIdx.x; e < G * QT_COLS; e += blockDim.x) {
         const int h = e / QT_COLS, c = e % QT_COLS;
@@ -877,16 +892,19 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
 
 // Merge an item's splits in rank space:
 //   M = max_s m_s,  U_h[r] = sum_s e^{m_s - M} u_s[r],  L_h = sum_s e^{m_s - M} l_s.
-// One CTA per (b, h, 256 columns of r): warp w takes the splits s = w, w + 8, ..., each
-// lane 8 columns (coalesced 128-byte rows), so every thread keeps 8 independent loads in
-// flight; the 8 warps' sums meet in shared memory.
+// One CTA per (b, h, 32 CPL columns of r): warp w takes the splits s = w, w + 8, ..., each
+// lane CPL columns (coalesced 128-byte rows; the loop is unrolled so that several splits'
+// loads are in flight); the 8 warps' sums meet in shared memory.  The host takes CPL = 2
+// when the CPL = 8 grid would leave SMs idle (the 147 spans of a dense batch-1 call), else
+// CPL = 8.
 constexpr int MG_THREADS = 256;
-constexpr int MG_COLS = 256;
+template <int CPL>
 __global__ void __launch_bounds__(MG_THREADS) k_merge_ra(const float *__restrict__ partials,
                                                          float *__restrict__ U,
                                                          float *__restrict__ Lsum, int n_split,
                                                          int BH, int rv,
                                                          const unsigned *__restrict__ status) {
+    constexpr int MG_COLS = 32 * CPL;
     __shared__ float red[MG_THREADS / 32][MG_COLS];
     __shared__ float s_m[MG_THREADS / 32];
     __shared__ float s_l[MG_THREADS / 32];
@@ -905,22 +923,22 @@ __global__ void __launch_bounds__(MG_THREADS) k_merge_ra(const float *__restrict
     M = s_m[0];
 #pragma unroll
     for (int w = 1; w < NW; ++w) M = fmaxf(M, s_m[w]);
-    float acc[8], l = 0.f;
+    float acc[CPL], l = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-#pragma unroll 4
+    for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
+#pragma unroll 8
     for (int sp = warp; sp < n_split; sp += NW) {
         const float *ps = p + sp * stride;
         const float wgt = expf(ps[0] - M);
         l = fmaf(wgt, ps[1], l);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < CPL; ++k) {
             const int r = r0 + lane + 32 * k;
             if (r < rv) acc[k] = fmaf(wgt, ps[2 + r], acc[k]);
         }
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) red[warp][lane + 32 * k] = acc[k];
+    for (int k = 0; k < CPL; ++k) red[warp][lane + 32 * k] = acc[k];
     if (lane == 0) s_l[warp] = l;
     __syncthreads();
     const int r = r0 + threadIdx.x;
@@ -938,18 +956,19 @@ __global__ void __launch_bounds__(MG_THREADS) k_merge_ra(const float *__restrict
     }
 }
 
-// out[b][h][j] = (U_h . B^V[:, g*hd + j]) / L_h.  One CTA per (b, g, 32 columns j): each
-// warp takes 4 rows j of Bvt, so the group's B^V slice is read once for its G heads with
-// 16-byte loads, several per thread in flight.  Within a warp, lane = 8 * jr + c: row j = j0 + 4 * warp + jr, 16-byte pieces c, c + 8, ... of
-// the row; the 8 lanes of a row then sum their partial dot products with shuffles.
-constexpr int PJ_ROWS = 32;
-template <int G>
+// out[b][h][j] = (U_h . B^V[:, g*hd + j]) / L_h.  One CTA per (b, g, 8 RPW columns j): each
+// warp takes RPW rows j of Bvt, so the group's B^V slice is read once for its G heads; the
+// 32 / RPW lanes of a row take its 16-byte pieces in turn (all in flight) and sum their
+// partial dot products with shuffles.  The host takes RPW = 1 (more, smaller CTAs) when
+// the RPW = 4 grid would leave SMs idle, else RPW = 4.
+template <int G, int RPW>
 __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
                                                     const float *__restrict__ Lsum,
                                                     const __nv_bfloat16 *__restrict__ Bvt,
                                                     float *__restrict__ out, int Hq, int Hkv,
                                                     int hd, int rv,
                                                     const unsigned *__restrict__ status) {
+    constexpr int PJ_ROWS = 8 * RPW, LPR = 32 / RPW;   // rows per CTA, lanes per row
     extern __shared__ float Us[];                 // [G][rv]
     const int g = blockIdx.x, b = blockIdx.y, j0 = blockIdx.z * PJ_ROWS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -961,14 +980,14 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
     }
     for (int e = threadIdx.x; e < G * rv; e += blockDim.x) Us[e] = U[bh0 * rv + e];
     __syncthreads();
-    const int jr = lane >> 3, c = lane & 7;
-    const int j = j0 + warp * 4 + jr;
+    const int c = lane % LPR;
+    const int j = j0 + warp * RPW + lane / LPR;
     const __nv_bfloat16 *row = Bvt + ((size_t)b * Hkv * hd + (size_t)g * hd + j) * rv;
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll 4
-    for (int pc = c; pc < rv / 8; pc += 8) {       // 16-byte piece pc: columns 8 pc .. 8 pc + 7
+    for (int pc = c; pc < rv / 8; pc += LPR) {     // 16-byte piece pc: columns 8 pc .. 8 pc + 7
         const uint4 w4 = *reinterpret_cast<const uint4 *>(row + pc * 8);
         const float bv[8] = {bf16lo(w4.x), bf16hi(w4.x), bf16lo(w4.y), bf16hi(w4.y),
                              bf16lo(w4.z), bf16hi(w4.z), bf16lo(w4.w), bf16hi(w4.w)};
@@ -980,7 +999,7 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
 #pragma unroll
     for (int h = 0; h < G; ++h) {
 #pragma unroll
-        for (int off = 4; off; off >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], off);
+        for (int off = LPR / 2; off; off >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], off);
         if (c == 0) out[(bh0 + h) * hd + j] = acc[h] / Lsum[bh0 + h];
     }
 }
@@ -1044,9 +1063,16 @@ cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams 
                      const DnParams *dp, const void *q, const void *Bkt, const void *Bvt,
                      __nv_bfloat16 *qt_hi, __nv_bfloat16 *qt_lo, float *U, float *Lsum,
                      float *out, cudaStream_t s) {
-    k_qtilde<G><<<dim3(d.n_kv_heads, d.batch, d.rank_k / QT_COLS), 256, 0, s>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
-        d.n_kv_heads, d.head_dim, d.rank_k, p.status);
+    // narrow slices only where the wide ones leave SMs without a CTA
+    const bool few = (int64_t)d.batch * d.n_kv_heads * (d.rank_k / 128) < sm_count();
+    if (few)
+        k_qtilde<G, 1><<<dim3(d.n_kv_heads, d.batch, d.rank_k / 32), 256, 0, s>>>(
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
+            d.n_kv_heads, d.head_dim, d.rank_k, p.status);
+    else
+        k_qtilde<G, 4><<<dim3(d.n_kv_heads, d.batch, d.rank_k / 128), 256, 0, s>>>(
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
+            d.n_kv_heads, d.head_dim, d.rank_k, p.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int n_split = p.n_split;
@@ -1063,16 +1089,20 @@ cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const int BH = d.batch * d.n_q_heads;
-    k_merge_ra<<<dim3(BH, (d.rank_v + MG_COLS - 1) / MG_COLS), MG_THREADS, 0, s>>>(
-        p.partials, U, Lsum, n_split, BH, d.rank_v, p.status);
+    if ((int64_t)BH * ((d.rank_v + 255) / 256) < sm_count())
+        k_merge_ra<2><<<dim3(BH, (d.rank_v + 63) / 64), MG_THREADS, 0, s>>>(
+            p.partials, U, Lsum, n_split, BH, d.rank_v, p.status);
+    else
+        k_merge_ra<8><<<dim3(BH, (d.rank_v + 255) / 256), MG_THREADS, 0, s>>>(
+            p.partials, U, Lsum, n_split, BH, d.rank_v, p.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t psmem = sizeof(float) * (size_t)G * d.rank_v;
-    auto kp = k_project_ra<G>;
+    const bool pj_few = (int64_t)d.n_kv_heads * d.batch * (d.head_dim / 32) < sm_count();
+    auto kp = pj_few ? k_project_ra<G, 1> : k_project_ra<G, 4>;
     if ((e = set_smem_limit((const void *)kp, psmem)) != cudaSuccess) return e;
-    kp<<<dim3(d.n_kv_heads, d.batch, d.head_dim / PJ_ROWS), 256, psmem, s>>>(
-        U, Lsum, (const __nv_bfloat16 *)Bvt, out,
-                                                       d.n_q_heads, d.n_kv_heads, d.head_dim,
-                                                       d.rank_v, p.status);
+    kp<<<dim3(d.n_kv_heads, d.batch, d.head_dim / (pj_few ? 8 : 32)), 256, psmem, s>>>(
+        U, Lsum, (const __nv_bfloat16 *)Bvt, out, d.n_q_heads, d.n_kv_heads, d.head_dim,
+        d.rank_v, p.status);
     return cudaGetLastError();
 }
 

@@ -58,6 +58,15 @@ static __device__ __forceinline__ void tma_load_4d(const CUtensorMap *map, uint6
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(su32(bar))
         : "memory");
 }
+// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global memory into this CTA's shared memory, completing on the mbarrier `bar`.
+static __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(su32(dst)), "l"(src), "r"(bytes), "r"(su32(bar))
+        : "memory");
+}
 static __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
