@@ -925,8 +925,13 @@ def main():
     step_bytes = wl.step_bytes(bytes_launch)
     hbm_peak, _, peak_kind = measured_peaks()
     achieved = bytes_launch / (attend_avg_ms / 1e3) / 1e9
-    traffic = profiled_traffic(w.name, "k_xkv_tc" if w.mode != "rcla" else "k_rcla_tc",
-                               "attend_tc.cu" if w.mode != "rcla" else "rcla_tc.cu")
+    if w.mode == "rcla":
+        traffic = profiled_traffic(w.name, "k_rcla_tc", "rcla_tc.cu")
+    elif args.path == "reassociated":
+        traffic = profiled_traffic(w.name, "k_xkv_ra_dense" if w.mode == "dense" else "k_xkv_ra",
+                                   "attend_ra.cu")
+    else:
+        traffic = profiled_traffic(w.name, "k_xkv_tc", "attend_tc.cu")
 
     kernel = ("rcla_decode_attend" if w.mode == "rcla" else
               "reassociated_attend" if args.path == "reassociated" else "reconstruct_attend")
@@ -952,8 +957,6 @@ def main():
                     "traffic": traffic, "flops_per_launch": wl.attend_flops(),
                     "hbm_gbs": achieved, "hbm_frac": achieved / hbm_peak,
                     "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms}
-    if args.path == "reassociated":
-        roofline["traffic"] = None            # the committed captures are of the explicit kernel
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
