@@ -47,9 +47,11 @@ def parse():
     p.add_argument("--path", choices=["explicit", "reassociated"], default="explicit",
                    help="xKV attention: explicit reconstruction (the method as the pages "
                         "state it) or its rank-space reassociation")
-    p.add_argument("--scoring", choices=["fused", "separate"], default="separate",
+    p.add_argument("--scoring", choices=["fused", "separate"], default=None,
                    help="selective xKV: one fused scoring + selection call per layer "
-                        "(xkv_score_select) or xkv_score_landmarks + xkv_select_chunks")
+                        "(xkv_score_select) or xkv_score_landmarks + xkv_select_chunks "
+                        "(default: separate, the faster of the two here; fused when "
+                        "--value-reserve is given, since reserved chunks go through it)")
     p.add_argument("--value-reserve", type=int, default=0,
                    help="selective xKV: also keep the N chunks of largest value range per "
                         "(sequence, KV head) (value-range-aware selection; the statistic and "
@@ -60,7 +62,10 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call directly instead of replaying a captured step")
-    return p.parse_args()
+    a = p.parse_args()
+    if a.scoring is None:
+        a.scoring = "fused" if a.value_reserve > 0 else "separate"
+    return a
 
 
 def measured_peaks():
@@ -437,7 +442,7 @@ def cpu_baseline(w, seed, budget_s=20.0):
                 if w.mode != "dense" else "dense reconstruct-attend of one (sequence, KV head)")
     # one unit alone sizes the sample: as many units per core as fit the budget
     t1 = _run_units(unit, 1, 1)
-    per_core = max(1, min(8, int(budget_s / max(t1, 1e-3) / 2)))
+    per_core = max(1, min(32, int(budget_s / max(t1, 1e-3) / 2)))
     n_units = cores * per_core
     wall = _run_units(unit, n_units, cores) if t1 < budget_s else t1
     if t1 >= budget_s:
