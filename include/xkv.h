@@ -150,7 +150,8 @@ xkv_status xkv_select_chunks(const xkv_dims *dims, const double *scores, int32_t
  *       return (in stream order) its first B * Hkv 32-bit words hold, per (b, g), the
  *       number of chunks rescored in fp64, or 0xFFFFFFFF when the unit was scored wholly
  *       in fp64 (a band wider than 512 chunks, e.g. many equal scores, or fp32 scores out
- *       of range); the rest is the fp64 scores of such units.
+ *       of range); the rest holds the fp64 scores of such units, the fp32 keys of every
+ *       chunk and the per-CTA flags of the scoring pass.
  * G = n_q_heads / n_kv_heads in 1..8 or 16; nC <= 16384.  A unit whose fp64 scores hold a
  * NaN (inputs outside the contract) gets every entry -1.  reserved [B][Hkv][n_reserved]
  * (or NULL with n_reserved = 0): chunks forced in as well, see the value-range-aware
@@ -300,7 +301,10 @@ size_t xkv_tail_workspace_bytes(const xkv_dims *dims, int32_t n_sel, int64_t T_m
  * xkv_reconstruct_attend; ws holds at least
  * xkv_workspace_bytes(dims, sel ? n_sel : 0, XKV_MODE_REASSOC) bytes.  Runs for bf16,
  * head_dim 128, G in {1, 2, 4, 5, 8}, ranks multiples of 128 up to 1024 (r_K up to 512
- * when G > 4) and chunks dividing 256; other shapes return XKV_ERR_UNSUPPORTED.
+ * when G > 4) and chunks dividing 256; other shapes return XKV_ERR_UNSUPPORTED.  Dense
+ * calls (sel == NULL) with 8, 16, 24 or 32 query heads read the window once for all heads
+ * of a sequence (per-sequence spans of 128-token tiles); the workspace then also holds
+ * an fp32 logit scratch of B * Hq * L floats (rounded up to whole tiles).
  */
 xkv_status xkv_reassociated_attend(const xkv_dims *dims, const void *Ak_win, const void *Av_win,
                                    const void *Bkt_layer, const void *Bvt_layer, const void *q,
