@@ -844,33 +844,44 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
     __shared__ float red[8][G][QT_COLS];
     const int g = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * QT_COLS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const __nv_bfloat16 *Bg =
+        Bkt + ((size_t)b * Hkv * hd + (size_t)g * hd) * rk + i0 + lane * CPL;
+    // this warp's rows j = warp, warp + 8, ... (hd <= 128: at most 16) are loaded before
+    // the query is staged, so the two loads overlap
+    constexpr int RPW = 16;
+    float bv[RPW][CPL];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+        const int j = warp + 8 * i;
+        if constexpr (CPL == 4) {
+            uint2 w2 = make_uint2(0u, 0u);
+            if (j < hd) w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
+            bv[i][0] = bf16lo(w2.x);
+            bv[i][1] = bf16hi(w2.x);
+            bv[i][2] = bf16lo(w2.y);
+            bv[i][3] = bf16hi(w2.y);
+        } else {
+            bv[i][0] = j < hd ? __bfloat162float(Bg[(size_t)j * rk]) : 0.f;
+        }
+    }
     for (int e = threadIdx.x; e < G * hd; e += blockDim.x)
         qs[e] = __bfloat162float(q[((size_t)b * Hq + (size_t)g * G) * hd + e]);
     __syncthreads();
-    const __nv_bfloat16 *Bg =
-        Bkt + ((size_t)b * Hkv * hd + (size_t)g * hd) * rk + i0 + lane * CPL;
     float acc[G][CPL];
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
-#pragma unroll 16
-    for (int j = warp; j < hd; j += 8) {            // every row's load in flight at once
-        float bv[CPL];
-        if constexpr (CPL == 4) {
-            const uint2 w2 = *reinterpret_cast<const uint2 *>(Bg + (size_t)j * rk);
-            bv[0] = bf16lo(w2.x);
-            bv[1] = bf16hi(w2.x);
-            bv[2] = bf16lo(w2.y);
-            bv[3] = bf16hi(w2.y);
-        } else {
-            bv[0] = __bfloat162float(Bg[(size_t)j * rk]);
-        }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float qv = qs[h * hd + j];
+    for (int i = 0; i < RPW; ++i) {
+        const int j = warp + 8 * i;
+        if (j < hd) {
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(qv, bv[c], acc[h][c]);
+            for (int h = 0; h < G; ++h) {
+                const float qv = qs[h * hd + j];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(qv, bv[i][c], acc[h][c]);
+            }
         }
     }
 #pragma unroll
@@ -892,6 +903,8 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
 
 // Merge an item's splits in rank space:
 //   M = max_s m_s,  U_h[r] = sum_s e^{m_s - M} u_s[r],  L_h = sum_s e^{m_s - M} l_s.
+// (A one-pass form with a running max per warp was measured slower at the 147 spans of a
+// dense batch-1 call.)
 // One CTA per (b, h, 32 CPL columns of r): warp w takes the splits s = w, w + 8, ..., each
 // lane CPL columns (coalesced 128-byte rows; the loop is unrolled so that several splits'
 // loads are in flight); the 8 warps' sums meet in shared memory.  The host takes CPL = 2
@@ -978,24 +991,38 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
             out[(bh0 + e / PJ_ROWS) * hd + j0 + e % PJ_ROWS] = __int_as_float(0x7fc00000);
         return;
     }
-    for (int e = threadIdx.x; e < G * rv; e += blockDim.x) Us[e] = U[bh0 * rv + e];
-    __syncthreads();
     const int c = lane % LPR;
     const int j = j0 + warp * RPW + lane / LPR;
     const __nv_bfloat16 *row = Bvt + ((size_t)b * Hkv * hd + (size_t)g * hd + j) * rv;
+    // the first pieces of the row are loaded before U is staged, so the two loads overlap
+    constexpr int PRE = 4;
+    uint4 pre[PRE];
+#pragma unroll
+    for (int i = 0; i < PRE; ++i) {
+        const int pc = c + i * LPR;
+        pre[i] = pc < rv / 8 ? *reinterpret_cast<const uint4 *>(row + pc * 8)
+                             : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int e = threadIdx.x; e < G * rv; e += blockDim.x) Us[e] = U[bh0 * rv + e];
+    __syncthreads();
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 4
-    for (int pc = c; pc < rv / 8; pc += LPR) {     // 16-byte piece pc: columns 8 pc .. 8 pc + 7
-        const uint4 w4 = *reinterpret_cast<const uint4 *>(row + pc * 8);
+    // 16-byte piece pc holds columns 8 pc .. 8 pc + 7 of the row
+    auto piece = [&](int pc, const uint4 &w4) {
         const float bv[8] = {bf16lo(w4.x), bf16hi(w4.x), bf16lo(w4.y), bf16hi(w4.y),
                              bf16lo(w4.z), bf16hi(w4.z), bf16lo(w4.w), bf16hi(w4.w)};
 #pragma unroll
         for (int h = 0; h < G; ++h)
 #pragma unroll
             for (int k = 0; k < 8; ++k) acc[h] = fmaf(Us[h * rv + pc * 8 + k], bv[k], acc[h]);
-    }
+    };
+#pragma unroll
+    for (int i = 0; i < PRE; ++i)
+        if (c + i * LPR < rv / 8) piece(c + i * LPR, pre[i]);
+#pragma unroll 4
+    for (int pc = c + PRE * LPR; pc < rv / 8; pc += LPR)
+        piece(pc, *reinterpret_cast<const uint4 *>(row + pc * 8));
 #pragma unroll
     for (int h = 0; h < G; ++h) {
 #pragma unroll
