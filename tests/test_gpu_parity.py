@@ -164,6 +164,21 @@ def test_select_edge_cases_with_ties(xkv, ora, nC, top_k, n_sink, n_recent):
     assert np.array_equal(got, ref)
 
 
+def test_select_ranked_bin_with_ties(xkv, ora):
+    """Distinct scores except a dozen chunks planted at exactly the k-th value: the radix
+    descent stops at a bin of a few keys (ranked directly, ties by index)."""
+    rng = np.random.default_rng(21)
+    B, Hkv, nC, k = 2, 3, 4096, 256
+    s = rng.standard_normal((B, Hkv, nC))
+    for b in range(B):
+        for g in range(Hkv):
+            v = np.sort(s[b, g, 1:nC - 4])[::-1][k - 6]
+            idx = rng.choice(np.arange(1, nC - 4), 12, replace=False)
+            s[b, g, idx] = v
+    ref = ora.select_chunks(s, k, 1, 4)
+    assert np.array_equal(_run_select(xkv, s, k, 1, 4), ref)
+
+
 def test_select_distinct_scores_extremes(xkv, ora):
     rng = np.random.default_rng(9)
     s = rng.standard_normal((1, 2, 3000)) * 1e300
