@@ -428,10 +428,10 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
 //           D_u[r][n] += A^V[t][r] P[n][t]  (M = 128 rank columns per block, N = NO,
 //           K = tokens), accumulated in tensor memory over the whole span;
 //   end:    the span's (m, l, u) partial in rank space, merged across spans by k_merge_ra.
-// A stage is 128 tokens x 128 rank columns in one copy of the 3D view (64, rows, column
-// blocks) of A: two 64-column atoms of 128 rows, 16 KB apart.  Logits use A K-major
-// (8-row groups 1 KB apart), the value product reads the same stage MN-major (64-column
-// atoms 16 KB apart, 8-token groups 1 KB apart).  TMEM: two logit buffers, then the
+// A stage is 128 tokens x 128 rank columns in 16 copies of the 3D view (64, rows, column
+// blocks) of A, one per 8-row group, each landing as two consecutive 64-column atoms (the
+// layout of k_xkv_ra): logits use A K-major (8-row groups 2 KB apart), the value product
+// reads the same stage MN-major (64-column atoms 1 KB apart, 8-token groups 2 KB apart).  TMEM: two logit buffers, then the
 // r_V / 128 accumulator blocks, NO columns each.  Warp roles: warp 0 TMEM + MMA issue,
 // warp 1 the copies, warps 2-5 the epilogue (thread = TMEM lane = token, or rank column
 // at the end).
@@ -458,6 +458,7 @@ struct DnParams {
     unsigned *status;
     int64_t L;
     int rk, rv, B;
+    int rows_all;                         // B * L: rows of the 3D views
     int tiles, tps, n_span, n_items;
     float qscale;                         // log2(e) / sqrt(hd)
 };
@@ -580,9 +581,18 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                                 break;
                             }
                             mbar_expect_tx(&sh->full[s], (uint32_t)DN_STAGE);
-                            // rows past the batch's last row read as zeros (full box bytes)
-                            tma_load_3d(m, &sh->full[s], smem + s * DN_STAGE, 0,
-                                        row0 + i * DN_TILE, st * 2);
+                            // 16 copies of one 8-row group each (both 64-column atoms):
+                            // many copies in flight stream faster than one 32 KB box.  A
+                            // group past the batch's last row re-reads the last group (its
+                            // rows are masked: logit -inf, weight 0)
+                            const int base = row0 + i * DN_TILE;
+#pragma unroll
+                            for (int gr = 0; gr < DN_TILE / 8; ++gr) {
+                                int row = base + gr * 8;
+                                row = row < p.rows_all - 8 ? row : p.rows_all - 8;
+                                tma_load_3d(m, &sh->full[s], smem + s * DN_STAGE + gr * 2048, 0,
+                                            row, st * 2);
+                            }
                         }
                 }
             }
@@ -627,7 +637,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                         for (int kk = 0; kk < 8; ++kk) {
                             const int k0 = st * 128 + kk * 16;
                             umma_f16(tmem + TM_Z + zb * NO,
-                                     smem_desc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                     smem_desc_sw128(a0 + (kk >> 2) * 1024 + (kk & 3) * 32, 16, 2048),
                                      smem_desc_sw128(qb + (k0 >> 6) * ATOM + ((k0 & 63) >> 4) * 32, 16, 1024),
                                      idZ, (st | kk) ? 1u : 0u);
                         }
@@ -657,7 +667,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
 #pragma unroll
                         for (int kt = 0; kt < 8; ++kt)
                             umma_f16(tmem + TM_U + st * NO,
-                                     smem_desc_sw128(a0 + kt * 2048, 16384, 1024),
+                                     smem_desc_sw128(a0 + kt * 4096, 1024, 2048),
                                      smem_desc_sw128(pb + pbi * PBUF + (kt >> 2) * ATOM + (kt & 3) * 32, 16, 1024),
                                      idU, (i | kt) ? 1u : 0u);
                         umma_arrive(&sh->empty[s]);
@@ -1226,10 +1236,7 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
         dp.n_items = d.batch * pl.n_span;
         dp.qscale = p.qscale;
         dpp = &dp;
-        // the 3D views with 128-row boxes: one copy per 128 x 128 stage
-        if (!make_map_bf16_sw128_cb(&maps[0], Ak, (uint64_t)d.batch * d.ctx_len, d.rank_k, 128, 2) ||
-            !make_map_bf16_sw128_cb(&maps[1], Av, (uint64_t)d.batch * d.ctx_len, d.rank_v, 128, 2))
-            return cudaErrorInvalidValue;
+        dp.rows_all = (int)((int64_t)d.batch * d.ctx_len);
     }
     switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_RA_G(GG) \
