@@ -113,6 +113,7 @@ __device__ __forceinline__ bool ra_wait(uint64_t *b, uint32_t parity, RaShared *
     if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
     if (!*(volatile int *)&sh->abort) {
         *(volatile int *)&sh->abort = 1;
+        grid_dep_wait();    // after q~'s clear of the status word
         if (p.status) atomicOr(p.status, 1u << XKV_ERR_TIMEOUT);
     }
     return false;
@@ -184,8 +185,10 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                 const int ci = gg / gpc, sub = gg % gpc;
                 int64_t c = w.c0 + ci;
                 if (p.sel) c = p.sel[((int64_t)w.b * p.Hkv + w.g) * p.n_sel + c];
-                if (gi < ng && (c < 0 || c >= nC) && p.status)   // the call fails: NaN outputs
+                if (gi < ng && (c < 0 || c >= nC) && p.status) {  // the call fails: NaN outputs
+                    grid_dep_wait();    // after q~'s clear of the status word
                     atomicOr(p.status, 1u << XKV_ERR_INVALID_ARG);
+                }
                 c = min64(max64(c, 0), nC - 1);                   // the copy stays in bounds
                 row = (int)((int64_t)w.b * p.L + c * p.C + sub * 8);
             }
@@ -298,6 +301,8 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                     *reinterpret_cast<const uint4 *>(src);
             }
         };
+        // q~ comes from the kernel before (the copies of A started without waiting for it)
+        grid_dep_wait();
         if (blockIdx.x < p.n_items) write_q(blockIdx.x);
         fence_async_smem();
         ra_epi_bar();
@@ -489,6 +494,7 @@ __device__ __forceinline__ bool dn_wait(uint64_t *b, uint32_t parity, DnShared *
     if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
     if (!*(volatile int *)&sh->abort) {
         *(volatile int *)&sh->abort = 1;
+        grid_dep_wait();    // after q~'s clear of the status word
         if (status) atomicOr(status, 1u << XKV_ERR_TIMEOUT);
     }
     return false;
@@ -529,7 +535,6 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
     unsigned char *pbuf = qbuf + (p.rk / 64) * ATOM;      // two P buffers
     DnShared *sh = reinterpret_cast<DnShared *>(pbuf + 2 * PBUF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t Lp = (int64_t)p.tiles * DN_TILE;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < DN_STAGES; ++s) {
@@ -705,6 +710,8 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                     *reinterpret_cast<const uint4 *>(src);
             }
         };
+        // q~ comes from the kernel before (the copies of A started without waiting for it)
+        grid_dep_wait();
         if (blockIdx.x < p.n_items) write_q(dn_decode(p, blockIdx.x).b);
         fence_async_smem();
         dn_epi_bar();
@@ -716,7 +723,11 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
             float m[HQ];
 #pragma unroll
             for (int h = 0; h < HQ; ++h) m[h] = -INFINITY;
-            float *zrow = p.z + (size_t)w.b * HQ * Lp;
+            // logits of tile (b, t): one contiguous block of HQ x 128 floats, so a tile's
+            // stores and loads stay within a few pages
+            auto zblk = [&](int i) {
+                return p.z + ((size_t)w.b * p.tiles + (size_t)(w.t0 + i)) * HQ * DN_TILE;
+            };
             // pass 1: logits to the scratch, running max
             for (int i = 0; i < w.nt; ++i, ++zt) {
                 const int zb = zt & 1;
@@ -734,12 +745,21 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                 for (int h = 0; h < HQ; ++h) {
                     const float zh = valid ? (v[h] + v[HQ + h]) * p.qscale : -INFINITY;
                     m[h] = fmaxf(m[h], zh);
-                    zrow[(size_t)h * Lp + t] = zh;
+                    zblk(i)[h * DN_TILE + lrow] = zh;
                 }
                 dn_epi_bar();
                 if (et == 0) mbar_arrive(&sh->zfree[zb]);
             }
             if (dead) break;
+            // the first tile's logits are loaded before the max reduction, each later
+            // tile's right after the previous P is published (same thread, program order)
+            float zl[HQ];
+            auto load_z = [&](int i) {
+                const float *zb = zblk(i);
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) zl[h] = __ldcg(zb + h * DN_TILE + lrow);
+            };
+            if (w.nt > 0) load_z(0);
             // the span's max per head
 #pragma unroll
             for (int h = 0; h < HQ; ++h) {
@@ -770,13 +790,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                     const bool fail = !dn_wait(&sh->pfree[pbi], ((pt >> 1) & 1) ^ 1, sh, p.status);
                     if (dn_epi_bar_any(fail)) { dead = true; break; }
                 }
-                const int64_t t = (int64_t)(w.t0 + i) * DN_TILE + lrow;
                 unsigned char *pdst = pbuf + pbi * PBUF;
-                // every logit load in flight before the first shared-memory store (the
-                // stores could otherwise order each load after the previous head's)
-                float zl[HQ];
-#pragma unroll
-                for (int h = 0; h < HQ; ++h) zl[h] = __ldcg(zrow + (size_t)h * Lp + t);
 #pragma unroll
                 for (int h = 0; h < HQ; ++h) {
                     const float pv = exp2f(zl[h] - m[h]);   // 0 past L
@@ -789,6 +803,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                 fence_async_smem();
                 dn_epi_bar();
                 if (et == 0) mbar_arrive(&sh->pfull[pbi]);
+                if (i + 1 < w.nt) load_z(i + 1);
             }
             if (dead) break;
 #pragma unroll
@@ -847,6 +862,9 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
                                                 int Hkv, int hd, int rk,
                                                 unsigned *__restrict__ status) {
     __shared__ float qs[G * 128];                  // [G][hd]
+    // the attention kernel after this one may start streaming the rows of A at once: it
+    // waits for this grid only where it reads q~ or writes the status word
+    grid_dep_launch();
     // the call's device-side error word starts clean: this kernel runs first in the call,
     // so the clear is ordered before every kernel that may set it
     if (status && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *status = 0u;
@@ -996,11 +1014,6 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
     const int g = blockIdx.x, b = blockIdx.y, j0 = blockIdx.z * PJ_ROWS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t bh0 = (size_t)b * Hq + (size_t)g * G;
-    if (status && *(volatile const unsigned *)status) {   // a device-side failure: NaN out
-        for (int e = threadIdx.x; e < G * PJ_ROWS; e += blockDim.x)
-            out[(bh0 + e / PJ_ROWS) * hd + j0 + e % PJ_ROWS] = __int_as_float(0x7fc00000);
-        return;
-    }
     const int c = lane % LPR;
     const int j = j0 + warp * RPW + lane / LPR;
     const __nv_bfloat16 *row = Bvt + ((size_t)b * Hkv * hd + (size_t)g * hd + j) * rv;
@@ -1012,6 +1025,11 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
         const int pc = c + i * LPR;
         pre[i] = pc < rv / 8 ? *reinterpret_cast<const uint4 *>(row + pc * 8)
                              : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (status && *(volatile const unsigned *)status) {   // a device-side failure: NaN out
+        for (int e = threadIdx.x; e < G * PJ_ROWS; e += blockDim.x)
+            out[(bh0 + e / PJ_ROWS) * hd + j0 + e % PJ_ROWS] = __int_as_float(0x7fc00000);
+        return;
     }
     for (int e = threadIdx.x; e < G * rv; e += blockDim.x) Us[e] = U[bh0 * rv + e];
     __syncthreads();
@@ -1081,8 +1099,7 @@ cudaError_t launch_dense_hq(const xkv_dims &d, const CUtensorMap *maps, const Dn
     cudaError_t e = set_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     const int grid = dp.n_items < sm_count() ? dp.n_items : sm_count();
-    k<<<grid, DN_THREADS, smem, s>>>(maps[0], maps[1], dp);
-    return cudaGetLastError();
+    return launch_chained(k, dim3(grid), dim3(DN_THREADS), smem, s, maps[0], maps[1], dp);
 }
 cudaError_t launch_dense(const xkv_dims &d, const CUtensorMap *maps, const DnParams &dp,
                          cudaStream_t s) {
@@ -1122,8 +1139,9 @@ cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams 
         auto k = k_xkv_ra<G>;
         if ((e = set_smem_limit((const void *)k, smem)) != cudaSuccess) return e;
         const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
-        k<<<grid, RA_THREADS, smem, s>>>(maps[0], maps[1], p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_chained(k, dim3(grid), dim3(RA_THREADS), smem, s, maps[0], maps[1], p)) !=
+            cudaSuccess)
+            return e;
     }
     const int BH = d.batch * d.n_q_heads;
     if ((int64_t)BH * ((d.rank_v + 255) / 256) < sm_count())
