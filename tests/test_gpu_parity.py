@@ -441,6 +441,22 @@ DENSE_CASES = [
 ]
 
 
+def test_reassociated_attend_dense_more_items_than_sms(xkv, ora):
+    """160 sequences of 4 tiles: one span per sequence, so 160 items on at most 148 CTAs
+    and some CTAs take a second item (the next item's Q~, the accumulator hand-back and
+    the buffer parities carried across items)."""
+    w = dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=160, ctx_len=512),
+                            rank_k=256, rank_v=384, name="dense_b160")
+    x = _layer_inputs(w)
+    units = [(b, g) for b in (0, 11, 12, 147, 148, 159) for g in (0, w.n_kv_heads - 1)]
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], None, w.chunk,
+                                 units=units)
+    got = _reassoc(xkv, w, x, None)[0]
+    G = w.n_q_heads // w.n_kv_heads
+    for b, g in units:
+        compare_outputs(got[b, g * G:(g + 1) * G], ref[b, g * G:(g + 1) * G], w.dtype)
+
+
 @pytest.mark.parametrize("w", DENSE_CASES, ids=lambda w: w.name)
 def test_reassociated_attend_dense_all_heads(xkv, ora, w):
     x = _layer_inputs(w)
