@@ -47,6 +47,8 @@
 // thread-block cluster per unit (keys gathered in CTA 0 over distributed shared memory);
 // its per-thread row reads missed L1 on every 16-byte load and its 256-thread tail left
 // most of the GPU idle, 58 us per layer against 44 us for the two-call path.
+#include <cstdlib>
+
 #include "sm100_util.cuh"
 #include "xkv_internal.cuh"
 
@@ -82,6 +84,7 @@ struct SsParams {
     int sps;              // stages per key-pass CTA (the last CTA may have fewer)
     int64_t n_stages;     // stages over all units' rows
     int64_t rows_total;   // landmark rows of all units
+    uint32_t spin;        // poll limit of the key pass's pipeline waits
     int Hq, Hkv, hd;
     int top_k, n_sink, n_recent, n_sel;
     const int32_t *reserved;   // [B][Hkv][n_res] chunks forced in as well, or null
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_ss_keys(const SsParams p) {
             int k = 0;
             for (; k < n_st; ++k) {
                 const int slot = k % SK_STAGES, n = k / SK_STAGES;
-                if (!mbar_wait_bounded(&empty[slot], (n & 1) ^ 1, &s_abort, SK_SPIN)) {
+                if (!mbar_wait_bounded(&empty[slot], (n & 1) ^ 1, &s_abort, p.spin)) {
                     *(volatile int *)&s_abort = 1;
                     break;
                 }
@@ -425,7 +428,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_ss_keys(const SsParams p) {
         for (int k = 0; k < n_st; ++k) {
             const int slot = k % SK_STAGES, n = k / SK_STAGES;
             int got = 0;
-            if (lane == 0) got = mbar_wait_bounded(&full[slot], n & 1, &s_abort, SK_SPIN) ? 1 : 0;
+            if (lane == 0) got = mbar_wait_bounded(&full[slot], n & 1, &s_abort, p.spin) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, got, 0)) {
                 if (lane == 0) *(volatile int *)&s_abort = 1;
                 bad = true;
@@ -947,6 +950,14 @@ cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q
     p.n_sel = n_sel;
     p.reserved = reserved;
     p.n_res = reserved ? n_res : 0;
+    // XKV_TEST_SS_SPIN (tests only, read on every call): a shorter poll limit for the key
+    // pass's pipeline waits, so a test can make them give up (the units then take the
+    // exact path); the drain of the copies in flight keeps its full bound
+    p.spin = SK_SPIN;
+    if (const char *e = getenv("XKV_TEST_SS_SPIN")) {
+        const long v = atol(e);
+        if (v > 0 && v < (long)SK_SPIN) p.spin = (uint32_t)v;
+    }
     const double slack = 1.0 + 0x1p-20;
     p.err_rel = (gamma_n(d.head_dim, 0x1p-24) + gamma_n(d.head_dim, 0x1p-53)) * slack;
     p.err_abs = d.head_dim * 0x1p-150 * slack;

@@ -1,8 +1,11 @@
-"""The device-side timeout path of the tensor-core attention kernel, exercised without
-faulting anything: a test-only variable shortens the poll limit of the MMA issuer's waits
-for staged data so that they give up; every other wait (and the drain of the copies and
-MMAs in flight) keeps its full bound.  The call must report XKV_ERR_TIMEOUT in its status
-word and NaN outputs, and the next call, with the normal limit, must be clean."""
+"""The device-side timeout paths, exercised without faulting anything: a test-only variable
+shortens the poll limit of one kernel's pipeline waits so that they give up; every other
+wait (and the drain of the copies and MMAs in flight) keeps its full bound.
+
+* The tensor-core attention kernel must report XKV_ERR_TIMEOUT in its status word and NaN
+  outputs, and the next call, with the normal limit, must be clean.
+* The fused selection's key pass must send the units it covers to the exact fp64 path:
+  the selection stays the oracle's, and the next call takes the fp32 path again."""
 import numpy as np
 import pytest
 import torch
@@ -56,3 +59,29 @@ def test_attention_wait_timeout_is_reported_then_the_next_call_is_clean(xkv, ora
     for b, gg in ((0, 1), (1, 6)):
         G = w.group
         compare_outputs(o[b, gg * G:(gg + 1) * G], ref[b, gg * G:(gg + 1) * G], w.dtype)
+
+
+def test_selection_key_pass_timeout_falls_back_to_the_exact_path(xkv, ora, monkeypatch):
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=8192, top_k=64)
+    x = synth.np_xkv_layer_inputs(w, seed=3, layer=1)
+    lm = ora.to_torch(ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    ref = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    d = xkv.dims_of(w)
+    lm_d, q_d = lm.to(DEV), x["q"].to(DEV)
+    ws = torch.zeros(xkv.xkv_score_select_workspace_bytes(d), dtype=torch.uint8, device=DEV)
+    sel = torch.full((w.batch, w.n_kv_heads, w.n_sel), -7, dtype=torch.int32, device=DEV)
+
+    def call():
+        xkv.xkv_score_select(d, lm_d, q_d, w.top_k, w.n_sink, w.n_recent, sel, ws)
+        torch.cuda.synchronize()
+        band = ws[:4 * w.batch * w.n_kv_heads].cpu().view(torch.int32).numpy().view(np.uint32)
+        return sel.cpu().numpy(), band
+
+    monkeypatch.setenv("XKV_TEST_SS_SPIN", "1")
+    got, band = call()
+    assert np.all(band == 0xFFFFFFFF), band          # every unit on the exact path
+    assert np.array_equal(got, ref)
+    monkeypatch.delenv("XKV_TEST_SS_SPIN")
+    got, band = call()
+    assert np.all(band != 0xFFFFFFFF), band
+    assert np.array_equal(got, ref)
