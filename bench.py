@@ -87,6 +87,24 @@ def measured_tflops_sustained():
 
 
 # --------------------------------------------------------------------------- clocks
+
+def _ra_kernels(w, n_sel):
+    """Kernels of one rank-space attention call, following the library's launch plan: q~,
+    the attention kernel, then the split merge and the projection, as one kernel when a
+    head has 32 or more splits (dense calls at small batch), else as two.  Dense calls
+    here take the head-batched kernel: one span of whole 128-token tiles per SM (148 spans)
+    over the batch; selective calls split each unit's rows into items of <= 256 rows."""
+    if n_sel == 0:
+        tiles = -(-w.ctx_len // 128)
+        ns = max(1, min(148 // w.batch, tiles))
+        tps = -(-tiles // ns)
+        n_split = -(-tiles // tps)
+    else:
+        n_split = -(-(n_sel * w.chunk) // 256)
+        per = -(-n_sel // n_split)
+        n_split = -(-n_sel // per)
+    return 3 if n_split >= 32 else 4
+
 class ClockSampler:
     """This GPU's SM clock and clock-event (throttle) reasons, polled through NVML (the
     source nvidia-smi reads) every ~2 ms on a thread while the timed region runs, so a
@@ -210,12 +228,12 @@ class XkvStep:
         self.out = torch.empty((w.n_layers, w.batch, w.n_q_heads, w.head_dim),
                                dtype=torch.float32, device=dev)
         self.q_in = torch.empty_like(self.qpool[0])   # e2e: per-step queries land here
-        # our kernels per layer: the fused score + select (or score, select), then status
-        # clear + attention + split merge (explicit) or q~ + attention + merge + projection
-        # (reassociated; q~ clears the status word)
-        n_sel_kernels = 0 if self.dense else (1 if scoring == "fused" else 2)
-        self.launches_per_step = w.n_layers * (n_sel_kernels +
-                                               (4 if path == "reassociated" else 3))
+        # our kernels per layer: the fused selection's key and selection grids (or score,
+        # select), then status clear + attention + split merge (explicit) or q~ +
+        # attention + merge-and-projection (reassociated; q~ clears the status word)
+        n_sel_kernels = 0 if self.dense else 2
+        n_attn = _ra_kernels(w, self.n_sel) if path == "reassociated" else 3
+        self.launches_per_step = w.n_layers * (n_sel_kernels + n_attn)
         torch.cuda.synchronize()
 
     def resident_bytes(self):

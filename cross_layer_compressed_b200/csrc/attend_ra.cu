@@ -17,6 +17,8 @@
 //                partials (m, l, u) in rank space
 //   k_merge_ra   merges an item's splits in rank space (U_h, L_h)
 //   k_project_ra o_h = U_h B^V_g / L_h
+// or, for calls with many splits, k_merge_project_ra, which does both, one slice of r_V
+// per CTA.
 // Warp roles of k_xkv_ra: warp 0 TMEM + MMA issue, warps 1-4 TMA producers, warps 5-8
 // epilogue.  A stage holds 128 columns of the item's rows; each 8-row group arrives in
 // one copy of a 3D view of A (64 elements x 8 rows x 2 column blocks) as two consecutive
@@ -432,7 +434,8 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
 //   pass 2, per tile: P[n][t] = exp2(z - m) as hi + lo bf16 rows, then
 //           D_u[r][n] += A^V[t][r] P[n][t]  (M = 128 rank columns per block, N = NO,
 //           K = tokens), accumulated in tensor memory over the whole span;
-//   end:    the span's (m, l, u) partial in rank space, merged across spans by k_merge_ra.
+//   end:    the span's (m, l, u) partial in rank space, merged across spans by k_merge_project_ra
+//           (k_merge_ra and k_project_ra when the spans are few).
 // A stage is 128 tokens x 128 rank columns in 16 copies of the 3D view (64, rows, column
 // blocks) of A, one per 8-row group, each landing as two consecutive 64-column atoms (the
 // layout of k_xkv_ra): logits use A K-major (8-row groups 2 KB apart), the value product
@@ -860,7 +863,8 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
                                                 __nv_bfloat16 *__restrict__ qt_hi,
                                                 __nv_bfloat16 *__restrict__ qt_lo, int Hq,
                                                 int Hkv, int hd, int rk,
-                                                unsigned *__restrict__ status) {
+                                                unsigned *__restrict__ status,
+                                                unsigned *__restrict__ arrived) {
     __shared__ float qs[G * 128];                  // [G][hd]
     // the attention kernel after this one may start streaming the rows of A at once: it
     // waits for this grid only where it reads q~ or writes the status word
@@ -868,6 +872,9 @@ __global__ void __launch_bounds__(256) k_qtilde(const __nv_bfloat16 *__restrict_
     // the call's device-side error word starts clean: this kernel runs first in the call,
     // so the clear is ordered before every kernel that may set it
     if (status && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *status = 0u;
+    // so do the per-(b, h) arrival counters of the merge + projection kernel
+    if ((blockIdx.x | blockIdx.y | blockIdx.z) == 0)
+        for (int e = threadIdx.x; e < Hq * gridDim.y; e += blockDim.x) arrived[e] = 0u;
     constexpr int QT_COLS = 32 * CPL;
     __shared__ float red[8][G][QT_COLS];
     const int g = blockIdx.x, b = blockIdx.y, i0 = blockIdx.z * QT_COLS;
@@ -1059,6 +1066,122 @@ __global__ void __launch_bounds__(256) k_project_ra(const float *__restrict__ U,
     }
 }
 
+// Merge of an item's splits in rank space fused with the projection, for calls with many
+// splits (dense calls at small batch: one span per SM, so ~148 / B splits per head).  For
+// a query head h of group g and a slice of W = 32 CPL rank columns r:
+//   M = max_s m_s,  w_s = e^{m_s - M},  L = sum_s w_s l_s,  U[r] = sum_s w_s u_s[r],
+//   y[j] = sum_{r in the slice} U[r] B^V[g*hd + j][r],
+// and the CTA of h that finishes last sums y over the slices in slice order and writes
+// o_h[j] = y[j] / L.  Every CTA of a head forms M and L from all splits in the same
+// order, so they agree bit for bit, and the order of the final sum does not depend on
+// which CTA is last: the output is reproducible.  The CTA's rows of B^V (128 rows x W
+// columns, two threads per row) are loaded first, since they do not depend on the merge.
+// Warp w takes the splits s = w, w + 8, ..., each lane CPL columns (coalesced 128-byte
+// rows).  The arrival counters are zeroed by k_qtilde, which runs first in every call.
+// Each head re-reads its group's B^V slice (from L2), so with few splits the two
+// separate kernels above, which read it once per group, are faster; the host takes this
+// kernel from MP_MIN_SPLITS splits on.
+constexpr int MP_THREADS = 256;
+constexpr int MP_HD = 128;
+constexpr int MP_MIN_CTAS = 296;   // about two CTAs per SM: the widest slices that keep this
+constexpr int MP_MIN_SPLITS = 32;
+template <int CPL>
+__global__ void __launch_bounds__(MP_THREADS) k_merge_project_ra(
+    const float *__restrict__ partials, const __nv_bfloat16 *__restrict__ Bvt,
+    float *__restrict__ yparts, unsigned *__restrict__ arrived, float *__restrict__ out,
+    int n_split, int BH, int Hq, int Hkv, int rv, const unsigned *__restrict__ status) {
+    constexpr int W = 32 * CPL, NW = MP_THREADS / 32, HALF = W / 2, NV = HALF / 8;
+    static_assert(MP_THREADS == 2 * MP_HD, "two threads per row of the B^V slice");
+    __shared__ float red[NW][W];
+    __shared__ float Us[W];
+    __shared__ float s_m[NW], s_l[NW];
+    __shared__ int s_last;
+    const int bh = blockIdx.x, sl = blockIdx.y, n_sl = gridDim.y, r0 = sl * W;
+    const int G = Hq / Hkv;
+    const int b = bh / Hq, g = (bh % Hq) / G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const uint4 *brow = reinterpret_cast<const uint4 *>(
+        Bvt + ((size_t)b * Hkv * MP_HD + (size_t)g * MP_HD + j) * rv + r0 + half * HALF);
+    uint4 bw[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) bw[i] = brow[i];
+    if (status && *(volatile const unsigned *)status) {
+        if (sl == 0 && threadIdx.x < MP_HD) out[(size_t)bh * MP_HD + threadIdx.x] = __int_as_float(0x7fc00000);
+        return;
+    }
+    const size_t stride = (size_t)BH * (rv + 2);
+    const float *p = partials + (size_t)bh * (rv + 2);
+    float M = -INFINITY;
+    for (int sp = threadIdx.x; sp < n_split; sp += MP_THREADS) M = fmaxf(M, p[sp * stride]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) s_m[warp] = M;
+    __syncthreads();
+    M = s_m[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) M = fmaxf(M, s_m[w]);
+    float acc[CPL], l = 0.f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
+#pragma unroll 8
+    for (int sp = warp; sp < n_split; sp += NW) {
+        const float *ps = p + sp * stride;
+        const float wgt = expf(ps[0] - M);
+        l = fmaf(wgt, ps[1], l);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) acc[k] = fmaf(wgt, ps[2 + r0 + lane + 32 * k], acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) red[warp][lane + 32 * k] = acc[k];
+    if (lane == 0) s_l[warp] = l;
+    __syncthreads();
+    if (threadIdx.x < W) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) sum += red[w][threadIdx.x];
+        Us[threadIdx.x] = sum;
+    }
+    __syncthreads();
+    float y = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const float bv[8] = {bf16lo(bw[i].x), bf16hi(bw[i].x), bf16lo(bw[i].y), bf16hi(bw[i].y),
+                             bf16lo(bw[i].z), bf16hi(bw[i].z), bf16lo(bw[i].w), bf16hi(bw[i].w)};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y = fmaf(Us[half * HALF + i * 8 + k], bv[k], y);
+    }
+    y += __shfl_xor_sync(0xffffffffu, y, 1);
+    if (half == 0) yparts[((size_t)bh * n_sl + sl) * MP_HD + j] = y;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&arrived[bh], 1u) == (unsigned)(n_sl - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (threadIdx.x < MP_HD) {
+        const float *yu = yparts + (size_t)bh * n_sl * MP_HD + threadIdx.x;
+        float sum = 0.f;
+        for (int t0 = 0; t0 < n_sl; t0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = t0 + i < n_sl ? __ldcg(yu + (size_t)(t0 + i) * MP_HD) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (t0 + i < n_sl) sum += v[i];
+        }
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) L += s_l[w];
+        out[(size_t)bh * MP_HD + threadIdx.x] = sum / L;
+    }
+}
+int mp_cpl(const xkv_dims &d) {
+    const int64_t bh = (int64_t)d.batch * d.n_q_heads;
+    for (int c = 4; c > 1; c /= 2)
+        if (bh * (d.rank_v / (32 * c)) >= MP_MIN_CTAS) return c;
+    return 1;
+}
 // Dense-mode plan: spans of whole 128-token tiles, about one span per SM over the batch.
 struct DnPlan {
     int tiles, tps, n_span;
@@ -1115,18 +1238,18 @@ cudaError_t launch_dense(const xkv_dims &d, const CUtensorMap *maps, const DnPar
 template <int G>
 cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams &p,
                      const DnParams *dp, const void *q, const void *Bkt, const void *Bvt,
-                     __nv_bfloat16 *qt_hi, __nv_bfloat16 *qt_lo, float *U, float *Lsum,
-                     float *out, cudaStream_t s) {
+                     __nv_bfloat16 *qt_hi, __nv_bfloat16 *qt_lo, float *yparts,
+                     unsigned *arrived, float *out, cudaStream_t s) {
     // narrow slices only where the wide ones leave SMs without a CTA
     const bool few = (int64_t)d.batch * d.n_kv_heads * (d.rank_k / 128) < sm_count();
     if (few)
         k_qtilde<G, 1><<<dim3(d.n_kv_heads, d.batch, d.rank_k / 32), 256, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
-            d.n_kv_heads, d.head_dim, d.rank_k, p.status);
+            d.n_kv_heads, d.head_dim, d.rank_k, p.status, arrived);
     else
         k_qtilde<G, 4><<<dim3(d.n_kv_heads, d.batch, d.rank_k / 128), 256, 0, s>>>(
             (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Bkt, qt_hi, qt_lo, d.n_q_heads,
-            d.n_kv_heads, d.head_dim, d.rank_k, p.status);
+            d.n_kv_heads, d.head_dim, d.rank_k, p.status, arrived);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int n_split = p.n_split;
@@ -1144,6 +1267,24 @@ cudaError_t launch_g(const xkv_dims &d, const CUtensorMap *maps, const RaParams 
             return e;
     }
     const int BH = d.batch * d.n_q_heads;
+    if (n_split >= MP_MIN_SPLITS) {
+        const dim3 mgrid(BH, d.rank_v / (32 * mp_cpl(d)));
+        switch (mp_cpl(d)) {
+#define XKV_MP(C)                                                                              \
+    case C:                                                                                    \
+        k_merge_project_ra<C><<<mgrid, MP_THREADS, 0, s>>>(p.partials, (const __nv_bfloat16 *)Bvt, \
+                                                           yparts, arrived, out, n_split, BH,  \
+                                                           d.n_q_heads, d.n_kv_heads, d.rank_v, \
+                                                           p.status);                          \
+        break;
+            XKV_MP(1) XKV_MP(2) XKV_MP(4)
+#undef XKV_MP
+            default: return cudaErrorInvalidValue;
+        }
+        return cudaGetLastError();
+    }
+    // few splits: merge, then project (U and L take the y and counter regions)
+    float *U = yparts, *Lsum = (float *)arrived;
     if ((int64_t)BH * ((d.rank_v + 255) / 256) < sm_count())
         k_merge_ra<2><<<dim3(BH, (d.rank_v + 63) / 64), MG_THREADS, 0, s>>>(
             p.partials, U, Lsum, n_split, BH, d.rank_v, p.status);
@@ -1177,13 +1318,22 @@ int ra_splits(const xkv_dims &d, int n_sel) {
     return (int)((rows + RA_ROWS - 1) / RA_ROWS);
 }
 
-// scratch: q~ hi and lo [B][Hq][r_K] bf16, U [B][Hq][r_V] and L [B][Hq] fp32, then the
-// partials [n_split][B][Hq][r_V + 2] fp32; each region starts on a 256-byte boundary
+// scratch: q~ hi and lo [B][Hq][r_K] bf16, the projected slices y [B][Hq][r_V / W][hd]
+// fp32 (W the merge + projection kernel's slice width; with few splits U [B][Hq][r_V]
+// instead, which fits), the arrival counters (or L) [B][Hq] 32-bit, then the partials
+// [n_split][B][Hq][r_V + 2] fp32; each region starts on a 256-byte boundary
 static size_t al256(size_t n) { return (n + 255) / 256 * 256; }
+static size_t y_bytes(const xkv_dims &d) {
+    return al256((size_t)d.batch * d.n_q_heads * (d.rank_v / (32 * mp_cpl(d))) * MP_HD *
+                 sizeof(float));
+}
+static size_t arrived_bytes(const xkv_dims &d) {
+    return al256((size_t)d.batch * d.n_q_heads * sizeof(unsigned));
+}
 size_t ra_scratch_bytes(const xkv_dims &d, int n_split) {
     const size_t bh = (size_t)d.batch * d.n_q_heads;
-    return 2 * al256(bh * d.rank_k * sizeof(__nv_bfloat16)) + al256(bh * d.rank_v * sizeof(float)) +
-           al256(bh * sizeof(float)) + (size_t)n_split * bh * (d.rank_v + 2) * sizeof(float);
+    return 2 * al256(bh * d.rank_k * sizeof(__nv_bfloat16)) + y_bytes(d) + arrived_bytes(d) +
+           (size_t)n_split * bh * (d.rank_v + 2) * sizeof(float);
 }
 
 // Dense calls with a supported head count run the head-batched kernel: partials per span,
@@ -1209,17 +1359,16 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
         return cudaErrorInvalidValue;
     const size_t bh = (size_t)d.batch * d.n_q_heads;
     const size_t qt_al = al256(bh * d.rank_k * sizeof(__nv_bfloat16));
-    const size_t u_al = al256(bh * d.rank_v * sizeof(float));
     char *sc = (char *)scratch;
     __nv_bfloat16 *qt_hi = (__nv_bfloat16 *)sc;
     __nv_bfloat16 *qt_lo = (__nv_bfloat16 *)(sc + qt_al);
-    float *U = (float *)(sc + 2 * qt_al);
-    float *Lsum = (float *)(sc + 2 * qt_al + u_al);
+    float *yparts = (float *)(sc + 2 * qt_al);
+    unsigned *arrived = (unsigned *)(sc + 2 * qt_al + y_bytes(d));
     RaParams p;
     p.qt_hi = qt_hi;
     p.qt_lo = qt_lo;
     p.sel = sel;
-    p.partials = (float *)(sc + 2 * qt_al + u_al + al256(bh * sizeof(float)));
+    p.partials = (float *)(sc + 2 * qt_al + y_bytes(d) + arrived_bytes(d));
     p.status = status;
     p.L = d.ctx_len;
     p.n_sel = n_sel;
@@ -1258,7 +1407,7 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
     }
     switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_RA_G(GG) \
-    case GG: return launch_g<GG>(d, maps, p, dpp, q, Bkt, Bvt, qt_hi, qt_lo, U, Lsum, out, s);
+    case GG: return launch_g<GG>(d, maps, p, dpp, q, Bkt, Bvt, qt_hi, qt_lo, yparts, arrived, out, s);
         XKV_RA_G(1) XKV_RA_G(2) XKV_RA_G(4) XKV_RA_G(5) XKV_RA_G(8)
 #undef XKV_RA_G
         default: return cudaErrorInvalidValue;

@@ -438,6 +438,12 @@ DENSE_CASES = [
                         n_q_heads=8, n_kv_heads=8, rank_k=256, rank_v=384, name="dense_hq8_g1"),
     dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=2048),
                         n_q_heads=24, n_kv_heads=6, rank_k=384, rank_v=640, name="dense_hq24"),
+    # 32 or more spans per sequence: the merge and the projection run as one kernel
+    # (slices of 32 and of 128 rank columns, one and four heads per group)
+    dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=8192),
+                        n_q_heads=8, n_kv_heads=8, rank_k=256, rank_v=384,
+                        name="dense_hq8_many_spans"),
+    synth.reduced(synth.LLAMA8B_DENSE_128K, batch=2, ctx_len=16384, name="dense_b2_many_spans"),
 ]
 
 
@@ -460,7 +466,7 @@ def test_reassociated_attend_dense_more_items_than_sms(xkv, ora):
 @pytest.mark.parametrize("w", DENSE_CASES, ids=lambda w: w.name)
 def test_reassociated_attend_dense_all_heads(xkv, ora, w):
     x = _layer_inputs(w)
-    units = None if w.ctx_len <= 4096 else [(0, 0), (0, w.n_kv_heads - 1)]
+    units = None if w.ctx_len <= 4096 else [(0, 0), (w.batch - 1, w.n_kv_heads - 1)]
     ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], None, w.chunk,
                                  units=units)
     got = _reassoc(xkv, w, x, None)[0]
