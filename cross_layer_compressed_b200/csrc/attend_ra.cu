@@ -28,6 +28,8 @@
 // 8-row groups 2 KB apart, the two column blocks 1 KB apart.  Every mbarrier wait is bounded; on
 // expiry the CTA sets XKV_ERR_TIMEOUT in the workspace status word, drains its copies
 // and MMAs (bounded), frees TMEM and returns, and the combine writes NaN outputs.
+#include <cstdlib>
+
 #include "sm100_util.cuh"
 
 namespace xkv {
@@ -69,6 +71,7 @@ struct RaParams {
     int n_sel, C, rk, rv, Hq, Hkv, B;
     int chunks_per_item, n_split, n_items;
     float qscale;                         // log2(e) / sqrt(hd)
+    uint32_t mma_spin;                    // poll limit of the MMA issuer's waits for staged data
 };
 
 struct RaItem {
@@ -111,8 +114,8 @@ __device__ __forceinline__ bool ra_epi_bar_any(bool flag) {
     return r != 0;
 }
 __device__ __forceinline__ bool ra_wait(uint64_t *b, uint32_t parity, RaShared *sh,
-                                        const RaParams &p) {
-    if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
+                                        const RaParams &p, uint32_t limit = RA_SPIN) {
+    if (mbar_wait_bounded(b, parity, &sh->abort, limit)) return true;
     if (!*(volatile int *)&sh->abort) {
         *(volatile int *)&sh->abort = 1;
         grid_dep_wait();    // after q~'s clear of the status word
@@ -214,9 +217,12 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
             }
         }
         if (!ok && pi == 0 && lane == 0) {
-            for (int s = 0; s < RA_STAGES; ++s)
+            // Every stage the four warps issued lands before the CTA may leave: the last
+            // RA_STAGES fills (each issued whole: a warp checks for abort only in its wait
+            // on `empty`, which completes for all four warps alike) complete their phase.
+            for (int j = it - RA_STAGES > 0 ? it - RA_STAGES : 0; j < it; ++j)
                 for (uint32_t i = 0; i < RA_SPIN; ++i)
-                    if (mbar_test(&sh->full[s], 0) || mbar_test(&sh->full[s], 1)) break;
+                    if (mbar_test(&sh->full[j % RA_STAGES], (uint32_t)(j / RA_STAGES) & 1)) break;
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                 const int nsk = p.rk / 128;
                 for (int st = 0; st < nsk && ok; ++st, ++it) {
                     const int s = it % RA_STAGES, n = it / RA_STAGES;
-                    if (!ra_wait(&sh->full[s], n & 1, sh, p)) { ok = false; break; }
+                    if (!ra_wait(&sh->full[s], n & 1, sh, p, p.mma_spin)) { ok = false; break; }
                     tcgen05_after();
                     const uint32_t a0 = sbase + s * RA_STAGE;
 #pragma unroll
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(RA_THREADS, 1)
                 const int nsv = p.rv / 128;
                 for (int st = 0; st < nsv && ok; ++st, ++it) {
                     const int s = it % RA_STAGES, n = it / RA_STAGES;
-                    if (!ra_wait(&sh->full[s], n & 1, sh, p)) { ok = false; break; }
+                    if (!ra_wait(&sh->full[s], n & 1, sh, p, p.mma_spin)) { ok = false; break; }
                     tcgen05_after();
                     const uint32_t a0 = sbase + s * RA_STAGE;
                     for (int kt = 0; kt < nk16; ++kt) {
@@ -469,6 +475,7 @@ struct DnParams {
     int rows_all;                         // B * L: rows of the 3D views
     int tiles, tps, n_span, n_items;
     float qscale;                         // log2(e) / sqrt(hd)
+    uint32_t mma_spin;                    // poll limit of the MMA issuer's waits for staged data
 };
 
 template <int HQ> struct DnCfg {
@@ -493,8 +500,8 @@ __device__ __forceinline__ bool dn_epi_bar_any(bool flag) {
     return r != 0;
 }
 __device__ __forceinline__ bool dn_wait(uint64_t *b, uint32_t parity, DnShared *sh,
-                                        unsigned *status) {
-    if (mbar_wait_bounded(b, parity, &sh->abort, RA_SPIN)) return true;
+                                        unsigned *status, uint32_t limit = RA_SPIN) {
+    if (mbar_wait_bounded(b, parity, &sh->abort, limit)) return true;
     if (!*(volatile int *)&sh->abort) {
         *(volatile int *)&sh->abort = 1;
         grid_dep_wait();    // after q~'s clear of the status word
@@ -635,7 +642,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                     tcgen05_after();
                     for (int st = 0; st < p.rk / 128; ++st, ++it) {
                         const int s = it % DN_STAGES, n = it / DN_STAGES;
-                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status)) {
+                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status, p.mma_spin)) {
                             ok = false;
                             break;
                         }
@@ -666,7 +673,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
                     tcgen05_after();
                     for (int st = 0; st < p.rv / 128; ++st, ++it) {
                         const int s = it % DN_STAGES, n = it / DN_STAGES;
-                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status)) {
+                        if (!dn_wait(&sh->full[s], n & 1, sh, p.status, p.mma_spin)) {
                             ok = false;
                             break;
                         }
@@ -1383,6 +1390,14 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
     p.n_split = (n_sel + p.chunks_per_item - 1) / p.chunks_per_item;
     p.n_items = d.batch * d.n_kv_heads * p.n_split;
     p.qscale = 1.4426950408889634f / sqrtf((float)d.head_dim);
+    // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the MMA
+    // issuer's waits on staged data, so a test can make them give up; every other wait,
+    // and the drain that follows, keeps its full bound
+    p.mma_spin = RA_SPIN;
+    if (const char *e = getenv("XKV_TEST_MMA_SPIN")) {
+        const long v = atol(e);
+        if (v > 0 && v < (long)RA_SPIN) p.mma_spin = (uint32_t)v;
+    }
     DnParams dp;
     const DnParams *dpp = nullptr;
     if (!sel && attend_ra_dense_heads(d)) {
@@ -1402,6 +1417,7 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
         dp.n_span = pl.n_span;
         dp.n_items = d.batch * pl.n_span;
         dp.qscale = p.qscale;
+        dp.mma_spin = p.mma_spin;
         dpp = &dp;
         dp.rows_all = (int)((int64_t)d.batch * d.ctx_len);
     }

@@ -2,10 +2,13 @@
 shortens the poll limit of one kernel's pipeline waits so that they give up; every other
 wait (and the drain of the copies and MMAs in flight) keeps its full bound.
 
-* The tensor-core attention kernel must report XKV_ERR_TIMEOUT in its status word and NaN
-  outputs, and the next call, with the normal limit, must be clean.
+* The tensor-core attention kernels (explicit, rank-space selective, rank-space dense)
+  must report XKV_ERR_TIMEOUT in the status word and NaN outputs, and the next call, with
+  the normal limit, must be clean.
 * The fused selection's key pass must send the units it covers to the exact fp64 path:
   the selection stays the oracle's, and the next call takes the fp32 path again."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -85,3 +88,54 @@ def test_selection_key_pass_timeout_falls_back_to_the_exact_path(xkv, ora, monke
     got, band = call()
     assert np.all(band != 0xFFFFFFFF), band
     assert np.array_equal(got, ref)
+
+
+def _rank_space_timeout_then_clean(xkv, ora, monkeypatch, w, sel, units):
+    x = synth.np_xkv_layer_inputs(w, seed=7, layer=0)
+    g = {k: x[k].to(DEV) for k in ("Ak", "Av", "Bkt", "Bvt", "q")}
+    d = xkv.dims_of(w)
+    n_sel = 0 if sel is None else sel.shape[2]
+    sel_d = None if sel is None else torch.from_numpy(sel).to(DEV)
+    ws = torch.zeros(xkv.xkv_workspace_bytes(d, n_sel, xkv.XKV_MODE_REASSOC), dtype=torch.uint8,
+                     device=DEV)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+
+    def call():
+        xkv.xkv_reassociated_attend(d, g["Ak"], g["Av"], g["Bkt"], g["Bvt"], g["q"], sel_d, n_sel,
+                                    out, ws)
+        torch.cuda.synchronize()
+        return int(ws[:4].cpu().view(torch.int32).item()), out.cpu().numpy()
+
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "1")
+    status, o = call()
+    assert status & (1 << xkv.XKV_ERR_TIMEOUT), status
+    assert np.all(np.isnan(o))
+    monkeypatch.delenv("XKV_TEST_MMA_SPIN")
+    status, o = call()
+    assert status == 0
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk,
+                                 units=units)
+    G = w.group
+    for b, gg in units:
+        compare_outputs(o[b, gg * G:(gg + 1) * G], ref[b, gg * G:(gg + 1) * G], w.dtype)
+
+
+def test_rank_space_selective_wait_timeout_is_reported_then_the_next_call_is_clean(
+        xkv, ora, monkeypatch):
+    """Selective rank-space kernel: the split merge and projection kernels see the status
+    word and write NaN."""
+    w = synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=4096, top_k=60, n_needles=0)
+    rng = np.random.default_rng(11)
+    sel = np.stack([np.sort(rng.choice(w.n_chunks, w.n_sel, replace=False))
+                    for _ in range(w.batch * w.n_kv_heads)]).reshape(
+        w.batch, w.n_kv_heads, w.n_sel).astype(np.int32)
+    _rank_space_timeout_then_clean(xkv, ora, monkeypatch, w, sel, [(0, 2), (1, 7)])
+
+
+def test_rank_space_dense_wait_timeout_is_reported_then_the_next_call_is_clean(
+        xkv, ora, monkeypatch):
+    """Head-batched dense kernel with 64 spans per sequence, so the merge + projection
+    kernel is the one that turns the status word into NaN outputs."""
+    w = dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=8192),
+                            n_q_heads=8, n_kv_heads=8, rank_k=256, rank_v=384, name="dense_g1")
+    _rank_space_timeout_then_clean(xkv, ora, monkeypatch, w, None, [(0, 0), (0, 5)])
