@@ -149,12 +149,11 @@ SplitPlan plan_rcla(const xkv_dims &d, int64_t rows) {
 
 void xkv::set_last_error(const char *msg) { g_last_error = msg; }
 
-// The switches are read once, on first use, and hold for the life of the process.
+// The switches are read on every call (a host-side lookup; no workspace size depends on
+// them), so a process can change them between calls.
 bool xkv::env_flag(EnvFlag f) {
-    static const bool flags[3] = {getenv("XKV_FORCE_SIMT") != nullptr,
-                                  getenv("XKV_NO_TC") != nullptr,
-                                  getenv("XKV_NO_PDL") != nullptr};
-    return flags[(int)f];
+    static const char *const names[3] = {"XKV_FORCE_SIMT", "XKV_NO_TC", "XKV_NO_PDL"};
+    return getenv(names[(int)f]) != nullptr;
 }
 
 extern "C" {

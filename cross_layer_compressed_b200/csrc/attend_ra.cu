@@ -28,8 +28,6 @@
 // 8-row groups 2 KB apart, the two column blocks 1 KB apart.  Every mbarrier wait is bounded; on
 // expiry the CTA sets XKV_ERR_TIMEOUT in the workspace status word, drains its copies
 // and MMAs (bounded), frees TMEM and returns, and the combine writes NaN outputs.
-#include <cstdlib>
-
 #include "sm100_util.cuh"
 
 namespace xkv {
@@ -1393,11 +1391,7 @@ cudaError_t launch_attend_ra(const xkv_dims &d, const void *Ak, const void *Av, 
     // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the MMA
     // issuer's waits on staged data, so a test can make them give up; every other wait,
     // and the drain that follows, keeps its full bound
-    p.mma_spin = RA_SPIN;
-    if (const char *e = getenv("XKV_TEST_MMA_SPIN")) {
-        const long v = atol(e);
-        if (v > 0 && v < (long)RA_SPIN) p.mma_spin = (uint32_t)v;
-    }
+    p.mma_spin = test_poll_limit("XKV_TEST_MMA_SPIN", RA_SPIN);
     DnParams dp;
     const DnParams *dpp = nullptr;
     if (!sel && attend_ra_dense_heads(d)) {

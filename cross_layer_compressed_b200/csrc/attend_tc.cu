@@ -35,8 +35,6 @@
 // Every wait on an mbarrier is bounded; on expiry the CTA records XKV_ERR_TIMEOUT in the
 // workspace status word, drains its own copies and MMAs (again bounded), frees TMEM and
 // returns; the combine kernel then writes NaN outputs.
-#include <cstdlib>
-
 #include "sm100_util.cuh"
 
 namespace xkv {
@@ -509,11 +507,7 @@ cudaError_t launch_attend_tc(const xkv_dims &d, const void *Ak, const void *Av, 
     // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the MMA
     // issuer's waits on staged data, so a test can make them give up; every other wait,
     // and the drain that follows, keeps its full bound
-    p.mma_spin = SPIN_LIMIT;
-    if (const char *e = getenv("XKV_TEST_MMA_SPIN")) {
-        const long v = atol(e);
-        if (v > 0 && v < (long)SPIN_LIMIT) p.mma_spin = (uint32_t)v;
-    }
+    p.mma_spin = test_poll_limit("XKV_TEST_MMA_SPIN", SPIN_LIMIT);
     *n_split_out = p.n_split;
     switch (d.n_q_heads / d.n_kv_heads) {
 #define XKV_G(GG) \

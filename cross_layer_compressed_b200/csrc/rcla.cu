@@ -13,8 +13,6 @@
 // The leader's update: when `update_row` >= 0, the CTAs of split 0 copy k_new / v_new
 // into that row of the cache, and every CTA reads that row from k_new / v_new (never
 // from the cache), so no CTA depends on another's write.
-#include <cstdlib>
-
 #include "sm100_util.cuh"
 
 namespace xkv {
@@ -201,6 +199,7 @@ struct RclaParams {
     int64_t L_max, n_rows, update_row;
     int rows_per_split, n_split, n_items;
     float qscale;                                // log2(e) / sqrt(hd)
+    uint32_t stage_spin;                         // poll limit of the waits for staged data
 };
 
 template <int G>
@@ -259,7 +258,7 @@ __global__ void __launch_bounds__(R3_THREADS, 1)
     auto wait_stage = [&](int &st) -> bool {   // CTA-uniform outcome
         st = n_used % R3_STAGES;
         const bool got = mbar_wait_bounded(&full[st], (uint32_t)((n_used / R3_STAGES) & 1),
-                                           &s_abort, R3_SPIN);
+                                           &s_abort, p.stage_spin);
         if (!got) s_abort = 1;
         return !__syncthreads_or(!got);
     };
@@ -435,10 +434,10 @@ __global__ void __launch_bounds__(R3_THREADS, 1)
                 p.partials[(((size_t)split * p.B + b) * p.Hq + (size_t)g * G + t) * 130] =
                     __int_as_float(0x7fc00000);
         }
-        if (t == 0) {
-            for (int st = 0; st < R3_STAGES; ++st)
+        if (t == 0) {   // the last R3_STAGES loads issued complete their phase
+            for (int j = n_loaded - R3_STAGES > 0 ? n_loaded - R3_STAGES : 0; j < n_loaded; ++j)
                 for (uint32_t k = 0; k < R3_SPIN; ++k)
-                    if (mbar_test(&full[st], 0) || mbar_test(&full[st], 1)) break;
+                    if (mbar_test(&full[j % R3_STAGES], (uint32_t)(j / R3_STAGES) & 1)) break;
         }
     }
 }
@@ -471,6 +470,9 @@ cudaError_t launch_rcla_tma_g(const xkv_dims &d, int slot, int64_t L_max, int64_
     p.n_split = plan.n_split;
     p.n_items = d.batch * d.n_kv_heads * plan.n_split;
     p.qscale = 1.4426950408889634f / sqrtf(128.f);
+    // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the
+    // waits on staged data, so a test can make them give up; the drain keeps its bound
+    p.stage_spin = test_poll_limit("XKV_TEST_MMA_SPIN", R3_SPIN);
     const size_t smem = 1024 + (size_t)R3_STAGES * R3_TILE +
                         sizeof(float) * (128 * G + (size_t)plan.rows_per_split * G + 4 * G * 128) +
                         R3_STAGES * sizeof(uint64_t);

@@ -65,6 +65,7 @@ struct RtParams {
     int64_t L_max, n_rows, update_row;
     int rows_per_split, n_split, n_items;
     float qscale;                              // log2(e) / sqrt(hd)
+    uint32_t mma_spin;                         // poll limit of the MMA warp's waits for staged data
 };
 
 struct RtItem {
@@ -107,16 +108,17 @@ __device__ __forceinline__ bool rt_epi_bar_any(bool flag) {
         : "memory");
     return r != 0;
 }
-__device__ __forceinline__ bool rt_wait(uint64_t *b, uint32_t parity, RtShared *sh) {
-    const bool ok = mbar_wait_bounded(b, parity, &sh->abort, RT_SPIN);
+__device__ __forceinline__ bool rt_wait(uint64_t *b, uint32_t parity, RtShared *sh,
+                                        uint32_t limit = RT_SPIN) {
+    const bool ok = mbar_wait_bounded(b, parity, &sh->abort, limit);
     if (!ok) *(volatile int *)&sh->abort = 1;
     return ok;
 }
 // warp-uniform bounded wait: lane 0 polls
 __device__ __forceinline__ bool rt_warp_wait(uint64_t *b, uint32_t parity, RtShared *sh,
-                                             int lane) {
+                                             int lane, uint32_t limit = RT_SPIN) {
     int got = 0;
-    if (lane == 0) got = rt_wait(b, parity, sh) ? 1 : 0;
+    if (lane == 0) got = rt_wait(b, parity, sh, limit) ? 1 : 0;
     return __shfl_sync(0xffffffffu, got, 0) != 0;
 }
 
@@ -204,10 +206,11 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                     }
                 }
             }
-            if (!ok) {                              // let this CTA's copies land
-                for (int s = 0; s < S; ++s)
+            if (!ok) {
+                // let this CTA's copies land: the last S fills issued complete their phase
+                for (int j = it - S > 0 ? it - S : 0; j < it; ++j)
                     for (uint32_t i = 0; i < RT_SPIN; ++i)
-                        if (mbar_test(&sh->full[s], 0) || mbar_test(&sh->full[s], 1)) break;
+                        if (mbar_test(&sh->full[j % S], (uint32_t)(j / S) & 1)) break;
             }
         }
         __syncwarp();
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 tcgen05_after();
                 for (int t = 0; t < w.tiles && ok; ++t, ++it) {
                     const int s = it % S, n = it / S;
-                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
+                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane, p.mma_spin)) { ok = false; break; }
                     tcgen05_after();
                     const int64_t nl = new_local - (int64_t)t * RT_ROWS;
                     if (nl >= 0 && nl < RT_ROWS)
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 tcgen05_after();
                 for (int t = 0; t < w.tiles && ok; ++t, ++it) {
                     const int s = it % S, n = it / S;
-                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane)) { ok = false; break; }
+                    if (!rt_warp_wait(&sh->full[s], n & 1, sh, lane, p.mma_spin)) { ok = false; break; }
                     tcgen05_after();
                     const int rows = min(RT_ROWS, w.nr - t * RT_ROWS);
                     const int nks = (rows + 15) / 16;
@@ -504,6 +507,10 @@ cudaError_t launch_rcla_tc(const xkv_dims &d, int slot, int64_t L_max, int64_t n
     p.n_split = plan.n_split;
     p.n_items = d.batch * d.n_kv_heads * plan.n_split;
     p.qscale = 1.4426950408889634f / sqrtf((float)RT_HD);
+    // XKV_TEST_MMA_SPIN (tests only, read on every call): a shorter poll limit for the MMA
+    // warp's waits on staged data, so a test can make them give up; every other wait, and
+    // the drain that follows, keeps its full bound
+    p.mma_spin = test_poll_limit("XKV_TEST_MMA_SPIN", RT_SPIN);
     switch (d.n_q_heads / d.n_kv_heads) {
         case 1: return launch_g<1>(tm, p, s);
         case 2: return launch_g<2>(tm, p, s);

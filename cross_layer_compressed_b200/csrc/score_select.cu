@@ -47,8 +47,6 @@
 // thread-block cluster per unit (keys gathered in CTA 0 over distributed shared memory);
 // its per-thread row reads missed L1 on every 16-byte load and its 256-thread tail left
 // most of the GPU idle, 58 us per layer against 44 us for the two-call path.
-#include <cstdlib>
-
 #include "sm100_util.cuh"
 #include "xkv_internal.cuh"
 
@@ -953,11 +951,7 @@ cudaError_t launch_score_select(const xkv_dims &d, const void *lm, const void *q
     // XKV_TEST_SS_SPIN (tests only, read on every call): a shorter poll limit for the key
     // pass's pipeline waits, so a test can make them give up (the units then take the
     // exact path); the drain of the copies in flight keeps its full bound
-    p.spin = SK_SPIN;
-    if (const char *e = getenv("XKV_TEST_SS_SPIN")) {
-        const long v = atol(e);
-        if (v > 0 && v < (long)SK_SPIN) p.spin = (uint32_t)v;
-    }
+    p.spin = test_poll_limit("XKV_TEST_SS_SPIN", SK_SPIN);
     const double slack = 1.0 + 0x1p-20;
     p.err_rel = (gamma_n(d.head_dim, 0x1p-24) + gamma_n(d.head_dim, 0x1p-53)) * slack;
     p.err_abs = d.head_dim * 0x1p-150 * slack;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+
 #include "xkv.h"
 
 namespace xkv {
@@ -163,6 +165,17 @@ void set_last_error(const char *msg);
 // CUDA-core R-CLA kernel, XKV_NO_PDL plain stream order for every launch.
 enum EnvFlag { ENV_FORCE_SIMT = 0, ENV_NO_TC = 1, ENV_NO_PDL = 2 };
 bool env_flag(EnvFlag f);
+// A test-only poll limit read from the environment on every call: the variable's value
+// when it is a whole decimal number in [0, full), else `full`.  A limit of 0 makes the
+// waits it governs give up without polling (mbarrier try_wait may itself suspend for a
+// while, so even a limit of 1 can succeed when the data is already close).
+inline uint32_t test_poll_limit(const char *name, uint32_t full) {
+    const char *e = getenv(name);
+    if (!e || !*e) return full;
+    char *end = nullptr;
+    const long v = strtol(e, &end, 10);
+    return (*end == '\0' && v >= 0 && v < (long)full) ? (uint32_t)v : full;
+}
 
 // Host-side checks of xkv_reconstruct_attend(_tail) and its launches, shared with the
 // allocation-free entry point.  attend_validate checks every argument rule, reports the

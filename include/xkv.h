@@ -35,7 +35,7 @@
  *  - Inputs holding NaN or Inf are outside the contract.
  *  - The library runs on compute capability 10.0 devices only (XKV_ERR_UNSUPPORTED
  *    otherwise).
- *  - Environment switches, read once per process on first use:
+ *  - Environment switches, read on every call:
  *      XKV_FORCE_SIMT  take the CUDA-core kernels for both attention paths instead of
  *                      the tensor-core ones (same results within the output tolerance)
  *      XKV_NO_TC       take the TMA + CUDA-core R-CLA kernel instead of the tensor-core one
@@ -238,7 +238,9 @@ xkv_status xkv_reconstruct_attend(const xkv_dims *dims, const void *Ak_win, cons
  *   q [B][Hq][hd], out [B][Hq][hd] fp32 (output)
  *   ws, ws_bytes: scratch of at least xkv_workspace_bytes(dims with ctx_len = L_max,
  *          0, XKV_MODE_RCLA) bytes.
- * dims->chunk, rank_k and rank_v are ignored.
+ * dims->chunk, rank_k and rank_v are ignored.  A bounded device-side wait that gives up
+ * makes the outputs of the (b, g) units whose rows it had not finished NaN (there is no
+ * status word on this path).
  */
 xkv_status rcla_decode_attend(const xkv_dims *dims, int32_t layer, const int32_t *leader_of,
                               int32_t n_layers, void *K_lead, void *V_lead, int64_t L_max,

@@ -604,6 +604,15 @@ def test_rcla_group_sizes(xkv, ora, G, length):
     assert np.array_equal(V.cpu().view(torch.int16).numpy().view(np.uint16), V_ref)
 
 
+@pytest.mark.parametrize("switch", ["XKV_NO_TC", "XKV_FORCE_SIMT"])
+@pytest.mark.parametrize("G,length", [(4, 5000), (5, 2100)])
+def test_rcla_other_kernels_bf16(xkv, ora, monkeypatch, switch, G, length):
+    """The TMA + CUDA-core kernel (XKV_NO_TC) and the plain CUDA-core kernel
+    (XKV_FORCE_SIMT) on bf16 caches the tensor-core kernel normally takes."""
+    monkeypatch.setenv(switch, "1")
+    test_rcla_group_sizes(xkv, ora, G, length)
+
+
 def test_rcla_outlier_values_are_attended(xkv, ora):
     """Rows whose V is 20x larger (1% of tokens) dominate nothing by themselves but must be
     carried exactly: compare against the oracle with the outliers present."""

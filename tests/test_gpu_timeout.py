@@ -1,10 +1,13 @@
 """The device-side timeout paths, exercised without faulting anything: a test-only variable
-shortens the poll limit of one kernel's pipeline waits so that they give up; every other
+sets the poll limit of one kernel's pipeline waits to 0, so that they give up at once (a
+single poll can succeed: mbarrier try_wait may suspend until the data lands); every other
 wait (and the drain of the copies and MMAs in flight) keeps its full bound.
 
 * The tensor-core attention kernels (explicit, rank-space selective, rank-space dense)
   must report XKV_ERR_TIMEOUT in the status word and NaN outputs, and the next call, with
   the normal limit, must be clean.
+* The R-CLA kernels (tensor-core, and TMA + CUDA-core) poison the partials of the items
+  they gave up on, so the outputs are NaN; the next call must match the oracle.
 * The fused selection's key pass must send the units it covers to the exact fp64 path:
   the selection stays the oracle's, and the next call takes the fp32 path again."""
 import dataclasses
@@ -50,7 +53,7 @@ def test_attention_wait_timeout_is_reported_then_the_next_call_is_clean(xkv, ora
         torch.cuda.synchronize()
         return int(ws[:4].cpu().view(torch.int32).item()), out.cpu().numpy()
 
-    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "1")
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "0")
     status, o = call()
     assert status & (1 << xkv.XKV_ERR_TIMEOUT), status
     assert np.all(np.isnan(o))
@@ -80,7 +83,7 @@ def test_selection_key_pass_timeout_falls_back_to_the_exact_path(xkv, ora, monke
         band = ws[:4 * w.batch * w.n_kv_heads].cpu().view(torch.int32).numpy().view(np.uint32)
         return sel.cpu().numpy(), band
 
-    monkeypatch.setenv("XKV_TEST_SS_SPIN", "1")
+    monkeypatch.setenv("XKV_TEST_SS_SPIN", "0")
     got, band = call()
     assert np.all(band == 0xFFFFFFFF), band          # every unit on the exact path
     assert np.array_equal(got, ref)
@@ -106,7 +109,7 @@ def _rank_space_timeout_then_clean(xkv, ora, monkeypatch, w, sel, units):
         torch.cuda.synchronize()
         return int(ws[:4].cpu().view(torch.int32).item()), out.cpu().numpy()
 
-    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "1")
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "0")
     status, o = call()
     assert status & (1 << xkv.XKV_ERR_TIMEOUT), status
     assert np.all(np.isnan(o))
@@ -139,3 +142,36 @@ def test_rank_space_dense_wait_timeout_is_reported_then_the_next_call_is_clean(
     w = dataclasses.replace(synth.reduced(synth.LLAMA8B_DENSE_128K, batch=1, ctx_len=8192),
                             n_q_heads=8, n_kv_heads=8, rank_k=256, rank_v=384, name="dense_g1")
     _rank_space_timeout_then_clean(xkv, ora, monkeypatch, w, None, [(0, 0), (0, 5)])
+
+
+@pytest.mark.parametrize("switch", [None, "XKV_NO_TC"], ids=["tensor_core", "tma"])
+def test_rcla_wait_timeout_gives_nan_then_the_next_call_is_clean(xkv, ora, monkeypatch, switch):
+    """A follower layer (no append, so both calls attend the same rows) over 20000 rows,
+    many items: every CTA gives up on its first item and poisons the items it owed."""
+    if switch:
+        monkeypatch.setenv(switch, "1")
+    length = 20000
+    w = dataclasses.replace(
+        synth.reduced(synth.QWEN3_8B_RCLA_32K, batch=1, ctx_len=length, n_layers=2,
+                      extra_rows=2, outlier_frac=0.0),
+        n_kv_heads=2, n_q_heads=8, name="rcla_timeout")
+    x = synth.np_rcla_inputs(w, seed=9, len_rows=length)
+    lo = ora.leader_map([0], 2)
+    K_ref = x["K_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    V_ref = x["V_lead"].view(torch.int16).numpy().view(np.uint16).copy()
+    ref = ora.rcla_decode_attend(1, lo, K_ref, V_ref, length, None, None, x["q"][1])
+    d = xkv.dims(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.L_max, dtype=w.dtype)
+    ws = torch.empty(xkv.xkv_workspace_bytes(d, 0, xkv.XKV_MODE_RCLA), dtype=torch.uint8,
+                     device=DEV)
+    K, V, q = x["K_lead"].to(DEV), x["V_lead"].to(DEV), x["q"][1].to(DEV)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device=DEV)
+
+    def call():
+        xkv.rcla_decode_attend(d, 1, lo, K, V, w.L_max, length, None, None, q, out, ws)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
+
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "0")
+    assert np.all(np.isnan(call()))
+    monkeypatch.delenv("XKV_TEST_MMA_SPIN")
+    compare_outputs(call(), ref, w.dtype)
