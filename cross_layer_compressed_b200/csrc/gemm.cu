@@ -51,6 +51,7 @@ struct GtParams {
     float *rho;
     int hd, chunk, Hkv;
     int64_t nC;
+    uint32_t mma_spin;       // poll limit of the MMA issuer's waits for staged data
 };
 
 struct GtShared {
@@ -94,8 +95,8 @@ __device__ __forceinline__ Tile gt_decode(const GtParams &p, int64_t t) {
 }
 
 __device__ __forceinline__ bool gt_wait(uint64_t *bar, uint32_t parity, GtShared *sh,
-                                        const GtParams &p) {
-    if (mbar_wait_bounded(bar, parity, &sh->abort, GT_SPIN)) return true;
+                                        const GtParams &p, uint32_t limit = GT_SPIN) {
+    if (mbar_wait_bounded(bar, parity, &sh->abort, limit)) return true;
     if (!*(volatile int *)&sh->abort) {
         *(volatile int *)&sh->abort = 1;
         if (p.status) atomicOr(p.status, 1u << XKV_ERR_TIMEOUT);
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
                 for (int kb = 0; kb < kb_tile; ++kb, ++it) {
                     const int s = (int)(it % GT_STAGES);
                     const uint32_t n = (uint32_t)(it / GT_STAGES);
-                    if (!gt_wait(&sh->full[s], n & 1, sh, p)) { ok = false; break; }
+                    if (!gt_wait(&sh->full[s], n & 1, sh, p, p.mma_spin)) { ok = false; break; }
                     tcgen05_after();
                     const uint32_t sa = base + s * GT_STAGE, sb = sa + GT_A_BYTES;
 #pragma unroll
@@ -550,6 +551,10 @@ cudaError_t launch_gemm(const GemmDesc &g, cudaStream_t s) {
     p.chunk = g.chunk;
     p.Hkv = g.Hkv;
     p.nC = g.nC;
+    // XKV_TEST_MMA_SPIN (tests only, read on every call): the poll limit of the MMA
+    // issuer's waits on staged data, so a test can make them give up; every other wait,
+    // and the drain that follows, keeps its full bound
+    p.mma_spin = test_poll_limit("XKV_TEST_MMA_SPIN", GT_SPIN);
     const size_t smem = 1024 + (size_t)GT_STAGES * GT_STAGE + sizeof(GtShared);
     cudaError_t e = set_smem_limit((const void *)k_gemm_tc, smem);
     if (e != cudaSuccess) return e;

@@ -8,6 +8,8 @@ wait (and the drain of the copies and MMAs in flight) keeps its full bound.
   the normal limit, must be clean.
 * The R-CLA kernels (tensor-core, and TMA + CUDA-core) poison the partials of the items
   they gave up on, so the outputs are NaN; the next call must match the oracle.
+* The factorization's tcgen05 products report XKV_ERR_TIMEOUT in the workspace status
+  word and leave NaN factors; the next call must match the oracle's truncated SVD.
 * The fused selection's key pass must send the units it covers to the exact fp64 path:
   the selection stays the oracle's, and the next call takes the fp32 path again."""
 import dataclasses
@@ -175,3 +177,34 @@ def test_rcla_wait_timeout_gives_nan_then_the_next_call_is_clean(xkv, ora, monke
     assert np.all(np.isnan(call()))
     monkeypatch.delenv("XKV_TEST_MMA_SPIN")
     compare_outputs(call(), ref, w.dtype)
+
+
+def test_factorization_product_timeout_is_reported_then_the_next_call_is_clean(
+        xkv, ora, monkeypatch):
+    W, B, L, Hkv, hd, r = 2, 2, 1000, 2, 64, 32
+    X, s = synth.np_window_caches(W, B, L, Hkv * hd, 96, r, 16.0, 0.05, 0)
+    Xs = synth.to_storage(X, "bf16")
+    d = xkv.dims(B, Hkv, Hkv, hd, L, chunk=8, rank_k=0, rank_v=0, dtype="bf16")
+    A = torch.empty((B, L, r), dtype=torch.bfloat16, device=DEV)
+    Bt = torch.empty((W, B, Hkv * hd, r), dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(xkv.xkv_factorize_workspace_bytes(d, W, r), dtype=torch.uint8, device=DEV)
+    om = torch.from_numpy(synth.np_test_matrix(W * Hkv * hd, r, 0)).to(DEV)
+    Xd = Xs.to(DEV)
+
+    def call():
+        xkv.xkv_factorize_window(d, W, r, Xd, om, 3, A, Bt, ws)
+        torch.cuda.synchronize()
+        return (int(ws[:4].cpu().view(torch.int32).item()), A.double().cpu().numpy(),
+                Bt.double().cpu().numpy())
+
+    monkeypatch.setenv("XKV_TEST_MMA_SPIN", "0")
+    status, A0, Bt0 = call()
+    assert status & (1 << xkv.XKV_ERR_TIMEOUT), status
+    assert np.all(np.isnan(A0)) and np.all(np.isnan(Bt0))
+    monkeypatch.delenv("XKV_TEST_MMA_SPIN")
+    status, A1, Bt1 = call()
+    assert status == 0
+    A_ref, Bt_ref, _ = ora.factorize_window(Xs.double().numpy(), r)
+    P_ref = ora.reconstruct_window(A_ref, Bt_ref)
+    err = np.abs(ora.reconstruct_window(A1, Bt1) - P_ref).max() / np.abs(P_ref).max()
+    assert err <= 2e-2, err
