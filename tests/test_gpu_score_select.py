@@ -8,7 +8,8 @@ made from landmarks built on the GPU.
   elements, so a selection made from them may differ from the oracle's selection from
   its own landmarks -- but only at certified near-ties: a chunk selected on one side only
   must score within 2 beta of the k-th candidate score, beta bounding how far any score
-  can move between the two landmark sets (parity section)."""
+  can move between the two landmark sets (the bound is derived in
+  parity_util.certify_near_ties)."""
 import dataclasses
 
 import numpy as np
