@@ -586,6 +586,24 @@ def profiled_traffic(workload: str, kernel: str, source: str):
     return None
 
 
+def count_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (every kernel one replay launches), or None
+    when the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        h = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(h, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(h, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kern = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kern)
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------ rank aggregation
 def max_over_ranks(x: float, world: int, device) -> float:
     """Max of a per-rank number over all ranks (the timed region's length)."""
@@ -933,12 +951,14 @@ def main():
         for slot in slots:
             wl.step(io=io[slot])
         torch.cuda.synchronize(dev)
-    graphs, e2e_graphs = {}, {}
+    graphs, e2e_graphs, graph_kernels = {}, {}, {}
     if use_graph:
         for slot in slots:
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g):
                 wl.step(slot)
+            graph_kernels[slot] = count_kernel_nodes(g)
+            g.instantiate()
             graphs[slot] = g
             if io:
                 g = torch.cuda.CUDAGraph()
@@ -1067,6 +1087,15 @@ def main():
                     "hbm_gbs": achieved, "hbm_frac": achieved / hbm_peak,
                     "bytes_per_launch": bytes_launch, "avg_launch_ms": attend_avg_ms}
 
+    # this library's kernels launched in the timed region: counted in the replayed graphs
+    # when the steps are graphs, else the launch plan
+    planned = wl.launches_per_step * args.steps
+    launches, launches_source = planned, "launch plan"
+    if use_graph and all(graph_kernels.get(sl) is not None for sl in slots):
+        launches = sum(graph_kernels[s % nq] for s in range(args.steps))
+        launches_source = "kernel nodes of the replayed CUDA graphs"
+        if launches != planned:
+            launches_source += f" (launch plan: {planned})"
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -1099,7 +1128,8 @@ def main():
             "config": cfg,
             "step_gbs": step_bytes / (ms_step / 1e3) / 1e9,
             "roofline": roofline,
-            "gpu_launches": wl.launches_per_step * args.steps,
+            "gpu_launches": launches,
+            "gpu_launches_source": launches_source,
             "score_select_avg_ms": select_avg_ms,
             "cuda_graph": use_graph,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
