@@ -88,23 +88,6 @@ def measured_tflops_sustained():
 
 # --------------------------------------------------------------------------- clocks
 
-def _ra_kernels(w, n_sel):
-    """Kernels of one rank-space attention call, following the library's launch plan: q~,
-    the attention kernel, then the split merge and the projection, as one kernel when a
-    head has 32 or more splits (dense calls at small batch), else as two.  Dense calls
-    here take the head-batched kernel: one span of whole 128-token tiles per SM (148 spans)
-    over the batch; selective calls split each unit's rows into items of <= 256 rows."""
-    if n_sel == 0:
-        tiles = -(-w.ctx_len // 128)
-        ns = max(1, min(148 // w.batch, tiles))
-        tps = -(-tiles // ns)
-        n_split = -(-tiles // tps)
-    else:
-        n_split = -(-(n_sel * w.chunk) // 256)
-        per = -(-n_sel // n_split)
-        n_split = -(-n_sel // per)
-    return 3 if n_split >= 32 else 4
-
 class ClockSampler:
     """This GPU's SM clock and clock-event (throttle) reasons, polled through NVML (the
     source nvidia-smi reads) every ~2 ms on a thread while the timed region runs, so a
@@ -165,6 +148,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------ workloads
+def _ra_kernels(w, n_sel):
+    """Kernels of one rank-space attention call, following the library's launch plan: q~,
+    the attention kernel, then the split merge and the projection, as one kernel when a
+    head has 32 or more splits (dense calls at small batch), else as two.  Dense calls
+    here take the head-batched kernel: one span of whole 128-token tiles per SM (148 spans)
+    over the batch; selective calls split each unit's rows into items of <= 256 rows."""
+    if n_sel == 0:
+        tiles = -(-w.ctx_len // 128)
+        ns = max(1, min(148 // w.batch, tiles))
+        tps = -(-tiles // ns)
+        n_split = -(-tiles // tps)
+    else:
+        n_split = -(-(n_sel * w.chunk) // 256)
+        per = -(-n_sel // n_split)
+        n_split = -(-n_sel // per)
+    return 3 if n_split >= 32 else 4
+
+
 class IoOverlap:
     """The host<->device copies of one end-to-end step, on a copy stream, overlapped with
     the layers: every layer's queries are issued at the start (after the copy stream has
