@@ -18,12 +18,13 @@
 //                              (M = hd = 128, N = tokens rounded up to 16)
 //                 so keys come out one token per TMEM lane and values one head-dim per
 //                 lane: neither epilogue needs a cross-thread reduction.
-//   warps 1-4     TMA producers.  Each 8-row group of the item's A rows is one 8 x 64
-//                 box (a selected chunk is 8 contiguous rows, so a group is one 128-byte
-//                 swizzle atom); the groups are spread over the four warps because the
-//                 per-box cost of the tensor-copy unit, not bandwidth, bounds how fast one
-//                 warp can feed a stage.  Warp 1 also loads the 16 KB B slice.
-//   warps 5-12    epilogue in two groups of four (group 1 takes rows / tokens 128..255).
+//   warps 1-8     TMA producers (warps 1-4 when G > 6).  Each 8-row group of the item's A
+//                 rows is one 8 x 64 box (a selected chunk is 8 contiguous rows, so a
+//                 group is one 128-byte swizzle atom); the groups are spread over the
+//                 warps (four boxes each) because the cost of issuing the boxes, not
+//                 bandwidth, bounds how fast one warp can feed a stage.  Warp 1 also loads
+//                 the 16 KB B slice.
+//   next 8 warps  epilogue in two groups of four (group 1 takes rows / tokens 128..255).
 //                 Key epilogue: thread = token, logits z_h = q_h . K_hat (fp32); then the
 //                 exact max / sum of the item's rows.  Value epilogue: thread = output
 //                 column j, o_h[j] = sum_t p_h[t] V_hat[t][j]; the groups' halves are
@@ -47,9 +48,17 @@ constexpr int TC_HD = 128;
 constexpr int A_TILE = TC_ROWS * TC_KS * 2;  // 32 KB: 32 row groups of 8 x 128 B
 constexpr int B_TILE = TC_HD * TC_KS * 2;    // 16 KB
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
-constexpr int W_MMA = 0, W_LOAD = 1, N_LOAD = 4, W_EPI = 5, N_EPI = 8;
-constexpr int TC_THREADS = 32 * (W_EPI + N_EPI);       // 416
+constexpr int W_MMA = 0, W_LOAD = 1, N_EPI = 8;
 constexpr int EPI_THREADS = 32 * N_EPI;                // 256
+// Producer warps: eight for groups of up to 6 query heads (544 threads, 96 registers
+// each, no spills); the larger groups' epilogue needs the 128 registers a 416-thread CTA
+// of four producer warps leaves it.
+template <int G>
+struct TcRoles {
+    static constexpr int N_LOAD = G <= 6 ? 8 : 4;
+    static constexpr int W_EPI = W_LOAD + N_LOAD;
+    static constexpr int THREADS = 32 * (W_EPI + N_EPI);
+};
 constexpr uint32_t SPIN_LIMIT = 1u << 24;
 
 struct TcShared {
@@ -145,7 +154,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *b, uint32_t parity, TcShared
 }
 
 template <int G>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TcRoles<G>::THREADS, 1)
     k_xkv_tc(const __grid_constant__ CUtensorMap tmAk, const __grid_constant__ CUtensorMap tmAv,
              const __grid_constant__ CUtensorMap tmBk, const __grid_constant__ CUtensorMap tmBv,
              const TcParams p) {
@@ -189,6 +198,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     grid_dep_wait();    // selection, query and status come from the kernels before
     grid_dep_launch();
 
+    constexpr int N_LOAD = TcRoles<G>::N_LOAD, W_EPI = TcRoles<G>::W_EPI;
     if (warp >= W_LOAD && warp < W_LOAD + N_LOAD) {
         // ------------------------------------------------------------ TMA producers
         const int pi = warp - W_LOAD;              // row groups pi, pi + 4, ... of an item
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                     unsigned char *st = smem + s * STAGE_BYTES;
                     if (pi == 0 && lane == 0) {
-                        // the stage's one arrival, with every byte its four warps will load
+                        // the stage's one arrival, with every byte the producer warps will load
                         mbar_expect_tx(&sh->full[s], (uint32_t)(ng * 1024 + B_TILE));
                         tma_load_2d(mB, &sh->full[s], st + A_TILE, ks * TC_KS, brow);
                     }
@@ -234,9 +244,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
         if (!ok && pi == 0 && lane == 0) {
-            // Every stage the four warps issued lands before the CTA may leave: the last
+            // Every stage the producer warps issued lands before the CTA may leave: the last
             // TC_STAGES fills (each issued whole: a warp checks for abort only in its wait
-            // on `empty`, which completes for all four warps alike) complete their phase.
+            // on `empty`, which completes for all of them alike) complete their phase.
             for (int j = it - TC_STAGES > 0 ? it - TC_STAGES : 0; j < it; ++j)
                 for (uint32_t i = 0; i < SPIN_LIMIT; ++i)
                     if (mbar_test(&sh->full[j % TC_STAGES], (uint32_t)(j / TC_STAGES) & 1)) break;
@@ -300,7 +310,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int et = threadIdx.x - 32 * W_EPI;  // 0..255
-        const int ew = warp - W_EPI;              // 0..7
+        const int ew = warp - W_EPI;              // 0..7 (each group of four covers the
+                                                  // four TMEM lane quadrants, warp & 3)
         const int grp = ew >> 2;                  // rows / tokens [128 grp, 128 grp + 128)
         const int quad = warp & 3;                // TMEM lane quadrant of this warp
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
@@ -455,7 +466,7 @@ cudaError_t launch_g(const CUtensorMap *maps, const TcParams &p, cudaStream_t s)
     cudaError_t e = set_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
-    return launch_chained(k, dim3(grid), dim3(TC_THREADS), smem, s, maps[0], maps[1], maps[2],
+    return launch_chained(k, dim3(grid), dim3(TcRoles<G>::THREADS), smem, s, maps[0], maps[1], maps[2],
                           maps[3], p);
 }
 

@@ -227,6 +227,20 @@ def test_reconstruct_attend_selective(xkv, ora, w):
     compare_outputs(got, ref, w.dtype)
 
 
+@pytest.mark.parametrize("G", [1, 2, 6, 7, 8, 16])
+def test_reconstruct_attend_group_sizes(xkv, ora, G):
+    """The tensor-core kernel for group sizes on both sides of its role split: eight
+    producer warps up to 6 query heads per KV head, four above (the larger epilogue needs
+    the registers)."""
+    w = dataclasses.replace(synth.reduced(synth.LLAMA8B_SR_32K, batch=2, ctx_len=2048, top_k=24),
+                            n_kv_heads=2, n_q_heads=2 * G, name=f"sr_g{G}")
+    x = _layer_inputs(w)
+    lm = _host_lm(ora, ora.build_landmarks(x["Ak"], x["Bkt"], w.n_kv_heads, w.head_dim, w.chunk))
+    sel = ora.select_chunks(ora.score_landmarks(lm, x["q"]), w.top_k, w.n_sink, w.n_recent)
+    ref = ora.reconstruct_attend(x["Ak"], x["Av"], x["Bkt"], x["Bvt"], x["q"], sel, w.chunk)
+    compare_outputs(_attend(xkv, w, x, sel), ref, w.dtype)
+
+
 @pytest.mark.parametrize("w", [LLAMA_R, QWEN14_R], ids=lambda w: w.name)
 def test_reconstruct_attend_cuda_core_path_bf16(xkv, ora, w, monkeypatch):
     """The CUDA-core kernel on bf16 shapes the tensor-core kernel normally takes."""
