@@ -160,7 +160,7 @@ cudaError_t launch_chained(void (*k)(P...), dim3 grid, dim3 block, size_t smem, 
 // Sets the calling thread's xkv_last_error() message (defined with the C ABI layer).
 void set_last_error(const char *msg);
 
-// Environment switches (documented in include/xkv.h), read once per process:
+// Environment switches (documented in include/xkv.h), read on every call:
 // XKV_FORCE_SIMT takes the CUDA-core kernels for both attentions, XKV_NO_TC the TMA +
 // CUDA-core R-CLA kernel, XKV_NO_PDL plain stream order for every launch.
 enum EnvFlag { ENV_FORCE_SIMT = 0, ENV_NO_TC = 1, ENV_NO_PDL = 2 };
